@@ -1,0 +1,268 @@
+"""Plain fp64 NumPy definition of each step of the packed joint-attention block.
+
+TEST INFRASTRUCTURE ONLY (see ``oracle/__init__.py``): slow, obviously correct,
+no blocking or fusion beyond what each definition states. Inputs arrive as
+float32 arrays holding exact bf16 values; every computation is float64.
+"""
+
+from __future__ import annotations
+
+import math
+from typing import Optional, Sequence
+
+import numpy as np
+
+MOD_IMG = 0  # modality id of image-latent tokens
+MOD_TXT = 1  # modality id of text tokens
+
+SHIFT, SCALE, GATE = 0, 1, 2  # order of the three modulation vectors
+
+
+# ---------------------------------------------------------------------------
+# Pack metadata  ([pack], [rope], [edit])
+# ---------------------------------------------------------------------------
+def pack_build(descs: Sequence, rope_axes: int):
+    """Per-sample cumulative offsets and per-token ids of a native-resolution pack.
+
+    [pack]: samples share one flat token buffer; sample s owns tokens
+    ``cu_seqlens[s] .. cu_seqlens[s+1]-1``.
+
+    Readings (the pages give no layout):
+      * inside a sample, image tokens come first, frame-major then row-major
+        (f, h, w), followed by the text tokens;
+      * an image token's position is (f, h, w); for 2D packs f = 0 ([rope]),
+        for edit packs the frame index tells source (0) from target (1) ([edit]);
+      * text token j sits on a 1D axis after the image grid: p = max(Hg, Wg) + j
+        on every axis, i.e. position (p, p, p);
+      * a text-only segment (frames = 0, empty grid) has positions 0, 1, 2, ...
+
+    Returns a dict with int32 ``cu_seqlens`` [S+1], int32 ``pos_ids`` [T][3]
+    (f, h, w), int32 ``tok_sample`` [T], uint8 ``tok_mod`` [T] (0 image,
+    1 text) and ``T``.
+    """
+    descs = [tuple(d.as_tuple()) if hasattr(d, "as_tuple") else tuple(d) for d in descs]
+    if rope_axes not in (2, 3):
+        raise ValueError("rope_axes must be 2 or 3")
+    n = []
+    for (F, Hg, Wg, L, *_rest) in descs:
+        if min(F, Hg, Wg, L) < 0:
+            raise ValueError("negative descriptor field")
+        if rope_axes == 2 and F > 1:
+            raise ValueError("a 2D pack holds one frame per sample")
+        if rope_axes == 3 and F > 2:
+            raise ValueError("an edit pack holds at most two frames per sample")
+        n.append(F * Hg * Wg + L)
+    S = len(descs)
+    cu = np.zeros(S + 1, dtype=np.int64)
+    cu[1:] = np.cumsum(np.asarray(n, dtype=np.int64))
+    T = int(cu[-1])
+    pos = np.zeros((T, 3), dtype=np.int32)
+    tok_sample = np.zeros(T, dtype=np.int32)
+    tok_mod = np.zeros(T, dtype=np.uint8)
+    for s, (F, Hg, Wg, L, *_rest) in enumerate(descs):
+        start = int(cu[s])
+        n_img = F * Hg * Wg
+        f, h, w = np.meshgrid(np.arange(F), np.arange(Hg), np.arange(Wg), indexing="ij")
+        pos[start:start + n_img, 0] = f.ravel()
+        pos[start:start + n_img, 1] = h.ravel()
+        pos[start:start + n_img, 2] = w.ravel()
+        p = max(Hg, Wg) + np.arange(L)
+        pos[start + n_img:start + n_img + L, :] = p[:, None]
+        tok_sample[start:start + n_img + L] = s
+        tok_mod[start + n_img:start + n_img + L] = MOD_TXT
+    return dict(cu_seqlens=cu.astype(np.int32), pos_ids=pos, tok_sample=tok_sample,
+                tok_mod=tok_mod, T=T)
+
+
+# ---------------------------------------------------------------------------
+# Modality-specific adaptive LayerNorm  ([norm], [fuse])
+# ---------------------------------------------------------------------------
+def adaln_params(c: np.ndarray, W: np.ndarray, hid: int) -> np.ndarray:
+    """Per-sample, per-modality shift / scale / gate vectors.
+
+    Reading: a plain linear map of the conditioning vector (no bias, no
+    activation): ``mod[s][m][j][i] = sum_c c[s][c] * W[c][(3*m + j)*hid + i]``
+    with m in {image, text} and j in {shift, scale, gate}.
+    Returns float64 [S][2][3][hid].
+    """
+    c = np.asarray(c, dtype=np.float64)
+    W = np.asarray(W, dtype=np.float64)
+    S = c.shape[0]
+    if W.shape != (c.shape[1], 6 * hid):
+        raise ValueError("W must be [C][6*hid]")
+    return (c @ W).reshape(S, 2, 3, hid)
+
+
+def layer_norm_rows(x: np.ndarray, eps: float) -> np.ndarray:
+    """LayerNorm without affine parameters over the last axis: population
+    variance, ``(x - mean) / sqrt(var + eps)``."""
+    x = np.asarray(x, dtype=np.float64)
+    mu = x.mean(axis=-1, keepdims=True)
+    var = np.mean((x - mu) ** 2, axis=-1, keepdims=True)
+    return (x - mu) / np.sqrt(var + eps)
+
+
+def adaln_modulate(x, mod, tok_sample, tok_mod, eps: float = 1e-6, rows=None):
+    """``x_mod[t] = LN(x[t]) * (1 + scale[s, m]) + shift[s, m]`` with s the
+    token's sample and m its modality ([norm]). Reading: eps = 1e-6, no affine
+    LayerNorm parameters. ``rows`` restricts the output to those token rows."""
+    x = np.asarray(x, dtype=np.float64)
+    tok_sample = np.asarray(tok_sample)
+    tok_mod = np.asarray(tok_mod)
+    if rows is not None:
+        x, tok_sample, tok_mod = x[rows], tok_sample[rows], tok_mod[rows]
+    ln = layer_norm_rows(x, eps)
+    shift = mod[tok_sample, tok_mod, SHIFT]
+    scale = mod[tok_sample, tok_mod, SCALE]
+    return ln * (1.0 + scale) + shift
+
+
+# ---------------------------------------------------------------------------
+# Per-sample 2D / 3D rotary embedding  ([rope], [edit])
+# ---------------------------------------------------------------------------
+def rope_split(D: int, rope_axes: int) -> int:
+    """Channels given to each axis. Reading: head_dim is split evenly across
+    the axes in whole pairs, ``d_a = 2 * floor(D / (2 * axes))``; the chunks are
+    contiguous in axis order ((h, w) for 2D, (f, h, w) for 3D) and any leftover
+    channels at the end are not rotated (D = 128, 3D: 42 | 42 | 42 | 2 kept)."""
+    if D % 2:
+        raise ValueError("head_dim must be even")
+    return 2 * (D // (2 * rope_axes))
+
+
+def rope_pair_angles(pos_ids: np.ndarray, D: int, rope_axes: int, base: float = 10000.0):
+    """Rotation angle of every channel pair for every token: float64 [T][D/2].
+
+    Pair i of an axis chunk of width d_a turns by
+    ``theta = pos_axis * base ** (-2 i / d_a)`` (reading: base 10000); pairs past
+    the last chunk get angle 0."""
+    pos_ids = np.asarray(pos_ids)
+    d_a = rope_split(D, rope_axes)
+    comps = (1, 2) if rope_axes == 2 else (0, 1, 2)  # which (f, h, w) entry drives each chunk
+    inv_freq = np.power(float(base), -np.arange(0, d_a, 2, dtype=np.float64) / d_a)  # [d_a/2]
+    theta = np.zeros((pos_ids.shape[0], D // 2), dtype=np.float64)
+    for a, comp in enumerate(comps):
+        p = pos_ids[:, comp].astype(np.float64)
+        theta[:, a * (d_a // 2):(a + 1) * (d_a // 2)] = p[:, None] * inv_freq[None, :]
+    return theta
+
+
+def rope_apply(x, pos_ids, rope_axes: int, base: float = 10000.0, rows=None):
+    """Rotate interleaved channel pairs ``(x[2i], x[2i+1])`` of every head by the
+    token's angles: ``x0' = x0 cos - x1 sin``, ``x1' = x0 sin + x1 cos``.
+    Reading: pairs are adjacent channels. x is [T][H][D]; returns float64."""
+    x = np.asarray(x, dtype=np.float64)
+    pos_ids = np.asarray(pos_ids)
+    if rows is not None:
+        x, pos_ids = x[rows], pos_ids[rows]
+    D = x.shape[-1]
+    theta = rope_pair_angles(pos_ids, D, rope_axes, base)[:, None, :]  # [T][1][D/2]
+    cos, sin = np.cos(theta), np.sin(theta)
+    x0, x1 = x[..., 0::2], x[..., 1::2]
+    out = np.empty_like(x)
+    out[..., 0::2] = x0 * cos - x1 * sin
+    out[..., 1::2] = x0 * sin + x1 * cos
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Block-diagonal variable-length attention  ([pack], [norm])
+# ---------------------------------------------------------------------------
+def varlen_attention(q, k, v, cu_seqlens, scale: Optional[float] = None,
+                     rows=None, chunk: int = 2048):
+    """Joint self-attention inside each sample of the pack: for sample s and
+    head h, ``O = softmax(Q K^T * scale) V`` over the sample's own tokens (image
+    and text together, no mask inside a sample, nothing across samples).
+    Reading: scale = 1/sqrt(D).
+
+    q, k, v: [T][H][D]. Returns (O float64 [T][H][D], lse float64 [H][T]) where
+    ``lse = log sum_j exp(s_ij)`` (natural log). With ``rows`` (sorted token
+    indices) only those query rows are computed; O is then [len(rows)][H][D] and
+    lse [H][len(rows)]. Query rows are processed ``chunk`` at a time only to
+    bound memory."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    T, H, D = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    rows = np.arange(T) if rows is None else np.asarray(rows, dtype=np.int64)
+    out = np.zeros((rows.shape[0], H, D), dtype=np.float64)
+    lse = np.zeros((H, rows.shape[0]), dtype=np.float64)
+    sample_of_row = np.searchsorted(cu, rows, side="right") - 1
+    for s in range(len(cu) - 1):
+        lo, hi = int(cu[s]), int(cu[s + 1])
+        sel = np.nonzero(sample_of_row == s)[0]
+        if sel.size == 0 or hi == lo:
+            continue
+        for h in range(H):
+            Ks = k[lo:hi, h, :]
+            Vs = v[lo:hi, h, :]
+            for c0 in range(0, sel.size, chunk):
+                idx = sel[c0:c0 + chunk]
+                Qc = q[rows[idx], h, :]
+                Sc = (Qc @ Ks.T) * scale
+                m = Sc.max(axis=1, keepdims=True)
+                P = np.exp(Sc - m)
+                l = P.sum(axis=1, keepdims=True)
+                out[idx, h, :] = (P @ Vs) / l
+                lse[h, idx] = (m + np.log(l))[:, 0]
+    return out, lse
+
+
+# ---------------------------------------------------------------------------
+# Gated residual  ([fuse])
+# ---------------------------------------------------------------------------
+def gated_residual(x, o, mod, tok_sample, tok_mod, rows=None):
+    """``y[t] = x[t] + gate[s, m] * O[t]`` with O viewed as [T][H*D] (head-major
+    columns). Reading: the gate multiplies the attention branch and is added to
+    the block input (adaLN-zero form; no output projection on this path)."""
+    x = np.asarray(x, dtype=np.float64)
+    tok_sample = np.asarray(tok_sample)
+    tok_mod = np.asarray(tok_mod)
+    if rows is not None:
+        x, tok_sample, tok_mod = x[rows], tok_sample[rows], tok_mod[rows]
+    o = np.asarray(o, dtype=np.float64).reshape(x.shape[0], -1)
+    gate = mod[tok_sample, tok_mod, GATE]
+    return x + gate * o
+
+
+# ---------------------------------------------------------------------------
+# The whole block
+# ---------------------------------------------------------------------------
+def block_fwd(x, q, k, v, mod, pack, rope_axes: int, base: float = 10000.0,
+              eps: float = 1e-6, rows=None):
+    """adaLN modulation, RoPE on Q and K, joint varlen attention and the gated
+    residual, in the order the fused chain names them ([fuse]). Returns
+    (x_mod, y, O) in float64, restricted to ``rows`` when given."""
+    tok_sample, tok_mod = pack["tok_sample"], pack["tok_mod"]
+    x_mod = adaln_modulate(x, mod, tok_sample, tok_mod, eps, rows=rows)
+    q_r = rope_apply(q, pack["pos_ids"], rope_axes, base, rows=rows) if rows is not None \
+        else rope_apply(q, pack["pos_ids"], rope_axes, base)
+    k_r = rope_apply(k, pack["pos_ids"], rope_axes, base)
+    if rows is not None:
+        # attention needs every key of the sampled rows' samples, but only the
+        # sampled query rows; scatter the roped query rows back in place.
+        q_full = np.zeros(np.asarray(q).shape, dtype=np.float64)
+        q_full[rows] = q_r
+        q_r = q_full
+    o, _ = varlen_attention(q_r, k_r, v, pack["cu_seqlens"], rows=rows)
+    y = gated_residual(x, o, mod, tok_sample, tok_mod, rows=rows)
+    return x_mod, y, o
+
+
+def useful_attention_flops(descs: Sequence, H: int, D: int) -> float:
+    """Useful attention FLOPs of a pack: ``4 * D * H * sum n_s^2`` over the real
+    samples (QK^T and PV, 2 FLOPs per multiply-add, only within-sample pairs,
+    the padding segment excluded)."""
+    tot = 0
+    for d in descs:
+        t = tuple(d.as_tuple()) if hasattr(d, "as_tuple") else tuple(d)
+        F, Hg, Wg, L = t[:4]
+        dummy = t[4] if len(t) > 4 else 0
+        if dummy:
+            continue
+        n = F * Hg * Wg + L
+        tot += n * n
+    return 4.0 * D * H * tot

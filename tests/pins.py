@@ -1,0 +1,350 @@
+"""Reusable pin checks for the oracle.
+
+Each ``check_*`` takes the oracle function(s) it pins as arguments and raises
+AssertionError when they break a property fixed by the pages, by mathematics or
+by an independent computation. ``test_oracle_pins.py`` runs them on the oracle;
+``test_oracle_mutations.py`` runs them on deliberately broken copies to show
+that each plausible slip is caught.
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+from oracle import brute
+from packgen import SampleDesc, make_random_pack
+
+
+# --------------------------------------------------------------------- pack
+def check_pack_vs_brute(pack_build):
+    for seed in range(6):
+        for axes in (2, 3):
+            w = make_random_pack(100 + seed, S=1 + seed % 4, H=1, D=8, rope_axes=axes)
+            p = pack_build(w.descs, axes)
+            cu, pos, ts, tm = brute.brute_pack(w.descs, axes)
+            assert p["cu_seqlens"].tolist() == cu
+            assert p["pos_ids"].tolist() == [list(t) for t in pos]
+            assert p["tok_sample"].tolist() == ts
+            assert p["tok_mod"].tolist() == tm
+
+
+def check_pack_tiny_closed_form(pack_build):
+    # The 544-token pack: sample A = 16x16 grid + 20 text, B = 8x32 grid + 12 text.
+    p = pack_build([SampleDesc(1, 16, 16, 20), SampleDesc(1, 8, 32, 12)], 2)
+    nA, nB = 16 * 16 + 20, 8 * 32 + 12
+    assert p["cu_seqlens"].tolist() == [0, nA, nA + nB]
+    pos = p["pos_ids"]
+    assert pos[0].tolist() == [0, 0, 0]
+    assert pos[17].tolist() == [0, 1, 1]          # row-major: 17 = 1*16 + 1
+    assert pos[255].tolist() == [0, 15, 15]
+    assert pos[256].tolist() == [16, 16, 16]      # first text token: max(16,16) + 0
+    assert pos[nA - 1].tolist() == [16 + 19] * 3
+    assert pos[nA + 31].tolist() == [0, 0, 31]    # B is 8 rows of 32
+    assert pos[nA + 32].tolist() == [0, 1, 0]
+    assert pos[nA + 256].tolist() == [32, 32, 32]  # max(8,32) + 0
+    assert int((p["tok_mod"] == 1).sum()) == 32
+    assert p["tok_sample"][nA - 1] == 0 and p["tok_sample"][nA] == 1
+
+
+def check_pack_edit_frames(pack_build):
+    # Edit pack: source (f=0) and target (f=1) share every (h, w) ([edit]).
+    p = pack_build([SampleDesc(2, 3, 4, 2)], 3)
+    pos = p["pos_ids"]
+    n_grid = 3 * 4
+    assert (pos[:n_grid, 0] == 0).all() and (pos[n_grid:2 * n_grid, 0] == 1).all()
+    assert (pos[:n_grid, 1:] == pos[n_grid:2 * n_grid, 1:]).all()
+    assert pos[2 * n_grid].tolist() == [4, 4, 4]
+
+
+# ---------------------------------------------------------------------- adaLN
+def check_mod_layout(adaln_params):
+    # W is a selector: column (3m + j)*hid + i reads conditioning entry
+    # code(m, j, i) = (7m + 3j + 5i) mod C, so each slot has a distinct source.
+    C, hid, S = 16, 5, 2
+    c = np.arange(S * C, dtype=np.float64).reshape(S, C) + 1.0
+    W = np.zeros((C, 6 * hid))
+    for m in range(2):
+        for j in range(3):
+            for i in range(hid):
+                W[(7 * m + 3 * j + 5 * i) % C, (3 * m + j) * hid + i] = 1.0
+    mod = adaln_params(c, W, hid)
+    assert mod.shape == (S, 2, 3, hid)
+    for s in range(S):
+        for m in range(2):
+            for j in range(3):
+                for i in range(hid):
+                    assert mod[s, m, j, i] == c[s, (7 * m + 3 * j + 5 * i) % C]
+
+
+def check_mod_vs_brute(adaln_params):
+    rng = np.random.default_rng(7)
+    c = rng.standard_normal((3, 6))
+    W = rng.standard_normal((6, 6 * 4))
+    got = adaln_params(c, W, 4)
+    ref = brute.brute_mod(c.tolist(), W.tolist(), 4)
+    assert np.allclose(got, np.array(ref), rtol=0, atol=1e-12)
+
+
+def check_layernorm_moments(layer_norm_rows):
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((20, 96)) * 3.0 + 1.5
+    eps = 1e-6
+    y = layer_norm_rows(x, eps)
+    var = x.var(axis=1)
+    assert np.allclose(y.mean(axis=1), 0.0, atol=1e-12)
+    # population variance of the output is var / (var + eps)
+    assert np.allclose(y.var(axis=1), var / (var + eps), atol=1e-12)
+    # a constant row maps to zero (0 / sqrt(eps))
+    assert np.allclose(layer_norm_rows(np.full((1, 8), 4.0), eps), 0.0)
+
+
+def check_adaln_zero_map(adaln_params, adaln_modulate, layer_norm_rows, gated_residual):
+    w = make_random_pack(11, S=3, H=2, D=8, rope_axes=2)
+    from oracle import pack_build  # descriptors -> per-token ids
+    p = pack_build(w.descs, 2)
+    mod = adaln_params(w.c, np.zeros_like(w.W), w.hid)
+    x = w.f32("x")
+    assert np.array_equal(adaln_modulate(x, mod, p["tok_sample"], p["tok_mod"], 1e-6),
+                          layer_norm_rows(x, 1e-6))
+    o = np.random.default_rng(0).standard_normal((w.T, w.H, w.D))
+    assert np.array_equal(gated_residual(x, o, mod, p["tok_sample"], p["tok_mod"]),
+                          x.astype(np.float64))
+
+
+def check_adaln_vs_brute(adaln_params, adaln_modulate, pack_build):
+    w = make_random_pack(12, S=3, H=2, D=8, rope_axes=2)
+    p = pack_build(w.descs, 2)
+    mod = adaln_params(w.c, w.W, w.hid)
+    x = w.f32("x")
+    got = adaln_modulate(x, mod, p["tok_sample"], p["tok_mod"], 1e-6)
+    for t in range(w.T):
+        s, m = int(p["tok_sample"][t]), int(p["tok_mod"][t])
+        ref = brute.brute_adaln_row(x[t].tolist(), mod[s, m, 0].tolist(), mod[s, m, 1].tolist(), 1e-6)
+        assert np.allclose(got[t], ref, rtol=0, atol=1e-12)
+
+
+# ----------------------------------------------------------------------- RoPE
+def _pos_rows(n, rng, hi=50):
+    return rng.integers(0, hi, size=(n, 3)).astype(np.int32)
+
+
+def check_rope_identity_and_norm(rope_apply):
+    rng = np.random.default_rng(5)
+    for D, axes in ((64, 2), (128, 2), (128, 3), (8, 2)):
+        x = rng.standard_normal((9, 3, D))
+        assert np.array_equal(rope_apply(x, np.zeros((9, 3), np.int32), axes), x)
+        y = rope_apply(x, _pos_rows(9, rng), axes)
+        n0 = x[..., 0::2] ** 2 + x[..., 1::2] ** 2
+        n1 = y[..., 0::2] ** 2 + y[..., 1::2] ** 2
+        assert np.allclose(n0, n1, rtol=1e-12, atol=1e-12)
+
+
+def check_rope_relative(rope_apply):
+    """<R(p) q, R(p') k> depends only on p - p' on every axis."""
+    rng = np.random.default_rng(6)
+    for D, axes in ((64, 2), (128, 2), (128, 3)):
+        q = rng.standard_normal((1, 1, D))
+        k = rng.standard_normal((1, 1, D))
+        for _ in range(5):
+            p = _pos_rows(1, rng)
+            pp = _pos_rows(1, rng)
+            shift = rng.integers(0, 30, size=(1, 3)).astype(np.int32)
+            a = np.sum(rope_apply(q, p, axes) * rope_apply(k, pp, axes))
+            b = np.sum(rope_apply(q, p + shift, axes) * rope_apply(k, pp + shift, axes))
+            assert abs(a - b) < 1e-9 * max(1.0, abs(a))
+        # and it does depend on the difference on each rotated axis
+        p = np.zeros((1, 3), np.int32)
+        comps = (1, 2) if axes == 2 else (0, 1, 2)
+        base_val = np.sum(rope_apply(q, p, axes) * rope_apply(k, p, axes))
+        for comp in comps:
+            pp = p.copy()
+            pp[0, comp] = 3
+            moved = np.sum(rope_apply(q, p, axes) * rope_apply(k, pp, axes))
+            assert abs(moved - base_val) > 1e-6
+
+
+def check_rope_textbook_1d(rope_apply):
+    """A 2D pack whose grid is one column wide (w = 0 everywhere) reduces to
+    textbook 1D RoPE on the h channels, written here as complex multiplication
+    z_i * exp(i * p * base**(-2i/d)) over the first d = D/2 channels, while the
+    w channels stay put."""
+    rng = np.random.default_rng(8)
+    for D in (64, 128):
+        d = D // 2
+        x = rng.standard_normal((7, 2, D))
+        h = np.arange(7)
+        pos = np.stack([np.zeros(7), h, np.zeros(7)], axis=1).astype(np.int32)
+        y = rope_apply(x, pos, 2)
+        z = x[..., 0:d:2] + 1j * x[..., 1:d:2]
+        omega = 10000.0 ** (-np.arange(d // 2) * 2.0 / d)
+        zr = z * np.exp(1j * h[:, None, None] * omega[None, None, :])
+        assert np.allclose(y[..., 0:d:2], zr.real, atol=1e-12)
+        assert np.allclose(y[..., 1:d:2], zr.imag, atol=1e-12)
+        assert np.array_equal(y[..., d:], x[..., d:])
+
+
+def check_rope_3d_layout(rope_apply):
+    """3D, D = 128: chunks of 42 channels for f, h, w; channels 126-127 are
+    never rotated; moving only the frame index touches only channels 0-41."""
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal((4, 1, 128))
+    base_pos = np.array([[0, 5, 7]] * 4, np.int32)
+    y0 = rope_apply(x, base_pos, 3)
+    pos_f = base_pos.copy()
+    pos_f[:, 0] = 1
+    y1 = rope_apply(x, pos_f, 3)
+    assert np.array_equal(y0[..., 42:], y1[..., 42:])
+    assert not np.allclose(y0[..., :42], y1[..., :42])
+    far = np.array([[9, 99, 999]] * 4, np.int32)
+    assert np.array_equal(rope_apply(x, far, 3)[..., 126:], x[..., 126:])
+    # angle of pair i of the h chunk at h = 1, recovered with atan2 from a unit pair
+    e = np.zeros((1, 1, 128))
+    e[..., 42::2] = 1.0  # the first channel of every pair from channel 42 on
+    ang = rope_apply(e, np.array([[0, 1, 0]], np.int32), 3)
+    got = np.arctan2(ang[0, 0, 43:84:2], ang[0, 0, 42:84:2])
+    assert np.allclose(got, 10000.0 ** (-np.arange(21) * 2.0 / 42), atol=1e-12)
+
+
+def check_rope_vs_brute(rope_apply, pack_build):
+    for axes in (2, 3):
+        w = make_random_pack(13 + axes, S=3, H=2, D=16, rope_axes=axes)
+        p = pack_build(w.descs, axes)
+        q = w.f32("q")
+        got = rope_apply(q, p["pos_ids"], axes)
+        for t in range(w.T):
+            for h in range(w.H):
+                ref = brute.brute_rope_vec(q[t, h].tolist(), p["pos_ids"][t].tolist(), axes)
+                assert np.allclose(got[t, h], ref, rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------------------ attention
+def _sdpa64(q, k, v):
+    """torch SDPA in float64 on CPU for one sample: q,k,v [n][H][D]."""
+    tq = torch.from_numpy(np.ascontiguousarray(q.transpose(1, 0, 2)))[None]
+    tk = torch.from_numpy(np.ascontiguousarray(k.transpose(1, 0, 2)))[None]
+    tv = torch.from_numpy(np.ascontiguousarray(v.transpose(1, 0, 2)))[None]
+    o = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv)
+    return o[0].numpy().transpose(1, 0, 2)
+
+
+def check_attention_vs_sdpa(varlen_attention):
+    rng = np.random.default_rng(20)
+    # a single-sample pack is ordinary full attention
+    for n, H, D in ((1, 1, 8), (37, 2, 64), (300, 3, 128)):
+        q, k, v = (rng.standard_normal((n, H, D)) for _ in range(3))
+        o, _ = varlen_attention(q, k, v, [0, n])
+        assert np.allclose(o, _sdpa64(q, k, v), rtol=1e-10, atol=1e-12)
+    # a pack is block-diagonal: each sample equals attention over itself alone
+    lens = [5, 130, 1, 64]
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    T, H, D = int(cu[-1]), 2, 16
+    q, k, v = (rng.standard_normal((T, H, D)) for _ in range(3))
+    o, _ = varlen_attention(q, k, v, cu)
+    for s in range(len(lens)):
+        lo, hi = cu[s], cu[s + 1]
+        assert np.allclose(o[lo:hi], _sdpa64(q[lo:hi], k[lo:hi], v[lo:hi]), rtol=1e-10, atol=1e-12)
+
+
+def check_attention_lse(varlen_attention):
+    from scipy.special import logsumexp
+    rng = np.random.default_rng(21)
+    lens = [3, 40]
+    cu = [0, 3, 43]
+    q, k, v = (rng.standard_normal((43, 2, 8)) for _ in range(3))
+    _, lse = varlen_attention(q, k, v, cu)
+    for s in range(2):
+        for h in range(2):
+            sc = q[cu[s]:cu[s + 1], h] @ k[cu[s]:cu[s + 1], h].T / math.sqrt(8)
+            assert np.allclose(lse[h, cu[s]:cu[s + 1]], logsumexp(sc, axis=1), atol=1e-12)
+    assert len(lens) == 2
+
+
+def check_attention_permutation(varlen_attention):
+    """Reordering the samples of a pack reorders the outputs, bit for bit."""
+    rng = np.random.default_rng(22)
+    lens = [7, 19, 3, 11]
+    H, D = 2, 8
+    segs = [tuple(rng.standard_normal((n, H, D)) for _ in range(3)) for n in lens]
+
+    def run(order):
+        q = np.concatenate([segs[i][0] for i in order])
+        k = np.concatenate([segs[i][1] for i in order])
+        v = np.concatenate([segs[i][2] for i in order])
+        cu = np.concatenate([[0], np.cumsum([lens[i] for i in order])])
+        o, _ = varlen_attention(q, k, v, cu)
+        return [o[cu[j]:cu[j + 1]] for j in range(len(order))]
+
+    ref = run([0, 1, 2, 3])
+    perm = [2, 0, 3, 1]
+    got = run(perm)
+    for j, i in enumerate(perm):
+        assert np.array_equal(got[j], ref[i])
+
+
+def check_attention_equal_v(varlen_attention):
+    """If every key of a sample carries the same value vector, every query of
+    that sample returns it (softmax weights sum to one)."""
+    rng = np.random.default_rng(23)
+    cu = [0, 4, 50, 51]
+    T, H, D = 51, 2, 8
+    q = rng.standard_normal((T, H, D)) * 4
+    k = rng.standard_normal((T, H, D)) * 4
+    v = np.zeros((T, H, D))
+    for s in range(3):
+        v[cu[s]:cu[s + 1]] = rng.standard_normal((1, H, D))
+    o, _ = varlen_attention(q, k, v, cu)
+    assert np.allclose(o, v, rtol=0, atol=1e-12)
+
+
+def check_attention_vs_brute(varlen_attention):
+    for seed, D in ((30, 8), (31, 64), (32, 8)):
+        rng = np.random.default_rng(seed)
+        lens = [int(x) for x in rng.integers(1, 41, size=int(rng.integers(1, 4)))]
+        H = int(rng.integers(1, 3))
+        cu = [0]
+        for n in lens:
+            cu.append(cu[-1] + n)
+        T = cu[-1]
+        q, k, v = (rng.standard_normal((T, H, D)) for _ in range(3))
+        o, _ = varlen_attention(q, k, v, cu)
+        ref = brute.brute_attention(q.tolist(), k.tolist(), v.tolist(), cu)
+        assert np.allclose(o, np.array(ref), rtol=0, atol=1e-12)
+
+
+def check_attention_rows_subset(varlen_attention):
+    rng = np.random.default_rng(24)
+    cu = [0, 10, 45, 46]
+    q, k, v = (rng.standard_normal((46, 2, 8)) for _ in range(3))
+    o, lse = varlen_attention(q, k, v, cu)
+    rows = np.array([0, 9, 10, 30, 45])
+    o2, lse2 = varlen_attention(q, k, v, cu, rows=rows, chunk=2)
+    assert np.array_equal(o2, o[rows]) or np.allclose(o2, o[rows], rtol=0, atol=1e-14)
+    assert np.allclose(lse2, lse[:, rows], rtol=0, atol=1e-14)
+
+
+# ----------------------------------------------------------------------- gate
+def check_gate(gated_residual, adaln_params, pack_build):
+    w = make_random_pack(40, S=2, H=2, D=8, rope_axes=2)
+    p = pack_build(w.descs, 2)
+    x = w.f32("x")
+    o = np.random.default_rng(1).standard_normal((w.T, w.H, w.D))
+    # a conditioning vector that is 1 in its first entry and a W whose gate
+    # columns read that entry: gate = 1, so y = x + O
+    c = np.zeros((w.S, 4))
+    c[:, 0] = 1.0
+    W = np.zeros((4, 6 * w.hid))
+    for m in range(2):
+        W[0, (3 * m + 2) * w.hid:(3 * m + 3) * w.hid] = 1.0
+    mod = adaln_params(c, W, w.hid)
+    y = gated_residual(x, o, mod, p["tok_sample"], p["tok_mod"])
+    assert np.allclose(y, x + o.reshape(w.T, w.hid), rtol=0, atol=1e-15)
+    # brute force with a random map
+    mod = adaln_params(w.c, w.W, w.hid)
+    y = gated_residual(x, o, mod, p["tok_sample"], p["tok_mod"])
+    for t in range(w.T):
+        s, m = int(p["tok_sample"][t]), int(p["tok_mod"][t])
+        ref = brute.brute_gate_row(x[t].tolist(), o[t].reshape(-1).tolist(), mod[s, m, 2].tolist())
+        assert np.allclose(y[t], ref, rtol=0, atol=1e-12)

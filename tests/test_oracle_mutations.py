@@ -1,0 +1,115 @@
+"""Plant plausible mistakes in copies of the oracle (on the CPU) and check
+that the pins catch each one. A pin set that passes a broken oracle would not
+be evidence of anything."""
+
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import mf_oracle as mo
+import pins
+
+
+def _rope_sign_flip(x, pos_ids, rope_axes, base=10000.0, rows=None):
+    x = np.asarray(x, dtype=np.float64)
+    th = mo.rope_pair_angles(np.asarray(pos_ids), x.shape[-1], rope_axes, base)[:, None, :]
+    out = np.empty_like(x)
+    out[..., 0::2] = x[..., 0::2] * np.cos(th) + x[..., 1::2] * np.sin(th)   # wrong sign
+    out[..., 1::2] = x[..., 0::2] * np.sin(th) + x[..., 1::2] * np.cos(th)
+    return out
+
+
+def _rope_half_split(x, pos_ids, rope_axes, base=10000.0, rows=None):
+    # pairs (i, i + D/2) instead of adjacent channels
+    x = np.asarray(x, dtype=np.float64)
+    D = x.shape[-1]
+    th = mo.rope_pair_angles(np.asarray(pos_ids), D, rope_axes, base)[:, None, :]
+    a, b = x[..., :D // 2], x[..., D // 2:]
+    return np.concatenate([a * np.cos(th) - b * np.sin(th), a * np.sin(th) + b * np.cos(th)], -1)
+
+
+def _rope_axes_swapped(x, pos_ids, rope_axes, base=10000.0, rows=None):
+    p = np.asarray(pos_ids).copy()
+    p[:, [1, 2]] = p[:, [2, 1]]
+    return mo.rope_apply(x, p, rope_axes, base)
+
+
+def _mod_shift_scale_swapped(c, W, hid):
+    m = mo.adaln_params(c, W, hid)
+    return m[:, :, [1, 0, 2], :]
+
+
+def _ln_sample_var(x, eps):
+    x = np.asarray(x, dtype=np.float64)
+    mu = x.mean(axis=-1, keepdims=True)
+    var = np.var(x, axis=-1, ddof=1, keepdims=True)
+    return (x - mu) / np.sqrt(var + eps)
+
+
+def _attention_ignores_pack(q, k, v, cu_seqlens, scale=None, rows=None, chunk=2048):
+    T = np.asarray(q).shape[0]
+    return mo.varlen_attention(q, k, v, [0, T], scale, rows, chunk)
+
+
+def _attention_no_scale(q, k, v, cu_seqlens, scale=None, rows=None, chunk=2048):
+    return mo.varlen_attention(q, k, v, cu_seqlens, 1.0, rows, chunk)
+
+
+def _attention_transposed_pv(q, k, v, cu_seqlens, scale=None, rows=None, chunk=2048):
+    # uses the key matrix instead of the value matrix (an operand mix-up)
+    return mo.varlen_attention(q, k, k, cu_seqlens, scale, rows, chunk)
+
+
+def _pack_text_from_zero(descs, rope_axes):
+    p = mo.pack_build(descs, rope_axes)
+    pos = p["pos_ids"].copy()
+    cu = p["cu_seqlens"]
+    for s, d in enumerate(descs):
+        F, Hg, Wg, L = d.as_tuple()[:4] if hasattr(d, "as_tuple") else d[:4]
+        n_img = F * Hg * Wg
+        pos[cu[s] + n_img:cu[s + 1], :] = np.arange(L)[:, None]
+    p["pos_ids"] = pos
+    return p
+
+
+def _pack_col_major(descs, rope_axes):
+    p = mo.pack_build(descs, rope_axes)
+    pos = p["pos_ids"].copy()
+    cu = p["cu_seqlens"]
+    for s, d in enumerate(descs):
+        F, Hg, Wg, L = d.as_tuple()[:4] if hasattr(d, "as_tuple") else d[:4]
+        f, w, h = np.meshgrid(np.arange(F), np.arange(Wg), np.arange(Hg), indexing="ij")
+        n_img = F * Hg * Wg
+        pos[cu[s]:cu[s] + n_img] = np.stack([f.ravel(), h.ravel(), w.ravel()], 1)
+    p["pos_ids"] = pos
+    return p
+
+
+def _gate_uses_scale(x, o, mod, tok_sample, tok_mod, rows=None):
+    m = mod[:, :, [0, 1, 1], :]
+    return mo.gated_residual(x, o, m, tok_sample, tok_mod, rows)
+
+
+MUTANTS = [
+    ("rope sign flip", lambda: pins.check_rope_relative(_rope_sign_flip) or
+     pins.check_rope_textbook_1d(_rope_sign_flip)),
+    ("rope half-split pairs", lambda: pins.check_rope_textbook_1d(_rope_half_split)),
+    ("rope h/w swapped", lambda: pins.check_rope_textbook_1d(_rope_axes_swapped)),
+    ("shift/scale swapped", lambda: pins.check_mod_layout(_mod_shift_scale_swapped)),
+    ("LN sample variance", lambda: pins.check_layernorm_moments(_ln_sample_var)),
+    ("attention across samples", lambda: pins.check_attention_vs_sdpa(_attention_ignores_pack)),
+    ("attention without 1/sqrt(D)", lambda: pins.check_attention_vs_sdpa(_attention_no_scale)),
+    ("K used as V", lambda: pins.check_attention_vs_brute(_attention_transposed_pv)),
+    ("text positions from 0", lambda: pins.check_pack_tiny_closed_form(_pack_text_from_zero)),
+    ("column-major grid", lambda: pins.check_pack_tiny_closed_form(_pack_col_major)),
+    ("gate reads scale", lambda: pins.check_gate(_gate_uses_scale, oracle.adaln_params,
+                                                 oracle.pack_build)),
+]
+
+
+@pytest.mark.parametrize("name,run", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_mutant_is_caught(name, run):
+    with pytest.raises(AssertionError):
+        run()
