@@ -1,0 +1,185 @@
+/*
+ * mf.h -- C ABI of libmf, the B200 (sm_100a) packed joint-attention block.
+ *
+ * The block is the data-parallel hot path of the Mage-Flow NR-MMDiT backbone:
+ * image-latent token grids and text tokens of several samples share one flat
+ * token buffer (a "pack"), delimited by per-sample cumulative offsets. One
+ * block forward runs modality-specific adaptive LayerNorm modulation, per-sample
+ * 2D RoPE (3D with a frame axis for edit packs) on Q and K, block-diagonal
+ * variable-length softmax attention and a gated residual.
+ *
+ * Sources (page title, then section); the pages describe the operations in
+ * words only:
+ *   [pack] picx.dev "Mage-Flow" summary, Methodology > Native-Resolution MMDiT
+ *          (NR-MMDiT), "Native-resolution packing": variable-length latent and
+ *          text sequences packed under a fixed token budget, attention run with
+ *          per-sample cumulative offsets.
+ *   [rope] gist.science "Resumo Tecnico: Mage-Flow", Metodologia > 2. NR-MMDiT,
+ *          "Empacotamento de Resolucao Nativa": per-sample 2D rotary embeddings.
+ *   [edit] picx.dev summary, Methodology > NR-MMDiT, "Conditioning": source and
+ *          target latents concatenated under a 3D RoPE with a frame dimension.
+ *   [norm] picx.dev summary, Methodology > NR-MMDiT: modality-specific
+ *          normalization and joint self-attention.
+ *   [fuse] picx.dev summary, Methodology > Training Infrastructure: fused
+ *          adaptive normalization / RoPE / gating in NR-MMDiT.
+ * Where the pages are silent the library follows one stated reading: RoPE
+ * splits head_dim evenly across the axes in whole adjacent-channel pairs, base
+ * 10000 by default, leftover channels unrotated; text token j of a sample sits
+ * at position max(grid_h, grid_w) + j on every axis; LayerNorm has no affine
+ * parameters; x_mod = LN(x) * (1 + scale) + shift; y = x + gate * attn.
+ *
+ * Conventions for every entry point:
+ *   - Tensors are dense, row-major, in device memory unless marked "host".
+ *     bf16 tensors are passed as mf_bf16 (the 16-bit pattern of a bfloat16).
+ *   - The caller owns and allocates all memory; the library never allocates
+ *     device memory. Scratch space is passed as (workspace, ws_bytes).
+ *   - Device pointers must be 16-byte aligned.
+ *   - Argument errors return MF_ERR_INVALID (or MF_ERR_UNSUPPORTED for shapes
+ *     outside the supported set) before anything is launched.
+ *   - Work is enqueued asynchronously on `stream`. A failure detected inside a
+ *     kernel (a bounded wait that ran out, an id out of range in device data)
+ *     is recorded in a per-device error word; mf_get_error() reports it.
+ *   - Supported shapes: head_dim D in {64, 128}; hid = H * D with H <= 128 and
+ *     hid <= 4096; S <= MF_MAX_SAMPLES; T < 2^24.
+ */
+#ifndef MF_H_
+#define MF_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MF_ABI_VERSION 1
+#define MF_MAX_SAMPLES 512
+#define MF_MAX_TOKENS (1 << 24)
+
+typedef uint16_t mf_bf16; /* bfloat16 bit pattern */
+
+typedef enum {
+  MF_OK = 0,
+  MF_ERR_INVALID = 1,     /* bad argument, or bad id found in device data */
+  MF_ERR_CUDA = 2,        /* a CUDA runtime call failed */
+  MF_ERR_TIMEOUT = 3,     /* a bounded device-side wait ran out */
+  MF_ERR_UNSUPPORTED = 4  /* valid but outside the supported shapes */
+} mf_status;
+
+/* One sample of a pack: `frames` latent grids of grid_h x grid_w tokens (frame
+ * major, then row major), then n_text text tokens. frames is 0 (a text-only
+ * segment), 1, or 2 (source + target of an edit; 3D RoPE only). is_dummy marks
+ * the padding segment of a training pack; the library computes it like any other
+ * sample (it only matters to FLOP accounting). */
+typedef struct {
+  int32_t frames;
+  int32_t grid_h;
+  int32_t grid_w;
+  int32_t n_text;
+  int32_t is_dummy;
+} mf_sample_desc;
+
+int32_t mf_abi_version(void);
+const char* mf_status_string(mf_status s);
+
+/* Pack metadata [pack], [rope], [edit].
+ * desc: host array of S descriptors. rope_axes: 2 (h, w) or 3 (f, h, w).
+ * budget: token budget (0 = none); T > budget is MF_ERR_INVALID.
+ * Outputs: cu_seqlens_h (host, S+1 int32, exclusive prefix sum of sample
+ * lengths), *T_out (host), and on the device cu_seqlens_d [S+1] int32,
+ * pos_ids_d [T][3] int32 (frame, h, w), tok_sample_d [T] int32 (sample of each
+ * token), tok_mod_d [T] uint8 (0 = image latent, 1 = text).
+ * If all four device pointers are NULL only the host outputs are written (a
+ * size query). Image token (f, h, w) has position (f, h, w) (f = 0 in 2D
+ * packs); text token j has (p, p, p) with p = max(grid_h, grid_w) + j. */
+mf_status mf_pack_build(const mf_sample_desc* desc, int32_t S, int32_t rope_axes,
+                        int32_t budget, int32_t* cu_seqlens_h, int32_t* cu_seqlens_d,
+                        int32_t* pos_ids_d, int32_t* tok_sample_d, uint8_t* tok_mod_d,
+                        int32_t* T_out, cudaStream_t stream);
+
+/* Modulation vectors [norm], [fuse]: mod[s][m][j][i] =
+ * sum_c c[s][c] * W[c][(3m + j) * hid + i], m in {image, text},
+ * j in {shift, scale, gate}. c: [S][C] fp32, W: [C][6*hid] fp32,
+ * mod: [S][2][3][hid] fp32 (written). fp32 accumulation in c order. */
+mf_status mf_adaln_params(const float* c, const float* W, int32_t S, int32_t C,
+                          int32_t hid, float* mod, cudaStream_t stream);
+
+/* Modality-specific adaLN [norm]: x_mod[t] = LN(x[t]) * (1 + scale[s,m]) +
+ * shift[s,m], LN without affine parameters, population variance, eps given.
+ * x, x_mod: [T][hid] bf16 (must not alias); mod from mf_adaln_params;
+ * tok_sample / tok_mod from mf_pack_build. A tok_sample outside [0, S) is
+ * recorded as MF_ERR_INVALID and that row is left unwritten. hid % 8 == 0. */
+mf_status mf_adaln_modulate(const mf_bf16* x, const float* mod, const int32_t* tok_sample,
+                            const uint8_t* tok_mod, int32_t T, int32_t S, int32_t hid,
+                            float eps, mf_bf16* x_mod, cudaStream_t stream);
+
+/* Per-sample RoPE on Q and K [rope], [edit]. q, k: [T][H][D] bf16; either may be
+ * NULL to skip it. q_out / k_out may equal q / k (in place). Channel pairs
+ * (2i, 2i+1) of the chunk of axis a (width d_a = 2 * floor(D / (2*rope_axes)),
+ * chunks in axis order (h, w) or (f, h, w)) turn by pos_a * base^(-2i / d_a);
+ * channels past the last chunk are copied. fp32 arithmetic, bf16 output. */
+mf_status mf_rope_apply(const mf_bf16* q, const mf_bf16* k, const int32_t* pos_ids,
+                        int32_t T, int32_t H, int32_t D, int32_t rope_axes, float base,
+                        mf_bf16* q_out, mf_bf16* k_out, cudaStream_t stream);
+
+/* Block-diagonal varlen attention [pack], [norm]: for every sample s and head h,
+ * O = softmax(Q K^T * softmax_scale) V over the sample's own tokens only.
+ * q, k, v, o: [T][H][D] bf16 (o must not alias inputs). cu_seqlens_d and
+ * cu_seqlens_h: the same S+1 offsets on device and host; T = cu_seqlens_h[S].
+ * pos_ids: NULL when q and k are already rotated, else [T][3] and RoPE with
+ * (rope_axes, base) is applied to q and k first (needs workspace).
+ * softmax_scale: finite and > 0 (the usual choice is 1/sqrt(D)).
+ * lse: NULL or [H][T] fp32, natural-log log-sum-exp of each row's scores.
+ * workspace: ws_bytes >= mf_workspace_size(T, H, D, pos_ids != NULL).
+ * QK^T and PV run on tcgen05 tensor cores, bf16 operands, fp32 accumulation;
+ * P is rounded to bf16 for PV. */
+mf_status mf_varlen_attn_fwd(const mf_bf16* q, const mf_bf16* k, const mf_bf16* v,
+                             const int32_t* cu_seqlens_d, const int32_t* cu_seqlens_h,
+                             int32_t S, int32_t H, int32_t D, float softmax_scale,
+                             const int32_t* pos_ids, int32_t rope_axes, float base,
+                             mf_bf16* o, float* lse, void* workspace, size_t ws_bytes,
+                             cudaStream_t stream);
+
+/* Gated residual [fuse]: y[t] = x[t] + gate[s,m] * o[t], o viewed as [T][H*D].
+ * x, o, y: [T][hid] bf16 (y may equal x). Same id checks as mf_adaln_modulate. */
+mf_status mf_gated_residual(const mf_bf16* x, const mf_bf16* o, const float* mod,
+                            const int32_t* tok_sample, const uint8_t* tok_mod, int32_t T,
+                            int32_t S, int32_t hid, mf_bf16* y, cudaStream_t stream);
+
+/* The whole block [fuse]: x_mod = adaLN(x); then RoPE on q and k, varlen
+ * attention with softmax scale 1/sqrt(D), and the gated residual fused into the
+ * attention epilogue: y = x + gate * O (O never reaches memory).
+ * x, x_mod, y: [T][hid] bf16; q, k, v: [T][H][D] bf16; mod, ids and offsets as
+ * above. workspace: ws_bytes >= mf_workspace_size(T, H, D, 1). */
+mf_status mf_block_fwd(const mf_bf16* x, const mf_bf16* q, const mf_bf16* k, const mf_bf16* v,
+                       const float* mod, const int32_t* cu_seqlens_d,
+                       const int32_t* cu_seqlens_h, const int32_t* pos_ids,
+                       const int32_t* tok_sample, const uint8_t* tok_mod, int32_t S, int32_t H,
+                       int32_t D, int32_t rope_axes, float base, float eps, mf_bf16* x_mod,
+                       mf_bf16* y, void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* Bytes of workspace mf_varlen_attn_fwd / mf_block_fwd need (with_rope != 0:
+ * room for the rotated Q and K). */
+size_t mf_workspace_size(int32_t T, int32_t H, int32_t D, int32_t with_rope);
+
+/* Synchronises `stream`, returns and clears the device error word of the
+ * current device (MF_OK if no kernel recorded a failure). */
+mf_status mf_get_error(cudaStream_t stream);
+
+/* Limit, in nanoseconds, of every device-side wait of later launches on the
+ * current device (default 2e9). A wait that runs out records MF_ERR_TIMEOUT,
+ * and the kernel winds down and returns. */
+mf_status mf_set_wait_limit_ns(uint64_t ns);
+
+/* Self-test of the error channel: launches one CTA that waits on an mbarrier
+ * no thread ever arrives at, with a limit of `limit_ns`. The wait runs out, the
+ * kernel records MF_ERR_TIMEOUT and returns (no trap, no hang). */
+mf_status mf_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MF_H_ */

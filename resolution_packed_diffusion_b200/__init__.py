@@ -1,0 +1,202 @@
+"""Python binding of libmf, the sm_100a packed joint-attention block.
+
+Argument marshalling only: every function here has the name and argument order
+of the C entry point in ``include/mf.h``; tensors stand in for pointers (their
+``data_ptr()`` is passed), ``None`` for NULL, and the current torch CUDA stream
+is used unless ``stream`` is given. Every step of the block runs in libmf's
+CUDA kernels. There is no CPU fallback: importing this package fails loudly if
+``libmf.so`` has not been built (``python -m resolution_packed_diffusion_b200.build``).
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Iterable, List, Optional, Sequence, Tuple
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmf.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "mf.h")
+
+MF_OK, MF_ERR_INVALID, MF_ERR_CUDA, MF_ERR_TIMEOUT, MF_ERR_UNSUPPORTED = 0, 1, 2, 3, 4
+MF_MAX_SAMPLES = 512
+
+
+class MFError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+class mf_sample_desc(ctypes.Structure):
+    _fields_ = [("frames", ctypes.c_int32), ("grid_h", ctypes.c_int32),
+                ("grid_w", ctypes.c_int32), ("n_text", ctypes.c_int32),
+                ("is_dummy", ctypes.c_int32)]
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with "
+                      "`python -m resolution_packed_diffusion_b200.build`")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int32
+_F = ctypes.c_float
+_SZ = ctypes.c_size_t
+_U64 = ctypes.c_uint64
+
+_SIGS = {
+    "mf_abi_version": (_I, []),
+    "mf_status_string": (ctypes.c_char_p, [_I]),
+    "mf_pack_build": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
+    "mf_adaln_params": (_I, [_P, _P, _I, _I, _I, _P, _P]),
+    "mf_adaln_modulate": (_I, [_P, _P, _P, _P, _I, _I, _I, _F, _P, _P]),
+    "mf_rope_apply": (_I, [_P, _P, _P, _I, _I, _I, _I, _F, _P, _P, _P]),
+    "mf_varlen_attn_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _F, _P, _I, _F, _P, _P, _P,
+                                _SZ, _P]),
+    "mf_gated_residual": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P, _P]),
+    "mf_block_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _F, _P,
+                          _P, _P, _SZ, _P]),
+    "mf_workspace_size": (_SZ, [_I, _I, _I, _I]),
+    "mf_get_error": (_I, [_P]),
+    "mf_set_wait_limit_ns": (_I, [_U64]),
+    "mf_selftest_wait_timeout": (_I, [_U64, _P]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _fn = getattr(lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+
+def header_symbols(path: str = HEADER_PATH) -> List[str]:
+    """Names of the functions ``include/mf.h`` declares."""
+    text = open(path).read()
+    return sorted(set(re.findall(r"^(?:const\s+)?\w+\s*\*?\s*(mf_\w+)\(", text, re.M)))
+
+
+def status_string(status: int) -> str:
+    return lib.mf_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != MF_OK:
+        raise MFError(status, where)
+
+
+def _ptr(t) -> Optional[int]:
+    """Device pointer of a contiguous CUDA tensor (None -> NULL)."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda:
+        raise ValueError("libmf entry points take device tensors")
+    if not t.is_contiguous():
+        raise ValueError("libmf entry points take contiguous tensors")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def make_descs(descs: Iterable) -> ctypes.Array:
+    """ctypes array of mf_sample_desc from (frames, grid_h, grid_w, n_text[, is_dummy])
+    tuples or objects with ``as_tuple()``."""
+    rows = [tuple(d.as_tuple()) if hasattr(d, "as_tuple") else tuple(d) for d in descs]
+    arr = (mf_sample_desc * max(1, len(rows)))()
+    for i, r in enumerate(rows):
+        r = tuple(r) + (0,) * (5 - len(r))
+        arr[i] = mf_sample_desc(*[int(v) for v in r[:5]])
+    return arr
+
+
+def abi_version() -> int:
+    return lib.mf_abi_version()
+
+
+def mf_pack_build(descs, rope_axes: int, budget: int = 0, cu_seqlens_d=None, pos_ids_d=None,
+                  tok_sample_d=None, tok_mod_d=None, stream=None) -> Tuple[np.ndarray, int]:
+    """Returns (cu_seqlens_h as int32 [S+1], T). With all device tensors None
+    this is a host-only size query."""
+    arr = make_descs(descs)
+    S = len(list(descs)) if not isinstance(descs, ctypes.Array) else len(descs)
+    cu_h = np.zeros(S + 1, dtype=np.int32)
+    T = ctypes.c_int32(0)
+    query = all(t is None for t in (cu_seqlens_d, pos_ids_d, tok_sample_d, tok_mod_d))
+    st = None if query else _stream(stream)
+    _check(lib.mf_pack_build(ctypes.cast(arr, _P), S, rope_axes, budget,
+                             cu_h.ctypes.data_as(_P), _ptr(cu_seqlens_d), _ptr(pos_ids_d),
+                             _ptr(tok_sample_d), _ptr(tok_mod_d), ctypes.byref(T), st),
+           "mf_pack_build")
+    return cu_h, int(T.value)
+
+
+def mf_adaln_params(c, W, S: int, C: int, hid: int, mod, stream=None) -> None:
+    _check(lib.mf_adaln_params(_ptr(c), _ptr(W), S, C, hid, _ptr(mod), _stream(stream)),
+           "mf_adaln_params")
+
+
+def mf_adaln_modulate(x, mod, tok_sample, tok_mod, T: int, S: int, hid: int, eps: float, x_mod,
+                      stream=None) -> None:
+    _check(lib.mf_adaln_modulate(_ptr(x), _ptr(mod), _ptr(tok_sample), _ptr(tok_mod), T, S, hid,
+                                 eps, _ptr(x_mod), _stream(stream)), "mf_adaln_modulate")
+
+
+def mf_rope_apply(q, k, pos_ids, T: int, H: int, D: int, rope_axes: int, base: float, q_out,
+                  k_out, stream=None) -> None:
+    _check(lib.mf_rope_apply(_ptr(q), _ptr(k), _ptr(pos_ids), T, H, D, rope_axes, base,
+                             _ptr(q_out), _ptr(k_out), _stream(stream)), "mf_rope_apply")
+
+
+def mf_varlen_attn_fwd(q, k, v, cu_seqlens_d, cu_seqlens_h: np.ndarray, S: int, H: int, D: int,
+                       softmax_scale: float, pos_ids, rope_axes: int, base: float, o, lse,
+                       workspace, ws_bytes: int, stream=None) -> None:
+    cu_h = np.ascontiguousarray(cu_seqlens_h, dtype=np.int32)
+    _check(lib.mf_varlen_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens_d),
+                                  cu_h.ctypes.data_as(_P), S, H, D, softmax_scale,
+                                  _ptr(pos_ids), rope_axes, base, _ptr(o), _ptr(lse),
+                                  _ptr(workspace), ws_bytes, _stream(stream)),
+           "mf_varlen_attn_fwd")
+
+
+def mf_gated_residual(x, o, mod, tok_sample, tok_mod, T: int, S: int, hid: int, y,
+                      stream=None) -> None:
+    _check(lib.mf_gated_residual(_ptr(x), _ptr(o), _ptr(mod), _ptr(tok_sample), _ptr(tok_mod),
+                                 T, S, hid, _ptr(y), _stream(stream)), "mf_gated_residual")
+
+
+def mf_block_fwd(x, q, k, v, mod, cu_seqlens_d, cu_seqlens_h: np.ndarray, pos_ids, tok_sample,
+                 tok_mod, S: int, H: int, D: int, rope_axes: int, base: float, eps: float, x_mod,
+                 y, workspace, ws_bytes: int, stream=None) -> None:
+    cu_h = np.ascontiguousarray(cu_seqlens_h, dtype=np.int32)
+    _check(lib.mf_block_fwd(_ptr(x), _ptr(q), _ptr(k), _ptr(v), _ptr(mod), _ptr(cu_seqlens_d),
+                            cu_h.ctypes.data_as(_P), _ptr(pos_ids), _ptr(tok_sample),
+                            _ptr(tok_mod), S, H, D, rope_axes, base, eps, _ptr(x_mod), _ptr(y),
+                            _ptr(workspace), ws_bytes, _stream(stream)), "mf_block_fwd")
+
+
+def mf_workspace_size(T: int, H: int, D: int, with_rope: int) -> int:
+    return int(lib.mf_workspace_size(T, H, D, with_rope))
+
+
+def mf_get_error(stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the device error word."""
+    return int(lib.mf_get_error(_stream(stream)))
+
+
+def mf_set_wait_limit_ns(ns: int) -> None:
+    _check(lib.mf_set_wait_limit_ns(int(ns)), "mf_set_wait_limit_ns")
+
+
+def mf_selftest_wait_timeout(limit_ns: int, stream=None) -> None:
+    _check(lib.mf_selftest_wait_timeout(int(limit_ns), _stream(stream)), "mf_selftest_wait_timeout")

@@ -1,0 +1,345 @@
+// mf_api.cu -- the C ABI of libmf (declared in include/mf.h): argument checks,
+// the per-device error word, workspace carving and kernel launches. No entry
+// point allocates device memory; every buffer comes from the caller.
+#include <cuda_runtime_api.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "mf.h"
+#include "mf_internal.h"
+
+namespace mf {
+
+// Per-device word where kernels record the first failure they detect.
+__device__ int g_mf_error;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
+
+struct DeviceState {
+  bool ready = false;
+  int* err = nullptr;
+  uint64_t wait_limit_ns = kDefaultWaitLimitNs;
+};
+
+DeviceState g_state[kMaxDevices];
+std::mutex g_mutex;
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+inline mf_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MF_OK : MF_ERR_CUDA; }
+
+bool valid_head_dim(int32_t D) { return D == 64 || D == 128; }
+
+// Checks host offsets: 0 = cu[0] <= cu[1] <= ... ; writes T.
+bool check_offsets(const int32_t* cu_h, int32_t S, int32_t* T) {
+  if (cu_h == nullptr || cu_h[0] != 0) return false;
+  for (int32_t s = 0; s < S; ++s)
+    if (cu_h[s + 1] < cu_h[s]) return false;
+  if (cu_h[S] > MF_MAX_TOKENS) return false;
+  *T = cu_h[S];
+  return true;
+}
+
+int32_t count_items(const int32_t* cu_h, int32_t S, int32_t H) {
+  int64_t n = 0;
+  for (int32_t s = 0; s < S; ++s) n += (static_cast<int64_t>(cu_h[s + 1] - cu_h[s]) + 127) / 128;
+  return static_cast<int32_t>(n * H);
+}
+
+}  // namespace
+
+cudaError_t get_ctl(KernelCtl* ctl) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceState& d = g_state[dev];
+  if (!d.ready) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_mf_error);
+    if (e != cudaSuccess) return e;
+    d.err = static_cast<int*>(p);
+    d.ready = true;
+  }
+  ctl->err = d.err;
+  ctl->wait_limit_ns = d.wait_limit_ns;
+  return cudaSuccess;
+}
+
+}  // namespace mf
+
+using namespace mf;
+
+extern "C" {
+
+int32_t mf_abi_version(void) { return MF_ABI_VERSION; }
+
+const char* mf_status_string(mf_status s) {
+  switch (s) {
+    case MF_OK: return "MF_OK";
+    case MF_ERR_INVALID: return "MF_ERR_INVALID";
+    case MF_ERR_CUDA: return "MF_ERR_CUDA";
+    case MF_ERR_TIMEOUT: return "MF_ERR_TIMEOUT";
+    case MF_ERR_UNSUPPORTED: return "MF_ERR_UNSUPPORTED";
+  }
+  return "MF_ERR_UNKNOWN";
+}
+
+mf_status mf_pack_build(const mf_sample_desc* desc, int32_t S, int32_t rope_axes, int32_t budget,
+                        int32_t* cu_seqlens_h, int32_t* cu_seqlens_d, int32_t* pos_ids_d,
+                        int32_t* tok_sample_d, uint8_t* tok_mod_d, int32_t* T_out,
+                        cudaStream_t stream) {
+  if (S < 0 || S > MF_MAX_SAMPLES || (S > 0 && desc == nullptr) || cu_seqlens_h == nullptr ||
+      T_out == nullptr || (rope_axes != 2 && rope_axes != 3) || budget < 0)
+    return MF_ERR_INVALID;
+  const int n_null = (cu_seqlens_d == nullptr) + (pos_ids_d == nullptr) +
+                     (tok_sample_d == nullptr) + (tok_mod_d == nullptr);
+  if (n_null != 0 && n_null != 4) return MF_ERR_INVALID;
+  int64_t acc = 0;
+  for (int32_t s = 0; s < S; ++s) {
+    const mf_sample_desc& d = desc[s];
+    if (d.frames < 0 || d.grid_h < 0 || d.grid_w < 0 || d.n_text < 0) return MF_ERR_INVALID;
+    if (d.frames > (rope_axes == 2 ? 1 : 2)) return MF_ERR_INVALID;
+    if (d.grid_h > MF_MAX_TOKENS || d.grid_w > MF_MAX_TOKENS || d.n_text > MF_MAX_TOKENS)
+      return MF_ERR_INVALID;
+    const int64_t n = static_cast<int64_t>(d.frames) * d.grid_h * d.grid_w + d.n_text;
+    acc += n;
+    if (acc > MF_MAX_TOKENS) return MF_ERR_INVALID;
+  }
+  if (budget > 0 && acc > budget) return MF_ERR_INVALID;
+  PackParams p;
+  p.S = S;
+  p.T = static_cast<int32_t>(acc);
+  p.cu[0] = 0;
+  for (int32_t s = 0; s < S; ++s) {
+    const mf_sample_desc& d = desc[s];
+    p.cu[s + 1] = p.cu[s] + d.frames * d.grid_h * d.grid_w + d.n_text;
+    p.frames[s] = d.frames;
+    p.grid_h[s] = d.grid_h;
+    p.grid_w[s] = d.grid_w;
+  }
+  for (int32_t s = 0; s <= S; ++s) cu_seqlens_h[s] = p.cu[s];
+  *T_out = p.T;
+  if (n_null == 4) return MF_OK;  // size query
+  if (!aligned16(cu_seqlens_d) || !aligned16(pos_ids_d) || !aligned16(tok_sample_d) ||
+      !aligned16(tok_mod_d))
+    return MF_ERR_INVALID;
+  return cuda_status(launch_pack_ids(p, cu_seqlens_d, pos_ids_d, tok_sample_d, tok_mod_d, stream));
+}
+
+mf_status mf_adaln_params(const float* c, const float* W, int32_t S, int32_t C, int32_t hid,
+                          float* mod, cudaStream_t stream) {
+  if (c == nullptr || W == nullptr || mod == nullptr || S < 1 || S > MF_MAX_SAMPLES || C < 1 ||
+      C > 1024 || hid < 8 || hid % 8 != 0 || hid > 16384)
+    return MF_ERR_INVALID;
+  if (!aligned16(c) || !aligned16(W) || !aligned16(mod)) return MF_ERR_INVALID;
+  return cuda_status(launch_adaln_params(c, W, S, C, hid, mod, stream));
+}
+
+mf_status mf_adaln_modulate(const mf_bf16* x, const float* mod, const int32_t* tok_sample,
+                            const uint8_t* tok_mod, int32_t T, int32_t S, int32_t hid, float eps,
+                            mf_bf16* x_mod, cudaStream_t stream) {
+  if (T < 0 || T > MF_MAX_TOKENS || S < 1 || S > MF_MAX_SAMPLES || hid < 8 || hid % 8 != 0 ||
+      !(eps >= 0.f) || !std::isfinite(eps))
+    return MF_ERR_INVALID;
+  if (hid > 4096) return MF_ERR_UNSUPPORTED;
+  if (T == 0) return MF_OK;
+  if (x == nullptr || mod == nullptr || tok_sample == nullptr || tok_mod == nullptr ||
+      x_mod == nullptr || !aligned16(x) || !aligned16(mod) || !aligned16(x_mod))
+    return MF_ERR_INVALID;
+  const size_t bytes = static_cast<size_t>(T) * hid * 2;
+  if (overlap(x, bytes, x_mod, bytes)) return MF_ERR_INVALID;
+  KernelCtl ctl;
+  if (get_ctl(&ctl) != cudaSuccess) return MF_ERR_CUDA;
+  return cuda_status(
+      launch_adaln_modulate(x, mod, tok_sample, tok_mod, T, S, hid, eps, x_mod, ctl, stream));
+}
+
+mf_status mf_rope_apply(const mf_bf16* q, const mf_bf16* k, const int32_t* pos_ids, int32_t T,
+                        int32_t H, int32_t D, int32_t rope_axes, float base, mf_bf16* q_out,
+                        mf_bf16* k_out, cudaStream_t stream) {
+  if (T < 0 || T > MF_MAX_TOKENS || H < 1 || H > 128 || (rope_axes != 2 && rope_axes != 3) ||
+      !(base > 0.f) || !std::isfinite(base))
+    return MF_ERR_INVALID;
+  if (!valid_head_dim(D)) return MF_ERR_UNSUPPORTED;
+  if (q == nullptr && k == nullptr) return MF_ERR_INVALID;
+  if ((q != nullptr) != (q_out != nullptr) || (k != nullptr) != (k_out != nullptr))
+    return MF_ERR_INVALID;
+  if (T == 0) return MF_OK;
+  if (pos_ids == nullptr || !aligned16(q) || !aligned16(k) || !aligned16(q_out) ||
+      !aligned16(k_out))
+    return MF_ERR_INVALID;
+  const size_t bytes = static_cast<size_t>(T) * H * D * 2;
+  // in place is allowed; a partial overlap is not
+  if (q && q != q_out && overlap(q, bytes, q_out, bytes)) return MF_ERR_INVALID;
+  if (k && k != k_out && overlap(k, bytes, k_out, bytes)) return MF_ERR_INVALID;
+  if (q_out && k_out && overlap(q_out, bytes, k_out, bytes)) return MF_ERR_INVALID;
+  RopeTable tab;
+  make_rope_table(D, rope_axes, base, &tab);
+  return cuda_status(launch_rope(q, k, pos_ids, T, H, D, tab, q_out, k_out, stream));
+}
+
+size_t mf_workspace_size(int32_t T, int32_t H, int32_t D, int32_t with_rope) {
+  if (T <= 0 || H <= 0 || D <= 0 || !with_rope) return 0;
+  return 2 * round_up(static_cast<size_t>(T) * H * D * 2, 256) + 256;
+}
+
+mf_status mf_varlen_attn_fwd(const mf_bf16* q, const mf_bf16* k, const mf_bf16* v,
+                             const int32_t* cu_seqlens_d, const int32_t* cu_seqlens_h, int32_t S,
+                             int32_t H, int32_t D, float softmax_scale, const int32_t* pos_ids,
+                             int32_t rope_axes, float base, mf_bf16* o, float* lse,
+                             void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  if (S < 1 || S > MF_MAX_SAMPLES || H < 1 || H > 128 || !std::isfinite(softmax_scale) ||
+      !(softmax_scale > 0.f))
+    return MF_ERR_INVALID;
+  if (!valid_head_dim(D)) return MF_ERR_UNSUPPORTED;
+  int32_t T = 0;
+  if (!check_offsets(cu_seqlens_h, S, &T)) return MF_ERR_INVALID;
+  if (T == 0) return MF_OK;
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || cu_seqlens_d == nullptr ||
+      !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      !aligned16(cu_seqlens_d) || !aligned16(lse))
+    return MF_ERR_INVALID;
+  const size_t bytes = static_cast<size_t>(T) * H * D * 2;
+  if (overlap(o, bytes, q, bytes) || overlap(o, bytes, k, bytes) || overlap(o, bytes, v, bytes))
+    return MF_ERR_INVALID;
+  if (lse && (overlap(lse, static_cast<size_t>(T) * H * 4, o, bytes)))
+    return MF_ERR_INVALID;
+  KernelCtl ctl;
+  if (get_ctl(&ctl) != cudaSuccess) return MF_ERR_CUDA;
+  const mf_bf16* qa = q;
+  const mf_bf16* ka = k;
+  if (pos_ids != nullptr) {
+    if ((rope_axes != 2 && rope_axes != 3) || !(base > 0.f) || !std::isfinite(base))
+      return MF_ERR_INVALID;
+    if (workspace == nullptr || !aligned16(workspace) || ws_bytes < mf_workspace_size(T, H, D, 1))
+      return MF_ERR_INVALID;
+    const uintptr_t w0 = round_up(reinterpret_cast<uintptr_t>(workspace), 256);
+    mf_bf16* wq = reinterpret_cast<mf_bf16*>(w0);
+    mf_bf16* wk = reinterpret_cast<mf_bf16*>(w0 + round_up(bytes, 256));
+    RopeTable tab;
+    make_rope_table(D, rope_axes, base, &tab);
+    cudaError_t e = launch_rope(q, k, pos_ids, T, H, D, tab, wq, wk, stream);
+    if (e != cudaSuccess) return MF_ERR_CUDA;
+    qa = wq;
+    ka = wk;
+  }
+  AttnEpilogue ep{};
+  ep.o = o;
+  ep.lse = lse;
+  return cuda_status(launch_attention(qa, ka, v, cu_seqlens_d, S, T, H, D, softmax_scale, ep,
+                                      count_items(cu_seqlens_h, S, H), ctl, stream));
+}
+
+mf_status mf_gated_residual(const mf_bf16* x, const mf_bf16* o, const float* mod,
+                            const int32_t* tok_sample, const uint8_t* tok_mod, int32_t T,
+                            int32_t S, int32_t hid, mf_bf16* y, cudaStream_t stream) {
+  if (T < 0 || T > MF_MAX_TOKENS || S < 1 || S > MF_MAX_SAMPLES || hid < 8 || hid % 8 != 0)
+    return MF_ERR_INVALID;
+  if (T == 0) return MF_OK;
+  if (x == nullptr || o == nullptr || mod == nullptr || tok_sample == nullptr ||
+      tok_mod == nullptr || y == nullptr || !aligned16(x) || !aligned16(o) || !aligned16(mod) ||
+      !aligned16(y))
+    return MF_ERR_INVALID;
+  const size_t bytes = static_cast<size_t>(T) * hid * 2;
+  if (y != x && overlap(x, bytes, y, bytes)) return MF_ERR_INVALID;
+  if (overlap(o, bytes, y, bytes)) return MF_ERR_INVALID;
+  KernelCtl ctl;
+  if (get_ctl(&ctl) != cudaSuccess) return MF_ERR_CUDA;
+  return cuda_status(
+      launch_gated_residual(x, o, mod, tok_sample, tok_mod, T, S, hid, y, ctl, stream));
+}
+
+mf_status mf_block_fwd(const mf_bf16* x, const mf_bf16* q, const mf_bf16* k, const mf_bf16* v,
+                       const float* mod, const int32_t* cu_seqlens_d, const int32_t* cu_seqlens_h,
+                       const int32_t* pos_ids, const int32_t* tok_sample, const uint8_t* tok_mod,
+                       int32_t S, int32_t H, int32_t D, int32_t rope_axes, float base, float eps,
+                       mf_bf16* x_mod, mf_bf16* y, void* workspace, size_t ws_bytes,
+                       cudaStream_t stream) {
+  if (S < 1 || S > MF_MAX_SAMPLES || H < 1 || H > 128 || (rope_axes != 2 && rope_axes != 3) ||
+      !(base > 0.f) || !std::isfinite(base) || !(eps >= 0.f) || !std::isfinite(eps))
+    return MF_ERR_INVALID;
+  if (!valid_head_dim(D) || H * D > 4096) return MF_ERR_UNSUPPORTED;
+  int32_t T = 0;
+  if (!check_offsets(cu_seqlens_h, S, &T)) return MF_ERR_INVALID;
+  if (T == 0) return MF_OK;
+  const int32_t hid = H * D;
+  if (x == nullptr || q == nullptr || k == nullptr || v == nullptr || mod == nullptr ||
+      cu_seqlens_d == nullptr || pos_ids == nullptr || tok_sample == nullptr ||
+      tok_mod == nullptr || x_mod == nullptr || y == nullptr || workspace == nullptr)
+    return MF_ERR_INVALID;
+  if (!aligned16(x) || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(mod) ||
+      !aligned16(cu_seqlens_d) || !aligned16(x_mod) || !aligned16(y) || !aligned16(workspace))
+    return MF_ERR_INVALID;
+  if (ws_bytes < mf_workspace_size(T, H, D, 1)) return MF_ERR_INVALID;
+  const size_t bytes = static_cast<size_t>(T) * hid * 2;
+  const void* ins[4] = {x, q, k, v};
+  for (const void* in : ins)
+    if (overlap(in, bytes, x_mod, bytes) || overlap(in, bytes, y, bytes)) return MF_ERR_INVALID;
+  if (overlap(x_mod, bytes, y, bytes)) return MF_ERR_INVALID;
+  if (overlap(workspace, ws_bytes, x_mod, bytes) || overlap(workspace, ws_bytes, y, bytes))
+    return MF_ERR_INVALID;
+  KernelCtl ctl;
+  if (get_ctl(&ctl) != cudaSuccess) return MF_ERR_CUDA;
+  cudaError_t e =
+      launch_adaln_modulate(x, mod, tok_sample, tok_mod, T, S, hid, eps, x_mod, ctl, stream);
+  if (e != cudaSuccess) return MF_ERR_CUDA;
+  const uintptr_t w0 = round_up(reinterpret_cast<uintptr_t>(workspace), 256);
+  mf_bf16* wq = reinterpret_cast<mf_bf16*>(w0);
+  mf_bf16* wk = reinterpret_cast<mf_bf16*>(w0 + round_up(bytes, 256));
+  RopeTable tab;
+  make_rope_table(D, rope_axes, base, &tab);
+  e = launch_rope(q, k, pos_ids, T, H, D, tab, wq, wk, stream);
+  if (e != cudaSuccess) return MF_ERR_CUDA;
+  AttnEpilogue ep{};
+  ep.x = x;
+  ep.mod = mod;
+  ep.tok_mod = tok_mod;
+  ep.y = y;
+  return cuda_status(launch_attention(wq, wk, v, cu_seqlens_d, S, T, H, D,
+                                      1.0f / std::sqrt(static_cast<float>(D)), ep,
+                                      count_items(cu_seqlens_h, S, H), ctl, stream));
+}
+
+mf_status mf_get_error(cudaStream_t stream) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return MF_ERR_CUDA;
+  KernelCtl ctl;
+  if (get_ctl(&ctl) != cudaSuccess) return MF_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_mf_error, sizeof(int)) != cudaSuccess) return MF_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_mf_error, &zero, sizeof(int)) != cudaSuccess) return MF_ERR_CUDA;
+  return static_cast<mf_status>(v);
+}
+
+mf_status mf_set_wait_limit_ns(uint64_t ns) {
+  if (ns == 0) return MF_ERR_INVALID;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MF_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return MF_ERR_INVALID;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  g_state[dev].wait_limit_ns = ns;
+  return MF_OK;
+}
+
+mf_status mf_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t stream) {
+  if (limit_ns == 0 || limit_ns > 10000000000ull) return MF_ERR_INVALID;
+  KernelCtl ctl;
+  if (get_ctl(&ctl) != cudaSuccess) return MF_ERR_CUDA;
+  return cuda_status(launch_selftest_wait(limit_ns, ctl, stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,118 @@
+"""The C-ABI library without a GPU: it loads, exports every symbol include/mf.h
+declares, and its host-side logic (pack offsets, argument checks, workspace
+sizing) matches the oracle and the header's contract. No compute is launched."""
+
+import ctypes
+
+import numpy as np
+import pytest
+
+import oracle
+from packgen import SampleDesc, make_random_pack, make_workload
+
+mf = pytest.importorskip("resolution_packed_diffusion_b200")
+
+
+def test_library_exports_every_declared_symbol():
+    names = mf.header_symbols()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(mf.lib, n), n
+        assert n in mf._SIGS, f"binding lacks {n}"
+    for needed in ("mf_pack_build", "mf_adaln_modulate", "mf_rope_apply", "mf_varlen_attn_fwd",
+                   "mf_gated_residual", "mf_block_fwd"):
+        assert needed in names
+
+
+def test_abi_version_and_status_strings():
+    assert mf.abi_version() == 1
+    assert mf.status_string(mf.MF_OK) == "MF_OK"
+    assert mf.status_string(mf.MF_ERR_TIMEOUT) == "MF_ERR_TIMEOUT"
+
+
+@pytest.mark.parametrize("idx", [1, 2, 3, 4, 5])
+def test_pack_offsets_match_oracle(idx):
+    w = make_workload(idx, with_arrays=False)
+    cu, T = mf.mf_pack_build(w.descs, w.rope_axes, w.budget)
+    ref = oracle.pack_build(w.descs, w.rope_axes)
+    assert T == ref["T"] == w.T
+    assert np.array_equal(cu, ref["cu_seqlens"])
+
+
+def test_pack_offsets_random_and_empty():
+    for seed in range(20):
+        axes = 2 + seed % 2
+        w = make_random_pack(seed, S=1 + seed % 7, H=1, D=8, rope_axes=axes, max_grid=9,
+                             max_text=11)
+        cu, T = mf.mf_pack_build(w.descs, axes, 0)
+        assert np.array_equal(cu, oracle.pack_build(w.descs, axes)["cu_seqlens"])
+    cu, T = mf.mf_pack_build([], 2, 0)
+    assert T == 0 and cu.tolist() == [0]
+
+
+@pytest.mark.parametrize("descs,axes,budget", [
+    ([(2, 4, 4, 3)], 2, 0),           # two frames need the 3D layout
+    ([(3, 4, 4, 3)], 3, 0),           # at most two frames
+    ([(1, -1, 4, 3)], 2, 0),          # negative grid
+    ([(1, 4, 4, -2)], 2, 0),          # negative text length
+    ([(1, 64, 64, 256)], 2, 1000),    # over the token budget
+    ([(1, 4, 4, 0)], 4, 0),           # bad rope_axes
+])
+def test_pack_rejects_invalid(descs, axes, budget):
+    with pytest.raises(mf.MFError) as e:
+        mf.mf_pack_build(descs, axes, budget)
+    assert e.value.status == mf.MF_ERR_INVALID
+
+
+def test_pack_rejects_too_many_samples():
+    with pytest.raises(mf.MFError):
+        mf.mf_pack_build([(1, 1, 1, 1)] * (mf.MF_MAX_SAMPLES + 1), 2, 0)
+
+
+def test_workspace_size():
+    assert mf.mf_workspace_size(0, 24, 128, 1) == 0
+    assert mf.mf_workspace_size(100, 24, 128, 0) == 0
+    n = 100 * 24 * 128 * 2
+    assert mf.mf_workspace_size(100, 24, 128, 1) >= 2 * n
+
+
+def test_host_argument_checks_without_gpu():
+    """Calls that fail validation return before touching the GPU."""
+    lib = mf.lib
+    cu = np.array([0, 10], dtype=np.int32)
+    P = ctypes.c_void_p
+    # head_dim 96 is outside the supported set
+    st = lib.mf_varlen_attn_fwd(P(16), P(16), P(16), P(16), cu.ctypes.data_as(P), 1, 2, 96,
+                                0.1, None, 2, 10000.0, P(4096), None, None, 0, None)
+    assert st == mf.MF_ERR_UNSUPPORTED
+    # misaligned output pointer
+    st = lib.mf_varlen_attn_fwd(P(16), P(16 + 4096), P(16 + 8192), P(16), cu.ctypes.data_as(P),
+                                1, 1, 64, 0.1, None, 2, 10000.0, P(1 << 20 | 8), None, None, 0,
+                                None)
+    assert st == mf.MF_ERR_INVALID
+    # non-monotone offsets
+    bad = np.array([0, 10, 5], dtype=np.int32)
+    st = lib.mf_varlen_attn_fwd(P(16), P(16), P(16), P(16), bad.ctypes.data_as(P), 2, 1, 64,
+                                0.1, None, 2, 10000.0, P(4096), None, None, 0, None)
+    assert st == mf.MF_ERR_INVALID
+    # non-positive softmax scale
+    st = lib.mf_varlen_attn_fwd(P(16), P(1 << 20), P(2 << 20), P(16), cu.ctypes.data_as(P), 1,
+                                1, 64, 0.0, None, 2, 10000.0, P(4 << 20), None, None, 0, None)
+    assert st == mf.MF_ERR_INVALID
+    # empty pack: nothing to do
+    z = np.array([0, 0], dtype=np.int32)
+    st = lib.mf_varlen_attn_fwd(None, None, None, None, z.ctypes.data_as(P), 1, 1, 64, 0.1,
+                                None, 2, 10000.0, None, None, None, 0, None)
+    assert st == mf.MF_OK
+    # adaLN: hid above the supported row length
+    st = lib.mf_adaln_modulate(P(16), P(16), P(16), P(16), 4, 1, 8192, 1e-6, P(1 << 30), None)
+    assert st == mf.MF_ERR_UNSUPPORTED
+    # RoPE with no tensor to rotate
+    st = lib.mf_rope_apply(None, None, P(16), 4, 1, 64, 2, 10000.0, None, None, None)
+    assert st == mf.MF_ERR_INVALID
+    # block forward with too small a workspace
+    cu2 = np.array([0, 128], dtype=np.int32)
+    st = lib.mf_block_fwd(P(1 << 24), P(2 << 24), P(3 << 24), P(4 << 24), P(5 << 24), P(16),
+                          cu2.ctypes.data_as(P), P(16), P(16), P(16), 1, 2, 64, 2, 10000.0,
+                          1e-6, P(6 << 24), P(7 << 24), P(8 << 24), 16, None)
+    assert st == mf.MF_ERR_INVALID

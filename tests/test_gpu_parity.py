@@ -1,0 +1,247 @@
+"""CUDA path (through the C ABI) against the CPU oracle on the same seeded
+inputs: every workload at full size, in the launch configuration the bench
+times, plus edge cases. Pack metadata must be bit-exact; bf16 outputs meet
+max-abs 2e-2 and relative RMS 5e-3 (see gpu_util for the storage-rounding rule
+above |8|); the fp32 modulation vectors meet 1e-5 absolute."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from packgen import SampleDesc, make_random_pack, make_workload
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import resolution_packed_diffusion_b200 as mf  # noqa: E402
+from gpu_util import (DevicePack, assert_bf16_close, dev_bf16, host_f32,  # noqa: E402
+                      oracle_pack, sample_rows)
+
+MOD_ATOL = 1e-5  # fp32 dot products of 128 terms of size ~0.02: rounding ~1e-7
+
+
+class Case:
+    def __init__(self, idx):
+        self.w = make_workload(idx)
+        self.dp = DevicePack(self.w)
+        self.pack = oracle_pack(self.w)
+        self.mod = oracle.adaln_params(self.w.c, self.w.W, self.w.hid)
+        T = self.w.T
+        self.rows = np.arange(T) if T <= 4096 else sample_rows(self.pack["cu_seqlens"], 24, idx)
+        self._k_r = None
+
+    @property
+    def k_r(self):
+        if self._k_r is None:
+            self._k_r = oracle.rope_apply(self.w.f32("k"), self.pack["pos_ids"], self.w.rope_axes)
+        return self._k_r
+
+
+_CASES = {}
+
+
+@pytest.fixture(scope="module", params=[1, 2, 3, 4, 5], ids=lambda i: f"cfg{i}")
+def case(request):
+    if request.param not in _CASES:
+        _CASES.clear()
+        torch.cuda.empty_cache()
+        _CASES[request.param] = Case(request.param)
+    return _CASES[request.param]
+
+
+def test_pack_ids_bit_exact(case):
+    dp, ref = case.dp, case.pack
+    assert np.array_equal(dp.cu_h, ref["cu_seqlens"])
+    assert np.array_equal(dp.cu_d.cpu().numpy(), ref["cu_seqlens"])
+    assert np.array_equal(dp.pos.cpu().numpy(), ref["pos_ids"])
+    assert np.array_equal(dp.tok_sample.cpu().numpy(), ref["tok_sample"])
+    assert np.array_equal(dp.tok_mod.cpu().numpy(), ref["tok_mod"])
+
+
+def test_adaln_params(case):
+    got = case.dp.mod.cpu().numpy().astype(np.float64)
+    assert np.abs(got - case.mod).max() <= MOD_ATOL
+
+
+def test_adaln_modulate(case):
+    dp, w = case.dp, case.w
+    x_mod = torch.empty_like(dp.x)
+    mf.mf_adaln_modulate(dp.x, dp.mod, dp.tok_sample, dp.tok_mod, dp.T, dp.S, dp.hid, w.eps, x_mod)
+    assert mf.mf_get_error() == mf.MF_OK
+    rows = case.rows
+    ref = oracle.adaln_modulate(w.f32("x"), case.mod, case.pack["tok_sample"],
+                                case.pack["tok_mod"], w.eps, rows=rows)
+    assert_bf16_close(host_f32(x_mod)[rows], ref, "x_mod")
+
+
+def test_rope(case):
+    dp, w = case.dp, case.w
+    q_out = torch.empty_like(dp.q)
+    k_out = torch.empty_like(dp.k)
+    mf.mf_rope_apply(dp.q, dp.k, dp.pos, dp.T, dp.H, dp.D, w.rope_axes, w.base, q_out, k_out)
+    rows = case.rows
+    ref_q = oracle.rope_apply(w.f32("q"), case.pack["pos_ids"], w.rope_axes, rows=rows)
+    assert_bf16_close(host_f32(q_out)[rows], ref_q, "rope q")
+    assert_bf16_close(host_f32(k_out)[rows], case.k_r[rows], "rope k")
+
+
+def test_attention_on_rotated_inputs(case):
+    """mf_varlen_attn_fwd with pos_ids = NULL: the inputs are taken as already
+    rotated, so this checks the tensor-core attention alone (and the LSE)."""
+    dp, w = case.dp, case.w
+    o, lse = dp.attention(dp.q, dp.k, dp.v, with_rope=False, lse=True)
+    assert mf.mf_get_error() == mf.MF_OK
+    rows = case.rows
+    ref_o, ref_lse = oracle.varlen_attention(w.f32("q"), w.f32("k"), w.f32("v"),
+                                             case.pack["cu_seqlens"], rows=rows)
+    assert_bf16_close(host_f32(o)[rows], ref_o, "attention O")
+    got_lse = lse.cpu().numpy()[:, rows].astype(np.float64)
+    assert np.abs(got_lse - ref_lse).max() <= 2e-2
+
+
+def test_attention_with_rope(case):
+    dp, w = case.dp, case.w
+    o, _ = dp.attention(dp.q, dp.k, dp.v, with_rope=True)
+    assert mf.mf_get_error() == mf.MF_OK
+    rows = case.rows
+    q_r = np.zeros((w.T, w.H, w.D))
+    q_r[rows] = oracle.rope_apply(w.f32("q"), case.pack["pos_ids"], w.rope_axes, rows=rows)
+    ref_o, _ = oracle.varlen_attention(q_r, case.k_r, w.f32("v"), case.pack["cu_seqlens"], rows=rows)
+    assert_bf16_close(host_f32(o)[rows], ref_o, "attention O (RoPE)")
+
+
+def test_gated_residual(case):
+    dp, w = case.dp, case.w
+    o = dp.v.reshape(dp.T, dp.hid)  # any bf16 tensor of the right shape serves as O
+    y = torch.empty_like(dp.x)
+    mf.mf_gated_residual(dp.x, o, dp.mod, dp.tok_sample, dp.tok_mod, dp.T, dp.S, dp.hid, y)
+    assert mf.mf_get_error() == mf.MF_OK
+    rows = case.rows
+    ref = oracle.gated_residual(w.f32("x"), w.f32("v"), case.mod, case.pack["tok_sample"],
+                                case.pack["tok_mod"], rows=rows)
+    assert_bf16_close(host_f32(y)[rows], ref, "gated residual y")
+
+
+def test_block_fwd(case):
+    """The fused block in the configuration bench.py times."""
+    dp, w = case.dp, case.w
+    x_mod, y = dp.block()
+    assert mf.mf_get_error() == mf.MF_OK
+    rows = case.rows
+    ref_xm, ref_y, _ = oracle.block_fwd(w.f32("x"), w.f32("q"), w.f32("k"), w.f32("v"), case.mod,
+                                        case.pack, w.rope_axes, rows=rows)
+    assert_bf16_close(host_f32(x_mod)[rows], ref_xm, "block x_mod")
+    assert_bf16_close(host_f32(y)[rows], ref_y, "block y")
+    # the attention branch alone, recovered from y: gate * O = y - x
+    gate = case.mod[case.pack["tok_sample"][rows], case.pack["tok_mod"][rows], 2]
+    x = w.f32("x")[rows].astype(np.float64)
+    # deterministic: a second run gives the same bits
+    x_mod2, y2 = dp.block()
+    assert torch.equal(x_mod, x_mod2) and torch.equal(y, y2)
+    assert gate.shape == x.shape
+
+
+# ------------------------------------------------------------------ edge cases
+EDGE_PACKS = [
+    # (descs, H, D, axes)
+    ([SampleDesc(0, 0, 0, 1)], 1, 64, 2),                                    # one token
+    ([SampleDesc(1, 1, 127, 0), SampleDesc(1, 8, 16, 0), SampleDesc(1, 1, 129, 0)], 2, 128, 2),
+    ([SampleDesc(0, 0, 0, 300), SampleDesc(1, 5, 7, 3)], 3, 64, 2),          # text-only sample
+    ([SampleDesc(1, 4, 4, 0), SampleDesc(0, 0, 0, 0), SampleDesc(1, 3, 3, 5)], 2, 128, 2),  # empty sample
+    ([SampleDesc(2, 6, 5, 7), SampleDesc(1, 9, 4, 2), SampleDesc(2, 3, 3, 0)], 2, 128, 3),  # mixed frames
+    ([SampleDesc(1, 16, 16, 255)], 1, 128, 2),                                # 511 tokens
+    ([SampleDesc(1, 16, 16, 1), SampleDesc(1, 16, 16, 0), SampleDesc(1, 16, 16, 2)], 4, 64, 2),
+]
+
+
+@pytest.mark.parametrize("k", range(len(EDGE_PACKS)))
+def test_edge_packs_full_compare(k):
+    descs, H, D, axes = EDGE_PACKS[k]
+    w = make_random_pack(500 + k, S=len(descs), H=H, D=D, rope_axes=axes, descs=descs)
+    dp = DevicePack(w)
+    pack = oracle_pack(w)
+    mod = oracle.adaln_params(w.c, w.W, w.hid)
+    x_mod, y = dp.block()
+    assert mf.mf_get_error() == mf.MF_OK
+    ref_xm, ref_y, _ = oracle.block_fwd(w.f32("x"), w.f32("q"), w.f32("k"), w.f32("v"), mod, pack,
+                                        axes)
+    assert_bf16_close(host_f32(x_mod), ref_xm, "edge x_mod")
+    assert_bf16_close(host_f32(y), ref_y, "edge y")
+    o, lse = dp.attention(dp.q, dp.k, dp.v, with_rope=False, lse=True)
+    ref_o, ref_lse = oracle.varlen_attention(w.f32("q"), w.f32("k"), w.f32("v"),
+                                             pack["cu_seqlens"])
+    assert_bf16_close(host_f32(o), ref_o, "edge O")
+    assert np.abs(lse.cpu().numpy() - ref_lse).max() <= 2e-2
+
+
+def test_empty_pack_is_a_no_op():
+    w = make_random_pack(600, S=2, H=2, D=64, rope_axes=2,
+                         descs=[SampleDesc(0, 0, 0, 0), SampleDesc(1, 0, 5, 0)])
+    cu_h, T = mf.mf_pack_build(w.descs, 2, 0)
+    assert T == 0
+    st = mf.lib.mf_block_fwd(None, None, None, None, None, None, cu_h.ctypes.data, None, None,
+                             None, 2, 2, 64, 2, 10000.0, 1e-6, None, None, None, 0, None)
+    assert st == mf.MF_OK
+
+
+def test_unaligned_pointer_rejected():
+    w = make_workload(1)
+    dp = DevicePack(w)
+    flat = torch.empty(dp.T * dp.hid + 8, dtype=torch.bfloat16, device="cuda")
+    x_mis = flat[1:1 + dp.T * dp.hid].view(dp.T, dp.hid)  # 2-byte offset
+    with pytest.raises(mf.MFError) as e:
+        mf.mf_adaln_modulate(x_mis, dp.mod, dp.tok_sample, dp.tok_mod, dp.T, dp.S, dp.hid, 1e-6,
+                             torch.empty_like(dp.x))
+    assert e.value.status == mf.MF_ERR_INVALID
+
+
+def test_device_offsets_disagreeing_with_host_are_reported():
+    w = make_workload(1)
+    dp = DevicePack(w)
+    bad_cu = dp.cu_d.clone()
+    bad_cu[-1] += 1  # device says T+1, host says T
+    o = torch.empty_like(dp.q)
+    mf.mf_varlen_attn_fwd(dp.q, dp.k, dp.v, bad_cu, dp.cu_h, dp.S, dp.H, dp.D, 0.125, None, 2,
+                          1e4, o, None, None, 0)
+    assert mf.mf_get_error() == mf.MF_ERR_INVALID
+    o2, _ = dp.attention(dp.q, dp.k, dp.v, with_rope=False)
+    assert mf.mf_get_error() == mf.MF_OK
+
+
+def test_bad_sample_id_in_device_data_is_reported():
+    w = make_workload(1)
+    dp = DevicePack(w)
+    ts = dp.tok_sample.clone()
+    ts[5] = dp.S + 3
+    x_mod = torch.zeros_like(dp.x)
+    mf.mf_adaln_modulate(dp.x, dp.mod, ts, dp.tok_mod, dp.T, dp.S, dp.hid, 1e-6, x_mod)
+    assert mf.mf_get_error() == mf.MF_ERR_INVALID
+    assert torch.count_nonzero(x_mod[5]) == 0          # the bad row is left alone
+    assert torch.count_nonzero(x_mod[4]) > 0
+
+
+def test_bounded_wait_times_out_and_context_survives():
+    mf.mf_selftest_wait_timeout(20_000_000)  # 20 ms, nothing ever arrives
+    assert mf.mf_get_error() == mf.MF_ERR_TIMEOUT
+    assert mf.mf_get_error() == mf.MF_OK     # cleared
+    w = make_workload(1)
+    dp = DevicePack(w)
+    x_mod, y = dp.block()
+    assert mf.mf_get_error() == mf.MF_OK
+    ref_xm, ref_y, _ = oracle.block_fwd(w.f32("x"), w.f32("q"), w.f32("k"), w.f32("v"),
+                                        oracle.adaln_params(w.c, w.W, w.hid), oracle_pack(w), 2)
+    assert_bf16_close(host_f32(y), ref_y, "y after timeout")
+
+
+def test_rope_in_place():
+    w = make_workload(1)
+    dp = DevicePack(w)
+    q = dp.q.clone()
+    mf.mf_rope_apply(q, None, dp.pos, dp.T, dp.H, dp.D, 2, 1e4, q, None)
+    ref = oracle.rope_apply(w.f32("q"), oracle_pack(w)["pos_ids"], 2)
+    assert_bf16_close(host_f32(q), ref, "rope in place")
