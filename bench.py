@@ -1,0 +1,436 @@
+"""Benchmark of the packed joint-attention block on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config I] [--impl reference]
+
+One step is one pass of the whole path over one synthetic pack: pack metadata
+(mf_pack_build), modulation vectors (mf_adaln_params) and the fused block
+(mf_block_fwd: adaLN modulation, RoPE, tcgen05 varlen attention with the gated
+residual epilogue). Inputs are resident in HBM when the timed region starts.
+
+Metric: useful attention TFLOP/s of the whole step, where useful FLOPs are
+4 * D * H * sum(n_s^2) over the real samples (the padding segment is computed but
+not counted). Also reported: block tokens/s, the attention kernel alone against
+the measured bf16 tensor peak (roofline), the end-to-end rate through host
+buffers (e2e) and the CPU oracle on a bounded sample (cpu_baseline).
+
+Multi-GPU: every rank runs its own replica pack (same shapes, its own seed); no
+data moves between ranks. Timing is the max over ranks of the CUDA-event time.
+``--impl reference`` times the CPU oracle (the only reference this method has)
+on rank 0; other ranks exit without work.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from packgen import make_workload  # noqa: E402
+
+DEFAULT_CONFIG = 2  # the 16384-token native-resolution training pack
+METRIC = "packed varlen attention useful TFLOP/s (% bf16 peak); block tokens/s at 1 B200"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+REF_ROW_STRIDE = 32  # reference arm: rows sampled per step (keeps a step near 0.3 s)
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_fwd_traffic.txt")
+ATTN_SRC = os.path.join(ROOT, "resolution_packed_diffusion_b200", "csrc", "attn_fwd.cu")
+
+
+# ----------------------------------------------------------------- helpers
+def useful_flops(w) -> float:
+    tot = 0
+    for d in w.descs:
+        if d.is_dummy:
+            continue
+        n = d.frames * d.grid_h * d.grid_w + d.n_text
+        tot += n * n
+    return 4.0 * w.D * w.H * tot
+
+
+def real_tokens(w) -> int:
+    return int(sum(d.frames * d.grid_h * d.grid_w + d.n_text for d in w.descs if not d.is_dummy))
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def rank_seed(index: int, rank: int) -> int:
+    """Seed of a rank's replica pack: rank 0 uses the workload's own seed."""
+    return 1000 + index + 7919 * rank
+
+
+def reduce_timing(ms: float, units: float, world: int):
+    """(max time over ranks, summed units over ranks); plain values at world 1."""
+    if world == 1:
+        return ms, units
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    u = torch.tensor([units], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(u.item())
+
+
+def attn_traffic_bytes(T_full: int):
+    """DRAM bytes per attention launch from the committed ncu summary, scaled
+    to this pack, or None when the kernel source changed since the capture."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    fields = {}
+    for line in open(TRAFFIC_FILE):
+        if "=" in line and not line.startswith("#"):
+            k, v = line.strip().split("=", 1)
+            fields[k.strip()] = v.strip()
+    sha = hashlib.sha256(open(ATTN_SRC, "rb").read()).hexdigest()[:16]
+    if fields.get("kernel_sha") != sha or "workload" not in fields:
+        return None
+    if fields.get("workload") != str(T_full):
+        return None
+    return float(fields["bytes_per_launch"])
+
+
+class ClockSampler:
+    """nvidia-smi sampled every 200 ms while the loop runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.gpu = gpu_index
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={gpu_index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------- CPU oracle
+def oracle_sample_step(w, heads, row_stride):
+    """One bounded oracle step on the workload: pack metadata, modulation
+    vectors, and, for every ``row_stride``-th token row, adaLN plus RoPE,
+    attention over the row's whole sample and the gated residual for ``heads``.
+    Returns (seconds, useful FLOPs of the sampled rows)."""
+    import oracle
+    from packgen import bf16_bits_to_f32
+    t0 = time.perf_counter()
+    pack = oracle.pack_build(w.descs, w.rope_axes)
+    mod = oracle.adaln_params(w.c, w.W, w.hid)
+    rows = np.arange(0, w.T, row_stride)
+    x = bf16_bits_to_f32(w.x_bits[rows])
+    oracle.adaln_modulate(x, mod, pack["tok_sample"][rows], pack["tok_mod"][rows], w.eps)
+    q = bf16_bits_to_f32(w.q_bits[:, heads])
+    k = bf16_bits_to_f32(w.k_bits[:, heads])
+    v = bf16_bits_to_f32(w.v_bits[:, heads])
+    k_r = oracle.rope_apply(k, pack["pos_ids"], w.rope_axes, w.base)
+    q_r = np.zeros(q.shape)
+    q_r[rows] = oracle.rope_apply(q, pack["pos_ids"], w.rope_axes, w.base, rows=rows)
+    o, _ = oracle.varlen_attention(q_r, k_r, v, pack["cu_seqlens"], rows=rows)
+    cols = np.concatenate([np.arange(h * w.D, (h + 1) * w.D) for h in heads])
+    oracle.gated_residual(x[:, cols], o, mod[..., cols], pack["tok_sample"][rows],
+                          pack["tok_mod"][rows])
+    dt = time.perf_counter() - t0
+    cu = pack["cu_seqlens"]
+    fl = 0.0
+    for s, d in enumerate(w.descs):
+        if d.is_dummy:
+            continue
+        n = int(cu[s + 1] - cu[s])
+        n_rows = int(((rows >= cu[s]) & (rows < cu[s + 1])).sum())
+        fl += 4.0 * w.D * len(heads) * n * n_rows
+    return dt, fl
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        blas = [i for i in info if i.get("user_api") == "blas"]
+        if blas:
+            return int(blas[0]["num_threads"]), blas[0].get("internal_api", "blas")
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0)), "unknown"
+
+
+def cpu_baseline(w, budget_s=12.0):
+    """The oracle as it stands, on a bounded sample of the same workload:
+    adaLN on all rows and RoPE + attention + gated residual for as many heads as
+    fit in about ``budget_s`` seconds; its throughput is the sample's useful
+    FLOPs over the sample's time."""
+    dt, fl = oracle_sample_step(w, [0], 4)
+    n = int(max(1, min(w.H, budget_s / max(dt, 1e-3))))
+    heads = list(range(n))
+    if n > 1:
+        dt, fl = oracle_sample_step(w, heads, 4)
+    threads, api = cpu_threads()
+    return {"value": fl / dt / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": (f"{w.name}: pack metadata, modulation vectors, then for every 4th token "
+                       f"row adaLN and, for {n} of {w.H} heads, RoPE + attention over the "
+                       f"row's sample + gated residual; fp64 NumPy ({api}); {dt:.1f} s"),
+            "seconds": dt}
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return
+    w = make_workload(args.config)
+    # warm-up and timed steps, each a one-head sample of the workload
+    for _ in range(args.warmup):
+        oracle_sample_step(w, [0], REF_ROW_STRIDE)
+    times, flops = [], 0.0
+    for _ in range(args.steps):
+        dt, fl = oracle_sample_step(w, [0], REF_ROW_STRIDE)
+        times.append(dt)
+        flops += fl
+    total = sum(times)
+    value = flops / total / 1e12
+    threads, api = cpu_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, args),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": (f"each step: {w.name}, pack metadata, modulation vectors, "
+                                    f"then for every {REF_ROW_STRIDE}th token row adaLN and, "
+                                    f"for head 0 of {w.H}, RoPE + attention over the row's "
+                                    f"sample + gated residual; fp64 NumPy ({api})")},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w, args):
+    return {"workload": w.name, "config_index": w.index, "T": w.T, "S": w.S, "H": w.H, "D": w.D,
+            "hid": w.hid, "real_tokens": real_tokens(w),
+            "samples": [list(d.as_tuple()) for d in w.descs], "rope_axes": w.rope_axes,
+            "parallelism": f"replicas x{args.gpus}",
+            "l2": ("inputs larger than L2: x, q, k, v total "
+                   f"{4 * w.T * w.hid * 2 / 1e6:.0f} MB vs 126 MB L2; no flush")}
+
+
+# ------------------------------------------------------------- GPU arm
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    import resolution_packed_diffusion_b200 as mf
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = make_workload(args.config, seed=rank_seed(args.config, rank))
+    T, H, D, hid, S = w.T, w.H, w.D, w.hid, w.S
+
+    def dbf16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    x, q, k, v = dbf16(w.x_bits), dbf16(w.q_bits), dbf16(w.k_bits), dbf16(w.v_bits)
+    c = torch.from_numpy(w.c).to(dev)
+    Wm = torch.from_numpy(w.W).to(dev)
+    cu_d = torch.empty(S + 1, dtype=torch.int32, device=dev)
+    pos = torch.empty((T, 3), dtype=torch.int32, device=dev)
+    ts = torch.empty(T, dtype=torch.int32, device=dev)
+    tm = torch.empty(T, dtype=torch.uint8, device=dev)
+    mod = torch.empty((S, 2, 3, hid), dtype=torch.float32, device=dev)
+    x_mod = torch.empty_like(x)
+    y = torch.empty_like(x)
+    ws_bytes = mf.mf_workspace_size(T, H, D, 1)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        cu_h, _ = mf.mf_pack_build(w.descs, w.rope_axes, w.budget, cu_d, pos, ts, tm, stream)
+        mf.mf_adaln_params(c, Wm, S, c.shape[1], hid, mod, stream)
+        mf.mf_block_fwd(x, q, k, v, mod, cu_d, cu_h, pos, ts, tm, S, H, D, w.rope_axes, w.base,
+                        w.eps, x_mod, y, ws, ws_bytes, stream)
+
+    launches_per_step = 5  # pack ids, adaLN params, adaLN modulate, RoPE, attention
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    clocks = ClockSampler(local_rank) if rank == 0 else None
+    for _ in range(args.warmup):
+        step()
+    if mf.mf_get_error(stream) != mf.MF_OK:
+        raise RuntimeError("device error during warm-up")
+    # attention-kernel events, one pair per timed step
+    ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for e in ev_a + ev_b:
+        e.record(stream)  # creates the CUDA events before the library records them
+    barrier()
+    torch.cuda.synchronize(dev)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        mf.mf_set_attn_timing_events(ev_a[i], ev_b[i])
+        step()
+    t1.record(stream)
+    mf.mf_set_attn_timing_events(None, None)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ms_total = t0.elapsed_time(t1)
+    attn_ms = [a.elapsed_time(b) for a, b in zip(ev_a, ev_b)]
+    clk = clocks.stop() if clocks else None
+    if mf.mf_get_error(stream) != mf.MF_OK:
+        raise RuntimeError("device error during the timed steps")
+
+    flops = useful_flops(w)
+    ms_step_local = ms_total / args.steps
+    ms_step, flops_all = reduce_timing(ms_step_local, flops, world)
+    tokens_all = reduce_timing(0.0, float(real_tokens(w)), world)[1]
+    value = flops_all / (ms_step * 1e-3) / 1e12
+
+    # ---- end to end through the public API with host buffers
+    pin = {n: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).pin_memory()
+           for n, a in (("x", w.x_bits), ("q", w.q_bits), ("k", w.k_bits), ("v", w.v_bits))}
+    c_h = torch.from_numpy(w.c).pin_memory()
+    W_h = torch.from_numpy(w.W).pin_memory()
+    y_h = torch.empty((T, hid), dtype=torch.int16).pin_memory()
+    xm_h = torch.empty((T, hid), dtype=torch.int16).pin_memory()
+    dst = {"x": x, "q": q, "k": k, "v": v}
+
+    def e2e_step():
+        for n, t in pin.items():
+            dst[n].view(torch.int16).copy_(t, non_blocking=True)
+        c.copy_(c_h, non_blocking=True)
+        Wm.copy_(W_h, non_blocking=True)
+        step()
+        y_h.copy_(y.view(torch.int16), non_blocking=True)
+        xm_h.copy_(x_mod.view(torch.int16), non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        e2e_step()
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms, _ = reduce_timing(e0.elapsed_time(e1) / e2e_steps, 0.0, world)
+    h2d = sum(t.numel() * t.element_size() for t in pin.values()) + \
+        c_h.numel() * 4 + W_h.numel() * 4
+    d2h = (y_h.numel() + xm_h.numel()) * 2
+
+    if rank != 0:
+        return
+    peaks, peak_src = load_peaks()
+    attn_avg = float(np.mean(attn_ms))
+    achieved = flops / (attn_avg * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(w, args),
+        "block_tokens_per_s": tokens_all / (ms_step * 1e-3),
+        "pct_bf16_peak": 100.0 * value / (peak * world),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
+                     "frac": achieved / peak, "traffic": attn_traffic_bytes(T),
+                     "kernel": "varlen_attn_kernel<128, gated>",
+                     "peak_source": f"{peak_src} bf16_tflops (burst)",
+                     "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
+                     "attn_ms": attn_avg},
+        "gpu_launches": launches_per_step * args.steps,
+        "e2e": {"value": flops_all / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                "ms_per_step": e2e_ms},
+        "clocks": clk,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", type=int, default=DEFAULT_CONFIG, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--impl", default="mf", choices=["mf", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_gpu(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

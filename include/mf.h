@@ -173,6 +173,13 @@ mf_status mf_get_error(cudaStream_t stream);
  * and the kernel winds down and returns. */
 mf_status mf_set_wait_limit_ns(uint64_t ns);
 
+/* Instrumentation: while both events are non-NULL, every later call of
+ * mf_varlen_attn_fwd / mf_block_fwd on the current device records `start` on its
+ * stream right before the attention kernel and `stop` right after it, so the
+ * caller can time that kernel alone (cudaEventElapsedTime). (NULL, NULL) turns it
+ * off. The events belong to the caller and must outlive the calls that use them. */
+mf_status mf_set_attn_timing_events(cudaEvent_t start, cudaEvent_t stop);
+
 /* Self-test of the error channel: launches one CTA that waits on an mbarrier
  * no thread ever arrives at, with a limit of `limit_ns`. The wait runs out, the
  * kernel records MF_ERR_TIMEOUT and returns (no trap, no hang). */

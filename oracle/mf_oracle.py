@@ -219,11 +219,11 @@ def gated_residual(x, o, mod, tok_sample, tok_mod, rows=None):
     columns). Reading: the gate multiplies the attention branch and is added to
     the block input (adaLN-zero form; no output projection on this path)."""
     x = np.asarray(x, dtype=np.float64)
+    o = np.asarray(o, dtype=np.float64).reshape(x.shape[0], -1)
     tok_sample = np.asarray(tok_sample)
     tok_mod = np.asarray(tok_mod)
     if rows is not None:
-        x, tok_sample, tok_mod = x[rows], tok_sample[rows], tok_mod[rows]
-    o = np.asarray(o, dtype=np.float64).reshape(x.shape[0], -1)
+        x, o, tok_sample, tok_mod = x[rows], o[rows], tok_sample[rows], tok_mod[rows]
     gate = mod[tok_sample, tok_mod, GATE]
     return x + gate * o
 
@@ -248,7 +248,11 @@ def block_fwd(x, q, k, v, mod, pack, rope_axes: int, base: float = 10000.0,
         q_full[rows] = q_r
         q_r = q_full
     o, _ = varlen_attention(q_r, k_r, v, pack["cu_seqlens"], rows=rows)
-    y = gated_residual(x, o, mod, tok_sample, tok_mod, rows=rows)
+    if rows is not None:
+        y = gated_residual(np.asarray(x)[rows], o, mod, np.asarray(tok_sample)[rows],
+                           np.asarray(tok_mod)[rows])
+    else:
+        y = gated_residual(x, o, mod, tok_sample, tok_mod)
     return x_mod, y, o
 
 

@@ -5,7 +5,7 @@ of the C entry point in ``include/mf.h``; tensors stand in for pointers (their
 ``data_ptr()`` is passed), ``None`` for NULL, and the current torch CUDA stream
 is used unless ``stream`` is given. Every step of the block runs in libmf's
 CUDA kernels. There is no CPU fallback: importing this package fails loudly if
-``libmf.so`` has not been built (``python -m resolution_packed_diffusion_b200.build``).
+``libmf.so`` has not been built (``python resolution_packed_diffusion_b200/build.py``).
 """
 
 from __future__ import annotations
@@ -39,7 +39,7 @@ class mf_sample_desc(ctypes.Structure):
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with "
-                      "`python -m resolution_packed_diffusion_b200.build`")
+                      "`python resolution_packed_diffusion_b200/build.py`")
 
 lib = ctypes.CDLL(LIB_PATH)
 
@@ -65,6 +65,7 @@ _SIGS = {
     "mf_get_error": (_I, [_P]),
     "mf_set_wait_limit_ns": (_I, [_U64]),
     "mf_selftest_wait_timeout": (_I, [_U64, _P]),
+    "mf_set_attn_timing_events": (_I, [_P, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -200,3 +201,11 @@ def mf_set_wait_limit_ns(ns: int) -> None:
 
 def mf_selftest_wait_timeout(limit_ns: int, stream=None) -> None:
     _check(lib.mf_selftest_wait_timeout(int(limit_ns), _stream(stream)), "mf_selftest_wait_timeout")
+
+
+def mf_set_attn_timing_events(start, stop) -> None:
+    """``start`` / ``stop``: torch.cuda.Event objects (already recorded once, so
+    that the CUDA event exists) or None to switch timing off."""
+    def handle(ev):
+        return None if ev is None else ev.cuda_event
+    _check(lib.mf_set_attn_timing_events(handle(start), handle(stop)), "mf_set_attn_timing_events")

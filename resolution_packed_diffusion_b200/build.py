@@ -1,6 +1,6 @@
 """Build libmf.so in-tree for sm_100a with nvcc.
 
-    python -m resolution_packed_diffusion_b200.build [-v]
+    python resolution_packed_diffusion_b200/build.py [-v]
 
 Each CUDA source is compiled to an object under ``_build/`` (in parallel) and
 linked into ``resolution_packed_diffusion_b200/libmf.so``. The CUDA runtime is

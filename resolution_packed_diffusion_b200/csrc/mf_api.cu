@@ -24,6 +24,8 @@ struct DeviceState {
   bool ready = false;
   int* err = nullptr;
   uint64_t wait_limit_ns = kDefaultWaitLimitNs;
+  cudaEvent_t attn_start = nullptr;  // instrumentation (mf_set_attn_timing_events)
+  cudaEvent_t attn_stop = nullptr;
 };
 
 DeviceState g_state[kMaxDevices];
@@ -56,6 +58,28 @@ int32_t count_items(const int32_t* cu_h, int32_t S, int32_t H) {
   int64_t n = 0;
   for (int32_t s = 0; s < S; ++s) n += (static_cast<int64_t>(cu_h[s + 1] - cu_h[s]) + 127) / 128;
   return static_cast<int32_t>(n * H);
+}
+
+// Runs the attention launcher between the caller's timing events, if any.
+cudaError_t timed_attention(const mf_bf16* q, const mf_bf16* k, const mf_bf16* v,
+                            const int32_t* cu_d, int32_t S, int32_t T, int32_t H, int32_t D,
+                            float scale, const AttnEpilogue& ep, int32_t items,
+                            const KernelCtl& ctl, cudaStream_t st) {
+  cudaEvent_t e0 = nullptr, e1 = nullptr;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDevices) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    e0 = g_state[dev].attn_start;
+    e1 = g_state[dev].attn_stop;
+  }
+  if (e0 != nullptr) {
+    cudaError_t e = cudaEventRecord(e0, st);
+    if (e != cudaSuccess) return e;
+  }
+  cudaError_t e = launch_attention(q, k, v, cu_d, S, T, H, D, scale, ep, items, ctl, st);
+  if (e != cudaSuccess) return e;
+  if (e1 != nullptr) e = cudaEventRecord(e1, st);
+  return e;
 }
 
 }  // namespace
@@ -240,8 +264,8 @@ mf_status mf_varlen_attn_fwd(const mf_bf16* q, const mf_bf16* k, const mf_bf16* 
   AttnEpilogue ep{};
   ep.o = o;
   ep.lse = lse;
-  return cuda_status(launch_attention(qa, ka, v, cu_seqlens_d, S, T, H, D, softmax_scale, ep,
-                                      count_items(cu_seqlens_h, S, H), ctl, stream));
+  return cuda_status(timed_attention(qa, ka, v, cu_seqlens_d, S, T, H, D, softmax_scale, ep,
+                                     count_items(cu_seqlens_h, S, H), ctl, stream));
 }
 
 mf_status mf_gated_residual(const mf_bf16* x, const mf_bf16* o, const float* mod,
@@ -309,9 +333,9 @@ mf_status mf_block_fwd(const mf_bf16* x, const mf_bf16* q, const mf_bf16* k, con
   ep.mod = mod;
   ep.tok_mod = tok_mod;
   ep.y = y;
-  return cuda_status(launch_attention(wq, wk, v, cu_seqlens_d, S, T, H, D,
-                                      1.0f / std::sqrt(static_cast<float>(D)), ep,
-                                      count_items(cu_seqlens_h, S, H), ctl, stream));
+  return cuda_status(timed_attention(wq, wk, v, cu_seqlens_d, S, T, H, D,
+                                     1.0f / std::sqrt(static_cast<float>(D)), ep,
+                                     count_items(cu_seqlens_h, S, H), ctl, stream));
 }
 
 mf_status mf_get_error(cudaStream_t stream) {
@@ -332,6 +356,17 @@ mf_status mf_set_wait_limit_ns(uint64_t ns) {
   if (dev < 0 || dev >= 64) return MF_ERR_INVALID;
   std::lock_guard<std::mutex> lock(g_mutex);
   g_state[dev].wait_limit_ns = ns;
+  return MF_OK;
+}
+
+mf_status mf_set_attn_timing_events(cudaEvent_t start, cudaEvent_t stop) {
+  if ((start == nullptr) != (stop == nullptr)) return MF_ERR_INVALID;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MF_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MF_ERR_INVALID;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  g_state[dev].attn_start = start;
+  g_state[dev].attn_stop = stop;
   return MF_OK;
 }
 
