@@ -160,6 +160,27 @@ mf_status mf_block_fwd(const mf_bf16* x, const mf_bf16* q, const mf_bf16* k, con
                        int32_t D, int32_t rope_axes, float base, float eps, mf_bf16* x_mod,
                        mf_bf16* y, void* workspace, size_t ws_bytes, cudaStream_t stream);
 
+/* mf_block_fwd without a workspace argument, for callers that cannot allocate
+ * device memory (for example a plugin inside a host application that owns all
+ * device memory and gives it no allocator, or a caller that must not make a call
+ * which can synchronise the device). The paper has no counterpart: this is a
+ * library convenience. Arguments and results are those of mf_block_fwd; the
+ * rotated Q and K go to a file-scope device array of MF_NOALLOC_SCRATCH_BYTES
+ * that every GPU loading the library holds until exit, so a pack needs
+ * mf_workspace_size(T, H, D, 1) <= MF_NOALLOC_SCRATCH_BYTES (about 5400 tokens at
+ * H*D = 3072); a larger pack returns MF_ERR_UNSUPPORTED and launches nothing.
+ * The function allocates nothing. Its first call on a device looks up the array's
+ * device address (cudaGetSymbolAddress) with that device current; make that
+ * first call before any stream capture. All calls share the array: calls that
+ * overlap on the GPU race and must be serialised by the caller. */
+#define MF_NOALLOC_SCRATCH_BYTES (64u << 20)
+mf_status mf_block_fwd_noalloc(const mf_bf16* x, const mf_bf16* q, const mf_bf16* k,
+                               const mf_bf16* v, const float* mod, const int32_t* cu_seqlens_d,
+                               const int32_t* cu_seqlens_h, const int32_t* pos_ids,
+                               const int32_t* tok_sample, const uint8_t* tok_mod, int32_t S,
+                               int32_t H, int32_t D, int32_t rope_axes, float base, float eps,
+                               mf_bf16* x_mod, mf_bf16* y, cudaStream_t stream);
+
 /* Bytes of workspace mf_varlen_attn_fwd / mf_block_fwd need (with_rope != 0:
  * room for the rotated Q and K). */
 size_t mf_workspace_size(int32_t T, int32_t H, int32_t D, int32_t with_rope);

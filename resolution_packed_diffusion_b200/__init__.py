@@ -23,6 +23,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "mf.h")
 
 MF_OK, MF_ERR_INVALID, MF_ERR_CUDA, MF_ERR_TIMEOUT, MF_ERR_UNSUPPORTED = 0, 1, 2, 3, 4
 MF_MAX_SAMPLES = 512
+MF_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 class MFError(RuntimeError):
@@ -66,6 +67,8 @@ _SIGS = {
     "mf_set_wait_limit_ns": (_I, [_U64]),
     "mf_selftest_wait_timeout": (_I, [_U64, _P]),
     "mf_set_attn_timing_events": (_I, [_P, _P]),
+    "mf_block_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F,
+                                  _F, _P, _P, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -209,3 +212,16 @@ def mf_set_attn_timing_events(start, stop) -> None:
     def handle(ev):
         return None if ev is None else ev.cuda_event
     _check(lib.mf_set_attn_timing_events(handle(start), handle(stop)), "mf_set_attn_timing_events")
+
+
+def mf_block_fwd_noalloc(x, q, k, v, mod, cu_seqlens_d, cu_seqlens_h: np.ndarray, pos_ids,
+                         tok_sample, tok_mod, S: int, H: int, D: int, rope_axes: int, base: float,
+                         eps: float, x_mod, y, stream=None) -> None:
+    """mf_block_fwd for callers that cannot allocate device memory: the rotated
+    Q and K live in the library's own fixed device array (see include/mf.h)."""
+    cu_h = np.ascontiguousarray(cu_seqlens_h, dtype=np.int32)
+    _check(lib.mf_block_fwd_noalloc(_ptr(x), _ptr(q), _ptr(k), _ptr(v), _ptr(mod),
+                                    _ptr(cu_seqlens_d), cu_h.ctypes.data_as(_P), _ptr(pos_ids),
+                                    _ptr(tok_sample), _ptr(tok_mod), S, H, D, rope_axes, base,
+                                    eps, _ptr(x_mod), _ptr(y), _stream(stream)),
+           "mf_block_fwd_noalloc")
