@@ -84,6 +84,11 @@ typedef struct {
 int32_t mf_abi_version(void);
 const char* mf_status_string(mf_status s);
 
+/* Text of the last CUDA runtime error a call on this host thread turned into
+ * MF_ERR_CUDA ("" if none). The string belongs to the library and stays valid
+ * until the next failing call on this thread. */
+const char* mf_last_error_detail(void);
+
 /* Pack metadata [pack], [rope], [edit].
  * desc: host array of S descriptors. rope_axes: 2 (h, w) or 3 (f, h, w).
  * budget: token budget (0 = none); T > budget is MF_ERR_INVALID.

@@ -29,7 +29,10 @@ MF_NOALLOC_SCRATCH_BYTES = 64 << 20
 class MFError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {status_string(status)}")
+        detail = ""
+        if status == MF_ERR_CUDA:
+            detail = " (" + lib.mf_last_error_detail().decode() + ")"
+        super().__init__(f"{where}: {status_string(status)}{detail}")
 
 
 class mf_sample_desc(ctypes.Structure):
@@ -53,6 +56,7 @@ _U64 = ctypes.c_uint64
 _SIGS = {
     "mf_abi_version": (_I, []),
     "mf_status_string": (ctypes.c_char_p, [_I]),
+    "mf_last_error_detail": (ctypes.c_char_p, []),
     "mf_pack_build": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
     "mf_adaln_params": (_I, [_P, _P, _I, _I, _I, _P, _P]),
     "mf_adaln_modulate": (_I, [_P, _P, _P, _P, _I, _I, _I, _F, _P, _P]),

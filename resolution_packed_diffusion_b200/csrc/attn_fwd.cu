@@ -9,24 +9,32 @@
 // block): for every sample s and head h, O = softmax(Q K^T * scale) V over the
 // sample's own keys; optionally y = x + gate[s, modality] * O.
 //
-// Design (one persistent CTA per SM, 6 warps):
-//   warp 0      TMA producer: Q tile (128 rows) per work item, then K and V
-//               tiles (128 rows) of the item's own sample only, in separate
-//               rings (K slots free once S = Q K^T is done, V slots once PV is).
-//   warp 1      tcgen05 issuer: S = Q K^T into one of two TMEM S buffers, then
-//               O += P V with P read from TMEM (the A operand) and V from shared
-//               memory (MN-major). Allocates / frees the 512 TMEM columns.
-//   warps 2..5  softmax + epilogue, one thread per query row (TMEM lane): read S
-//               from TMEM, online softmax in the exp2 domain with a lazy
-//               rescale (O is rescaled only when the running max grows by more
-//               than 2^8), write P as packed bf16 to TMEM, then O / l and the
-//               epilogue from TMEM.
-// Work items are (sample, head, 128-row query tile), ordered longest sample
-// first and, inside a sample, query tiles of one head next to each other so
-// that concurrently running CTAs stream the same K/V tiles through L2. Key tiles
-// start at the sample's first token and never leave the sample: tiles of other
-// samples are never visited; only the last key tile of a sample can be partial
-// and only it is masked.
+// Design (one persistent CTA per SM, 10 warps). A work item is (sample, head,
+// 256-row query block) = two 128-row query tiles A and B that share every K/V
+// tile the CTA loads, which halves K/V traffic per FLOP and lets the softmax of
+// one tile overlap the MMAs of the other:
+//   warp 0      TMA producer: the item's Q tiles, then K and V tiles (128 keys)
+//               of the item's own sample only, in separate 2-stage rings.
+//   warp 1      tcgen05 issuer. Per key tile c, in this order:
+//                 PV_A(c)  O_A += P_A V_c   (P_A read from TMEM as the A operand)
+//                 S_A(c+1) = Q_A K_{c+1}^T  (overwrites S_A/P_A in TMEM)
+//                 PV_B(c), S_B(c+1)
+//               MMAs from one thread execute in issue order, so S_X(c+1) never
+//               overwrites P_X(c) before PV_X(c) has read it, and the commit that
+//               signals S_X(c+1) also covers PV_X(c).
+//   warps 2..5  softmax + epilogue of tile A, one thread per query row (TMEM
+//   warps 6..9  lane); the same for tile B. Online softmax in the exp2 domain:
+//               exponentials are taken against the running reference max while
+//               the tile max is tracked alongside; only when the max grows by
+//               more than 2^8 is O rescaled in TMEM and the tile redone (exact
+//               after the final 1/l). P is packed to bf16 into the first 64
+//               columns of the tile's S region.
+// TMEM (512 columns): S_A/P_A | S_B/P_B | O_A | O_B.
+// Work items are ordered longest sample first and, inside a sample, the query
+// blocks of one head next to each other so that concurrently running CTAs stream
+// the same K/V tiles through L2. Key tiles start at the sample's first token and
+// never leave the sample: tiles of other samples are never visited; only the
+// last key tile of a sample can be partial and only it is masked.
 //
 // Every wait is bounded (mbar_wait); on expiry the CTA records MF_ERR_TIMEOUT,
 // lets its in-flight copies and MMAs finish, frees TMEM and returns.
@@ -43,36 +51,39 @@ namespace mf {
 namespace {
 
 constexpr int BM = 128;              // query rows per tile (MMA M)
+constexpr int QB = 2 * BM;           // query rows per work item (tiles A and B)
 constexpr int BN = 128;              // key rows per tile (MMA N of QK^T, K of PV)
-constexpr int NUM_THREADS = 192;     // 6 warps
-constexpr uint32_t TMEM_COLS = 512;  // S0 | S1 | O | P0 | P1
-constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O = 256, TM_P0 = 384, TM_P1 = 448;
+constexpr int NUM_THREADS = 320;     // 10 warps: TMA, MMA, 2 x 4 softmax
+constexpr uint32_t kSoftmaxWarpsPerTile = 4;
+constexpr uint32_t TMEM_COLS = 512;
+// TMEM columns of tile x: S_X (fp32) with P_X (bf16x2) in its first 64 columns,
+// and O_X (fp32, D columns)
+__host__ __device__ constexpr uint32_t tm_s(int x) { return 128u * x; }
+__host__ __device__ constexpr uint32_t tm_o(int x) { return 256u + 128u * x; }
 constexpr int BOX_BYTES = 128 * 128;  // one TMA box: 128 rows x 64 bf16 (128 B), swizzled
-constexpr int NK = 2;                 // K tile ring stages (freed after S = Q K^T)
-constexpr int NV = 3;                 // V tile ring stages (freed after O += P V)
+constexpr int NK = 2;                 // K tile ring stages
+constexpr int NV = 2;                 // V tile ring stages
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: rescale O only past 2^8 growth
 
 template <int D>
 struct Layout {
   static constexpr int kBoxes = D / 64;  // 64-column boxes per 128-row tile
   static constexpr int TILE_BYTES = BM * D * 2;
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + TILE_BYTES;
+  static constexpr int OFF_Q = 0;  // Q_A, Q_B
+  static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
   static constexpr int OFF_V = OFF_K + NK * TILE_BYTES;
   static constexpr int OFF_BAR = OFF_V + NV * TILE_BYTES;
-  // barriers (arrival count 1 unless arrivals() says 4)
+  // barriers (arrival count 1 unless arrivals() says one per softmax warp)
   static constexpr int B_Q_FULL = 0, B_Q_EMPTY = 1;
   static constexpr int B_K_FULL = 2;                 // NK
   static constexpr int B_K_EMPTY = B_K_FULL + NK;    // NK
   static constexpr int B_V_FULL = B_K_EMPTY + NK;    // NV
   static constexpr int B_V_EMPTY = B_V_FULL + NV;    // NV
-  static constexpr int B_S_FULL = B_V_EMPTY + NV;    // 2
-  static constexpr int B_S_FREE = B_S_FULL + 2;      // 2, one arrival per softmax warp
-  static constexpr int B_P_FULL = B_S_FREE + 2;      // 2, one arrival per softmax warp
-  static constexpr int B_PV_DONE = B_P_FULL + 2;     // 2
-  static constexpr int B_O_FULL = B_PV_DONE + 2;
-  static constexpr int B_O_EMPTY = B_O_FULL + 1;     // one arrival per softmax warp
-  static constexpr int B_DRAIN = B_O_EMPTY + 1;
+  static constexpr int B_S_FULL = B_V_EMPTY + NV;    // [tile]
+  static constexpr int B_P_FULL = B_S_FULL + 2;      // [tile], one arrival per softmax warp
+  static constexpr int B_O_FULL = B_P_FULL + 2;      // [tile]
+  static constexpr int B_O_EMPTY = B_O_FULL + 2;     // [tile], one arrival per softmax warp
+  static constexpr int B_DRAIN = B_O_EMPTY + 2;
   static constexpr int NUM_BARS = B_DRAIN + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;  // tmem slot, abort, bad flag
   static constexpr int OFF_CU = OFF_MISC + 16;
@@ -85,9 +96,8 @@ struct Layout {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget of one CTA");
 
   __device__ static uint32_t arrivals(int i) {
-    return (i == B_S_FREE || i == B_S_FREE + 1 || i == B_P_FULL || i == B_P_FULL + 1 ||
-            i == B_O_EMPTY)
-               ? 4u
+    return (i == B_P_FULL || i == B_P_FULL + 1 || i == B_O_EMPTY || i == B_O_EMPTY + 1)
+               ? kSoftmaxWarpsPerTile
                : 1u;
   }
 };
@@ -101,10 +111,11 @@ struct AttnArgs {
 };
 
 struct WorkItem {
-  int32_t s, qt, h, row0, kv0, n, nkv;
+  int32_t s, qb, h, row0, kv0, n, nkv;
+  bool has_b;  // tile B holds at least one row of the sample
 };
 
-__device__ __forceinline__ WorkItem decode_item(int w, int S, int H, const int32_t* s_cu,
+__device__ __forceinline__ WorkItem decode_item(int w, int S, const int32_t* s_cu,
                                                 const int32_t* s_order, const int32_t* s_istart) {
   int lo = 0, hi = S - 1;  // largest r with istart[r] <= w
   while (lo < hi) {
@@ -116,11 +127,12 @@ __device__ __forceinline__ WorkItem decode_item(int w, int S, int H, const int32
   const int local = w - s_istart[lo];
   it.kv0 = s_cu[it.s];
   it.n = s_cu[it.s + 1] - it.kv0;
-  const int nq = (it.n + BM - 1) / BM;
+  const int nq = (it.n + QB - 1) / QB;
   it.h = local / nq;
-  it.qt = local - it.h * nq;
-  it.row0 = it.kv0 + it.qt * BM;
+  it.qb = local - it.h * nq;
+  it.row0 = it.kv0 + it.qb * QB;
   it.nkv = (it.n + BN - 1) / BN;
+  it.has_b = (it.n - it.qb * QB) > BM;
   return it;
 }
 
@@ -140,6 +152,8 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint6
 }
 
 template <int D, bool GATED>
+// Registers are split per SM sub-partition: with 10 warps, two sub-partitions
+// hold three warps each, which caps a thread at 16384 / (3 * 32) = 168.
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     varlen_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
                        const __grid_constant__ CUtensorMap tmap_k,
@@ -202,7 +216,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int r = 0; r < S; ++r) {
       s_istart[r] = acc;
       const int n = s_cu[s_order[r] + 1] - s_cu[s_order[r]];
-      acc += ((n + BM - 1) / BM) * H;
+      acc += ((n + QB - 1) / QB) * H;
     }
     s_istart[S] = acc;
     if (*bad_flag) atomicCAS(args.ctl.err, 0, static_cast<int>(MF_ERR_INVALID));
@@ -217,8 +231,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (warp == 0) {
     // ============================================================ TMA producer
-    // Order of loads: Q, K_0, then (K_{j+1}, V_j) -- the MMA warp consumes
-    // S_j = Q K_j^T before O += P_{j-1} V_{j-1}, so K runs one tile ahead of V.
+    // Order of loads: Q_A (and Q_B), K_0, then (K_{j+1}, V_j): the MMA warp
+    // consumes S(j+1) before PV_B(j), so K runs one tile ahead of V.
     if (lane == 0) {
       uint32_t kc = 0, vc = 0;  // K / V tiles issued so far (global over items)
       int n_item = 0;
@@ -246,12 +260,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         return true;
       };
       for (int w = blockIdx.x; w < total_items && ok; w += gridDim.x, ++n_item) {
-        const WorkItem wi = decode_item(w, S, H, s_cu, s_order, s_istart);
+        const WorkItem wi = decode_item(w, S, s_cu, s_order, s_istart);
         if (!mbar_wait(&bars[L::B_Q_EMPTY], (n_item & 1) ^ 1, args.ctl, abort_flag)) break;
-        mbar_expect_tx(&bars[L::B_Q_FULL], L::TILE_BYTES);
+        const int ntiles = wi.has_b ? 2 : 1;
+        mbar_expect_tx(&bars[L::B_Q_FULL], ntiles * L::TILE_BYTES);
+        for (int x = 0; x < ntiles; ++x)
 #pragma unroll
-        for (int b = 0; b < L::kBoxes; ++b)
-          tma_load_2d(sQ + b * BOX_BYTES, &tmap_q, &bars[L::B_Q_FULL], wi.h * D + 64 * b, wi.row0);
+          for (int b = 0; b < L::kBoxes; ++b)
+            tma_load_2d(sQ + x * L::TILE_BYTES + b * BOX_BYTES, &tmap_q, &bars[L::B_Q_FULL],
+                        wi.h * D + 64 * b, wi.row0 + x * BM);
         if (!load_k(wi, 0)) break;
         for (int j = 0; j < wi.nkv; ++j) {
           if (j + 1 < wi.nkv && !load_k(wi, j + 1)) { ok = false; break; }
@@ -279,60 +296,77 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, 0, 0);
       constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, 0, 1);
       const uint32_t qaddr = smem_u32(sQ), kaddr = smem_u32(sK), vaddr = smem_u32(sV);
-      uint32_t it = 0;
+      uint32_t kv = 0;           // key tiles consumed so far (global over items)
+      uint32_t itx[2] = {0, 0};  // tiles processed per query tile slot (global)
+      int nit[2] = {0, 0};       // items processed per query tile slot
       int n_item = 0;
       bool ok = true;
+      // S_X(c) = Q_X K_c^T into S_X; K-major operands, 128-byte swizzle; a
+      // 16-element K step is a 32-byte advance inside a 64-column box.
+      auto issue_s = [&](int x, uint32_t c) {
+        const int st = c % NK;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (kk >> 2) * BOX_BYTES + (kk & 3) * 32;
+          const uint64_t adesc = sdesc_sw128(qaddr + x * L::TILE_BYTES + koff, 16, 1024);
+          const uint64_t bdesc = sdesc_sw128(kaddr + st * L::TILE_BYTES + koff, 16, 1024);
+          umma_ss(tmem + tm_s(x), adesc, bdesc, IDESC_S, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&bars[L::B_S_FULL + x]);
+      };
+      // O_X += P_X V_c; V is MN-major (LBO = distance between 64-column boxes,
+      // SBO = 8 rows of 128 B); P_X comes from TMEM, 8 columns per 16 keys.
+      auto issue_pv = [&](int x, uint32_t c, bool first) {
+        const int st = c % NV;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint64_t bdesc =
+              sdesc_sw128(vaddr + st * L::TILE_BYTES + kk * 16 * 128, BOX_BYTES, 1024);
+          umma_ts(tmem + tm_o(x), tmem + tm_s(x) + kk * 8, bdesc, IDESC_PV,
+                  (first && kk == 0) ? 0u : 1u);
+        }
+      };
+      auto wait = [&](int bar, uint32_t parity) -> bool {
+        return mbar_wait(&bars[bar], parity, args.ctl, abort_flag);
+      };
       for (int w = blockIdx.x; w < total_items && ok; w += gridDim.x, ++n_item) {
-        const WorkItem wi = decode_item(w, S, H, s_cu, s_order, s_istart);
-        if (!mbar_wait(&bars[L::B_Q_FULL], n_item & 1, args.ctl, abort_flag)) break;
-        // O += P V for global iteration c (first = first key tile of the item)
-        auto issue_pv = [&](uint32_t c, bool first) -> bool {
-          const int st = c % NV;
-          const int b = c & 1;
-          if (!mbar_wait(&bars[L::B_V_FULL + st], (c / NV) & 1, args.ctl, abort_flag)) return false;
-          if (!mbar_wait(&bars[L::B_P_FULL + b], (c >> 1) & 1, args.ctl, abort_flag)) return false;
-          if (first && !mbar_wait(&bars[L::B_O_EMPTY], (n_item & 1) ^ 1, args.ctl, abort_flag))
-            return false;
-          tc_fence_after();
-          const uint32_t p_col = tmem + (b ? TM_P1 : TM_P0);
-#pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk) {
-            // V tile: 16 key rows x D columns, MN-major, 128-byte swizzle;
-            // LBO = distance between 64-column boxes, SBO = 8 rows of 128 B.
-            const uint64_t bdesc =
-                sdesc_sw128(vaddr + st * L::TILE_BYTES + kk * 16 * 128, BOX_BYTES, 1024);
-            umma_ts(tmem + TM_O, p_col + kk * 8, bdesc, IDESC_PV, (first && kk == 0) ? 0u : 1u);
-          }
-          umma_commit(&bars[L::B_V_EMPTY + st]);
-          umma_commit(&bars[L::B_PV_DONE + b]);
-          return true;
-        };
+        const WorkItem wi = decode_item(w, S, s_cu, s_order, s_istart);
+        const int ntiles = wi.has_b ? 2 : 1;
+        if (!wait(L::B_Q_FULL, n_item & 1)) break;
+        // prologue: S_A(0), S_B(0)
+        if (!wait(L::B_K_FULL + kv % NK, (kv / NK) & 1)) break;
+        tc_fence_after();
+        for (int x = 0; x < ntiles; ++x) issue_s(x, kv);
+        umma_commit(&bars[L::B_K_EMPTY + kv % NK]);
+        if (wi.nkv == 1) umma_commit(&bars[L::B_Q_EMPTY]);
         for (int j = 0; j < wi.nkv && ok; ++j) {
-          const uint32_t c = it + j;
-          const int st = c % NK;
-          const int b = c & 1;
-          if (!mbar_wait(&bars[L::B_K_FULL + st], (c / NK) & 1, args.ctl, abort_flag)) { ok = false; break; }
-          if (!mbar_wait(&bars[L::B_S_FREE + b], ((c >> 1) & 1) ^ 1, args.ctl, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t s_col = tmem + (b ? TM_S1 : TM_S0);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            // Q and K tiles: K-major, 128-byte swizzle; a 16-element K step is a
-            // 32-byte advance inside a 64-column box.
-            const uint32_t koff = (kk >> 2) * BOX_BYTES + (kk & 3) * 32;
-            const uint64_t adesc = sdesc_sw128(qaddr + koff, 16, 1024);
-            const uint64_t bdesc = sdesc_sw128(kaddr + st * L::TILE_BYTES + koff, 16, 1024);
-            umma_ss(s_col, adesc, bdesc, IDESC_S, kk > 0 ? 1u : 0u);
+          const uint32_t c = kv + j;
+          const bool more = j + 1 < wi.nkv;
+          if (!wait(L::B_V_FULL + c % NV, (c / NV) & 1)) { ok = false; break; }
+          if (more && !wait(L::B_K_FULL + (c + 1) % NK, ((c + 1) / NK) & 1)) { ok = false; break; }
+          for (int x = 0; x < ntiles; ++x) {
+            // PV_X(j) once softmax X has written P_X(j) (and, on the item's first
+            // tile, once the previous item's epilogue has read O_X)
+            if (!wait(L::B_P_FULL + x, (itx[x] + j) & 1)) { ok = false; break; }
+            if (j == 0 && !wait(L::B_O_EMPTY + x, (nit[x] & 1) ^ 1)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv(x, c, j == 0);
+            if (more) issue_s(x, c + 1);
           }
-          umma_commit(&bars[L::B_K_EMPTY + st]);
-          umma_commit(&bars[L::B_S_FULL + b]);
-          if (j == wi.nkv - 1) umma_commit(&bars[L::B_Q_EMPTY]);
-          if (j > 0 && !issue_pv(c - 1, j == 1)) { ok = false; break; }
+          if (!ok) break;
+          umma_commit(&bars[L::B_V_EMPTY + c % NV]);
+          if (more) {
+            umma_commit(&bars[L::B_K_EMPTY + (c + 1) % NK]);
+            if (j + 2 == wi.nkv) umma_commit(&bars[L::B_Q_EMPTY]);
+          }
         }
         if (!ok) break;
-        if (!issue_pv(it + wi.nkv - 1, wi.nkv == 1)) { ok = false; break; }
-        umma_commit(&bars[L::B_O_FULL]);
-        it += wi.nkv;
+        for (int x = 0; x < ntiles; ++x) {
+          umma_commit(&bars[L::B_O_FULL + x]);
+          itx[x] += wi.nkv;
+          ++nit[x];
+        }
+        kv += wi.nkv;
       }
       // every MMA this thread issued completes before TMEM is released
       umma_commit(&bars[L::B_DRAIN]);
@@ -341,115 +375,144 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     __syncwarp();
   } else {
     // ============================================================ softmax + epilogue
-    const int wq = warp & 3;          // TMEM sub-partition of this warp
-    const int row = wq * 32 + lane;   // query row of this thread inside the tile
+    const int x = (warp - 2) >> 2;    // query tile: 0 = A (warps 2-5), 1 = B (warps 6-9)
+    const int wq = warp & 3;          // TMEM lane quarter of this warp
+    const int row = wq * 32 + lane;   // query row inside the tile
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t s_col = tmem + lane_base + tm_s(x);
+    const uint32_t o_col = tmem + lane_base + tm_o(x);
     const float scale_log2 = args.scale_log2;
-    uint32_t it = 0;
-    int n_item = 0;
+    uint32_t it = 0;  // tiles of this query tile slot processed (global)
+    int n_item = 0;   // items with this tile present
     bool ok = true;
-    for (int w = blockIdx.x; w < total_items && ok; w += gridDim.x, ++n_item) {
-      const WorkItem wi = decode_item(w, S, H, s_cu, s_order, s_istart);
+    for (int w = blockIdx.x; w < total_items && ok; w += gridDim.x) {
+      const WorkItem wi = decode_item(w, S, s_cu, s_order, s_istart);
+      if (x == 1 && !wi.has_b) continue;
       const int last_cols = wi.n - (wi.nkv - 1) * BN;  // valid keys in the last tile
       float m_ref = 0.f;  // reference max (scaled, log2 units)
       float l = 0.f;
       for (int j = 0; j < wi.nkv; ++j, ++it) {
-        const int b = it & 1;
-        if (!warp_wait(&bars[L::B_S_FULL + b], (it >> 1) & 1, args.ctl, abort_flag)) { ok = false; break; }
+        if (!warp_wait(&bars[L::B_S_FULL + x], it & 1, args.ctl, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        uint32_t sr[128];
-        const uint32_t s_addr = tmem + lane_base + (b ? TM_S1 : TM_S0);
-        tmem_ld32(s_addr + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-        tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-        tmem_ld32(s_addr + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
-        tmem_ld32(s_addr + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[L::B_S_FREE + b]);
-        float* sv = reinterpret_cast<float*>(sr);
-        if (j == wi.nkv - 1 && last_cols < BN) {
+        const bool masked = (j == wi.nkv - 1) && (last_cols < BN);
+        // scores of this row from TMEM (fp32), masked past the sample's end
+        auto load_scores = [&](uint32_t (&sr)[BN]) {
 #pragma unroll
-          for (int cidx = 0; cidx < BN; ++cidx)
-            if (cidx >= last_cols) sv[cidx] = -INFINITY;
-        }
-        float mx = sv[0];
+          for (int cc = 0; cc < BN; cc += 32)
+            tmem_ld32(s_col + cc, *reinterpret_cast<uint32_t(*)[32]>(&sr[cc]));
+          tmem_ld_wait();
+          if (masked) {
 #pragma unroll
-        for (int cidx = 1; cidx < BN; ++cidx) mx = fmaxf(mx, sv[cidx]);
-        const float m_tile = mx * scale_log2;
-        if (j == 0) {
-          m_ref = m_tile;
-        } else if (m_tile > m_ref + RESCALE_THRESHOLD) {
-          // O holds sum_j 2^(s' - m_ref) v_j: bring it to the new reference.
-          const uint32_t cprev = it - 1;
-          if (!warp_wait(&bars[L::B_PV_DONE + (cprev & 1)], (cprev >> 1) & 1, args.ctl, abort_flag)) {
-            ok = false;
-            break;
+            for (int cidx = 0; cidx < BN; ++cidx)
+              if (cidx >= last_cols) sr[cidx] = __float_as_uint(-INFINITY);
           }
-          tc_fence_after();
-          const float factor = ex2_approx(m_ref - m_tile);
-          l *= factor;
+        };
+        // P = 2^(s * scale * log2 e - m_ref) packed to bf16 pairs; row sum in ls
+        auto exponentiate = [&](const uint32_t (&sr)[BN], uint32_t (&pp)[BN / 2], float (&ls)[4]) {
 #pragma unroll
-          for (int cc = 0; cc < D; cc += 32) {
-            uint32_t orr[32];
-            tmem_ld32(tmem + lane_base + TM_O + cc, orr);
-            tmem_ld_wait();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * factor);
-            tmem_st32(tmem + lane_base + TM_O + cc, orr);
+          for (int e = 0; e < BN / 2; ++e) {
+            const float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * e]), scale_log2, -m_ref));
+            const float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * e + 1]), scale_log2, -m_ref));
+            ls[(2 * e) & 3] += p0;
+            ls[(2 * e + 1) & 3] += p1;
+            pp[e] = pack_bf16x2(p0, p1);
           }
-          tmem_st_wait();
-          m_ref = m_tile;
-        }
-        // P = 2^(s * scale * log2 e - m_ref), packed to bf16 pairs
-        uint32_t pp[64];
-        float lsum = 0.f;
+        };
+        uint32_t pp[BN / 2];
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};
+        {
+          uint32_t sr[BN];
+          load_scores(sr);
+          if (j > 0) {
+            // exponentials against the current reference, tile max alongside
+            float mx8[8];
 #pragma unroll
-        for (int e = 0; e < 64; ++e) {
-          const float p0 = ex2_approx(fmaf(sv[2 * e], scale_log2, -m_ref));
-          const float p1 = ex2_approx(fmaf(sv[2 * e + 1], scale_log2, -m_ref));
-          lsum += p0 + p1;
-          pp[e] = pack_bf16x2(p0, p1);
-        }
-        l += lsum;
-        if (it >= 2) {  // PV of iteration it-2 has read this P buffer
-          if (!warp_wait(&bars[L::B_PV_DONE + b], ((it >> 1) & 1) ^ 1, args.ctl, abort_flag)) {
-            ok = false;
-            break;
+            for (int e = 0; e < 8; ++e) mx8[e] = -INFINITY;
+#pragma unroll
+            for (int e = 0; e < BN / 2; ++e) {
+              const float x0 = fmaf(__uint_as_float(sr[2 * e]), scale_log2, -m_ref);
+              const float x1 = fmaf(__uint_as_float(sr[2 * e + 1]), scale_log2, -m_ref);
+              mx8[(2 * e) & 7] = fmaxf(mx8[(2 * e) & 7], x0);
+              mx8[(2 * e + 1) & 7] = fmaxf(mx8[(2 * e + 1) & 7], x1);
+              const float p0 = ex2_approx(x0);
+              const float p1 = ex2_approx(x1);
+              ls[(2 * e) & 3] += p0;
+              ls[(2 * e + 1) & 3] += p1;
+              pp[e] = pack_bf16x2(p0, p1);
+            }
+            const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+            if (mx > RESCALE_THRESHOLD) {
+              // The max grew by more than 2^8: move the reference up, bring O and
+              // l along (PV_X(j-1) is complete: S_X(j) was issued after it), and
+              // redo the tile from the scores, still in TMEM.
+              const float factor = ex2_approx(-mx);
+              l *= factor;
+#pragma unroll
+              for (int cc = 0; cc < D; cc += 32) {
+                uint32_t orr[32];
+                tmem_ld32(o_col + cc, orr);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                  orr[e] = __float_as_uint(__uint_as_float(orr[e]) * factor);
+                tmem_st32(o_col + cc, orr);
+              }
+              tmem_st_wait();
+              m_ref += mx;
+#pragma unroll
+              for (int e = 0; e < 4; ++e) ls[e] = 0.f;
+              uint32_t sr2[BN];
+              load_scores(sr2);
+              exponentiate(sr2, pp, ls);
+            }
+          } else {
+            // first tile of the item: the reference is the tile max
+            float mx8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(sr[e]);
+#pragma unroll
+            for (int cidx = 8; cidx < BN; cidx += 8)
+#pragma unroll
+              for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(mx8[e], __uint_as_float(sr[cidx + e]));
+            m_ref = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                          fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * scale_log2;
+            exponentiate(sr, pp, ls);
           }
-          tc_fence_after();
         }
-        const uint32_t p_addr = tmem + lane_base + (b ? TM_P1 : TM_P0);
-        tmem_st32(p_addr + 0, *reinterpret_cast<uint32_t(*)[32]>(&pp[0]));
-        tmem_st32(p_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&pp[32]));
+        l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        tmem_st32(s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(&pp[0]));
+        tmem_st32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&pp[32]));
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[L::B_P_FULL + b]);
+        if (lane == 0) mbar_arrive(&bars[L::B_P_FULL + x]);
       }
       if (!ok) break;
       // ---------------------------------------------------------- epilogue
-      if (!warp_wait(&bars[L::B_O_FULL], n_item & 1, args.ctl, abort_flag)) break;
+      if (!warp_wait(&bars[L::B_O_FULL + x], n_item & 1, args.ctl, abort_flag)) break;
       tc_fence_after();
-      const float inv_l = 1.f / l;
-      const bool row_valid = (wi.qt * BM + row) < wi.n;
-      const int t = wi.row0 + row;
       uint32_t ov[D];
 #pragma unroll
       for (int cc = 0; cc < D; cc += 32)
-        tmem_ld32(tmem + lane_base + TM_O + cc, *reinterpret_cast<uint32_t(*)[32]>(&ov[cc]));
+        tmem_ld32(o_col + cc, *reinterpret_cast<uint32_t(*)[32]>(&ov[cc]));
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[L::B_O_EMPTY]);
-      if (row_valid) {
+      if (lane == 0) mbar_arrive(&bars[L::B_O_EMPTY + x]);
+      ++n_item;
+      const float inv_l = 1.f / l;
+      const int r_in_sample = wi.qb * QB + x * BM + row;
+      const int t = wi.row0 + x * BM + row;
+      if (r_in_sample < wi.n) {
+        const int col0 = wi.h * D;  // first column of this head in [T][H*D]
         if constexpr (GATED) {
           const int hid = H * D;
           const int m = __ldg(args.ep.tok_mod + t) ? 1 : 0;
           const float* gate =
-              args.ep.mod + ((static_cast<size_t>(wi.s) * 2 + m) * 3 + 2) * hid + wi.h * D;
-          const uint4* xr = reinterpret_cast<const uint4*>(args.ep.x + static_cast<size_t>(t) * hid + wi.h * D);
-          uint4* yr = reinterpret_cast<uint4*>(args.ep.y + static_cast<size_t>(t) * hid + wi.h * D);
+              args.ep.mod + ((static_cast<size_t>(wi.s) * 2 + m) * 3 + 2) * hid + col0;
+          const uint4* xr = reinterpret_cast<const uint4*>(args.ep.x + static_cast<size_t>(t) * hid + col0);
+          uint4* yr = reinterpret_cast<uint4*>(args.ep.y + static_cast<size_t>(t) * hid + col0);
 #pragma unroll
           for (int c8 = 0; c8 < D / 8; ++c8) {
             const uint4 xv = __ldg(xr + c8);
@@ -469,7 +532,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             yr[c8] = make_uint4(outw[0], outw[1], outw[2], outw[3]);
           }
         } else {
-          uint4* orow = reinterpret_cast<uint4*>(args.ep.o + (static_cast<size_t>(t) * H + wi.h) * D);
+          uint4* orow = reinterpret_cast<uint4*>(args.ep.o + static_cast<size_t>(t) * H * D + col0);
 #pragma unroll
           for (int c8 = 0; c8 < D / 8; ++c8) {
             uint32_t outw[4];
@@ -561,6 +624,12 @@ int sm_count_dev() {
 }
 
 }  // namespace
+
+int32_t attention_work_items(const int32_t* cu_h, int32_t S, int32_t H) {
+  int64_t n = 0;
+  for (int32_t s = 0; s < S; ++s) n += (static_cast<int64_t>(cu_h[s + 1] - cu_h[s]) + QB - 1) / QB;
+  return static_cast<int32_t>(n * H);
+}
 
 cudaError_t launch_attention(const mf_bf16* q, const mf_bf16* k, const mf_bf16* v,
                              const int32_t* cu_seqlens_d, int32_t S, int32_t T, int32_t H,

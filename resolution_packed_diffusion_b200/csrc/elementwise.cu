@@ -109,34 +109,56 @@ __global__ void __launch_bounds__(256) pack_ids_kernel(const PackParams p, int32
 }
 
 // ------------------------------------------------------------ adaLN params
-// mod[s][n] = sum_c c[s][c] * W[c][n], n in [0, 6*hid): one thread per column,
-// eight samples per pass with their conditioning rows staged in shared memory.
+// mod[s][n] = sum_c c[s][c] * W[c][n], n in [0, 6*hid). A 256-thread CTA covers
+// 64 columns with 4 slices of the conditioning dimension (so 4x more CTAs than
+// columns/256 and enough loads in flight to stream W); the slices are summed in
+// shared memory. Eight samples per pass.
 constexpr int kParamSamples = 8;
 constexpr int kMaxCond = 1024;
+constexpr int kParamCols = 64;
+constexpr int kParamSlices = 4;
 
 __global__ void __launch_bounds__(256) adaln_params_kernel(const float* __restrict__ c,
                                                            const float* __restrict__ W, int S,
                                                            int C, int N, float* __restrict__ mod) {
   __shared__ float s_c[kParamSamples][kMaxCond];
-  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  __shared__ float s_part[kParamSlices][kParamSamples][kParamCols];
+  const int col = threadIdx.x % kParamCols;
+  const int slice = threadIdx.x / kParamCols;
+  const int n = blockIdx.x * kParamCols + col;
+  const int per_slice = (C + kParamSlices - 1) / kParamSlices;
+  const int c0 = slice * per_slice;
+  const int c1 = min(C, c0 + per_slice);
   for (int s0 = 0; s0 < S; s0 += kParamSamples) {
     const int ns = min(kParamSamples, S - s0);
     __syncthreads();
     for (int i = threadIdx.x; i < ns * C; i += blockDim.x)
       s_c[i / C][i % C] = c[static_cast<size_t>(s0 + i / C) * C + (i % C)];
     __syncthreads();
-    if (n < N) {
-      float acc[kParamSamples];
+    float acc[kParamSamples];
 #pragma unroll
-      for (int u = 0; u < kParamSamples; ++u) acc[u] = 0.f;
-      for (int cc = 0; cc < C; ++cc) {
+    for (int u = 0; u < kParamSamples; ++u) acc[u] = 0.f;
+    if (n < N) {
+#pragma unroll 4
+      for (int cc = c0; cc < c1; ++cc) {
         const float w = __ldg(W + static_cast<size_t>(cc) * N + n);
 #pragma unroll
         for (int u = 0; u < kParamSamples; ++u) acc[u] = fmaf(s_c[u][cc], w, acc[u]);
       }
+    }
 #pragma unroll
-      for (int u = 0; u < kParamSamples; ++u)
-        if (u < ns) mod[static_cast<size_t>(s0 + u) * N + n] = acc[u];
+    for (int u = 0; u < kParamSamples; ++u) s_part[slice][u][col] = acc[u];
+    __syncthreads();
+    // slice sums in a fixed order: the result does not depend on scheduling
+    for (int i = threadIdx.x; i < ns * kParamCols; i += blockDim.x) {
+      const int u = i / kParamCols, cl = i % kParamCols;
+      const int nn = blockIdx.x * kParamCols + cl;
+      if (nn < N) {
+        float v = s_part[0][u][cl];
+#pragma unroll
+        for (int sl = 1; sl < kParamSlices; ++sl) v += s_part[sl][u][cl];
+        mod[static_cast<size_t>(s0 + u) * N + nn] = v;
+      }
     }
   }
 }
@@ -145,8 +167,10 @@ __global__ void __launch_bounds__(256) adaln_params_kernel(const float* __restri
 // One warp per token row; the row stays in registers as packed bf16 (NCH
 // 16-byte chunks per lane) across the mean pass, the variance pass and the
 // output pass.
+// The register cap (up to three 256-thread CTAs per SM) keeps enough
+// rows in flight to cover HBM latency.
 template <int NCH>
-__global__ void __launch_bounds__(256) adaln_modulate_kernel(
+__global__ void __launch_bounds__(256, (NCH <= 4 ? 3 : (NCH <= 12 ? 2 : 1))) adaln_modulate_kernel(
     const uint4* __restrict__ x, const float* __restrict__ mod,
     const int32_t* __restrict__ tok_sample, const uint8_t* __restrict__ tok_mod, int T, int S,
     int hid, float eps, uint4* __restrict__ x_mod, KernelCtl ctl) {
@@ -325,7 +349,7 @@ cudaError_t launch_pack_ids(const PackParams& p, int32_t* cu_d, int32_t* pos,
 cudaError_t launch_adaln_params(const float* c, const float* W, int32_t S, int32_t C,
                                 int32_t hid, float* mod, cudaStream_t st) {
   const int N = 6 * hid;
-  adaln_params_kernel<<<(N + 255) / 256, 256, 0, st>>>(c, W, S, C, N, mod);
+  adaln_params_kernel<<<(N + kParamCols - 1) / kParamCols, 256, 0, st>>>(c, W, S, C, N, mod);
   return cudaGetLastError();
 }
 

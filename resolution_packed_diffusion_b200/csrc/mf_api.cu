@@ -5,6 +5,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
 #include <mutex>
 
 #include "mf.h"
@@ -40,7 +41,14 @@ inline bool overlap(const void* a, size_t na, const void* b, size_t nb) {
 
 inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-inline mf_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MF_OK : MF_ERR_CUDA; }
+thread_local char g_last_detail[256] = {0};
+
+inline mf_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return MF_OK;
+  snprintf(g_last_detail, sizeof(g_last_detail), "%s: %s", cudaGetErrorName(e),
+           cudaGetErrorString(e));
+  return MF_ERR_CUDA;
+}
 
 bool valid_head_dim(int32_t D) { return D == 64 || D == 128; }
 
@@ -55,9 +63,7 @@ bool check_offsets(const int32_t* cu_h, int32_t S, int32_t* T) {
 }
 
 int32_t count_items(const int32_t* cu_h, int32_t S, int32_t H) {
-  int64_t n = 0;
-  for (int32_t s = 0; s < S; ++s) n += (static_cast<int64_t>(cu_h[s + 1] - cu_h[s]) + 127) / 128;
-  return static_cast<int32_t>(n * H);
+  return attention_work_items(cu_h, S, H);
 }
 
 // Runs the attention launcher between the caller's timing events, if any.
@@ -110,6 +116,8 @@ using namespace mf;
 extern "C" {
 
 int32_t mf_abi_version(void) { return MF_ABI_VERSION; }
+
+const char* mf_last_error_detail(void) { return g_last_detail; }
 
 const char* mf_status_string(mf_status s) {
   switch (s) {
@@ -187,7 +195,7 @@ mf_status mf_adaln_modulate(const mf_bf16* x, const float* mod, const int32_t* t
   const size_t bytes = static_cast<size_t>(T) * hid * 2;
   if (overlap(x, bytes, x_mod, bytes)) return MF_ERR_INVALID;
   KernelCtl ctl;
-  if (get_ctl(&ctl) != cudaSuccess) return MF_ERR_CUDA;
+  if (cudaError_t ge = get_ctl(&ctl); ge != cudaSuccess) return cuda_status(ge);
   return cuda_status(
       launch_adaln_modulate(x, mod, tok_sample, tok_mod, T, S, hid, eps, x_mod, ctl, stream));
 }
@@ -243,7 +251,7 @@ mf_status mf_varlen_attn_fwd(const mf_bf16* q, const mf_bf16* k, const mf_bf16* 
   if (lse && (overlap(lse, static_cast<size_t>(T) * H * 4, o, bytes)))
     return MF_ERR_INVALID;
   KernelCtl ctl;
-  if (get_ctl(&ctl) != cudaSuccess) return MF_ERR_CUDA;
+  if (cudaError_t ge = get_ctl(&ctl); ge != cudaSuccess) return cuda_status(ge);
   const mf_bf16* qa = q;
   const mf_bf16* ka = k;
   if (pos_ids != nullptr) {
@@ -257,7 +265,7 @@ mf_status mf_varlen_attn_fwd(const mf_bf16* q, const mf_bf16* k, const mf_bf16* 
     RopeTable tab;
     make_rope_table(D, rope_axes, base, &tab);
     cudaError_t e = launch_rope(q, k, pos_ids, T, H, D, tab, wq, wk, stream);
-    if (e != cudaSuccess) return MF_ERR_CUDA;
+    if (e != cudaSuccess) return cuda_status(e);
     qa = wq;
     ka = wk;
   }
@@ -282,7 +290,7 @@ mf_status mf_gated_residual(const mf_bf16* x, const mf_bf16* o, const float* mod
   if (y != x && overlap(x, bytes, y, bytes)) return MF_ERR_INVALID;
   if (overlap(o, bytes, y, bytes)) return MF_ERR_INVALID;
   KernelCtl ctl;
-  if (get_ctl(&ctl) != cudaSuccess) return MF_ERR_CUDA;
+  if (cudaError_t ge = get_ctl(&ctl); ge != cudaSuccess) return cuda_status(ge);
   return cuda_status(
       launch_gated_residual(x, o, mod, tok_sample, tok_mod, T, S, hid, y, ctl, stream));
 }
@@ -317,17 +325,17 @@ mf_status mf_block_fwd(const mf_bf16* x, const mf_bf16* q, const mf_bf16* k, con
   if (overlap(workspace, ws_bytes, x_mod, bytes) || overlap(workspace, ws_bytes, y, bytes))
     return MF_ERR_INVALID;
   KernelCtl ctl;
-  if (get_ctl(&ctl) != cudaSuccess) return MF_ERR_CUDA;
+  if (cudaError_t ge = get_ctl(&ctl); ge != cudaSuccess) return cuda_status(ge);
   cudaError_t e =
       launch_adaln_modulate(x, mod, tok_sample, tok_mod, T, S, hid, eps, x_mod, ctl, stream);
-  if (e != cudaSuccess) return MF_ERR_CUDA;
+  if (e != cudaSuccess) return cuda_status(e);
   const uintptr_t w0 = round_up(reinterpret_cast<uintptr_t>(workspace), 256);
   mf_bf16* wq = reinterpret_cast<mf_bf16*>(w0);
   mf_bf16* wk = reinterpret_cast<mf_bf16*>(w0 + round_up(bytes, 256));
   RopeTable tab;
   make_rope_table(D, rope_axes, base, &tab);
   e = launch_rope(q, k, pos_ids, T, H, D, tab, wq, wk, stream);
-  if (e != cudaSuccess) return MF_ERR_CUDA;
+  if (e != cudaSuccess) return cuda_status(e);
   AttnEpilogue ep{};
   ep.x = x;
   ep.mod = mod;
@@ -339,9 +347,10 @@ mf_status mf_block_fwd(const mf_bf16* x, const mf_bf16* q, const mf_bf16* k, con
 }
 
 mf_status mf_get_error(cudaStream_t stream) {
-  if (cudaStreamSynchronize(stream) != cudaSuccess) return MF_ERR_CUDA;
+  cudaError_t se = cudaStreamSynchronize(stream);
+  if (se != cudaSuccess) return cuda_status(se);
   KernelCtl ctl;
-  if (get_ctl(&ctl) != cudaSuccess) return MF_ERR_CUDA;
+  if (cudaError_t ge = get_ctl(&ctl); ge != cudaSuccess) return cuda_status(ge);
   int v = 0;
   if (cudaMemcpyFromSymbol(&v, g_mf_error, sizeof(int)) != cudaSuccess) return MF_ERR_CUDA;
   const int zero = 0;
@@ -373,7 +382,7 @@ mf_status mf_set_attn_timing_events(cudaEvent_t start, cudaEvent_t stop) {
 mf_status mf_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t stream) {
   if (limit_ns == 0 || limit_ns > 10000000000ull) return MF_ERR_INVALID;
   KernelCtl ctl;
-  if (get_ctl(&ctl) != cudaSuccess) return MF_ERR_CUDA;
+  if (cudaError_t ge = get_ctl(&ctl); ge != cudaSuccess) return cuda_status(ge);
   return cuda_status(launch_selftest_wait(limit_ns, ctl, stream));
 }
 

@@ -66,6 +66,9 @@ struct AttnEpilogue {
   mf_bf16* y;             // gated residual output [T][H*D], or NULL
 };
 
+// Work items (sample, head, 256-row query block) of a pack, from host offsets.
+int32_t attention_work_items(const int32_t* cu_h, int32_t S, int32_t H);
+
 cudaError_t launch_attention(const mf_bf16* q, const mf_bf16* k, const mf_bf16* v,
                              const int32_t* cu_seqlens_d, int32_t S, int32_t T, int32_t H,
                              int32_t D, float softmax_scale, const AttnEpilogue& ep,
