@@ -70,6 +70,7 @@ _SIGS = {
     "mf_get_error": (_I, [_P]),
     "mf_set_wait_limit_ns": (_I, [_U64]),
     "mf_selftest_wait_timeout": (_I, [_U64, _P]),
+    "mf_selftest_exp2_poly": (_I, [_P, _P, _I, _P]),
     "mf_set_attn_timing_events": (_I, [_P, _P]),
     "mf_block_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F,
                                   _F, _P, _P, _P]),
@@ -204,6 +205,10 @@ def mf_get_error(stream=None) -> int:
 
 def mf_set_wait_limit_ns(ns: int) -> None:
     _check(lib.mf_set_wait_limit_ns(int(ns)), "mf_set_wait_limit_ns")
+
+
+def mf_selftest_exp2_poly(x, y, n: int, stream=None) -> None:
+    _check(lib.mf_selftest_exp2_poly(_ptr(x), _ptr(y), n, _stream(stream)), "mf_selftest_exp2_poly")
 
 
 def mf_selftest_wait_timeout(limit_ns: int, stream=None) -> None:

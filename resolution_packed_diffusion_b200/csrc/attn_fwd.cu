@@ -9,7 +9,7 @@
 // block): for every sample s and head h, O = softmax(Q K^T * scale) V over the
 // sample's own keys; optionally y = x + gate[s, modality] * O.
 //
-// Design (one persistent CTA per SM, 10 warps). A work item is (sample, head,
+// Design (one persistent CTA per SM, 12 warps). A work item is (sample, head,
 // 256-row query block) = two 128-row query tiles A and B that share every K/V
 // tile the CTA loads, which halves K/V traffic per FLOP and lets the softmax of
 // one tile overlap the MMAs of the other:
@@ -22,8 +22,10 @@
 //               MMAs from one thread execute in issue order, so S_X(c+1) never
 //               overwrites P_X(c) before PV_X(c) has read it, and the commit that
 //               signals S_X(c+1) also covers PV_X(c).
-//   warps 2..5  softmax + epilogue of tile A, one thread per query row (TMEM
-//   warps 6..9  lane); the same for tile B. Online softmax in the exp2 domain:
+//   warps 2..3  idle (they complete the first warpgroup, which gives most of its
+//               registers to the softmax warpgroups with setmaxnreg).
+//   warps 4..7  softmax + epilogue of tile A, one thread per query row (TMEM
+//   warps 8..11 lane); the same for tile B. Online softmax in the exp2 domain:
 //               exponentials are taken against the running reference max while
 //               the tile max is tracked alongside; only when the max grows by
 //               more than 2^8 is O rescaled in TMEM and the tile redone (exact
@@ -53,7 +55,17 @@ namespace {
 constexpr int BM = 128;              // query rows per tile (MMA M)
 constexpr int QB = 2 * BM;           // query rows per work item (tiles A and B)
 constexpr int BN = 128;              // key rows per tile (MMA N of QK^T, K of PV)
-constexpr int NUM_THREADS = 320;     // 10 warps: TMA, MMA, 2 x 4 softmax
+constexpr int NUM_THREADS = 384;     // 3 warpgroups: {TMA, MMA, 2 idle}, softmax A, softmax B
+// Registers: launched at 168 per thread (384 x 168 = 64512 of the 65536), then
+// the first warpgroup gives up to 104 and the softmax warpgroups take 200 each:
+// 128 * (104 + 200 + 200) = 64512, the launch's own total. 104 keeps the fully
+// unrolled MMA issue (16 MMAs per key tile, issued back to back: measured 8%
+// faster than a rolled loop) free of spills.
+constexpr int kLaunchRegs = 168;
+constexpr int kRegsControl = 104;
+constexpr int kRegsSoftmax = 200;
+static_assert(128 * (kRegsControl + 2 * kRegsSoftmax) <= NUM_THREADS * kLaunchRegs,
+              "register split exceeds the launch allocation");
 constexpr uint32_t kSoftmaxWarpsPerTile = 4;
 constexpr uint32_t TMEM_COLS = 512;
 // TMEM columns of tile x: S_X (fp32) with P_X (bf16x2) in its first 64 columns,
@@ -64,6 +76,15 @@ constexpr int BOX_BYTES = 128 * 128;  // one TMA box: 128 rows x 64 bf16 (128 B)
 constexpr int NK = 2;                 // K tile ring stages
 constexpr int NV = 2;                 // V tile ring stages
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: rescale O only past 2^8 growth
+// Of every 8 key pairs, this many are exponentiated on the FMA pipe
+// (exp2_poly) and the rest on the MUFU unit. Measured on B200 (edit pack,
+// attention alone): 0 -> 1165, 2 -> 1044, 3 -> 1003 useful TFLOP/s: the softmax is
+// bound by issue slots, not by the MUFU, so every exponential goes to the MUFU.
+constexpr int kPolyPairsOf8 = 0;
+
+__device__ __forceinline__ float exp2_mixed(float x, int pair) {
+  return (pair % 8) < kPolyPairsOf8 ? exp2_poly(x) : ex2_approx(x);
+}
 
 template <int D>
 struct Layout {
@@ -152,8 +173,8 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint6
 }
 
 template <int D, bool GATED>
-// Registers are split per SM sub-partition: with 10 warps, two sub-partitions
-// hold three warps each, which caps a thread at 16384 / (3 * 32) = 168.
+// Registers are split per SM sub-partition: with 12 warps each sub-partition
+// holds three, which caps a thread at 16384 / (3 * 32) = 170 -> 168 at launch.
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     varlen_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
                        const __grid_constant__ CUtensorMap tmap_k,
@@ -229,6 +250,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t* sK = smem + L::OFF_K;
   uint8_t* sV = smem + L::OFF_V;
 
+  // Each role sets its register budget inside its own branch: code after a
+  // join of differently budgeted paths is compiled for the smaller budget.
+  if (warp < 4) {
+  regs_dec<kRegsControl>();
   if (warp == 0) {
     // ============================================================ TMA producer
     // Order of loads: Q_A (and Q_B), K_0, then (K_{j+1}, V_j): the MMA warp
@@ -301,30 +326,34 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int nit[2] = {0, 0};       // items processed per query tile slot
       int n_item = 0;
       bool ok = true;
+      // Shared-memory descriptors are built once per operand base; a byte offset
+      // o inside shared memory moves the start-address field by o >> 4 (the
+      // field cannot carry: shared addresses stay below 256 KB).
+      const uint64_t qdesc = sdesc_sw128(qaddr, 16, 1024);
+      const uint64_t kdesc = sdesc_sw128(kaddr, 16, 1024);
+      const uint64_t vdesc = sdesc_sw128(vaddr, BOX_BYTES, 1024);
       // S_X(c) = Q_X K_c^T into S_X; K-major operands, 128-byte swizzle; a
       // 16-element K step is a 32-byte advance inside a 64-column box.
       auto issue_s = [&](int x, uint32_t c) {
-        const int st = c % NK;
+        const uint64_t a0 = qdesc + static_cast<uint64_t>((x * L::TILE_BYTES) >> 4);
+        const uint64_t b0 = kdesc + static_cast<uint64_t>(((c % NK) * L::TILE_BYTES) >> 4);
+        const uint32_t d = tmem + tm_s(x);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t koff = (kk >> 2) * BOX_BYTES + (kk & 3) * 32;
-          const uint64_t adesc = sdesc_sw128(qaddr + x * L::TILE_BYTES + koff, 16, 1024);
-          const uint64_t bdesc = sdesc_sw128(kaddr + st * L::TILE_BYTES + koff, 16, 1024);
-          umma_ss(tmem + tm_s(x), adesc, bdesc, IDESC_S, kk > 0 ? 1u : 0u);
+          const uint32_t koff = ((kk >> 2) * BOX_BYTES + (kk & 3) * 32) >> 4;
+          umma_ss(d, a0 + koff, b0 + koff, IDESC_S, kk > 0 ? 1u : 0u);
         }
         umma_commit(&bars[L::B_S_FULL + x]);
       };
       // O_X += P_X V_c; V is MN-major (LBO = distance between 64-column boxes,
       // SBO = 8 rows of 128 B); P_X comes from TMEM, 8 columns per 16 keys.
       auto issue_pv = [&](int x, uint32_t c, bool first) {
-        const int st = c % NV;
+        const uint64_t b0 = vdesc + static_cast<uint64_t>(((c % NV) * L::TILE_BYTES) >> 4);
+        const uint32_t d = tmem + tm_o(x);
+        const uint32_t a = tmem + tm_s(x);
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t bdesc =
-              sdesc_sw128(vaddr + st * L::TILE_BYTES + kk * 16 * 128, BOX_BYTES, 1024);
-          umma_ts(tmem + tm_o(x), tmem + tm_s(x) + kk * 8, bdesc, IDESC_PV,
-                  (first && kk == 0) ? 0u : 1u);
-        }
+        for (int kk = 0; kk < BN / 16; ++kk)
+          umma_ts(d, a + kk * 8, b0 + ((kk * 16 * 128) >> 4), IDESC_PV, (first && kk == 0) ? 0u : 1u);
       };
       auto wait = [&](int bar, uint32_t parity) -> bool {
         return mbar_wait(&bars[bar], parity, args.ctl, abort_flag);
@@ -373,9 +402,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       drain_wait(&bars[L::B_DRAIN], 0, args.ctl.wait_limit_ns);
     }
     __syncwarp();
+  }
   } else {
+    regs_inc<kRegsSoftmax>();
     // ============================================================ softmax + epilogue
-    const int x = (warp - 2) >> 2;    // query tile: 0 = A (warps 2-5), 1 = B (warps 6-9)
+    const int x = (warp - 4) >> 2;    // query tile: 0 = A (warps 4-7), 1 = B (warps 8-11)
     const int wq = warp & 3;          // TMEM lane quarter of this warp
     const int row = wq * 32 + lane;   // query row inside the tile
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
@@ -407,66 +438,34 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               if (cidx >= last_cols) sr[cidx] = __float_as_uint(-INFINITY);
           }
         };
-        // P = 2^(s * scale * log2 e - m_ref) packed to bf16 pairs; row sum in ls
-        auto exponentiate = [&](const uint32_t (&sr)[BN], uint32_t (&pp)[BN / 2], float (&ls)[4]) {
+        // P = 2^(s * scale * log2 e - m_ref) for the row's 128 keys, packed to 64
+        // bf16 pairs; the row sum goes to four packed fp32 accumulators and the
+        // largest P (as bf16 pairs) to four max accumulators. Per key pair: one
+        // packed FMA, two ex2, one bf16 pack, one packed add, one bf16x2 max.
+        const uint64_t scale2 = f2_pack(scale_log2, scale_log2);
+        auto exponentiate = [&](const uint32_t (&sr)[BN], uint32_t (&pp)[BN / 2], uint64_t (&ls)[4],
+                                uint32_t (&pmax)[4]) {
+          const uint64_t neg_m2 = f2_pack(-m_ref, -m_ref);
 #pragma unroll
           for (int e = 0; e < BN / 2; ++e) {
-            const float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * e]), scale_log2, -m_ref));
-            const float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * e + 1]), scale_log2, -m_ref));
-            ls[(2 * e) & 3] += p0;
-            ls[(2 * e + 1) & 3] += p1;
+            const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])),
+                                       scale2, neg_m2);
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            const float p0 = exp2_mixed(x0, e);
+            const float p1 = exp2_mixed(x1, e);
             pp[e] = pack_bf16x2(p0, p1);
+            ls[e & 3] = f2_add(ls[e & 3], f2_pack(p0, p1));
+            pmax[e & 3] = bf16x2_max(pmax[e & 3], pp[e]);
           }
         };
         uint32_t pp[BN / 2];
-        float ls[4] = {0.f, 0.f, 0.f, 0.f};
+        uint64_t ls[4] = {0, 0, 0, 0};  // packed (0.f, 0.f)
+        uint32_t pmax[4] = {0, 0, 0, 0};
         {
           uint32_t sr[BN];
           load_scores(sr);
-          if (j > 0) {
-            // exponentials against the current reference, tile max alongside
-            float mx8[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) mx8[e] = -INFINITY;
-#pragma unroll
-            for (int e = 0; e < BN / 2; ++e) {
-              const float x0 = fmaf(__uint_as_float(sr[2 * e]), scale_log2, -m_ref);
-              const float x1 = fmaf(__uint_as_float(sr[2 * e + 1]), scale_log2, -m_ref);
-              mx8[(2 * e) & 7] = fmaxf(mx8[(2 * e) & 7], x0);
-              mx8[(2 * e + 1) & 7] = fmaxf(mx8[(2 * e + 1) & 7], x1);
-              const float p0 = ex2_approx(x0);
-              const float p1 = ex2_approx(x1);
-              ls[(2 * e) & 3] += p0;
-              ls[(2 * e + 1) & 3] += p1;
-              pp[e] = pack_bf16x2(p0, p1);
-            }
-            const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-            if (mx > RESCALE_THRESHOLD) {
-              // The max grew by more than 2^8: move the reference up, bring O and
-              // l along (PV_X(j-1) is complete: S_X(j) was issued after it), and
-              // redo the tile from the scores, still in TMEM.
-              const float factor = ex2_approx(-mx);
-              l *= factor;
-#pragma unroll
-              for (int cc = 0; cc < D; cc += 32) {
-                uint32_t orr[32];
-                tmem_ld32(o_col + cc, orr);
-                tmem_ld_wait();
-#pragma unroll
-                for (int e = 0; e < 32; ++e)
-                  orr[e] = __float_as_uint(__uint_as_float(orr[e]) * factor);
-                tmem_st32(o_col + cc, orr);
-              }
-              tmem_st_wait();
-              m_ref += mx;
-#pragma unroll
-              for (int e = 0; e < 4; ++e) ls[e] = 0.f;
-              uint32_t sr2[BN];
-              load_scores(sr2);
-              exponentiate(sr2, pp, ls);
-            }
-          } else {
+          if (j == 0) {
             // first tile of the item: the reference is the tile max
             float mx8[8];
 #pragma unroll
@@ -477,10 +476,55 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(mx8[e], __uint_as_float(sr[cidx + e]));
             m_ref = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                           fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * scale_log2;
-            exponentiate(sr, pp, ls);
           }
+          exponentiate(sr, pp, ls, pmax);
         }
-        l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        // Largest P of the tile above 2^8 (bf16 256 = 0x4380; P >= 0, so bit
+        // patterns order like values; inf and NaN also land above): the max grew
+        // by more than 2^8. Move the reference to the tile max, bring O and l
+        // along (PV_X(j-1) is complete: S_X(j) was issued after it) and redo the
+        // tile from the scores, still in TMEM.
+        const uint32_t pm = bf16x2_max(bf16x2_max(pmax[0], pmax[1]), bf16x2_max(pmax[2], pmax[3]));
+        if ((pm & 0xFFFFu) > 0x4380u || (pm >> 16) > 0x4380u) {
+          uint32_t sr2[BN];
+          load_scores(sr2);
+          float mx8[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(sr2[e]);
+#pragma unroll
+          for (int cidx = 8; cidx < BN; cidx += 8)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(mx8[e], __uint_as_float(sr2[cidx + e]));
+          const float m_new = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                    fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * scale_log2;
+          const float factor = ex2_approx(m_ref - m_new);
+          l *= factor;
+#pragma unroll 1
+          for (int cc = 0; cc < D; cc += 32) {
+            uint32_t orr[32];
+            tmem_ld32(o_col + cc, orr);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * factor);
+            tmem_st32(o_col + cc, orr);
+          }
+          tmem_st_wait();
+          m_ref = m_new;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            ls[e] = 0;
+            pmax[e] = 0;
+          }
+          exponentiate(sr2, pp, ls, pmax);
+        }
+        {
+          float a0, a1, b0, b1, c0, c1, d0, d1;
+          f2_unpack(ls[0], a0, a1);
+          f2_unpack(ls[1], b0, b1);
+          f2_unpack(ls[2], c0, c1);
+          f2_unpack(ls[3], d0, d1);
+          l += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
+        }
         tmem_st32(s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(&pp[0]));
         tmem_st32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&pp[32]));
         tmem_st_wait();
@@ -490,63 +534,71 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       if (!ok) break;
       // ---------------------------------------------------------- epilogue
+      // O row in chunks of 32 columns: normalise by 1/l and write (y = x + gate
+      // * O in the fused block, else O); then release O_X to the next item.
       if (!warp_wait(&bars[L::B_O_FULL + x], n_item & 1, args.ctl, abort_flag)) break;
       tc_fence_after();
-      uint32_t ov[D];
+      const float inv_l = 1.f / l;
+      const int r_in_sample = wi.qb * QB + x * BM + row;
+      const int t = wi.row0 + x * BM + row;
+      const bool row_valid = r_in_sample < wi.n;
+      const int col0 = wi.h * D;  // first column of this head in [T][H*D]
+      const int hid = H * D;
+      const float* gate = nullptr;
+      if constexpr (GATED) {
+        const int m = row_valid ? (__ldg(args.ep.tok_mod + t) ? 1 : 0) : 0;
+        gate = args.ep.mod + ((static_cast<size_t>(wi.s) * 2 + m) * 3 + 2) * hid + col0;
+      }
+#pragma unroll 1
+      for (int cc = 0; cc < D; cc += 32) {
+        uint32_t ov[32];
+        tmem_ld32(o_col + cc, ov);
+        tmem_ld_wait();
+        if (row_valid) {
+          if constexpr (GATED) {
+            const uint4* xr =
+                reinterpret_cast<const uint4*>(args.ep.x + static_cast<size_t>(t) * hid + col0 + cc);
+            uint4* yr = reinterpret_cast<uint4*>(args.ep.y + static_cast<size_t>(t) * hid + col0 + cc);
 #pragma unroll
-      for (int cc = 0; cc < D; cc += 32)
-        tmem_ld32(o_col + cc, *reinterpret_cast<uint32_t(*)[32]>(&ov[cc]));
-      tmem_ld_wait();
+            for (int c8 = 0; c8 < 4; ++c8) {
+              const uint4 xv = __ldg(xr + c8);
+              const float4 g0 = __ldg(reinterpret_cast<const float4*>(gate + cc + c8 * 8));
+              const float4 g1 = __ldg(reinterpret_cast<const float4*>(gate + cc + c8 * 8 + 4));
+              const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+              const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+              uint32_t outw[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float x0 = __uint_as_float(xw[e] << 16);
+                const float x1 = __uint_as_float(xw[e] & 0xFFFF0000u);
+                const float o0 = __uint_as_float(ov[c8 * 8 + 2 * e]) * inv_l;
+                const float o1 = __uint_as_float(ov[c8 * 8 + 2 * e + 1]) * inv_l;
+                outw[e] = pack_bf16x2(fmaf(gv[2 * e], o0, x0), fmaf(gv[2 * e + 1], o1, x1));
+              }
+              yr[c8] = make_uint4(outw[0], outw[1], outw[2], outw[3]);
+            }
+          } else {
+            uint4* orow =
+                reinterpret_cast<uint4*>(args.ep.o + static_cast<size_t>(t) * hid + col0 + cc);
+#pragma unroll
+            for (int c8 = 0; c8 < 4; ++c8) {
+              uint32_t outw[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                outw[e] = pack_bf16x2(__uint_as_float(ov[c8 * 8 + 2 * e]) * inv_l,
+                                      __uint_as_float(ov[c8 * 8 + 2 * e + 1]) * inv_l);
+              orow[c8] = make_uint4(outw[0], outw[1], outw[2], outw[3]);
+            }
+          }
+        }
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[L::B_O_EMPTY + x]);
       ++n_item;
-      const float inv_l = 1.f / l;
-      const int r_in_sample = wi.qb * QB + x * BM + row;
-      const int t = wi.row0 + x * BM + row;
-      if (r_in_sample < wi.n) {
-        const int col0 = wi.h * D;  // first column of this head in [T][H*D]
-        if constexpr (GATED) {
-          const int hid = H * D;
-          const int m = __ldg(args.ep.tok_mod + t) ? 1 : 0;
-          const float* gate =
-              args.ep.mod + ((static_cast<size_t>(wi.s) * 2 + m) * 3 + 2) * hid + col0;
-          const uint4* xr = reinterpret_cast<const uint4*>(args.ep.x + static_cast<size_t>(t) * hid + col0);
-          uint4* yr = reinterpret_cast<uint4*>(args.ep.y + static_cast<size_t>(t) * hid + col0);
-#pragma unroll
-          for (int c8 = 0; c8 < D / 8; ++c8) {
-            const uint4 xv = __ldg(xr + c8);
-            const float4 g0 = __ldg(reinterpret_cast<const float4*>(gate + c8 * 8));
-            const float4 g1 = __ldg(reinterpret_cast<const float4*>(gate + c8 * 8 + 4));
-            const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-            const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-            uint32_t outw[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float x0 = __uint_as_float(xw[e] << 16);
-              const float x1 = __uint_as_float(xw[e] & 0xFFFF0000u);
-              const float o0 = __uint_as_float(ov[c8 * 8 + 2 * e]) * inv_l;
-              const float o1 = __uint_as_float(ov[c8 * 8 + 2 * e + 1]) * inv_l;
-              outw[e] = pack_bf16x2(fmaf(gv[2 * e], o0, x0), fmaf(gv[2 * e + 1], o1, x1));
-            }
-            yr[c8] = make_uint4(outw[0], outw[1], outw[2], outw[3]);
-          }
-        } else {
-          uint4* orow = reinterpret_cast<uint4*>(args.ep.o + static_cast<size_t>(t) * H * D + col0);
-#pragma unroll
-          for (int c8 = 0; c8 < D / 8; ++c8) {
-            uint32_t outw[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              outw[e] = pack_bf16x2(__uint_as_float(ov[c8 * 8 + 2 * e]) * inv_l,
-                                    __uint_as_float(ov[c8 * 8 + 2 * e + 1]) * inv_l);
-            orow[c8] = make_uint4(outw[0], outw[1], outw[2], outw[3]);
-          }
-        }
-        if (args.ep.lse != nullptr)
-          args.ep.lse[static_cast<size_t>(wi.h) * args.T + t] =
-              (m_ref + __log2f(l)) * 0.69314718055994530942f;
-      }
+      if (row_valid && args.ep.lse != nullptr)
+        args.ep.lse[static_cast<size_t>(wi.h) * args.T + t] =
+            (m_ref + __log2f(l)) * 0.69314718055994530942f;
     }
   }
 
@@ -600,8 +652,15 @@ cudaError_t launch_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(varlen_attn_kernel<D, GATED>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    // The setmaxnreg split assumes the kernel was built with exactly
+    // kLaunchRegs registers per thread; with fewer the softmax warpgroups'
+    // setmaxnreg.inc could never be satisfied, so refuse to launch.
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, varlen_attn_kernel<D, GATED>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
+    e = cudaFuncSetAttribute(varlen_attn_kernel<D, GATED>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }

@@ -336,7 +336,18 @@ __global__ void selftest_wait_kernel(KernelCtl ctl) {
   __syncthreads();
 }
 
+__global__ void selftest_exp2_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) y[i] = exp2_poly(x[i]);
+}
+
 }  // namespace
+
+cudaError_t launch_selftest_exp2(const float* x, float* y, int32_t n, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  selftest_exp2_kernel<<<(n + 255) / 256, 256, 0, st>>>(x, y, n);
+  return cudaGetLastError();
+}
 
 // ------------------------------------------------------------ launchers
 cudaError_t launch_pack_ids(const PackParams& p, int32_t* cu_d, int32_t* pos,

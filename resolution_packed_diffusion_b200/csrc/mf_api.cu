@@ -379,6 +379,11 @@ mf_status mf_set_attn_timing_events(cudaEvent_t start, cudaEvent_t stop) {
   return MF_OK;
 }
 
+mf_status mf_selftest_exp2_poly(const float* x, float* y, int32_t n, cudaStream_t stream) {
+  if (n < 0 || (n > 0 && (x == nullptr || y == nullptr))) return MF_ERR_INVALID;
+  return cuda_status(launch_selftest_exp2(x, y, n, stream));
+}
+
 mf_status mf_selftest_wait_timeout(uint64_t limit_ns, cudaStream_t stream) {
   if (limit_ns == 0 || limit_ns > 10000000000ull) return MF_ERR_INVALID;
   KernelCtl ctl;

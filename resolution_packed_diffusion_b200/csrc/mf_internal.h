@@ -74,6 +74,7 @@ cudaError_t launch_attention(const mf_bf16* q, const mf_bf16* k, const mf_bf16* 
                              int32_t D, float softmax_scale, const AttnEpilogue& ep,
                              int32_t num_items, const KernelCtl& ctl, cudaStream_t st);
 
+cudaError_t launch_selftest_exp2(const float* x, float* y, int32_t n, cudaStream_t st);
 cudaError_t launch_selftest_wait(uint64_t limit_ns, const KernelCtl& ctl, cudaStream_t st);
 
 }  // namespace mf

@@ -220,6 +220,62 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// 2^x on the FMA pipe, for x <= 127 (used for part of the softmax exponentials
+// so that they do not all queue on the MUFU unit). Range reduction x = j + f,
+// j = round(x) (adding and subtracting 1.5 * 2^23 rounds to the nearest
+// integer; f = x - j is exact), 2^f from a degree-3 minimax polynomial on
+// [-1/2, 1/2] (coefficients from fit_exp2_poly.py, Remez exchange; maximum
+// relative error 7.5e-5), and 2^j added to the exponent field. Inputs below
+// -125 are clamped there (the result, about 2e-38, stands for zero).
+__device__ __forceinline__ float exp2_poly(float x) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  x = fmaxf(x, -125.0f);
+  const float t = x + kRound;
+  const float f = x - (t - kRound);
+  float p = fmaf(5.517166853e-02f, f, 2.426111251e-01f);
+  p = fmaf(p, f, 6.932609677e-01f);
+  p = fmaf(p, f, 9.999280572e-01f);
+  const int j = __float_as_int(t) - 0x4B400000;  // t's bits are 0x4B400000 + j
+  return __int_as_float(__float_as_int(p) + (j << 23));
+}
+
+// Per-warpgroup register budget (all 128 threads of the warpgroup execute it).
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// Packed fp32 pairs (sm_100 f32x2 instructions): one instruction for two
+// elements' worth of FMA / add. A pair travels as a 64-bit register (x in the low half).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// Element-wise max of two bf16 pairs.
+__device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

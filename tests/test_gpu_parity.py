@@ -245,3 +245,20 @@ def test_rope_in_place():
     mf.mf_rope_apply(q, None, dp.pos, dp.T, dp.H, dp.D, 2, 1e4, q, None)
     ref = oracle.rope_apply(w.f32("q"), oracle_pack(w)["pos_ids"], 2)
     assert_bf16_close(host_f32(q), ref, "rope in place")
+
+
+def test_exp2_poly_against_float64():
+    """The polynomial 2^x the softmax uses for part of its exponentials: relative
+    error within the 7.5e-5 of its fit (plus float32 rounding), on the range the
+    softmax feeds it, and the clamp below -125."""
+    x = torch.cat([torch.linspace(-125.0, 127.0, 200001), torch.tensor([0.0, -0.5, 0.5, 8.0, -1e30])])
+    x = x.float().cuda()
+    y = torch.empty_like(x)
+    mf.mf_selftest_exp2_poly(x, y, x.numel())
+    torch.cuda.synchronize()
+    xs = x.cpu().double().numpy()
+    ys = y.cpu().double().numpy()
+    ref = np.exp2(np.maximum(xs, -125.0))
+    rel = np.abs(ys / ref - 1.0)
+    assert rel.max() <= 8e-5, rel.max()
+    assert ys[-1] < 1e-37  # -1e30 stands for zero
