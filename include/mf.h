@@ -207,8 +207,9 @@ mf_status mf_set_wait_limit_ns(uint64_t ns);
 mf_status mf_set_attn_timing_events(cudaEvent_t start, cudaEvent_t stop);
 
 /* Self-test of the polynomial 2^x the attention softmax uses for part of its
- * exponentials: y[i] = exp2_poly(x[i]) for n device floats (x <= 127; inputs
- * below -125 are treated as -125). Relative error <= 7.5e-5 by construction. */
+ * exponentials: y[i] = 2^x[i] for n device floats, evaluated pairwise exactly
+ * as in the softmax (x <= 127; inputs below -125 are treated as -125). Relative
+ * error <= 7.5e-5 by construction. */
 mf_status mf_selftest_exp2_poly(const float* x, float* y, int32_t n, cudaStream_t stream);
 
 /* Self-test of the error channel: launches one CTA that waits on an mbarrier

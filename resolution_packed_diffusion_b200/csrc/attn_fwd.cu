@@ -75,16 +75,12 @@ __host__ __device__ constexpr uint32_t tm_o(int x) { return 256u + 128u * x; }
 constexpr int BOX_BYTES = 128 * 128;  // one TMA box: 128 rows x 64 bf16 (128 B), swizzled
 constexpr int NK = 2;                 // K tile ring stages
 constexpr int NV = 2;                 // V tile ring stages
-constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: rescale O only past 2^8 growth
 // Of every 8 key pairs, this many are exponentiated on the FMA pipe
-// (exp2_poly) and the rest on the MUFU unit. Measured on B200 (edit pack,
-// attention alone): 0 -> 1165, 2 -> 1044, 3 -> 1003 useful TFLOP/s: the softmax is
-// bound by issue slots, not by the MUFU, so every exponential goes to the MUFU.
-constexpr int kPolyPairsOf8 = 0;
+// (exp2_poly2) and the rest on the MUFU unit, which the two softmax warpgroups
+// share. Measured on B200 (edit pack, attention alone, two runs each):
+// 0 -> 1032, 1 -> 1053, 2 -> 1145 / 1084, 3 -> 1066 / 1002 useful TFLOP/s.
+constexpr int kPolyPairsOf8 = 2;
 
-__device__ __forceinline__ float exp2_mixed(float x, int pair) {
-  return (pair % 8) < kPolyPairsOf8 ? exp2_poly(x) : ex2_approx(x);
-}
 
 template <int D>
 struct Layout {
@@ -452,8 +448,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                        scale2, neg_m2);
             float x0, x1;
             f2_unpack(x2, x0, x1);
-            const float p0 = exp2_mixed(x0, e);
-            const float p1 = exp2_mixed(x1, e);
+            float p0, p1;
+            if ((e % 8) < kPolyPairsOf8) {
+              exp2_poly2(x0, x1, p0, p1);
+            } else {
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+            }
             pp[e] = pack_bf16x2(p0, p1);
             ls[e & 3] = f2_add(ls[e & 3], f2_pack(p0, p1));
             pmax[e & 3] = bf16x2_max(pmax[e & 3], pp[e]);

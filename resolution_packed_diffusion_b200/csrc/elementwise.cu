@@ -336,16 +336,25 @@ __global__ void selftest_wait_kernel(KernelCtl ctl) {
   __syncthreads();
 }
 
+// Pairs (2i, 2i+1) through exp2_poly2, as the attention softmax uses it; a
+// trailing odd element is paired with itself.
 __global__ void selftest_exp2_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) y[i] = exp2_poly(x[i]);
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i < n) {
+    const float a = x[i];
+    const float b = (i + 1 < n) ? x[i + 1] : a;
+    float pa, pb;
+    exp2_poly2(a, b, pa, pb);
+    y[i] = pa;
+    if (i + 1 < n) y[i + 1] = pb;
+  }
 }
 
 }  // namespace
 
 cudaError_t launch_selftest_exp2(const float* x, float* y, int32_t n, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
-  selftest_exp2_kernel<<<(n + 255) / 256, 256, 0, st>>>(x, y, n);
+  selftest_exp2_kernel<<<(n / 2 + 256) / 256, 256, 0, st>>>(x, y, n);
   return cudaGetLastError();
 }
 

@@ -220,25 +220,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe, for x <= 127 (used for part of the softmax exponentials
-// so that they do not all queue on the MUFU unit). Range reduction x = j + f,
-// j = round(x) (adding and subtracting 1.5 * 2^23 rounds to the nearest
-// integer; f = x - j is exact), 2^f from a degree-3 minimax polynomial on
-// [-1/2, 1/2] (coefficients from fit_exp2_poly.py, Remez exchange; maximum
-// relative error 7.5e-5), and 2^j added to the exponent field. Inputs below
-// -125 are clamped there (the result, about 2e-38, stands for zero).
-__device__ __forceinline__ float exp2_poly(float x) {
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  x = fmaxf(x, -125.0f);
-  const float t = x + kRound;
-  const float f = x - (t - kRound);
-  float p = fmaf(5.517166853e-02f, f, 2.426111251e-01f);
-  p = fmaf(p, f, 6.932609677e-01f);
-  p = fmaf(p, f, 9.999280572e-01f);
-  const int j = __float_as_int(t) - 0x4B400000;  // t's bits are 0x4B400000 + j
-  return __int_as_float(__float_as_int(p) + (j << 23));
-}
-
 // Per-warpgroup register budget (all 128 threads of the warpgroup execute it).
 template <int N>
 __device__ __forceinline__ void regs_dec() {
@@ -274,6 +255,33 @@ __device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
   uint32_t r;
   asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
   return r;
+}
+
+// 2^x for a pair of inputs on the FMA pipe (f32x2 instructions), x <= 127; used
+// for part of the softmax exponentials so that they do not all queue on the
+// MUFU unit. Range reduction x = j + f with j = round(x): t = x + 1.5 * 2^23
+// rounds to the nearest integer, -j = 1.5 * 2^23 - t and f = x - j are exact.
+// 2^f from a degree-3 minimax polynomial on [-1/2, 1/2] (coefficients from
+// fit_exp2_poly.py, Remez exchange; maximum relative error 7.5e-5). 2^j is added
+// to the exponent field: t's bits are 0x4B400000 + j and 0x4B400000 << 23
+// vanishes modulo 2^32, so (bits(t) << 23) is j << 23. Inputs below -125 are
+// clamped there (the result, about 2e-38, stands for zero).
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& p0, float& p1) {
+  const uint64_t round2 = f2_pack(12582912.0f, 12582912.0f);
+  const uint64_t x2 = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+  const uint64_t t2 = f2_add(x2, round2);
+  uint64_t nj2;  // -j = 1.5 * 2^23 - t
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(nj2) : "l"(round2), "l"(t2));
+  const uint64_t f2 = f2_add(x2, nj2);
+  uint64_t p2 = f2_fma(f2_pack(5.517166853e-02f, 5.517166853e-02f), f2,
+                       f2_pack(2.426111251e-01f, 2.426111251e-01f));
+  p2 = f2_fma(p2, f2, f2_pack(6.932609677e-01f, 6.932609677e-01f));
+  p2 = f2_fma(p2, f2, f2_pack(9.999280572e-01f, 9.999280572e-01f));
+  float q0, q1, t0, t1;
+  f2_unpack(p2, q0, q1);
+  f2_unpack(t2, t0, t1);
+  p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
