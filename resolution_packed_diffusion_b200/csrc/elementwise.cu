@@ -110,22 +110,27 @@ __global__ void __launch_bounds__(256) pack_ids_kernel(const PackParams p, int32
 
 // ------------------------------------------------------------ adaLN params
 // mod[s][n] = sum_c c[s][c] * W[c][n], n in [0, 6*hid). A 256-thread CTA covers
-// 64 columns with 4 slices of the conditioning dimension (so 4x more CTAs than
-// columns/256 and enough loads in flight to stream W); the slices are summed in
-// shared memory. Eight samples per pass.
+// 128 columns: 32 threads read float4 column groups, 8 warps split the
+// conditioning dimension into slices, and the slice sums meet in shared memory
+// in a fixed order (the result does not depend on scheduling). Eight samples
+// per pass share each W load.
 constexpr int kParamSamples = 8;
 constexpr int kMaxCond = 1024;
-constexpr int kParamCols = 64;
-constexpr int kParamSlices = 4;
+constexpr int kParamSlices = 8;
+constexpr int kParamCols4 = 32;  // float4 column groups per CTA
 
 __global__ void __launch_bounds__(256) adaln_params_kernel(const float* __restrict__ c,
-                                                           const float* __restrict__ W, int S,
-                                                           int C, int N, float* __restrict__ mod) {
-  __shared__ float s_c[kParamSamples][kMaxCond];
-  __shared__ float s_part[kParamSlices][kParamSamples][kParamCols];
-  const int col = threadIdx.x % kParamCols;
-  const int slice = threadIdx.x / kParamCols;
-  const int n = blockIdx.x * kParamCols + col;
+                                                           const float4* __restrict__ W4, int S,
+                                                           int C, int N4, float4* __restrict__ mod4) {
+  // the conditioning rows and, after them, the slice partial sums share one
+  // 32 KB buffer
+  __shared__ __align__(16) unsigned char buf[kParamSamples * kMaxCond * 4];
+  static_assert(sizeof(float4) * kParamSlices * kParamSamples * kParamCols4 <= sizeof(buf), "");
+  auto s_c = reinterpret_cast<float(*)[kMaxCond]>(buf);
+  auto s_part = reinterpret_cast<float4(*)[kParamSamples][kParamCols4]>(buf);
+  const int g = threadIdx.x & 31;      // column group inside the CTA
+  const int slice = threadIdx.x >> 5;  // slice of the conditioning dimension
+  const int n4 = blockIdx.x * kParamCols4 + g;
   const int per_slice = (C + kParamSlices - 1) / kParamSlices;
   const int c0 = slice * per_slice;
   const int c1 = min(C, c0 + per_slice);
@@ -135,29 +140,38 @@ __global__ void __launch_bounds__(256) adaln_params_kernel(const float* __restri
     for (int i = threadIdx.x; i < ns * C; i += blockDim.x)
       s_c[i / C][i % C] = c[static_cast<size_t>(s0 + i / C) * C + (i % C)];
     __syncthreads();
-    float acc[kParamSamples];
+    float4 acc[kParamSamples];
 #pragma unroll
-    for (int u = 0; u < kParamSamples; ++u) acc[u] = 0.f;
-    if (n < N) {
+    for (int u = 0; u < kParamSamples; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (n4 < N4) {
 #pragma unroll 4
       for (int cc = c0; cc < c1; ++cc) {
-        const float w = __ldg(W + static_cast<size_t>(cc) * N + n);
+        const float4 w = __ldg(W4 + static_cast<size_t>(cc) * N4 + n4);
 #pragma unroll
-        for (int u = 0; u < kParamSamples; ++u) acc[u] = fmaf(s_c[u][cc], w, acc[u]);
+        for (int u = 0; u < kParamSamples; ++u) {
+          const float cv = s_c[u][cc];
+          acc[u].x = fmaf(cv, w.x, acc[u].x);
+          acc[u].y = fmaf(cv, w.y, acc[u].y);
+          acc[u].z = fmaf(cv, w.z, acc[u].z);
+          acc[u].w = fmaf(cv, w.w, acc[u].w);
+        }
       }
     }
+    __syncthreads();  // every thread is done with s_c
 #pragma unroll
-    for (int u = 0; u < kParamSamples; ++u) s_part[slice][u][col] = acc[u];
+    for (int u = 0; u < kParamSamples; ++u) s_part[slice][u][g] = acc[u];
     __syncthreads();
-    // slice sums in a fixed order: the result does not depend on scheduling
-    for (int i = threadIdx.x; i < ns * kParamCols; i += blockDim.x) {
-      const int u = i / kParamCols, cl = i % kParamCols;
-      const int nn = blockIdx.x * kParamCols + cl;
-      if (nn < N) {
-        float v = s_part[0][u][cl];
+    for (int i = threadIdx.x; i < ns * kParamCols4; i += blockDim.x) {
+      const int u = i / kParamCols4, gg = i % kParamCols4;
+      const int nn4 = blockIdx.x * kParamCols4 + gg;
+      if (nn4 < N4) {
+        float4 v = s_part[0][u][gg];
 #pragma unroll
-        for (int sl = 1; sl < kParamSlices; ++sl) v += s_part[sl][u][cl];
-        mod[static_cast<size_t>(s0 + u) * N + nn] = v;
+        for (int sl = 1; sl < kParamSlices; ++sl) {
+          const float4 q = s_part[sl][u][gg];
+          v.x += q.x; v.y += q.y; v.z += q.z; v.w += q.w;
+        }
+        mod4[static_cast<size_t>(s0 + u) * N4 + nn4] = v;
       }
     }
   }
@@ -166,7 +180,9 @@ __global__ void __launch_bounds__(256) adaln_params_kernel(const float* __restri
 // ------------------------------------------------------------ adaLN modulate
 // One warp per token row; the row stays in registers as packed bf16 (NCH
 // 16-byte chunks per lane) across the mean pass, the variance pass and the
-// output pass.
+// output pass. Each CTA takes a contiguous range of rows (its warps
+// interleaved inside it), so the rows an SM works on at a time mostly share a
+// sample and modality and their shift / scale vectors stay in L1.
 // The register cap (up to three 256-thread CTAs per SM) keeps enough
 // rows in flight to cover HBM latency.
 template <int NCH>
@@ -175,10 +191,12 @@ __global__ void __launch_bounds__(256, (NCH <= 4 ? 3 : (NCH <= 12 ? 2 : 1))) ada
     const int32_t* __restrict__ tok_sample, const uint8_t* __restrict__ tok_mod, int T, int S,
     int hid, float eps, uint4* __restrict__ x_mod, KernelCtl ctl) {
   const int lane = threadIdx.x & 31;
-  const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  const int wpb = blockDim.x >> 5;
   const int nchunk = hid >> 3;
   const float inv_hid = 1.f / static_cast<float>(hid);
-  for (int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < T; row += nwarps) {
+  const int per_block = (T + gridDim.x - 1) / gridDim.x;
+  const int row_end = min(T, (blockIdx.x + 1) * per_block);
+  for (int row = blockIdx.x * per_block + (threadIdx.x >> 5); row < row_end; row += wpb) {
     const int s = __ldg(tok_sample + row);
     const int m = __ldg(tok_mod + row);
     if (s < 0 || s >= S || m > 1) {
@@ -269,6 +287,8 @@ __global__ void __launch_bounds__(256) rope_kernel(const uint4* q, const uint4* 
         sn[j] = 0.f;
       }
     }
+    // four heads per step: 8 independent 16-byte loads in flight per thread
+#pragma unroll 4
     for (int h = 0; h < H; ++h) {
       const size_t off = (static_cast<size_t>(t) * H + h) * cpr + cch;
 #pragma unroll
@@ -277,13 +297,13 @@ __global__ void __launch_bounds__(256) rope_kernel(const uint4* q, const uint4* 
         uint4* dst = which ? k_out : q_out;
         if (src == nullptr) continue;
         float f[8], o[8];
-        unpack8(src[off], f);
+        unpack8(__ldcs(src + off), f);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           o[2 * j] = f[2 * j] * cs[j] - f[2 * j + 1] * sn[j];
           o[2 * j + 1] = f[2 * j] * sn[j] + f[2 * j + 1] * cs[j];
         }
-        dst[off] = pack8(o);
+        __stcs(dst + off, pack8(o));
       }
     }
   }
@@ -368,8 +388,9 @@ cudaError_t launch_pack_ids(const PackParams& p, int32_t* cu_d, int32_t* pos,
 
 cudaError_t launch_adaln_params(const float* c, const float* W, int32_t S, int32_t C,
                                 int32_t hid, float* mod, cudaStream_t st) {
-  const int N = 6 * hid;
-  adaln_params_kernel<<<(N + kParamCols - 1) / kParamCols, 256, 0, st>>>(c, W, S, C, N, mod);
+  const int N4 = 6 * hid / 4;  // hid % 8 == 0, so whole float4 groups
+  adaln_params_kernel<<<(N4 + kParamCols4 - 1) / kParamCols4, 256, 0, st>>>(
+      c, reinterpret_cast<const float4*>(W), S, C, N4, reinterpret_cast<float4*>(mod));
   return cudaGetLastError();
 }
 
@@ -379,7 +400,9 @@ cudaError_t launch_adaln_modulate(const mf_bf16* x, const float* mod, const int3
                                   cudaStream_t st) {
   const int nchunk = hid / 8;
   const int per_lane = (nchunk + 31) / 32;
-  const int grid = grid_for(static_cast<long long>(T) * 32, 256, 8);
+  // resident CTAs only (persistent): 3, 2 or 1 per SM by the register cap
+  const int per_sm = per_lane <= 4 ? 3 : (per_lane <= 12 ? 2 : 1);
+  const int grid = grid_for(static_cast<long long>(T) * 32, 256, per_sm);
   auto X = reinterpret_cast<const uint4*>(x);
   auto XM = reinterpret_cast<uint4*>(x_mod);
 #define MF_ADALN_CASE(N)                                                                   \
