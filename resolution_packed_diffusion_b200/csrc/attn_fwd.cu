@@ -153,6 +153,14 @@ __device__ __forceinline__ WorkItem decode_item(int w, int S, const int32_t* s_c
   return it;
 }
 
+// k-th work item of CTA b among G CTAs: rounds of G items in longest-first
+// order, dealt forwards in even rounds and backwards in odd ones, which evens
+// out the CTAs' totals when item sizes fall along the order. Every role of a CTA
+// walks the same sequence.
+__device__ __forceinline__ int snake_item(int k, int b, int G) {
+  return k * G + ((k & 1) ? (G - 1 - b) : b);
+}
+
 // Wait with every lane of a warp and agree on the outcome.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const KernelCtl& ctl,
                                           volatile int* abort_flag) {
@@ -280,7 +288,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ++vc;
         return true;
       };
-      for (int w = blockIdx.x; w < total_items && ok; w += gridDim.x, ++n_item) {
+      for (int k = 0, w = snake_item(0, blockIdx.x, gridDim.x); w < total_items && ok;
+           w = snake_item(++k, blockIdx.x, gridDim.x), ++n_item) {
         const WorkItem wi = decode_item(w, S, s_cu, s_order, s_istart);
         if (!mbar_wait(&bars[L::B_Q_EMPTY], (n_item & 1) ^ 1, args.ctl, abort_flag)) break;
         const int ntiles = wi.has_b ? 2 : 1;
@@ -354,7 +363,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       auto wait = [&](int bar, uint32_t parity) -> bool {
         return mbar_wait(&bars[bar], parity, args.ctl, abort_flag);
       };
-      for (int w = blockIdx.x; w < total_items && ok; w += gridDim.x, ++n_item) {
+      for (int k = 0, w = snake_item(0, blockIdx.x, gridDim.x); w < total_items && ok;
+           w = snake_item(++k, blockIdx.x, gridDim.x), ++n_item) {
         const WorkItem wi = decode_item(w, S, s_cu, s_order, s_istart);
         const int ntiles = wi.has_b ? 2 : 1;
         if (!wait(L::B_Q_FULL, n_item & 1)) break;
@@ -412,7 +422,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t it = 0;  // tiles of this query tile slot processed (global)
     int n_item = 0;   // items with this tile present
     bool ok = true;
-    for (int w = blockIdx.x; w < total_items && ok; w += gridDim.x) {
+    for (int k = 0, w = snake_item(0, blockIdx.x, gridDim.x); w < total_items && ok;
+         w = snake_item(++k, blockIdx.x, gridDim.x)) {
       const WorkItem wi = decode_item(w, S, s_cu, s_order, s_istart);
       if (x == 1 && !wi.has_b) continue;
       const int last_cols = wi.n - (wi.nkv - 1) * BN;  // valid keys in the last tile
@@ -537,36 +548,40 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // ---------------------------------------------------------- epilogue
       // O row in chunks of 32 columns: normalise by 1/l and write (y = x + gate
       // * O in the fused block, else O); then release O_X to the next item.
-      if (!warp_wait(&bars[L::B_O_FULL + x], n_item & 1, args.ctl, abort_flag)) break;
-      tc_fence_after();
-      const float inv_l = 1.f / l;
       const int r_in_sample = wi.qb * QB + x * BM + row;
       const int t = wi.row0 + x * BM + row;
       const bool row_valid = r_in_sample < wi.n;
       const int col0 = wi.h * D;  // first column of this head in [T][H*D]
       const int hid = H * D;
       const float* gate = nullptr;
+      // the block input row (the epilogue's only DRAM read) is requested before
+      // waiting for the last PV, so its latency overlaps that MMA
+      uint4 xv[GATED ? D / 8 : 1];
       if constexpr (GATED) {
         const int m = row_valid ? (__ldg(args.ep.tok_mod + t) ? 1 : 0) : 0;
         gate = args.ep.mod + ((static_cast<size_t>(wi.s) * 2 + m) * 3 + 2) * hid + col0;
+        const uint4* xr = reinterpret_cast<const uint4*>(args.ep.x + static_cast<size_t>(t) * hid + col0);
+#pragma unroll
+        for (int c8 = 0; c8 < D / 8; ++c8) xv[c8] = row_valid ? __ldg(xr + c8) : make_uint4(0, 0, 0, 0);
       }
-#pragma unroll 1
+      if (!warp_wait(&bars[L::B_O_FULL + x], n_item & 1, args.ctl, abort_flag)) break;
+      tc_fence_after();
+      const float inv_l = 1.f / l;
+#pragma unroll
       for (int cc = 0; cc < D; cc += 32) {
         uint32_t ov[32];
         tmem_ld32(o_col + cc, ov);
         tmem_ld_wait();
         if (row_valid) {
           if constexpr (GATED) {
-            const uint4* xr =
-                reinterpret_cast<const uint4*>(args.ep.x + static_cast<size_t>(t) * hid + col0 + cc);
             uint4* yr = reinterpret_cast<uint4*>(args.ep.y + static_cast<size_t>(t) * hid + col0 + cc);
 #pragma unroll
             for (int c8 = 0; c8 < 4; ++c8) {
-              const uint4 xv = __ldg(xr + c8);
+              const uint4 xc = xv[cc / 8 + c8];
               const float4 g0 = __ldg(reinterpret_cast<const float4*>(gate + cc + c8 * 8));
               const float4 g1 = __ldg(reinterpret_cast<const float4*>(gate + cc + c8 * 8 + 4));
               const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-              const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+              const uint32_t xw[4] = {xc.x, xc.y, xc.z, xc.w};
               uint32_t outw[4];
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
