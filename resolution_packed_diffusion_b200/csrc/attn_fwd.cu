@@ -43,7 +43,12 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include <algorithm>
 #include <cstdint>
+#include <functional>
+#include <queue>
+#include <utility>
+#include <vector>
 
 #include "mf_internal.h"
 #include "mf_ptx.cuh"
@@ -119,7 +124,21 @@ struct Layout {
   }
 };
 
+// Per-CTA work lists computed on the host (greedy longest-processing-time
+// assignment), passed in the kernel parameters. CTA b runs ids[start[b]],
+// ids[start[b] + 1], ... up to an entry of kSchedEnd. valid == 0 means "use the
+// snake order" (too many items, or CTAs, for the table).
+constexpr int kMaxSchedItems = 4096;
+constexpr int kMaxSchedCtas = 160;
+constexpr int32_t kSchedEnd = 0x7fffffff;
+struct Schedule {
+  int32_t valid;
+  int32_t start[kMaxSchedCtas];
+  int32_t ids[kMaxSchedItems + kMaxSchedCtas];  // items plus one end mark per CTA
+};
+
 struct AttnArgs {
+  Schedule sched;
   const int32_t* cu_seqlens;
   int32_t S, T, H;
   float scale_log2;  // softmax_scale * log2(e)
@@ -182,7 +201,8 @@ template <int D, bool GATED>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     varlen_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
                        const __grid_constant__ CUtensorMap tmap_k,
-                       const __grid_constant__ CUtensorMap tmap_v, const AttnArgs args) {
+                       const __grid_constant__ CUtensorMap tmap_v,
+                       const __grid_constant__ AttnArgs args) {
   using L = Layout<D>;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the 128-byte-swizzled TMA / UMMA tiles
@@ -249,6 +269,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   const uint32_t tmem = *tmem_slot;
   const int total_items = *bad_flag ? 0 : s_istart[S];
+  // k-th work item of this CTA (at least total_items once the list is exhausted)
+  auto item_k = [&](int k) -> int {
+    return args.sched.valid ? args.sched.ids[args.sched.start[blockIdx.x] + k]
+                            : snake_item(k, blockIdx.x, gridDim.x);
+  };
 
   uint8_t* sQ = smem + L::OFF_Q;
   uint8_t* sK = smem + L::OFF_K;
@@ -288,8 +313,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ++vc;
         return true;
       };
-      for (int k = 0, w = snake_item(0, blockIdx.x, gridDim.x); w < total_items && ok;
-           w = snake_item(++k, blockIdx.x, gridDim.x), ++n_item) {
+      for (int k = 0, w = item_k(0); w < total_items && ok; w = item_k(++k), ++n_item) {
         const WorkItem wi = decode_item(w, S, s_cu, s_order, s_istart);
         if (!mbar_wait(&bars[L::B_Q_EMPTY], (n_item & 1) ^ 1, args.ctl, abort_flag)) break;
         const int ntiles = wi.has_b ? 2 : 1;
@@ -363,8 +387,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       auto wait = [&](int bar, uint32_t parity) -> bool {
         return mbar_wait(&bars[bar], parity, args.ctl, abort_flag);
       };
-      for (int k = 0, w = snake_item(0, blockIdx.x, gridDim.x); w < total_items && ok;
-           w = snake_item(++k, blockIdx.x, gridDim.x), ++n_item) {
+      for (int k = 0, w = item_k(0); w < total_items && ok; w = item_k(++k), ++n_item) {
         const WorkItem wi = decode_item(w, S, s_cu, s_order, s_istart);
         const int ntiles = wi.has_b ? 2 : 1;
         if (!wait(L::B_Q_FULL, n_item & 1)) break;
@@ -422,8 +445,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t it = 0;  // tiles of this query tile slot processed (global)
     int n_item = 0;   // items with this tile present
     bool ok = true;
-    for (int k = 0, w = snake_item(0, blockIdx.x, gridDim.x); w < total_items && ok;
-         w = snake_item(++k, blockIdx.x, gridDim.x)) {
+    for (int k = 0, w = item_k(0); w < total_items && ok; w = item_k(++k)) {
       const WorkItem wi = decode_item(w, S, s_cu, s_order, s_istart);
       if (x == 1 && !wi.has_b) continue;
       const int last_cols = wi.n - (wi.nkv - 1) * BN;  // valid keys in the last tile
@@ -698,6 +720,62 @@ int sm_count_dev() {
   return cached[dev];
 }
 
+// Greedy longest-processing-time schedule over the items in the kernel's own
+// numbering (samples longest first, ties by pack order; inside a sample
+// item = head * query_blocks + query_block). An item over nkv key tiles costs
+// nkv + 1 periods whether it holds one query tile or two: a lone tile's softmax
+// is not hidden behind a second tile's MMAs, and timing showed it nearly as
+// slow. Each item goes to the least-loaded CTA (lowest index on ties). The table is used only when this
+// beats the snake order's estimated makespan by more than 1%: where the two
+// tie (equal items, or one item per CTA) the snake order measured a little
+// faster. Leaves s->valid = 0 for the snake order, and when the table cannot
+// hold the items.
+void build_schedule(const int32_t* cu_h, int32_t S, int32_t H, int grid, Schedule* s) {
+  s->valid = 0;
+  std::vector<int> order(S);
+  for (int i = 0; i < S; ++i) order[i] = i;
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) {
+    return (cu_h[a + 1] - cu_h[a]) > (cu_h[b + 1] - cu_h[b]);
+  });
+  int64_t total = 0;
+  for (int i = 0; i < S; ++i) total += static_cast<int64_t>((cu_h[i + 1] - cu_h[i] + QB - 1) / QB) * H;
+  if (total > kMaxSchedItems || grid > kMaxSchedCtas || grid <= 0) return;
+  std::vector<std::vector<int32_t>> lists(grid);
+  std::vector<int64_t> snake_load(grid, 0);
+  using Slot = std::pair<int64_t, int>;  // (load, cta)
+  std::priority_queue<Slot, std::vector<Slot>, std::greater<Slot>> heap;
+  for (int b = 0; b < grid; ++b) heap.push({0, b});
+  int64_t greedy_max = 0;
+  int32_t id = 0;
+  for (int r = 0; r < S; ++r) {
+    const int n = cu_h[order[r] + 1] - cu_h[order[r]];
+    const int nq = (n + QB - 1) / QB;
+    const int64_t nkv = (n + BN - 1) / BN;
+    for (int h = 0; h < H; ++h) {
+      for (int qb = 0; qb < nq; ++qb, ++id) {
+        const int64_t cost = nkv + 1;
+        const int k = id / grid, i = id - k * grid;
+        snake_load[(k & 1) ? grid - 1 - i : i] += cost;
+        Slot sl = heap.top();
+        heap.pop();
+        lists[sl.second].push_back(id);
+        sl.first += cost;
+        greedy_max = std::max(greedy_max, sl.first);
+        heap.push(sl);
+      }
+    }
+  }
+  const int64_t snake_max = *std::max_element(snake_load.begin(), snake_load.end());
+  if (greedy_max * 100 >= snake_max * 99) return;
+  int32_t pos = 0;
+  for (int b = 0; b < grid; ++b) {
+    s->start[b] = pos;
+    for (int32_t v : lists[b]) s->ids[pos++] = v;
+    s->ids[pos++] = kSchedEnd;
+  }
+  s->valid = 1;
+}
+
 }  // namespace
 
 int32_t attention_work_items(const int32_t* cu_h, int32_t S, int32_t H) {
@@ -707,16 +785,17 @@ int32_t attention_work_items(const int32_t* cu_h, int32_t S, int32_t H) {
 }
 
 cudaError_t launch_attention(const mf_bf16* q, const mf_bf16* k, const mf_bf16* v,
-                             const int32_t* cu_seqlens_d, int32_t S, int32_t T, int32_t H,
-                             int32_t D, float softmax_scale, const AttnEpilogue& ep,
-                             int32_t num_items, const KernelCtl& ctl, cudaStream_t st) {
+                             const int32_t* cu_seqlens_d, const int32_t* cu_seqlens_h, int32_t S,
+                             int32_t T, int32_t H, int32_t D, float softmax_scale,
+                             const AttnEpilogue& ep, int32_t num_items, const KernelCtl& ctl,
+                             cudaStream_t st) {
   if (num_items <= 0) return cudaSuccess;
   CUtensorMap mq, mk, mv;
   const int32_t cols = H * D;
   if (!make_tile_map(&mq, q, T, cols) || !make_tile_map(&mk, k, T, cols) ||
       !make_tile_map(&mv, v, T, cols))
     return cudaErrorInvalidValue;
-  AttnArgs a;
+  static thread_local AttnArgs a;  // ~17 KB: kept off the host stack
   a.cu_seqlens = cu_seqlens_d;
   a.S = S;
   a.T = T;
@@ -726,6 +805,7 @@ cudaError_t launch_attention(const mf_bf16* q, const mf_bf16* k, const mf_bf16* 
   a.ctl = ctl;
   const int sms = sm_count_dev();
   const int grid = num_items < sms ? num_items : sms;
+  build_schedule(cu_seqlens_h, S, H, grid, &a.sched);
   const bool gated = ep.y != nullptr;
   if (D == 128) {
     return gated ? launch_t<128, true>(mq, mk, mv, a, grid, st)

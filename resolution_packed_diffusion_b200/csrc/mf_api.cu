@@ -68,9 +68,9 @@ int32_t count_items(const int32_t* cu_h, int32_t S, int32_t H) {
 
 // Runs the attention launcher between the caller's timing events, if any.
 cudaError_t timed_attention(const mf_bf16* q, const mf_bf16* k, const mf_bf16* v,
-                            const int32_t* cu_d, int32_t S, int32_t T, int32_t H, int32_t D,
-                            float scale, const AttnEpilogue& ep, int32_t items,
-                            const KernelCtl& ctl, cudaStream_t st) {
+                            const int32_t* cu_d, const int32_t* cu_h, int32_t S, int32_t T,
+                            int32_t H, int32_t D, float scale, const AttnEpilogue& ep,
+                            int32_t items, const KernelCtl& ctl, cudaStream_t st) {
   cudaEvent_t e0 = nullptr, e1 = nullptr;
   int dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDevices) {
@@ -82,7 +82,7 @@ cudaError_t timed_attention(const mf_bf16* q, const mf_bf16* k, const mf_bf16* v
     cudaError_t e = cudaEventRecord(e0, st);
     if (e != cudaSuccess) return e;
   }
-  cudaError_t e = launch_attention(q, k, v, cu_d, S, T, H, D, scale, ep, items, ctl, st);
+  cudaError_t e = launch_attention(q, k, v, cu_d, cu_h, S, T, H, D, scale, ep, items, ctl, st);
   if (e != cudaSuccess) return e;
   if (e1 != nullptr) e = cudaEventRecord(e1, st);
   return e;
@@ -272,7 +272,7 @@ mf_status mf_varlen_attn_fwd(const mf_bf16* q, const mf_bf16* k, const mf_bf16* 
   AttnEpilogue ep{};
   ep.o = o;
   ep.lse = lse;
-  return cuda_status(timed_attention(qa, ka, v, cu_seqlens_d, S, T, H, D, softmax_scale, ep,
+  return cuda_status(timed_attention(qa, ka, v, cu_seqlens_d, cu_seqlens_h, S, T, H, D, softmax_scale, ep,
                                      count_items(cu_seqlens_h, S, H), ctl, stream));
 }
 
@@ -341,7 +341,7 @@ mf_status mf_block_fwd(const mf_bf16* x, const mf_bf16* q, const mf_bf16* k, con
   ep.mod = mod;
   ep.tok_mod = tok_mod;
   ep.y = y;
-  return cuda_status(timed_attention(wq, wk, v, cu_seqlens_d, S, T, H, D,
+  return cuda_status(timed_attention(wq, wk, v, cu_seqlens_d, cu_seqlens_h, S, T, H, D,
                                      1.0f / std::sqrt(static_cast<float>(D)), ep,
                                      count_items(cu_seqlens_h, S, H), ctl, stream));
 }

@@ -70,9 +70,10 @@ struct AttnEpilogue {
 int32_t attention_work_items(const int32_t* cu_h, int32_t S, int32_t H);
 
 cudaError_t launch_attention(const mf_bf16* q, const mf_bf16* k, const mf_bf16* v,
-                             const int32_t* cu_seqlens_d, int32_t S, int32_t T, int32_t H,
-                             int32_t D, float softmax_scale, const AttnEpilogue& ep,
-                             int32_t num_items, const KernelCtl& ctl, cudaStream_t st);
+                             const int32_t* cu_seqlens_d, const int32_t* cu_seqlens_h, int32_t S,
+                             int32_t T, int32_t H, int32_t D, float softmax_scale,
+                             const AttnEpilogue& ep, int32_t num_items, const KernelCtl& ctl,
+                             cudaStream_t st);
 
 cudaError_t launch_selftest_exp2(const float* x, float* y, int32_t n, cudaStream_t st);
 cudaError_t launch_selftest_wait(uint64_t limit_ns, const KernelCtl& ctl, cudaStream_t st);

@@ -179,6 +179,64 @@ def test_edge_packs_full_compare(k):
     assert np.abs(lse.cpu().numpy() - ref_lse).max() <= 2e-2
 
 
+def _expect_host_table(lengths, H, sms, cap=4096):
+    """Which work order the attention launch should pick for these sample
+    lengths: the host's greedy per-CTA table (True) or the in-kernel snake
+    order (False). Restates the launch rule: items of ceil(n/256) query blocks
+    per head at nkv + 1 periods each, longest sample first; the table is used
+    when it fits and its greedy makespan beats the snake deal's by over 1%."""
+    import heapq
+    order = sorted(range(len(lengths)), key=lambda s: -lengths[s])
+    costs = []
+    for s in order:
+        n = lengths[s]
+        costs += [(n + 127) // 128 + 1] * (((n + 255) // 256) * H)
+    G = min(sms, len(costs))
+    if len(costs) > cap or G <= 0:
+        return False
+    snake = [0] * G
+    for i, c in enumerate(costs):
+        k, b = divmod(i, G)
+        snake[G - 1 - b if k & 1 else b] += c
+    heap = [(0, b) for b in range(G)]
+    greedy = 0
+    for c in costs:
+        load, b = heapq.heappop(heap)
+        greedy = max(greedy, load + c)
+        heapq.heappush(heap, (load + c, b))
+    return greedy * 100 < max(snake) * 99
+
+
+SCHEDULE_PACKS = [
+    # (descs, H, D, expected work order)
+    ([SampleDesc(1, 64, 64, 0), SampleDesc(1, 40, 40, 100), SampleDesc(1, 24, 24, 10),
+      SampleDesc(1, 10, 10, 5), SampleDesc(0, 0, 0, 77)], 8, 128, "table"),
+    ([SampleDesc(1, 32, 32, 0)] * 4, 16, 128, "snake"),                 # equal items: a tie
+    ([SampleDesc(1, 16, 16, 0)] * 300, 16, 64, "snake"),               # 4800 items: over the table
+]
+
+
+@pytest.mark.parametrize("k", range(len(SCHEDULE_PACKS)), ids=[p[3] + str(i) for i, p in
+                                                             enumerate(SCHEDULE_PACKS)])
+def test_attention_under_each_work_order(k):
+    """Both work orders (host greedy table, in-kernel snake deal, and the snake
+    fallback when the table cannot hold the items) cover every item once."""
+    descs, H, D, kind = SCHEDULE_PACKS[k]
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    lengths = [d.frames * d.grid_h * d.grid_w + d.n_text for d in descs]
+    assert _expect_host_table(lengths, H, sms) == (kind == "table")
+    w = make_random_pack(700 + k, S=len(descs), H=H, D=D, rope_axes=2, descs=descs)
+    dp = DevicePack(w)
+    pack = oracle_pack(w)
+    o, lse = dp.attention(dp.q, dp.k, dp.v, with_rope=False, lse=True)
+    assert mf.mf_get_error() == mf.MF_OK
+    rows = sample_rows(pack["cu_seqlens"], 8, 700 + k)
+    ref_o, ref_lse = oracle.varlen_attention(w.f32("q"), w.f32("k"), w.f32("v"),
+                                             pack["cu_seqlens"], rows=rows)
+    assert_bf16_close(host_f32(o)[rows], ref_o, "attention O")
+    assert np.abs(lse.cpu().numpy()[:, rows].astype(np.float64) - ref_lse).max() <= 2e-2
+
+
 def test_empty_pack_is_a_no_op():
     w = make_random_pack(600, S=2, H=2, D=64, rope_axes=2,
                          descs=[SampleDesc(0, 0, 0, 0), SampleDesc(1, 0, 5, 0)])
