@@ -26,10 +26,12 @@
 //               registers to the softmax warpgroups with setmaxnreg).
 //   warps 4..7  softmax + epilogue of tile A, one thread per query row (TMEM
 //   warps 8..11 lane); the same for tile B. Online softmax in the exp2 domain:
-//               exponentials are taken against the running reference max while
-//               the tile max is tracked alongside; only when the max grows by
-//               more than 2^8 is O rescaled in TMEM and the tile redone (exact
-//               after the final 1/l). P is packed to bf16 into the first 64
+//               the reference max is the first key tile's row max, and
+//               exponentials of later tiles are taken against it as long as the
+//               tile's row sum stays below 2^32 (which bounds every P); only
+//               then is the reference moved to the tile max, O rescaled in TMEM
+//               and the tile redone (exact after the final 1/l: a stale
+//               reference scales numerator and denominator alike). P is packed to bf16 into the first 64
 //               columns of the tile's S region.
 // TMEM (512 columns): S_A/P_A | S_B/P_B | O_A | O_B.
 // Work items are ordered longest sample first and, inside a sample, the query
@@ -85,6 +87,8 @@ constexpr int NV = 2;                 // V tile ring stages
 // share. Measured on B200 (edit pack, attention alone, two runs each):
 // 0 -> 1032, 1 -> 1053, 2 -> 1145 / 1084, 3 -> 1066 / 1002 useful TFLOP/s.
 constexpr int kPolyPairsOf8 = 2;
+// Redo bound on a tile's row sum (see the softmax loop).
+constexpr float kRedoSum = 4294967296.f;  // 2^32
 
 
 template <int D>
@@ -468,12 +472,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         };
         // P = 2^(s * scale * log2 e - m_ref) for the row's 128 keys, packed to 64
-        // bf16 pairs; the row sum goes to four packed fp32 accumulators and the
-        // largest P (as bf16 pairs) to four max accumulators. Per key pair: one
-        // packed FMA, two ex2, one bf16 pack, one packed add, one bf16x2 max.
+        // bf16 pairs; the row sum goes to four packed fp32 accumulators. Per key
+        // pair: one packed FMA, two ex2, one bf16 pack, one packed add.
         const uint64_t scale2 = f2_pack(scale_log2, scale_log2);
-        auto exponentiate = [&](const uint32_t (&sr)[BN], uint32_t (&pp)[BN / 2], uint64_t (&ls)[4],
-                                uint32_t (&pmax)[4]) {
+        auto exponentiate = [&](const uint32_t (&sr)[BN], uint32_t (&pp)[BN / 2], uint64_t (&ls)[4]) {
           const uint64_t neg_m2 = f2_pack(-m_ref, -m_ref);
 #pragma unroll
           for (int e = 0; e < BN / 2; ++e) {
@@ -490,47 +492,51 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             pp[e] = pack_bf16x2(p0, p1);
             ls[e & 3] = f2_add(ls[e & 3], f2_pack(p0, p1));
-            pmax[e & 3] = bf16x2_max(pmax[e & 3], pp[e]);
           }
+        };
+        // row max of a tile's scores (scaled to log2 units)
+        auto tile_max = [&](const uint32_t (&sr)[BN]) -> float {
+          float m4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) m4[e] = __uint_as_float(sr[e]);
+#pragma unroll
+          for (int cidx = 4; cidx < BN - 4; cidx += 8)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              m4[e] = max3f(m4[e], __uint_as_float(sr[cidx + e]), __uint_as_float(sr[cidx + 4 + e]));
+#pragma unroll
+          for (int e = 0; e < 4; ++e) m4[e] = fmaxf(m4[e], __uint_as_float(sr[BN - 4 + e]));
+          return fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * scale_log2;
+        };
+        auto row_sum = [](const uint64_t (&ls)[4]) -> float {
+          float a0, a1, b0, b1, c0, c1, d0, d1;
+          f2_unpack(ls[0], a0, a1);
+          f2_unpack(ls[1], b0, b1);
+          f2_unpack(ls[2], c0, c1);
+          f2_unpack(ls[3], d0, d1);
+          return ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
         };
         uint32_t pp[BN / 2];
         uint64_t ls[4] = {0, 0, 0, 0};  // packed (0.f, 0.f)
-        uint32_t pmax[4] = {0, 0, 0, 0};
         {
           uint32_t sr[BN];
           load_scores(sr);
-          if (j == 0) {
-            // first tile of the item: the reference is the tile max
-            float mx8[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(sr[e]);
-#pragma unroll
-            for (int cidx = 8; cidx < BN; cidx += 8)
-#pragma unroll
-              for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(mx8[e], __uint_as_float(sr[cidx + e]));
-            m_ref = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                          fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * scale_log2;
-          }
-          exponentiate(sr, pp, ls, pmax);
+          if (j == 0) m_ref = tile_max(sr);  // first tile of the item: the reference is its max
+          exponentiate(sr, pp, ls);
         }
-        // Largest P of the tile above 2^8 (bf16 256 = 0x4380; P >= 0, so bit
-        // patterns order like values; inf and NaN also land above): the max grew
-        // by more than 2^8. Move the reference to the tile max, bring O and l
-        // along (PV_X(j-1) is complete: S_X(j) was issued after it) and redo the
-        // tile from the scores, still in TMEM.
-        const uint32_t pm = bf16x2_max(bf16x2_max(pmax[0], pmax[1]), bf16x2_max(pmax[2], pmax[3]));
-        if ((pm & 0xFFFFu) > 0x4380u || (pm >> 16) > 0x4380u) {
+        // A tile row sum above 2^32 (or inf / NaN) means some P may be out of
+        // range: the max grew by more than 2^25 over the reference. Move the
+        // reference to the tile max, bring O and l along (PV_X(j-1) is complete:
+        // S_X(j) was issued after it) and redo the tile from the scores, still in
+        // TMEM. Below the bound every P <= 2^32 and O, l stay far from overflow.
+        // The TMEM loads and stores below are warp-collective (.sync.aligned), so
+        // the whole warp takes the branch when any row needs it; for the other
+        // rows moving the reference up to their own tile max is just as exact.
+        float tile_sum = row_sum(ls);
+        if (__any_sync(0xffffffffu, !(tile_sum <= kRedoSum))) {
           uint32_t sr2[BN];
           load_scores(sr2);
-          float mx8[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(sr2[e]);
-#pragma unroll
-          for (int cidx = 8; cidx < BN; cidx += 8)
-#pragma unroll
-            for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(mx8[e], __uint_as_float(sr2[cidx + e]));
-          const float m_new = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                    fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * scale_log2;
+          const float m_new = fmaxf(m_ref, tile_max(sr2));
           const float factor = ex2_approx(m_ref - m_new);
           l *= factor;
 #pragma unroll 1
@@ -545,20 +551,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tmem_st_wait();
           m_ref = m_new;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            ls[e] = 0;
-            pmax[e] = 0;
-          }
-          exponentiate(sr2, pp, ls, pmax);
+          for (int e = 0; e < 4; ++e) ls[e] = 0;
+          exponentiate(sr2, pp, ls);
+          tile_sum = row_sum(ls);
         }
-        {
-          float a0, a1, b0, b1, c0, c1, d0, d1;
-          f2_unpack(ls[0], a0, a1);
-          f2_unpack(ls[1], b0, b1);
-          f2_unpack(ls[2], c0, c1);
-          f2_unpack(ls[3], d0, d1);
-          l += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
-        }
+        l += tile_sum;
         tmem_st32(s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(&pp[0]));
         tmem_st32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&pp[32]));
         tmem_st_wait();

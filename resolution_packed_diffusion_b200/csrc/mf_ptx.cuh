@@ -220,6 +220,13 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// Three-input maximum (sm_100): one instruction for two elements of a running max.
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // Per-warpgroup register budget (all 128 threads of the warpgroup execute it).
 template <int N>
 __device__ __forceinline__ void regs_dec() {
@@ -257,18 +264,19 @@ __device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
   return r;
 }
 
-// 2^x for a pair of inputs on the FMA pipe (f32x2 instructions), x <= 127; used
+// 2^x for a pair of inputs on the FMA pipe (f32x2 instructions); used
 // for part of the softmax exponentials so that they do not all queue on the
 // MUFU unit. Range reduction x = j + f with j = round(x): t = x + 1.5 * 2^23
 // rounds to the nearest integer, -j = 1.5 * 2^23 - t and f = x - j are exact.
 // 2^f from a degree-3 minimax polynomial on [-1/2, 1/2] (coefficients from
 // fit_exp2_poly.py, Remez exchange; maximum relative error 7.5e-5). 2^j is added
 // to the exponent field: t's bits are 0x4B400000 + j and 0x4B400000 << 23
-// vanishes modulo 2^32, so (bits(t) << 23) is j << 23. Inputs below -125 are
-// clamped there (the result, about 2e-38, stands for zero).
+// vanishes modulo 2^32, so (bits(t) << 23) is j << 23. Inputs are clamped to
+// [-125, 127]: below, the result (about 2e-38) stands for zero; above, it stays
+// finite and at least 2^127, so an overflowing input is still seen as huge.
 __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& p0, float& p1) {
   const uint64_t round2 = f2_pack(12582912.0f, 12582912.0f);
-  const uint64_t x2 = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+  const uint64_t x2 = f2_pack(fmaxf(fminf(x0, 127.0f), -125.0f), fmaxf(fminf(x1, 127.0f), -125.0f));
   const uint64_t t2 = f2_add(x2, round2);
   uint64_t nj2;  // -j = 1.5 * 2^23 - t
   asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(nj2) : "l"(round2), "l"(t2));

@@ -237,6 +237,40 @@ def test_attention_under_each_work_order(k):
     assert np.abs(lse.cpu().numpy()[:, rows].astype(np.float64) - ref_lse).max() <= 2e-2
 
 
+@pytest.mark.parametrize("step,shift", [(29.0, 0), (29.0, 64), (3.0, 0)],
+                         ids=["jumps_at_tiles", "jumps_mid_tile", "creeps"])
+def test_attention_when_the_row_max_keeps_growing(step, shift):
+    """Scores that climb in steps of 128 keys (starting `shift` keys into a
+    128-key tile): by about `step` log2 units per step for some rows (29 forces
+    the kernel to move its reference max: at a tile's first half with shift 0,
+    at its second half with shift 64; 3 keeps the stale reference, with P up to
+    2^12), fall for others, barely move for the rest. The online softmax must
+    still match the exact one."""
+    from packgen import f32_to_bf16_bits
+    descs = [SampleDesc(1, 24, 25, 0), SampleDesc(1, 7, 9, 3)]  # 600 and 66 tokens
+    H, D = 2, 64
+    w = make_random_pack(800, S=len(descs), H=H, D=D, rope_axes=2, descs=descs)
+    rng = np.random.default_rng(801)
+    T = w.T
+    u = np.full(D, 1.0 / 8.0)  # |u|^2 = 1
+    # x = s * log2(e) / sqrt(D) = a * b * 0.18: b rises by step / (a * 0.18) per tile
+    a = rng.choice([4.0, -4.0, 0.5], size=(T, H))
+    tile = (np.arange(T) % 600 + shift) // 128
+    b = 1.0 + tile * step / (4.0 * 0.125 * 1.4426950408889634)
+    q = a[:, :, None] * u + 0.05 * rng.standard_normal((T, H, D))
+    k = b[:, None, None] * u + 0.05 * rng.standard_normal((T, H, D))
+    w.q_bits = f32_to_bf16_bits(q.astype(np.float32))
+    w.k_bits = f32_to_bf16_bits(k.astype(np.float32))
+    dp = DevicePack(w)
+    pack = oracle_pack(w)
+    o, lse = dp.attention(dp.q, dp.k, dp.v, with_rope=False, lse=True)
+    assert mf.mf_get_error() == mf.MF_OK
+    ref_o, ref_lse = oracle.varlen_attention(w.f32("q"), w.f32("k"), w.f32("v"), pack["cu_seqlens"])
+    assert_bf16_close(host_f32(o), ref_o, "attention O")
+    # the LSE carries the exact max, up to ~120 in these rows: relative bound
+    assert np.all(np.abs(lse.cpu().numpy() - ref_lse) <= 2e-2 * np.maximum(1.0, np.abs(ref_lse) / 8))
+
+
 def test_empty_pack_is_a_no_op():
     w = make_random_pack(600, S=2, H=2, D=64, rope_axes=2,
                          descs=[SampleDesc(0, 0, 0, 0), SampleDesc(1, 0, 5, 0)])
