@@ -43,7 +43,9 @@ UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 REF_ROW_STRIDE = 32  # reference arm: rows sampled per step (keeps a step near 0.3 s)
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_fwd_traffic.txt")
-ATTN_SRC = os.path.join(ROOT, "resolution_packed_diffusion_b200", "csrc", "attn_fwd.cu")
+# the attention kernel's sources: the traffic summary applies while they are unchanged
+ATTN_SRC = [os.path.join(ROOT, "resolution_packed_diffusion_b200", "csrc", f)
+            for f in ("attn_fwd.cu", "mf_ptx.cuh", "mf_internal.h")]
 
 
 # ----------------------------------------------------------------- helpers
@@ -99,7 +101,10 @@ def attn_traffic_bytes(T_full: int):
         if "=" in line and not line.startswith("#"):
             k, v = line.strip().split("=", 1)
             fields[k.strip()] = v.strip()
-    sha = hashlib.sha256(open(ATTN_SRC, "rb").read()).hexdigest()[:16]
+    h = hashlib.sha256()
+    for f in ATTN_SRC:
+        h.update(open(f, "rb").read())
+    sha = h.hexdigest()[:16]
     if fields.get("kernel_sha") != sha or "workload" not in fields:
         return None
     if fields.get("workload") != str(T_full):
