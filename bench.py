@@ -293,11 +293,11 @@ def run_gpu(args, rank, world, local_rank):
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step():
+    def step(bx=x, bq=q, bk=k, bv=v, bc=c, bW=Wm, bxm=x_mod, by=y):
         cu_h, _ = mf.mf_pack_build(w.descs, w.rope_axes, w.budget, cu_d, pos, ts, tm, stream)
-        mf.mf_adaln_params(c, Wm, S, c.shape[1], hid, mod, stream)
-        mf.mf_block_fwd(x, q, k, v, mod, cu_d, cu_h, pos, ts, tm, S, H, D, w.rope_axes, w.base,
-                        w.eps, x_mod, y, ws, ws_bytes, stream)
+        mf.mf_adaln_params(bc, bW, S, bc.shape[1], hid, mod, stream)
+        mf.mf_block_fwd(bx, bq, bk, bv, mod, cu_d, cu_h, pos, ts, tm, S, H, D, w.rope_axes, w.base,
+                        w.eps, bxm, by, ws, ws_bytes, stream)
 
     launches_per_step = 5  # pack ids, adaLN params, adaLN modulate, RoPE, attention
 
@@ -340,41 +340,73 @@ def run_gpu(args, rank, world, local_rank):
     tokens_all = reduce_timing(0.0, float(real_tokens(w)), world)[1]
     value = flops_all / (ms_step * 1e-3) / 1e12
 
-    # ---- end to end through the public API with host buffers
+    # ---- end to end through the public API with host buffers. Every step copies
+    # its inputs from pinned host memory and its outputs (y and x_mod) back. Two
+    # device buffer sets and three streams (host-to-device copies, compute,
+    # device-to-host copies) let step i's outputs travel back while step i+1's
+    # inputs come in: PCIe carries both directions at once.
     pin = {n: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).pin_memory()
            for n, a in (("x", w.x_bits), ("q", w.q_bits), ("k", w.k_bits), ("v", w.v_bits))}
     c_h = torch.from_numpy(w.c).pin_memory()
     W_h = torch.from_numpy(w.W).pin_memory()
-    y_h = torch.empty((T, hid), dtype=torch.int16).pin_memory()
-    xm_h = torch.empty((T, hid), dtype=torch.int16).pin_memory()
-    dst = {"x": x, "q": q, "k": k, "v": v}
+    sets = [dict(x=x, q=q, k=k, v=v, c=c, W=Wm, x_mod=x_mod, y=y)]
+    sets.append({n: torch.empty_like(t) for n, t in sets[0].items()})
+    out_h = [{n: torch.empty((T, hid), dtype=torch.int16).pin_memory() for n in ("y", "x_mod")}
+             for _ in range(2)]
+    s_in = torch.cuda.Stream(dev)
+    s_out = torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]    # inputs of set b landed
+    ev_done = [torch.cuda.Event() for _ in range(2)]  # step on set b finished
+    ev_out = [torch.cuda.Event() for _ in range(2)]   # outputs of set b copied back
+    for b in range(2):
+        for e in (ev_done[b], ev_out[b]):
+            e.record(stream)
 
-    def e2e_step():
-        for n, t in pin.items():
-            dst[n].view(torch.int16).copy_(t, non_blocking=True)
-        c.copy_(c_h, non_blocking=True)
-        Wm.copy_(W_h, non_blocking=True)
-        step()
-        y_h.copy_(y.view(torch.int16), non_blocking=True)
-        xm_h.copy_(x_mod.view(torch.int16), non_blocking=True)
+    def e2e_step(i):
+        b = i & 1
+        bs = sets[b]
+        s_in.wait_event(ev_done[b])  # the step that last read set b is finished
+        with torch.cuda.stream(s_in):
+            for n, t in pin.items():
+                bs[n].view(torch.int16).copy_(t, non_blocking=True)
+            bs["c"].copy_(c_h, non_blocking=True)
+            bs["W"].copy_(W_h, non_blocking=True)
+        ev_in[b].record(s_in)
+        stream.wait_event(ev_in[b])
+        stream.wait_event(ev_out[b])  # set b's previous outputs are back on the host
+        step(bs["x"], bs["q"], bs["k"], bs["v"], bs["c"], bs["W"], bs["x_mod"], bs["y"])
+        ev_done[b].record(stream)
+        s_out.wait_event(ev_done[b])
+        with torch.cuda.stream(s_out):
+            for n in ("y", "x_mod"):
+                out_h[b][n].copy_(bs[n].view(torch.int16), non_blocking=True)
+        ev_out[b].record(s_out)
 
     e2e_steps = max(3, min(args.steps, 20))
-    for _ in range(2):
-        e2e_step()
+    for i in range(2):
+        e2e_step(i)
+    torch.cuda.synchronize(dev)
     barrier()
     torch.cuda.synchronize(dev)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
+    s_in.wait_event(e0)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    stream.wait_stream(s_out)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
     e2e_ms, _ = reduce_timing(e0.elapsed_time(e1) / e2e_steps, 0.0, world)
     h2d = sum(t.numel() * t.element_size() for t in pin.values()) + \
         c_h.numel() * 4 + W_h.numel() * 4
-    d2h = (y_h.numel() + xm_h.numel()) * 2
+    d2h = sum(t.numel() * t.element_size() for t in out_h[0].values())
+    if mf.mf_get_error(stream) != mf.MF_OK:
+        raise RuntimeError("device error during the end-to-end steps")
+    if not all(np.array_equal(out_h[b][n].numpy(), out_h[0][n].numpy())
+               for b in range(2) for n in ("y", "x_mod")):
+        raise RuntimeError("end-to-end outputs differ between the two buffer sets")
 
     if rank != 0:
         return
