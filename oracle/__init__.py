@@ -45,6 +45,7 @@ from .mf_oracle import (  # noqa: F401
     adaln_modulate,
     adaln_params,
     block_fwd,
+    cfg_combine,
     gated_residual,
     layer_norm_rows,
     pack_build,

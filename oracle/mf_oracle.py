@@ -256,6 +256,46 @@ def block_fwd(x, q, k, v, mod, pack, rope_axes: int, base: float = 10000.0,
     return x_mod, y, o
 
 
+# ---------------------------------------------------------------------------
+# Packed classifier-free guidance  ([cfg])
+# ---------------------------------------------------------------------------
+def cfg_combine(v, descs: Sequence, pairs: Sequence, w: float) -> np.ndarray:
+    """Classifier-free guidance over a packed-CFG pack.
+
+    [cfg]: the conditional and the unconditional branch of an image run as two
+    samples of one pack, in a single forward. The pages do not give the
+    combine; the reading taken is the usual classifier-free guidance form,
+    applied to the image tokens of each (conditional, unconditional) pair:
+    ``out = v_u + w * (v_c - v_u)``, where row i of a pair's output takes row i
+    of each sample's image tokens (a sample's image tokens come first, see
+    ``pack_build``). Both samples of a pair must have the same number of image
+    tokens; their text tokens (prompt vs. empty prompt) are not part of it.
+
+    v: [T][C] per-token outputs of the pack; pairs: (cond, uncond) sample
+    indices. Returns float64 [sum of the pairs' image-token counts][C], pairs in
+    the order given.
+    """
+    v = np.asarray(v, dtype=np.float64)
+    rows = [tuple(d.as_tuple()) if hasattr(d, "as_tuple") else tuple(d) for d in descs]
+    n_tok = [F * Hg * Wg + L for (F, Hg, Wg, L, *_r) in rows]
+    n_img = [F * Hg * Wg for (F, Hg, Wg, _L, *_r) in rows]
+    cu = np.concatenate([[0], np.cumsum(n_tok)]).astype(np.int64)
+    if v.shape[0] != cu[-1]:
+        raise ValueError("v has the wrong number of rows for the pack")
+    out = []
+    for (c, u) in pairs:
+        if not (0 <= c < len(rows) and 0 <= u < len(rows)) or c == u:
+            raise ValueError("bad pair")
+        if n_img[c] != n_img[u]:
+            raise ValueError("the two branches of a pair need the same image grid")
+        n = n_img[c]
+        v_c = v[cu[c]:cu[c] + n]
+        v_u = v[cu[u]:cu[u] + n]
+        out.append(v_u + w * (v_c - v_u))
+    C = v.shape[1] if v.ndim == 2 else 0
+    return np.concatenate(out, axis=0) if out else np.zeros((0, C))
+
+
 def useful_attention_flops(descs: Sequence, H: int, D: int) -> float:
     """Useful attention FLOPs of a pack: ``4 * D * H * sum n_s^2`` over the real
     samples (QK^T and PV, 2 FLOPs per multiply-add, only within-sample pairs,

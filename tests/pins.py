@@ -348,3 +348,63 @@ def check_gate(gated_residual, adaln_params, pack_build):
         s, m = int(p["tok_sample"][t]), int(p["tok_mod"][t])
         ref = brute.brute_gate_row(x[t].tolist(), o[t].reshape(-1).tolist(), mod[s, m, 2].tolist())
         assert np.allclose(y[t], ref, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# Packed CFG combine  ([cfg])
+# ---------------------------------------------------------------------------
+_CFG_DESCS = [(1, 3, 4, 5), (0, 0, 0, 7), (1, 3, 4, 2), (1, 2, 2, 1), (1, 2, 2, 6)]
+_CFG_PAIRS = [(0, 2), (4, 3)]  # (cond, uncond): 12 and 4 image tokens
+
+
+def check_cfg_special_weights(cfg_combine):
+    """w = 0 returns the unconditional branch, w = 1 the conditional one, and
+    equal branches are left alone at any w (guidance has nothing to act on)."""
+    rng = np.random.default_rng(50)
+    T = sum(F * H * W + L for (F, H, W, L) in _CFG_DESCS)
+    # dyadic values, as bf16 inputs are: u + (c - u) is then exactly c in float64
+    v = rng.integers(-512, 512, size=(T, 8)) / 64.0
+    cu = np.concatenate([[0], np.cumsum([F * H * W + L for (F, H, W, L) in _CFG_DESCS])])
+    want_u = np.concatenate([v[cu[3]:cu[3] + 4] if u == 3 else v[cu[2]:cu[2] + 12]
+                             for (_c, u) in _CFG_PAIRS])
+    want_c = np.concatenate([v[cu[0]:cu[0] + 12], v[cu[4]:cu[4] + 4]])
+    assert np.array_equal(cfg_combine(v, _CFG_DESCS, _CFG_PAIRS, 0.0), want_u)
+    assert np.array_equal(cfg_combine(v, _CFG_DESCS, _CFG_PAIRS, 1.0), want_c)
+    v2 = v.copy()
+    v2[cu[2]:cu[2] + 12] = v2[cu[0]:cu[0] + 12]
+    v2[cu[3]:cu[3] + 4] = v2[cu[4]:cu[4] + 4]
+    for w in (0.0, 3.5, -2.0):
+        assert np.array_equal(cfg_combine(v2, _CFG_DESCS, _CFG_PAIRS, w), want_c)
+
+
+def check_cfg_row_map(cfg_combine):
+    """Which rows are combined: with v[t] = t in every channel, row i of pair
+    (c, u) is cu[u] + i + w * (cu[c] - cu[u]) (closed form of the row map:
+    image tokens first, same index i in both samples), and text rows never
+    enter."""
+    T = sum(F * H * W + L for (F, H, W, L) in _CFG_DESCS)
+    v = np.repeat(np.arange(T, dtype=np.float64)[:, None], 3, axis=1)
+    cu = [0, 17, 24, 38, 43, 53]
+    w = 4.25
+    got = cfg_combine(v, _CFG_DESCS, _CFG_PAIRS, w)
+    want = [cu[2] + i + w * (cu[0] - cu[2]) for i in range(12)] + \
+           [cu[3] + i + w * (cu[4] - cu[3]) for i in range(4)]
+    assert got.shape == (16, 3)
+    assert np.allclose(got, np.repeat(np.array(want)[:, None], 3, axis=1), rtol=0, atol=1e-12)
+
+
+def check_cfg_pack_order(cfg_combine):
+    """Reordering the samples of the pack (and renumbering the pairs) leaves the
+    guided output unchanged."""
+    rng = np.random.default_rng(51)
+    n = [F * H * W + L for (F, H, W, L) in _CFG_DESCS]
+    cu = np.concatenate([[0], np.cumsum(n)])
+    v = rng.standard_normal((cu[-1], 5))
+    perm = [3, 0, 4, 2, 1]  # new position -> old sample
+    descs2 = [_CFG_DESCS[o] for o in perm]
+    v2 = np.concatenate([v[cu[o]:cu[o + 1]] for o in perm])
+    where = {o: i for i, o in enumerate(perm)}
+    pairs2 = [(where[c], where[u]) for (c, u) in _CFG_PAIRS]
+    a = cfg_combine(v, _CFG_DESCS, _CFG_PAIRS, 2.5)
+    b = cfg_combine(v2, descs2, pairs2, 2.5)
+    assert np.array_equal(a, b)

@@ -92,6 +92,24 @@ def _gate_uses_scale(x, o, mod, tok_sample, tok_mod, rows=None):
     return mo.gated_residual(x, o, m, tok_sample, tok_mod, rows)
 
 
+def _cfg_branches_swapped(v, descs, pairs, w):
+    return mo.cfg_combine(v, descs, [(u, c) for (c, u) in pairs], w)
+
+
+def _cfg_text_rows(v, descs, pairs, w):
+    # takes the pair's rows from the end of each sample (its text tokens) instead
+    rows = [tuple(d) for d in descs]
+    n = [F * H * W + L for (F, H, W, L, *_r) in rows]
+    cu = np.concatenate([[0], np.cumsum(n)])
+    out = []
+    for (c, u) in pairs:
+        k = rows[c][0] * rows[c][1] * rows[c][2]
+        vc = np.asarray(v, dtype=np.float64)[cu[c + 1] - k:cu[c + 1]]
+        vu = np.asarray(v, dtype=np.float64)[cu[u + 1] - k:cu[u + 1]]
+        out.append(vu + w * (vc - vu))
+    return np.concatenate(out)
+
+
 MUTANTS = [
     ("rope sign flip", lambda: pins.check_rope_relative(_rope_sign_flip) or
      pins.check_rope_textbook_1d(_rope_sign_flip)),
@@ -106,6 +124,8 @@ MUTANTS = [
     ("column-major grid", lambda: pins.check_pack_tiny_closed_form(_pack_col_major)),
     ("gate reads scale", lambda: pins.check_gate(_gate_uses_scale, oracle.adaln_params,
                                                  oracle.pack_build)),
+    ("CFG branches swapped", lambda: pins.check_cfg_special_weights(_cfg_branches_swapped)),
+    ("CFG rows from the text end", lambda: pins.check_cfg_row_map(_cfg_text_rows)),
 ]
 
 

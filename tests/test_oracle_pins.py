@@ -149,3 +149,21 @@ def test_useful_flops_closed_form():
     assert w2.descs[-1].is_dummy == 1
     real = sum((d.frames * d.grid_h * d.grid_w + d.n_text) ** 2 for d in w2.descs[:-1])
     assert oracle.useful_attention_flops(w2.descs, 24, 128) == 4 * 128 * 24 * real
+
+
+def test_cfg_special_weights():
+    pins.check_cfg_special_weights(oracle.cfg_combine)
+
+
+def test_cfg_row_map():
+    pins.check_cfg_row_map(oracle.cfg_combine)
+
+
+def test_cfg_pack_order():
+    pins.check_cfg_pack_order(oracle.cfg_combine)
+
+
+def test_cfg_rejects_mismatched_grids():
+    import pytest as _pt
+    with _pt.raises(ValueError):
+        oracle.cfg_combine(np.zeros((17 + 7 + 14 + 5 + 10, 2)), pins._CFG_DESCS, [(0, 3)], 1.0)
