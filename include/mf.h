@@ -22,6 +22,8 @@
  *          normalization and joint self-attention.
  *   [fuse] picx.dev summary, Methodology > Training Infrastructure: fused
  *          adaptive normalization / RoPE / gating in NR-MMDiT.
+ *   [cfg]  picx.dev summary, Methodology > NR-MMDiT, "Packed CFG inference":
+ *          the conditional and unconditional branches packed into one forward.
  * Where the pages are silent the library follows one stated reading: RoPE
  * splits head_dim evenly across the axes in whole adjacent-channel pairs, base
  * 10000 by default, leftover channels unrotated; text token j of a sample sits
@@ -185,6 +187,24 @@ mf_status mf_block_fwd_noalloc(const mf_bf16* x, const mf_bf16* q, const mf_bf16
                                const int32_t* tok_sample, const uint8_t* tok_mod, int32_t S,
                                int32_t H, int32_t D, int32_t rope_axes, float base, float eps,
                                mf_bf16* x_mod, mf_bf16* y, cudaStream_t stream);
+
+/* Packed classifier-free guidance [cfg]: the two branches of an image are two
+ * samples of one pack. For each pair (cond, uncond) of sample indices whose
+ * samples hold the same number n of image tokens (frames * grid_h * grid_w),
+ * output rows [o, o + n) = v_u + w * (v_c - v_u), row i taken from image token
+ * i of each sample (a sample's image tokens come first), o = the sum of the
+ * earlier pairs' n. The pages name packed CFG but not its combine; this is the
+ * usual guidance form. desc: host, S samples (they fix T and the offsets);
+ * pairs: host, P >= 1 pairs of distinct samples, P <= MF_MAX_SAMPLES / 2.
+ * v: [T][C] bf16; out: [sum n][C] bf16, must not overlap v; C % 8 == 0; w finite.
+ * fp32 arithmetic (fma(w, c - u, u)), bf16 round-to-nearest-even output. */
+typedef struct {
+  int32_t cond;
+  int32_t uncond;
+} mf_cfg_pair;
+mf_status mf_cfg_combine(const mf_bf16* v, const mf_sample_desc* desc, int32_t S,
+                         const mf_cfg_pair* pairs, int32_t P, int32_t C, float w, mf_bf16* out,
+                         cudaStream_t stream);
 
 /* Bytes of workspace mf_varlen_attn_fwd / mf_block_fwd need (with_rope != 0:
  * room for the rotated Q and K). */

@@ -82,6 +82,8 @@ class Workload:
     v_bits: Optional[np.ndarray] = None
     c: Optional[np.ndarray] = None  # [S][COND_DIM] float32
     W: Optional[np.ndarray] = None  # [COND_DIM][6*hid] float32
+    # packed-CFG packs: (conditional, unconditional) sample index pairs
+    cfg_pairs: List[tuple] = dataclasses.field(default_factory=list)
 
     @property
     def hid(self) -> int:
@@ -112,7 +114,8 @@ CONFIGS = {
             pad_to_budget=True),
     3: dict(name="packed CFG at 1024x1024, 8464 tokens, 24 heads x 128",
             H=24, D=128, rope_axes=2, budget=0,
-            samples=[(1, 64, 64, 256), (1, 64, 64, 16)]),
+            samples=[(1, 64, 64, 256), (1, 64, 64, 16)],
+            cfg_pairs=[(0, 1)]),  # (conditional, unconditional) branch samples
     4: dict(name="edit pack, source+target 64x64, 3D RoPE, 16896 tokens, 24 heads x 128",
             H=24, D=128, rope_axes=3, budget=0,
             samples=[(2, 64, 64, 256), (2, 64, 64, 256)]),
@@ -156,7 +159,8 @@ def make_workload(index: int, with_arrays: bool = True, seed: Optional[int] = No
         if fill > 0:
             descs.append(SampleDesc(0, 0, 0, fill, 1))
     w = Workload(index=index, name=spec["name"], descs=descs, H=spec["H"], D=spec["D"],
-                 rope_axes=spec["rope_axes"], budget=spec["budget"], seed=seed)
+                 rope_axes=spec["rope_axes"], budget=spec["budget"], seed=seed,
+                 cfg_pairs=list(spec.get("cfg_pairs", [])))
     if with_arrays:
         fill_arrays(w, rng)
     return w

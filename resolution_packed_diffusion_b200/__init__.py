@@ -74,6 +74,7 @@ _SIGS = {
     "mf_set_attn_timing_events": (_I, [_P, _P]),
     "mf_block_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F,
                                   _F, _P, _P, _P]),
+    "mf_cfg_combine": (_I, [_P, _P, _I, _P, _I, _I, _F, _P, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -234,3 +235,20 @@ def mf_block_fwd_noalloc(x, q, k, v, mod, cu_seqlens_d, cu_seqlens_h: np.ndarray
                                     _ptr(tok_sample), _ptr(tok_mod), S, H, D, rope_axes, base,
                                     eps, _ptr(x_mod), _ptr(y), _stream(stream)),
            "mf_block_fwd_noalloc")
+
+
+class mf_cfg_pair(ctypes.Structure):
+    _fields_ = [("cond", ctypes.c_int32), ("uncond", ctypes.c_int32)]
+
+
+def mf_cfg_combine(v, descs, pairs, C: int, w: float, out, stream=None) -> None:
+    """Packed classifier-free guidance: ``pairs`` are (cond, uncond) sample
+    indices; ``out`` gets v_u + w (v_c - v_u) over each pair's image tokens."""
+    arr = make_descs(descs)
+    S = len(list(descs))
+    pl = list(pairs)
+    parr = (mf_cfg_pair * max(1, len(pl)))()
+    for i, (c, u) in enumerate(pl):
+        parr[i] = mf_cfg_pair(int(c), int(u))
+    _check(lib.mf_cfg_combine(_ptr(v), ctypes.cast(arr, _P), S, ctypes.cast(parr, _P), len(pl),
+                              C, w, _ptr(out), _stream(stream)), "mf_cfg_combine")

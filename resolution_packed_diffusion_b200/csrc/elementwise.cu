@@ -258,6 +258,37 @@ __global__ void __launch_bounds__(256, (NCH <= 4 ? 3 : (NCH <= 12 ? 2 : 1))) ada
   }
 }
 
+// ------------------------------------------------------------ packed CFG combine
+// One thread per 16-byte chunk of output rows (grid-stride): the chunk's pair by
+// binary search of the row map in the kernel parameters, then out = fma(w,
+// c - u, u) in fp32 on the two branches' chunks (picx.dev "Mage-Flow" summary,
+// Methodology > NR-MMDiT, "Packed CFG inference"; the combine is the usual
+// classifier-free guidance form).
+__global__ void __launch_bounds__(256) cfg_combine_kernel(const uint4* __restrict__ v,
+                                                          const CfgTable tab, int C, float w,
+                                                          uint4* __restrict__ out) {
+  const int cpr = C >> 3;  // chunks per row
+  const long long total = static_cast<long long>(tab.out0[tab.P]) * cpr;
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long gi = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; gi < total;
+       gi += stride) {
+    const int r = static_cast<int>(gi / cpr);
+    const int c = static_cast<int>(gi - static_cast<long long>(r) * cpr);
+    int lo = 0, hi = tab.P - 1;  // last pair with out0[p] <= r
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (tab.out0[mid] <= r) lo = mid; else hi = mid - 1;
+    }
+    const int i = r - tab.out0[lo];
+    float fc[8], fu[8], o[8];
+    unpack8(__ldcs(v + static_cast<size_t>(tab.cond0[lo] + i) * cpr + c), fc);
+    unpack8(__ldcs(v + static_cast<size_t>(tab.uncond0[lo] + i) * cpr + c), fu);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) o[e] = fmaf(w, fc[e] - fu[e], fu[e]);
+    __stcs(out + gi, pack8(o));
+  }
+}
+
 // ------------------------------------------------------------ RoPE
 // One thread per (token, 8-channel chunk): it computes the four pair angles of
 // its chunk once and applies them to that chunk of every head of q and k.
@@ -442,6 +473,16 @@ cudaError_t launch_gated_residual(const mf_bf16* x, const mf_bf16* o, const floa
   gated_residual_kernel<<<grid, 256, 0, st>>>(
       reinterpret_cast<const uint4*>(x), reinterpret_cast<const uint4*>(o), mod, tok_sample,
       tok_mod, T, S, hid, reinterpret_cast<uint4*>(y), ctl);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_cfg_combine(const mf_bf16* v, const CfgTable& tab, int32_t C, float w,
+                               mf_bf16* out, cudaStream_t st) {
+  const long long work = static_cast<long long>(tab.out0[tab.P]) * (C / 8);
+  if (work == 0) return cudaSuccess;
+  const int grid = grid_for(work, 256, 8);
+  cfg_combine_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(v), tab, C, w,
+                                           reinterpret_cast<uint4*>(out));
   return cudaGetLastError();
 }
 

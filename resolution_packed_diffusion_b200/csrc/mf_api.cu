@@ -346,6 +346,45 @@ mf_status mf_block_fwd(const mf_bf16* x, const mf_bf16* q, const mf_bf16* k, con
                                      count_items(cu_seqlens_h, S, H), ctl, stream));
 }
 
+mf_status mf_cfg_combine(const mf_bf16* v, const mf_sample_desc* desc, int32_t S,
+                         const mf_cfg_pair* pairs, int32_t P, int32_t C, float w, mf_bf16* out,
+                         cudaStream_t stream) {
+  if (desc == nullptr || pairs == nullptr || S < 1 || S > MF_MAX_SAMPLES || P < 1 ||
+      P > kMaxCfgPairs || C < 8 || C % 8 != 0 || !std::isfinite(w))
+    return MF_ERR_INVALID;
+  // offsets and image-token counts of the samples, from the descriptors
+  static thread_local CfgTable tab;
+  int64_t cu[MF_MAX_SAMPLES + 1];
+  int64_t n_img[MF_MAX_SAMPLES];
+  cu[0] = 0;
+  for (int32_t s = 0; s < S; ++s) {
+    const mf_sample_desc& d = desc[s];
+    if (d.frames < 0 || d.grid_h < 0 || d.grid_w < 0 || d.n_text < 0) return MF_ERR_INVALID;
+    n_img[s] = static_cast<int64_t>(d.frames) * d.grid_h * d.grid_w;
+    cu[s + 1] = cu[s] + n_img[s] + d.n_text;
+    if (cu[s + 1] > MF_MAX_TOKENS) return MF_ERR_INVALID;
+  }
+  const int64_t T = cu[S];
+  int64_t rows = 0;
+  tab.P = P;
+  for (int32_t p = 0; p < P; ++p) {
+    const int32_t c = pairs[p].cond, u = pairs[p].uncond;
+    if (c < 0 || c >= S || u < 0 || u >= S || c == u || n_img[c] != n_img[u])
+      return MF_ERR_INVALID;
+    tab.out0[p] = static_cast<int32_t>(rows);
+    tab.cond0[p] = static_cast<int32_t>(cu[c]);
+    tab.uncond0[p] = static_cast<int32_t>(cu[u]);
+    rows += n_img[c];
+    if (rows > MF_MAX_TOKENS) return MF_ERR_INVALID;
+  }
+  tab.out0[P] = static_cast<int32_t>(rows);
+  if (rows == 0) return MF_OK;
+  if (v == nullptr || out == nullptr || !aligned16(v) || !aligned16(out)) return MF_ERR_INVALID;
+  if (overlap(v, static_cast<size_t>(T) * C * 2, out, static_cast<size_t>(rows) * C * 2))
+    return MF_ERR_INVALID;
+  return cuda_status(launch_cfg_combine(v, tab, C, w, out, stream));
+}
+
 mf_status mf_get_error(cudaStream_t stream) {
   cudaError_t se = cudaStreamSynchronize(stream);
   if (se != cudaSuccess) return cuda_status(se);

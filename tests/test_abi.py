@@ -116,3 +116,22 @@ def test_host_argument_checks_without_gpu():
                           cu2.ctypes.data_as(P), P(16), P(16), P(16), 1, 2, 64, 2, 10000.0,
                           1e-6, P(6 << 24), P(7 << 24), P(8 << 24), 16, None)
     assert st == mf.MF_ERR_INVALID
+
+
+def test_cfg_combine_argument_checks_launch_nothing():
+    """Invalid pairs, widths or weights are refused on the host (no GPU is
+    touched: the checks come before any launch)."""
+    descs = mf.make_descs([(1, 3, 4, 5), (0, 0, 0, 7), (1, 3, 4, 2), (1, 2, 2, 1)])
+    fake = 1 << 20  # 16-byte aligned stand-in pointers, never dereferenced
+
+    def call(pairs, C=8, w=1.0, S=4):
+        parr = (mf.mf_cfg_pair * max(1, len(pairs)))(*[mf.mf_cfg_pair(c, u) for c, u in pairs])
+        return mf.lib.mf_cfg_combine(fake, ctypes.cast(descs, ctypes.c_void_p), S,
+                                     ctypes.cast(parr, ctypes.c_void_p), len(pairs), C, w,
+                                     fake + (1 << 30), None)
+    assert call([(0, 3)]) == mf.MF_ERR_INVALID      # 12 vs 4 image tokens
+    assert call([(2, 2)]) == mf.MF_ERR_INVALID      # a sample paired with itself
+    assert call([(0, 4)]) == mf.MF_ERR_INVALID      # out of range
+    assert call([(0, 2)], C=12) == mf.MF_ERR_INVALID
+    assert call([(0, 2)], w=float("inf")) == mf.MF_ERR_INVALID
+    assert call([]) == mf.MF_ERR_INVALID            # no pairs
