@@ -14,6 +14,7 @@
 #include <cmath>
 #include <cstdint>
 
+#include "cfg_internal.h"
 #include "mf_internal.h"
 #include "mf_ptx.cuh"
 

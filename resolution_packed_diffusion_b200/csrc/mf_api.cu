@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "mf.h"
+#include "cfg_internal.h"
 #include "mf_internal.h"
 
 namespace mf {

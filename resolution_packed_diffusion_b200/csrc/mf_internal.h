@@ -75,18 +75,6 @@ cudaError_t launch_attention(const mf_bf16* q, const mf_bf16* k, const mf_bf16* 
                              const AttnEpilogue& ep, int32_t num_items, const KernelCtl& ctl,
                              cudaStream_t st);
 
-// Row map of a packed-CFG combine: pair p writes output rows [out0[p],
-// out0[p + 1]) from rows cond0[p] + i and uncond0[p] + i of v.
-constexpr int kMaxCfgPairs = MF_MAX_SAMPLES / 2;
-struct CfgTable {
-  int32_t P;
-  int32_t out0[kMaxCfgPairs + 1];
-  int32_t cond0[kMaxCfgPairs];
-  int32_t uncond0[kMaxCfgPairs];
-};
-cudaError_t launch_cfg_combine(const mf_bf16* v, const CfgTable& tab, int32_t C, float w,
-                               mf_bf16* out, cudaStream_t st);
-
 cudaError_t launch_selftest_exp2(const float* x, float* y, int32_t n, cudaStream_t st);
 cudaError_t launch_selftest_wait(uint64_t limit_ns, const KernelCtl& ctl, cudaStream_t st);
 
