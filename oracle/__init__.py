@@ -48,6 +48,7 @@ from .mf_oracle import (  # noqa: F401
     cfg_combine,
     gated_residual,
     layer_norm_rows,
+    modality_linear,
     pack_build,
     rope_apply,
     rope_pair_angles,

@@ -114,3 +114,8 @@ def brute_attention(q, k, v, cu, scale=None):
 
 def brute_gate_row(xrow, orow, gate):
     return [float(xrow[i]) + float(gate[i]) * float(orow[i]) for i in range(len(xrow))]
+
+
+def brute_linear_row(x_row, w_rows):
+    """One output row of a linear map: one dot product per output feature."""
+    return [sum(a * b for a, b in zip(x_row, w)) for w in w_rows]

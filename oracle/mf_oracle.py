@@ -257,6 +257,31 @@ def block_fwd(x, q, k, v, mod, pack, rope_axes: int, base: float = 10000.0,
 
 
 # ---------------------------------------------------------------------------
+# Modality-specific linear layer  ([norm])
+# ---------------------------------------------------------------------------
+def modality_linear(x, W, tok_mod) -> np.ndarray:
+    """The per-modality projection of an MMDiT block.
+
+    [norm]: the backbone is an MMDiT with modality-specific normalization and
+    joint self-attention; in an MMDiT the image and the text stream also keep
+    their own projection weights, and the joint attention runs on the
+    concatenation. Reading (the pages give no layer shapes): one linear map per
+    modality, no bias, ``out[t] = x[t] @ W[m(t)].T`` with m(t) = tok_mod[t]
+    (0 image, 1 text) and W stored as [2][N][K] (out features, in features).
+
+    x: [T][K]; returns float64 [T][N].
+    """
+    x = np.asarray(x, dtype=np.float64)
+    W = np.asarray(W, dtype=np.float64)
+    tok_mod = np.asarray(tok_mod)
+    out = np.zeros((x.shape[0], W.shape[1]), dtype=np.float64)
+    for m in (MOD_IMG, MOD_TXT):
+        sel = tok_mod == m
+        out[sel] = x[sel] @ W[m].T
+    return out
+
+
+# ---------------------------------------------------------------------------
 # Packed classifier-free guidance  ([cfg])
 # ---------------------------------------------------------------------------
 def cfg_combine(v, descs: Sequence, pairs: Sequence, w: float) -> np.ndarray:

@@ -408,3 +408,51 @@ def check_cfg_pack_order(cfg_combine):
     a = cfg_combine(v, _CFG_DESCS, _CFG_PAIRS, 2.5)
     b = cfg_combine(v2, descs2, pairs2, 2.5)
     assert np.array_equal(a, b)
+
+
+# ---------------------------------------------------------------------------
+# Modality-specific linear layer  ([norm])
+# ---------------------------------------------------------------------------
+def _linear_case(seed=60, K=8, N=6):
+    w = make_random_pack(seed, S=4, H=1, D=8, rope_axes=2, max_grid=4, max_text=5)
+    p = oracle_pack_ids(w)
+    rng = np.random.default_rng(seed + 1)
+    x = rng.standard_normal((w.T, K))
+    W = rng.standard_normal((2, N, K))
+    return w, p, x, W
+
+
+def oracle_pack_ids(w):
+    """Modality of every token of a pack, written out from the descriptors
+    (image tokens first in each sample, then text), independent of the
+    oracle's pack_build."""
+    mods = []
+    for d in w.descs:
+        mods += [0] * (d.frames * d.grid_h * d.grid_w) + [1] * d.n_text
+    return np.asarray(mods, dtype=np.uint8)
+
+
+def check_linear_vs_brute(modality_linear):
+    w, tm, x, W = _linear_case()
+    out = modality_linear(x, W, tm)
+    assert out.shape == (w.T, W.shape[1])
+    assert (tm == 0).any() and (tm == 1).any()
+    for t in range(w.T):
+        ref = brute.brute_linear_row(x[t].tolist(), W[int(tm[t])].tolist())
+        assert np.allclose(out[t], ref, rtol=0, atol=1e-12)
+
+
+def check_linear_routing(modality_linear):
+    """Zero text weights zero exactly the text rows (and vice versa); identity
+    weights return the input."""
+    w, tm, x, W = _linear_case(K=6, N=6)
+    W0 = W.copy()
+    W0[1] = 0.0
+    out = modality_linear(x, W0, tm)
+    assert np.all(out[tm == 1] == 0.0) and np.all(out[tm == 0] != 0.0)
+    W1 = W.copy()
+    W1[0] = 0.0
+    out = modality_linear(x, W1, tm)
+    assert np.all(out[tm == 0] == 0.0) and np.all(out[tm == 1] != 0.0)
+    eye = np.stack([np.eye(6), np.eye(6)])
+    assert np.array_equal(modality_linear(x, eye, tm), x)

@@ -110,6 +110,20 @@ def _cfg_text_rows(v, descs, pairs, w):
     return np.concatenate(out)
 
 
+def _linear_modality_swapped(x, W, tok_mod):
+    return mo.modality_linear(x, np.asarray(W)[::-1], tok_mod)
+
+
+def _linear_untransposed(x, W, tok_mod):
+    x = np.asarray(x, dtype=np.float64)
+    W = np.asarray(W, dtype=np.float64)
+    out = np.zeros((x.shape[0], W.shape[1]))
+    for m in (0, 1):
+        sel = np.asarray(tok_mod) == m
+        out[sel] = x[sel][:, :W.shape[1]] @ W[m][:, :W.shape[1]]  # W used as [K][N]
+    return out
+
+
 MUTANTS = [
     ("rope sign flip", lambda: pins.check_rope_relative(_rope_sign_flip) or
      pins.check_rope_textbook_1d(_rope_sign_flip)),
@@ -126,6 +140,9 @@ MUTANTS = [
                                                  oracle.pack_build)),
     ("CFG branches swapped", lambda: pins.check_cfg_special_weights(_cfg_branches_swapped)),
     ("CFG rows from the text end", lambda: pins.check_cfg_row_map(_cfg_text_rows)),
+    ("linear weights of the other modality",
+     lambda: pins.check_linear_routing(_linear_modality_swapped)),
+    ("linear weight not transposed", lambda: pins.check_linear_vs_brute(_linear_untransposed)),
 ]
 
 

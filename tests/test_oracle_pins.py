@@ -167,3 +167,16 @@ def test_cfg_rejects_mismatched_grids():
     import pytest as _pt
     with _pt.raises(ValueError):
         oracle.cfg_combine(np.zeros((17 + 7 + 14 + 5 + 10, 2)), pins._CFG_DESCS, [(0, 3)], 1.0)
+
+
+def test_linear_vs_brute():
+    pins.check_linear_vs_brute(oracle.modality_linear)
+
+
+def test_linear_routing():
+    pins.check_linear_routing(oracle.modality_linear)
+
+
+def test_linear_modality_ids_match_pack_build():
+    w, tm, _x, _W = pins._linear_case()
+    assert np.array_equal(tm, oracle.pack_build(w.descs, 2)["tok_mod"])
