@@ -468,6 +468,72 @@ def run_gpu(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def run_linear(args, rank, world, local_rank):
+    """`--op linear`: the modality-specific linear layer as the block's fused
+    Q, K, V projection (hid -> 3 hid) over the workload's pack."""
+    import torch
+    import resolution_packed_diffusion_b200 as mf
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = make_workload(args.config, with_arrays=False, seed=rank_seed(args.config, rank))
+    cu_h, T = mf.mf_pack_build(w.descs, w.rope_axes, w.budget)
+    K, N = w.hid, 3 * w.hid
+    g = torch.Generator(device=dev)
+    g.manual_seed(rank_seed(args.config, rank))
+    x = torch.randn((T, K), device=dev, generator=g).to(torch.bfloat16)
+    W = (torch.randn((2, N, K), device=dev, generator=g) / K ** 0.5).to(torch.bfloat16)
+    cu_d = torch.empty(w.S + 1, dtype=torch.int32, device=dev)
+    pos = torch.empty((T, 3), dtype=torch.int32, device=dev)
+    ts = torch.empty(T, dtype=torch.int32, device=dev)
+    tm = torch.empty(T, dtype=torch.uint8, device=dev)
+    mf.mf_pack_build(w.descs, w.rope_axes, w.budget, cu_d, pos, ts, tm)
+    out = torch.empty((T, N), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    clocks = ClockSampler(local_rank) if rank == 0 else None
+    for _ in range(args.warmup):
+        mf.mf_modality_linear(x, W, tm, w.descs, K, N, out, stream)
+    barrier()
+    torch.cuda.synchronize(dev)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        mf.mf_modality_linear(x, W, tm, w.descs, K, N, out, stream)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop() if clocks else None
+    if mf.mf_get_error(stream) != mf.MF_OK:
+        raise RuntimeError("device error in the linear layer")
+    flops = 2.0 * T * K * N
+    ms_step, flops_all = reduce_timing(t0.elapsed_time(t1) / args.steps, flops, world)
+    if rank != 0:
+        return
+    peaks, peak_src = load_peaks()
+    achieved = flops / (ms_step * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    print(json.dumps({
+        "metric": "modality-specific linear (fused QKV projection) TFLOP/s", "op": "linear",
+        "value": flops_all / (ms_step * 1e-3) / 1e12, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "config_index": args.config, "T": T, "K": K, "N": N,
+                   "l2": "x, W and out total %d MB vs 126 MB L2; no flush"
+                         % ((T * K + 2 * N * K + T * N) * 2 >> 20)},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
+                     "frac": achieved / peak, "traffic": None, "kernel": "modality_linear_kernel",
+                     "peak_source": f"{peak_src} bf16_tflops (burst)"},
+        "gpu_launches": args.steps, "clocks": clk}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -476,6 +542,9 @@ def main():
     ap.add_argument("--config", type=int, default=DEFAULT_CONFIG, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--impl", default="mf", choices=["mf", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", default="block", choices=["block", "linear"],
+                    help="block: the packed joint-attention block (the default line); "
+                         "linear: the modality-specific linear layer as a QKV projection")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -493,7 +562,10 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        run_gpu(args, rank, world, local_rank)
+        if args.op == "linear":
+            run_linear(args, rank, world, local_rank)
+        else:
+            run_gpu(args, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist

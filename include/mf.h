@@ -206,6 +206,19 @@ mf_status mf_cfg_combine(const mf_bf16* v, const mf_sample_desc* desc, int32_t S
                          const mf_cfg_pair* pairs, int32_t P, int32_t C, float w, mf_bf16* out,
                          cudaStream_t stream);
 
+/* Modality-specific linear layer [norm]: out[t] = x[t] W[m]^T with m = tok_mod[t]
+ * (0 image, 1 text): the image and the text stream of the MMDiT keep their own
+ * projection weights. x: [T][K] bf16; W: [2][N][K] bf16 (out features by in
+ * features, image weights first); out: [T][N] bf16 (must not overlap x or W).
+ * tok_mod: [T] device, from mf_pack_build of the same desc; desc: host, S
+ * samples (they fix T and where each modality's rows lie). K % 64 == 0,
+ * N % 256 == 0, T <= 131072 (else MF_ERR_UNSUPPORTED). tcgen05 tensor cores,
+ * bf16 operands, fp32 accumulation over K, bf16 round-to-nearest-even output.
+ * A row whose tok_mod is neither 0 nor 1 is left unwritten. */
+mf_status mf_modality_linear(const mf_bf16* x, const mf_bf16* W, const uint8_t* tok_mod,
+                             const mf_sample_desc* desc, int32_t S, int32_t K, int32_t N,
+                             mf_bf16* out, cudaStream_t stream);
+
 /* Bytes of workspace mf_varlen_attn_fwd / mf_block_fwd need (with_rope != 0:
  * room for the rotated Q and K). */
 size_t mf_workspace_size(int32_t T, int32_t H, int32_t D, int32_t with_rope);

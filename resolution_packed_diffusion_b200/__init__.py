@@ -75,6 +75,7 @@ _SIGS = {
     "mf_block_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F,
                                   _F, _P, _P, _P]),
     "mf_cfg_combine": (_I, [_P, _P, _I, _P, _I, _I, _F, _P, _P]),
+    "mf_modality_linear": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -252,3 +253,11 @@ def mf_cfg_combine(v, descs, pairs, C: int, w: float, out, stream=None) -> None:
         parr[i] = mf_cfg_pair(int(c), int(u))
     _check(lib.mf_cfg_combine(_ptr(v), ctypes.cast(arr, _P), S, ctypes.cast(parr, _P), len(pl),
                               C, w, _ptr(out), _stream(stream)), "mf_cfg_combine")
+
+
+def mf_modality_linear(x, W, tok_mod, descs, K: int, N: int, out, stream=None) -> None:
+    """out[t] = x[t] W[tok_mod[t]]^T: W is [2][N][K] (image weights first)."""
+    arr = make_descs(descs)
+    S = len(list(descs))
+    _check(lib.mf_modality_linear(_ptr(x), _ptr(W), _ptr(tok_mod), ctypes.cast(arr, _P), S, K, N,
+                                  _ptr(out), _stream(stream)), "mf_modality_linear")

@@ -1,0 +1,334 @@
+// gemm.cu -- the modality-specific linear layer of the MMDiT block on sm_100a
+// tensor cores: out[t] = x[t] W[m(t)]^T, m(t) the token's modality (0 image,
+// 1 text), W stored [2][N][K].
+//
+// Source (page title, section): picx.dev "Mage-Flow" summary, Methodology >
+// Native-Resolution MMDiT (an MMDiT with modality-specific normalization and
+// joint self-attention: the image and the text stream keep their own weights).
+//
+// Design (one persistent CTA per SM, 8 warps). The output is cut into 128-row x
+// 256-column tiles; a 128-row tile of the pack whose tokens are all of one
+// modality is one job per column tile; a tile that holds both modalities (at
+// an image / text boundary) is two jobs, each computed with its modality's
+// weights and writing only its own rows.
+//   warp 0      TMA producer: 128 x 64 slices of x and 256 x 64 slices of W
+//               (128-byte swizzle, no multicast) into a 4-stage ring.
+//   warp 1      tcgen05 issuer: D (fp32, TMEM) += A B^T with M = 128, N = 256,
+//               K = 16, both operands K-major in shared memory; two TMEM
+//               accumulators of 256 columns alternate between jobs so that a
+//               job's epilogue overlaps the next job's MMAs.
+//   warps 2..3  idle.
+//   warps 4..7  epilogue: one output row per thread (its TMEM lane), 32 columns
+//               at a time, rounded to bf16 and stored if the row exists and is
+//               of the job's modality.
+// Jobs are walked in an order that keeps the 148 concurrent CTAs on a few
+// 128-row tiles of x at a time (all column tiles of a row tile back to back),
+// so that x tiles and the weights stream through L2. Every wait is bounded.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include <cstdint>
+#include <vector>
+
+#include "gemm_internal.h"
+#include "mf_internal.h"
+#include "mf_ptx.cuh"
+
+namespace mf {
+
+namespace {
+
+constexpr int GM = 128;             // rows per tile (MMA M)
+constexpr int GN = 256;             // output columns per tile (MMA N)
+constexpr int GK = 64;              // K per stage: one 128-byte swizzle atom
+constexpr int kStages = 4;
+constexpr int A_BYTES = GM * GK * 2;
+constexpr int B_BYTES = GN * GK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int kThreads = 256;
+constexpr uint32_t kTmemCols = 512;  // two accumulators of GN columns
+
+struct GemmLayout {
+  static constexpr int OFF_STAGES = 0;
+  static constexpr int OFF_BAR = kStages * STAGE_BYTES;
+  static constexpr int B_FULL = 0;                    // [kStages]
+  static constexpr int B_EMPTY = B_FULL + kStages;    // [kStages]
+  static constexpr int B_ACC_FULL = B_EMPTY + kStages;  // [2]
+  static constexpr int B_ACC_EMPTY = B_ACC_FULL + 2;    // [2], one arrival per epilogue warp
+  static constexpr int B_DRAIN = B_ACC_EMPTY + 2;
+  static constexpr int NUM_BARS = B_DRAIN + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;  // tmem slot, abort flag
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget of one CTA");
+};
+
+struct GemmArgs {
+  GemmJobs jobs;
+  int32_t T, K, N;
+  const uint8_t* tok_mod;
+  mf_bf16* out;
+  KernelCtl ctl;
+};
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const KernelCtl& ctl,
+                                          volatile int* abort_flag) {
+  const bool ok = mbar_wait(bar, parity, ctl, abort_flag);
+  return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > limit_ns) return;
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    modality_linear_kernel(const __grid_constant__ CUtensorMap tmap_x,
+                           const __grid_constant__ CUtensorMap tmap_w,
+                           const __grid_constant__ GemmArgs args) {
+  using L = GemmLayout;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < L::NUM_BARS; ++i)
+      mbar_init(&bars[i], (i == L::B_ACC_EMPTY || i == L::B_ACC_EMPTY + 1) ? 4u : 1u);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_map(&tmap_x);
+    tma_prefetch_map(&tmap_w);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int nN = args.N / GN;
+  const int nK = args.K / GK;
+  const int units = args.jobs.n * nN;
+
+  if (warp == 0) {
+    // ============================================================ TMA producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        const int job = args.jobs.job[u / nN];
+        const int tile = job & 0x7fff, m = job >> 15, nt = u % nN;
+        for (int kb = 0; kb < nK; ++kb, ++it) {
+          const int st = it % kStages;
+          if (!mbar_wait(&bars[L::B_EMPTY + st], ((it / kStages) & 1) ^ 1, args.ctl, abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + L::OFF_STAGES + st * STAGE_BYTES;
+          mbar_expect_tx(&bars[L::B_FULL + st], STAGE_BYTES);
+          tma_load_2d(sa, &tmap_x, &bars[L::B_FULL + st], kb * GK, tile * GM);
+          tma_load_2d(sa + A_BYTES, &tmap_w, &bars[L::B_FULL + st], kb * GK,
+                      m * args.N + nt * GN);
+        }
+      }
+      // every copy this thread started lands before the CTA can exit
+      for (int st = 0; st < kStages; ++st)
+        if (it > static_cast<uint32_t>(st)) {
+          const uint32_t last = it - 1 - ((it - 1 - st) % kStages);
+          drain_wait(&bars[L::B_FULL + st], (last / kStages) & 1, args.ctl.wait_limit_ns);
+        }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ============================================================ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC = idesc_bf16_f32(GM, GN, 0, 0);
+      const uint32_t base = smem_u32(smem + L::OFF_STAGES);
+      const uint64_t desc0 = sdesc_sw128(base, 16, 1024);
+      uint32_t it = 0, ul = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++ul) {
+        const uint32_t acc = ul & 1;
+        if (!mbar_wait(&bars[L::B_ACC_EMPTY + acc], ((ul >> 1) & 1) ^ 1, args.ctl, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + acc * GN;
+        for (int kb = 0; kb < nK; ++kb, ++it) {
+          const int st = it % kStages;
+          if (!mbar_wait(&bars[L::B_FULL + st], (it / kStages) & 1, args.ctl, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t a0 = desc0 + static_cast<uint64_t>((st * STAGE_BYTES) >> 4);
+          const uint64_t b0 = desc0 + static_cast<uint64_t>((st * STAGE_BYTES + A_BYTES) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < GK / 16; ++kk)  // a 16-element K step is 32 bytes inside the atom
+            umma_ss(d, a0 + kk * 2, b0 + kk * 2, IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(&bars[L::B_EMPTY + st]);
+        }
+        if (!ok) break;
+        umma_commit(&bars[L::B_ACC_FULL + acc]);
+      }
+      umma_commit(&bars[L::B_DRAIN]);
+      drain_wait(&bars[L::B_DRAIN], 0, args.ctl.wait_limit_ns);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ============================================================ epilogue
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+    uint32_t ul = 0;
+    for (int u = blockIdx.x; u < units; u += gridDim.x, ++ul) {
+      const int job = args.jobs.job[u / nN];
+      const int tile = job & 0x7fff, m = job >> 15, nt = u % nN;
+      const uint32_t acc = ul & 1;
+      if (!warp_wait(&bars[L::B_ACC_FULL + acc], (ul >> 1) & 1, args.ctl, abort_flag)) break;
+      tc_fence_after();
+      const int t = tile * GM + row;
+      const bool keep = t < args.T && __ldg(args.tok_mod + t) == m;
+      uint4* orow = reinterpret_cast<uint4*>(args.out + static_cast<size_t>(t) * args.N + nt * GN);
+#pragma unroll 1
+      for (int cc = 0; cc < GN; cc += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_base + acc * GN + cc, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) asm volatile("" : "+r"(v[e]));
+        if (keep) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 o;
+            o.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1]));
+            o.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
+            o.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
+            o.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
+            orow[cc / 8 + q] = o;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[L::B_ACC_EMPTY + acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// [rows][cols] bf16, box = 64 columns x box_rows rows, 128-byte swizzle; rows
+// past the end read as zeros.
+bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+int sms() {
+  static int cached[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+}  // namespace
+
+bool build_gemm_jobs(const int32_t* mods_per_sample_img, const int32_t* mods_per_sample_txt,
+                     int32_t S, int32_t T, GemmJobs* jobs) {
+  const int tiles = (T + GM - 1) / GM;
+  if (tiles > kMaxGemmTiles) return false;
+  std::vector<uint8_t> has(static_cast<size_t>(tiles), 0);  // bit m: modality m present
+  int64_t row = 0;
+  for (int32_t s = 0; s < S; ++s) {
+    const int64_t runs[2] = {mods_per_sample_img[s], mods_per_sample_txt[s]};
+    for (int m = 0; m < 2; ++m) {
+      if (runs[m] > 0) {
+        for (int64_t tl = row / GM; tl <= (row + runs[m] - 1) / GM; ++tl) has[tl] |= 1u << m;
+        row += runs[m];
+      }
+    }
+  }
+  if (row != T) return false;
+  int n = 0;
+  for (int tl = 0; tl < tiles; ++tl)
+    for (int m = 0; m < 2; ++m)
+      if (has[tl] & (1u << m)) jobs->job[n++] = static_cast<uint16_t>(tl | (m << 15));
+  jobs->n = n;
+  return true;
+}
+
+cudaError_t launch_modality_linear(const mf_bf16* x, const mf_bf16* W, const uint8_t* tok_mod,
+                                   const GemmJobs& jobs, int32_t T, int32_t K, int32_t N,
+                                   mf_bf16* out, const KernelCtl& ctl, cudaStream_t st) {
+  if (jobs.n == 0) return cudaSuccess;
+  CUtensorMap mx, mw;
+  if (!make_map(&mx, x, T, K, GM) || !make_map(&mw, W, 2LL * N, K, GN))
+    return cudaErrorInvalidValue;
+  static thread_local GemmArgs a;
+  a.jobs = jobs;
+  a.T = T;
+  a.K = K;
+  a.N = N;
+  a.tok_mod = tok_mod;
+  a.out = out;
+  a.ctl = ctl;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(
+        modality_linear_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GemmLayout::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  const int units = jobs.n * (N / GN);
+  const int grid = units < sms() ? units : sms();
+  modality_linear_kernel<<<grid, kThreads, GemmLayout::SMEM_BYTES, st>>>(mx, mw, a);
+  return cudaGetLastError();
+}
+
+}  // namespace mf

@@ -10,6 +10,7 @@
 
 #include "mf.h"
 #include "cfg_internal.h"
+#include "gemm_internal.h"
 #include "mf_internal.h"
 
 namespace mf {
@@ -384,6 +385,39 @@ mf_status mf_cfg_combine(const mf_bf16* v, const mf_sample_desc* desc, int32_t S
   if (overlap(v, static_cast<size_t>(T) * C * 2, out, static_cast<size_t>(rows) * C * 2))
     return MF_ERR_INVALID;
   return cuda_status(launch_cfg_combine(v, tab, C, w, out, stream));
+}
+
+mf_status mf_modality_linear(const mf_bf16* x, const mf_bf16* W, const uint8_t* tok_mod,
+                             const mf_sample_desc* desc, int32_t S, int32_t K, int32_t N,
+                             mf_bf16* out, cudaStream_t stream) {
+  if (desc == nullptr || S < 1 || S > MF_MAX_SAMPLES || K < 64 || K % 64 != 0 || N < 256 ||
+      N % 256 != 0 || N > (1 << 20))
+    return MF_ERR_INVALID;
+  int32_t n_img[MF_MAX_SAMPLES], n_txt[MF_MAX_SAMPLES];
+  int64_t T = 0;
+  for (int32_t s = 0; s < S; ++s) {
+    const mf_sample_desc& d = desc[s];
+    if (d.frames < 0 || d.grid_h < 0 || d.grid_w < 0 || d.n_text < 0) return MF_ERR_INVALID;
+    const int64_t ni = static_cast<int64_t>(d.frames) * d.grid_h * d.grid_w;
+    if (ni > MF_MAX_TOKENS) return MF_ERR_INVALID;
+    n_img[s] = static_cast<int32_t>(ni);
+    n_txt[s] = d.n_text;
+    T += ni + d.n_text;
+    if (T > MF_MAX_TOKENS) return MF_ERR_INVALID;
+  }
+  if (T == 0) return MF_OK;
+  if (x == nullptr || W == nullptr || tok_mod == nullptr || out == nullptr || !aligned16(x) ||
+      !aligned16(W) || !aligned16(out))
+    return MF_ERR_INVALID;
+  const size_t xb = static_cast<size_t>(T) * K * 2, wb = static_cast<size_t>(2) * N * K * 2,
+               ob = static_cast<size_t>(T) * N * 2;
+  if (overlap(out, ob, x, xb) || overlap(out, ob, W, wb)) return MF_ERR_INVALID;
+  static thread_local GemmJobs jobs;
+  if (!build_gemm_jobs(n_img, n_txt, S, static_cast<int32_t>(T), &jobs)) return MF_ERR_UNSUPPORTED;
+  KernelCtl ctl;
+  if (cudaError_t ge = get_ctl(&ctl); ge != cudaSuccess) return cuda_status(ge);
+  return cuda_status(launch_modality_linear(x, W, tok_mod, jobs, static_cast<int32_t>(T), K, N,
+                                            out, ctl, stream));
 }
 
 mf_status mf_get_error(cudaStream_t stream) {
