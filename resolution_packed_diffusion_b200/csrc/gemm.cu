@@ -21,9 +21,9 @@
 //   warps 4..7  epilogue: one output row per thread (its TMEM lane), 32 columns
 //               at a time, rounded to bf16 and stored if the row exists and is
 //               of the job's modality.
-// Jobs are walked in an order that keeps the 148 concurrent CTAs on a few
-// 128-row tiles of x at a time (all column tiles of a row tile back to back),
-// so that x tiles and the weights stream through L2. Every wait is bounded.
+// Units (job, column tile) are walked in column blocks of up to 12 tiles, every
+// row tile inside a block: a block of weights stays in L2 while x streams past
+// it once per block (see unit_coords). Every wait is bounded.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -65,10 +65,42 @@ struct GemmLayout {
 struct GemmArgs {
   GemmJobs jobs;
   int32_t T, K, N;
+  int32_t nb;  // column tiles per block of the traversal (divides N / GN)
   const uint8_t* tok_mod;
   mf_bf16* out;
   KernelCtl ctl;
 };
+
+// L2 cache policy for the weight slices: re-read by every row tile, they are
+// kept in L2 (evict_last) while the output streams past it (streaming stores).
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// 2D tiled TMA load with an L2 cache policy (no multicast).
+__device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                                 int32_t x, int32_t y, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(policy)
+      : "memory");
+}
+
+// Unit u of the traversal -> (job, column tile): column tiles in blocks of nb;
+// inside a block every job (row tile) in turn, the block's column tiles of a
+// job back to back. The ~148 units in flight then cover about 148 / nb row
+// tiles and one block of weights, which stays in L2 while x streams once per
+// block.
+__device__ __forceinline__ void unit_coords(int u, int n_jobs, int nb, int& job_idx, int& nt) {
+  const int per_block = n_jobs * nb;
+  const int b = u / per_block;
+  const int r = u - b * per_block;
+  job_idx = r / nb;
+  nt = b * nb + (r - job_idx * nb);
+}
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const KernelCtl& ctl,
                                           volatile int* abort_flag) {
@@ -122,11 +154,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ============================================================ TMA producer
     if (lane == 0) {
+      const uint64_t keep = policy_evict_last();
       uint32_t it = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-        const int job = args.jobs.job[u / nN];
-        const int tile = job & 0x7fff, m = job >> 15, nt = u % nN;
+        int ji, nt;
+        unit_coords(u, args.jobs.n, args.nb, ji, nt);
+        const int job = args.jobs.job[ji];
+        const int tile = job & 0x7fff, m = job >> 15;
         for (int kb = 0; kb < nK; ++kb, ++it) {
           const int st = it % kStages;
           if (!mbar_wait(&bars[L::B_EMPTY + st], ((it / kStages) & 1) ^ 1, args.ctl, abort_flag)) {
@@ -136,8 +171,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* sa = smem + L::OFF_STAGES + st * STAGE_BYTES;
           mbar_expect_tx(&bars[L::B_FULL + st], STAGE_BYTES);
           tma_load_2d(sa, &tmap_x, &bars[L::B_FULL + st], kb * GK, tile * GM);
-          tma_load_2d(sa + A_BYTES, &tmap_w, &bars[L::B_FULL + st], kb * GK,
-                      m * args.N + nt * GN);
+          tma_load_2d_hint(sa + A_BYTES, &tmap_w, &bars[L::B_FULL + st], kb * GK,
+                           m * args.N + nt * GN, keep);
         }
       }
       // every copy this thread started lands before the CTA can exit
@@ -189,8 +224,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
     uint32_t ul = 0;
     for (int u = blockIdx.x; u < units; u += gridDim.x, ++ul) {
-      const int job = args.jobs.job[u / nN];
-      const int tile = job & 0x7fff, m = job >> 15, nt = u % nN;
+      int ji, nt;
+      unit_coords(u, args.jobs.n, args.nb, ji, nt);
+      const int job = args.jobs.job[ji];
+      const int tile = job & 0x7fff, m = job >> 15;
       const uint32_t acc = ul & 1;
       if (!warp_wait(&bars[L::B_ACC_FULL + acc], (ul >> 1) & 1, args.ctl, abort_flag)) break;
       tc_fence_after();
@@ -212,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             o.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
             o.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
             o.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
-            orow[cc / 8 + q] = o;
+            __stcs(orow + cc / 8 + q, o);
           }
         }
       }
@@ -315,6 +352,11 @@ cudaError_t launch_modality_linear(const mf_bf16* x, const mf_bf16* W, const uin
   a.N = N;
   a.tok_mod = tok_mod;
   a.out = out;
+  // column-tile block: the largest divisor of N / GN that is at most 12
+  const int nN = N / GN;
+  a.nb = 1;
+  for (int d = 1; d <= 12 && d <= nN; ++d)
+    if (nN % d == 0) a.nb = d;
   a.ctl = ctl;
   static bool attr_set[64] = {false};
   int dev = 0;
