@@ -47,12 +47,15 @@ from .mf_oracle import (  # noqa: F401
     block_fwd,
     cfg_combine,
     gated_residual,
+    gelu_tanh,
     layer_norm_rows,
+    mmdit_block_fwd,
     modality_linear,
     pack_build,
     rope_apply,
     rope_pair_angles,
     rope_split,
+    store_bf16,
     useful_attention_flops,
     varlen_attention,
 )

@@ -119,3 +119,49 @@ def brute_gate_row(xrow, orow, gate):
 def brute_linear_row(x_row, w_rows):
     """One output row of a linear map: one dot product per output feature."""
     return [sum(a * b for a, b in zip(x_row, w)) for w in w_rows]
+
+
+def brute_gelu(v):
+    return 0.5 * v * (1.0 + math.tanh(math.sqrt(2.0 / math.pi) * (v + 0.044715 * v * v * v)))
+
+
+def brute_mmdit_block(x, Wq, Wk, Wv, Wo, Wup, Wdown, mod_attn, mod_mlp, descs, H, D, rope_axes,
+                      base=10000.0, eps=1e-6):
+    """The whole block, token by token and channel by channel, with no rounding
+    of intermediates: adaLN, per-modality q/k/v, RoPE, per-sample attention,
+    output projection and gate, second adaLN, GELU MLP and gate. Nested lists
+    in, nested lists out ([T][H*D])."""
+    cu, pos, ts, tm = brute_pack(descs, rope_axes)
+    T = len(ts)
+    hid = H * D
+
+    def mod_vec(mod, t, j):
+        return [float(mod[ts[t]][tm[t]][j][i]) for i in range(hid)]
+
+    x1 = [brute_adaln_row(x[t], mod_vec(mod_attn, t, 0), mod_vec(mod_attn, t, 1), eps)
+          for t in range(T)]
+    q = [brute_linear_row(x1[t], Wq[tm[t]]) for t in range(T)]
+    k = [brute_linear_row(x1[t], Wk[tm[t]]) for t in range(T)]
+    v = [brute_linear_row(x1[t], Wv[tm[t]]) for t in range(T)]
+
+    def heads(rows, rotate):
+        out = []
+        for t in range(T):
+            hs = []
+            for h in range(H):
+                vec = rows[t][h * D:(h + 1) * D]
+                hs.append(brute_rope_vec(vec, pos[t], rope_axes, base) if rotate else vec)
+            out.append(hs)
+        return out
+
+    o = brute_attention(heads(q, True), heads(k, True), heads(v, False), cu)
+    y = []
+    for t in range(T):
+        orow = [o[t][h][d] for h in range(H) for d in range(D)]
+        a = brute_linear_row(orow, Wo[tm[t]])
+        y1 = brute_gate_row(x[t], a, mod_vec(mod_attn, t, 2))
+        x2 = brute_adaln_row(y1, mod_vec(mod_mlp, t, 0), mod_vec(mod_mlp, t, 1), eps)
+        hmid = [brute_gelu(val) for val in brute_linear_row(x2, Wup[tm[t]])]
+        m = brute_linear_row(hmid, Wdown[tm[t]])
+        y.append(brute_gate_row(y1, m, mod_vec(mod_mlp, t, 2)))
+    return y

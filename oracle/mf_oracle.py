@@ -259,7 +259,16 @@ def block_fwd(x, q, k, v, mod, pack, rope_axes: int, base: float = 10000.0,
 # ---------------------------------------------------------------------------
 # Modality-specific linear layer  ([norm])
 # ---------------------------------------------------------------------------
-def modality_linear(x, W, tok_mod) -> np.ndarray:
+def gelu_tanh(x) -> np.ndarray:
+    """GELU in its tanh form, 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))).
+
+    Reading: the pages do not describe the MLP branch of the block; the form
+    taken is the one DiT-family blocks use."""
+    x = np.asarray(x, dtype=np.float64)
+    return 0.5 * x * (1.0 + np.tanh(math.sqrt(2.0 / math.pi) * (x + 0.044715 * x ** 3)))
+
+
+def modality_linear(x, W, tok_mod, act: str = "none") -> np.ndarray:
     """The per-modality projection of an MMDiT block.
 
     [norm]: the backbone is an MMDiT with modality-specific normalization and
@@ -269,7 +278,8 @@ def modality_linear(x, W, tok_mod) -> np.ndarray:
     modality, no bias, ``out[t] = x[t] @ W[m(t)].T`` with m(t) = tok_mod[t]
     (0 image, 1 text) and W stored as [2][N][K] (out features, in features).
 
-    x: [T][K]; returns float64 [T][N].
+    x: [T][K]; act: "none" or "gelu" (gelu_tanh applied to every output);
+    returns float64 [T][N].
     """
     x = np.asarray(x, dtype=np.float64)
     W = np.asarray(W, dtype=np.float64)
@@ -278,7 +288,63 @@ def modality_linear(x, W, tok_mod) -> np.ndarray:
     for m in (MOD_IMG, MOD_TXT):
         sel = tok_mod == m
         out[sel] = x[sel] @ W[m].T
+    if act == "gelu":
+        out = gelu_tanh(out)
+    elif act != "none":
+        raise ValueError("act must be 'none' or 'gelu'")
     return out
+
+
+# ---------------------------------------------------------------------------
+# The whole MMDiT block around the joint-attention path  ([norm], [fuse])
+# ---------------------------------------------------------------------------
+def store_bf16(a) -> np.ndarray:
+    """The bf16 value a block stores for an intermediate result (round to
+    float32, then to bf16 nearest-even), back in float64."""
+    from packgen import bf16_bits_to_f32, f32_to_bf16_bits
+    return bf16_bits_to_f32(f32_to_bf16_bits(np.asarray(a, dtype=np.float32))).astype(np.float64)
+
+
+def mmdit_block_fwd(x, Wq, Wk, Wv, Wo, Wup, Wdown, mod_attn, mod_mlp, pack, H: int, D: int,
+                    rope_axes: int, base: float = 10000.0, eps: float = 1e-6, rows=None,
+                    store=store_bf16):
+    """One NR-MMDiT block forward over a pack.
+
+    [norm]: modality-specific normalization and joint self-attention; [fuse]:
+    adaptive normalization / RoPE / gating. Reading (the pages give the
+    operations, not the block's wiring): the DiT-family block with two gated
+    branches, each with its own modulation vectors (shift, scale, gate) per
+    sample and modality, and modality-specific projections:
+        x1 = adaLN(x; mod_attn)
+        q, k, v = x1 Wq[m]^T, x1 Wk[m]^T, x1 Wv[m]^T       (per token modality m)
+        o  = joint varlen attention of RoPE(q), RoPE(k), v  (per sample)
+        y1 = x + gate_attn * (o Wo[m]^T)
+        x2 = adaLN(y1; mod_mlp)
+        y  = y1 + gate_mlp * (GELU(x2 Wup[m]^T) Wdown[m]^T)
+    Every intermediate is stored in bf16 (``store``), as the GPU block stores
+    them; the final y is returned unrounded (float64). ``rows`` restricts the
+    output to those rows (keys and values are still computed for every row).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    T = x.shape[0]
+    ts, tm = np.asarray(pack["tok_sample"]), np.asarray(pack["tok_mod"])
+    r = np.arange(T) if rows is None else np.asarray(rows)
+    x1 = store(adaln_modulate(x, mod_attn, ts, tm, eps))
+    k = store(modality_linear(x1, Wk, tm)).reshape(T, H, D)
+    v = store(modality_linear(x1, Wv, tm)).reshape(T, H, D)
+    q = np.zeros((T, H, D))
+    q[r] = store(modality_linear(x1[r], Wq, tm[r])).reshape(-1, H, D)
+    q_r = np.zeros((T, H, D))
+    q_r[r] = store(rope_apply(q[r], np.asarray(pack["pos_ids"])[r], rope_axes, base))
+    k_r = store(rope_apply(k, pack["pos_ids"], rope_axes, base))
+    o, _ = varlen_attention(q_r, k_r, v, pack["cu_seqlens"], rows=r)
+    o = store(o).reshape(len(r), H * D)
+    a = store(modality_linear(o, Wo, tm[r]))
+    y1 = store(gated_residual(x[r], a, mod_attn, ts[r], tm[r]))
+    x2 = store(adaln_modulate(y1, mod_mlp, ts[r], tm[r], eps))
+    h = store(modality_linear(x2, Wup, tm[r], "gelu"))
+    mlp = store(modality_linear(h, Wdown, tm[r]))
+    return gated_residual(y1, mlp, mod_mlp, ts[r], tm[r])
 
 
 # ---------------------------------------------------------------------------

@@ -456,3 +456,102 @@ def check_linear_routing(modality_linear):
     assert np.all(out[tm == 0] == 0.0) and np.all(out[tm == 1] != 0.0)
     eye = np.stack([np.eye(6), np.eye(6)])
     assert np.array_equal(modality_linear(x, eye, tm), x)
+
+
+def check_gelu(gelu_tanh):
+    """GELU(0) = 0; GELU(x) - GELU(-x) = x for any x (x Phi(x) has that odd part,
+    and so does the tanh form); GELU(x) -> x and -> 0 far out; and within 2e-3
+    of the exact x Phi(x) (the tanh form's known small deviation)."""
+    from scipy.special import erf
+    x = np.linspace(-8.0, 8.0, 4001)
+    g = gelu_tanh(x)
+    assert gelu_tanh(np.array([0.0]))[0] == 0.0
+    assert np.allclose(g - gelu_tanh(-x), x, rtol=0, atol=1e-12)
+    assert abs(gelu_tanh(np.array([12.0]))[0] - 12.0) < 1e-12
+    assert abs(gelu_tanh(np.array([-12.0]))[0]) < 1e-12
+    exact = 0.5 * x * (1.0 + erf(x / math.sqrt(2.0)))
+    dev = np.abs(g - exact).max()
+    assert 1e-5 < dev < 2e-3, dev  # close to, but not, the exact form
+
+
+def check_linear_gelu(modality_linear, gelu_tanh):
+    """act='gelu' is GELU applied after the linear map, row by row."""
+    w, tm, x, W = _linear_case(seed=61)
+    assert np.allclose(modality_linear(x, W, tm, "gelu"), gelu_tanh(modality_linear(x, W, tm)),
+                       rtol=0, atol=1e-14)
+
+
+# ---------------------------------------------------------------------------
+# The whole MMDiT block  ([norm], [fuse])
+# ---------------------------------------------------------------------------
+def _mmdit_case(seed=70, H=2, D=8, F=24, descs=None):
+    descs = descs or [SampleDesc(1, 2, 3, 2), SampleDesc(1, 3, 2, 3)]
+    w = make_random_pack(seed, S=len(descs), H=H, D=D, rope_axes=2, descs=descs)
+    rng = np.random.default_rng(seed + 1)
+    hid = H * D
+    ws = dict(Wq=rng.standard_normal((2, hid, hid)) / 4, Wk=rng.standard_normal((2, hid, hid)) / 4,
+              Wv=rng.standard_normal((2, hid, hid)) / 4, Wo=rng.standard_normal((2, hid, hid)) / 4,
+              Wup=rng.standard_normal((2, F, hid)) / 4, Wdown=rng.standard_normal((2, hid, F)) / 5)
+    mods = dict(mod_attn=rng.standard_normal((w.S, 2, 3, hid)) * 0.3,
+                mod_mlp=rng.standard_normal((w.S, 2, 3, hid)) * 0.3)
+    return w, ws, mods
+
+
+def _ident(a):
+    return np.asarray(a, dtype=np.float64)
+
+
+def check_mmdit_vs_brute(mmdit_block_fwd, pack_build):
+    w, ws, mods = _mmdit_case()
+    p = pack_build(w.descs, 2)
+    x = w.f32("x")
+    y = mmdit_block_fwd(x, **ws, **mods, pack=p, H=w.H, D=w.D, rope_axes=2, store=_ident)
+    ref = brute.brute_mmdit_block(x.tolist(), *[ws[k].tolist() for k in
+                                                ("Wq", "Wk", "Wv", "Wo", "Wup", "Wdown")],
+                                  mods["mod_attn"].tolist(), mods["mod_mlp"].tolist(),
+                                  w.descs, w.H, w.D, 2)
+    assert np.allclose(y, np.asarray(ref), rtol=0, atol=1e-10)
+
+
+def check_mmdit_zero_branches(mmdit_block_fwd, pack_build):
+    """Zero output and down-projection weights leave the input unchanged, bit
+    for bit, whatever the rest."""
+    w, ws, mods = _mmdit_case(seed=71)
+    p = pack_build(w.descs, 2)
+    x = w.f32("x")
+    ws = dict(ws, Wo=np.zeros_like(ws["Wo"]), Wdown=np.zeros_like(ws["Wdown"]))
+    y = mmdit_block_fwd(x, **ws, **mods, pack=p, H=w.H, D=w.D, rope_axes=2)
+    assert np.array_equal(y, x.astype(np.float64))
+
+
+def check_mmdit_reduces_to_path(mmdit_block_fwd, block_fwd, adaln_modulate, pack_build):
+    """With identity q/k/v/out projections and a silent MLP branch (zero down
+    projection), the block is the packed joint-attention path with q = k = v =
+    adaLN(x)."""
+    w, ws, mods = _mmdit_case(seed=72)
+    p = pack_build(w.descs, 2)
+    x = w.f32("x")
+    hid = w.H * w.D
+    eye = np.stack([np.eye(hid), np.eye(hid)])
+    ws = dict(ws, Wq=eye, Wk=eye, Wv=eye, Wo=eye, Wdown=np.zeros_like(ws["Wdown"]))
+    y = mmdit_block_fwd(x, **ws, **mods, pack=p, H=w.H, D=w.D, rope_axes=2, store=_ident)
+    x1 = adaln_modulate(x, mods["mod_attn"], p["tok_sample"], p["tok_mod"])
+    qkv = x1.reshape(w.T, w.H, w.D)
+    _, ref, _ = block_fwd(x, qkv, qkv, qkv, mods["mod_attn"], p, 2)
+    assert np.allclose(y, ref, rtol=0, atol=1e-12)
+
+
+def check_mmdit_branch_gates(mmdit_block_fwd, pack_build):
+    """The MLP branch answers to its own gate: zero MLP gates give the result of
+    a zero down projection; zero attention gates leave the MLP acting on x."""
+    w, ws, mods = _mmdit_case(seed=73)
+    p = pack_build(w.descs, 2)
+    x = w.f32("x")
+    m2 = mods["mod_mlp"].copy()
+    m2[:, :, 2] = 0.0
+    a = mmdit_block_fwd(x, **ws, mod_attn=mods["mod_attn"], mod_mlp=m2, pack=p, H=w.H, D=w.D,
+                        rope_axes=2, store=_ident)
+    b = mmdit_block_fwd(x, **dict(ws, Wdown=np.zeros_like(ws["Wdown"])), **mods, pack=p, H=w.H,
+                        D=w.D, rope_axes=2, store=_ident)
+    assert np.allclose(a, b, rtol=0, atol=1e-13)
+    assert not np.allclose(a, x, atol=1e-6)

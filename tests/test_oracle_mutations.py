@@ -124,6 +124,34 @@ def _linear_untransposed(x, W, tok_mod):
     return out
 
 
+def _gelu_sigmoid_form(x):
+    x = np.asarray(x, dtype=np.float64)
+    return x / (1.0 + np.exp(-1.702 * x))  # another approximation, not this one
+
+
+def _gelu_no_cubic(x):
+    x = np.asarray(x, dtype=np.float64)
+    return 0.5 * x * (1.0 + np.tanh(math.sqrt(2.0 / math.pi) * x))
+
+
+def _mmdit_gelu_after_down(x, Wq, Wk, Wv, Wo, Wup, Wdown, mod_attn, mod_mlp, pack, H, D,
+                           rope_axes, base=10000.0, eps=1e-6, rows=None, store=mo.store_bf16):
+    # the activation after the second MLP layer instead of between the two
+    full = mo.mmdit_block_fwd(x, Wq, Wk, Wv, Wo, Wup, Wdown, mod_attn, mod_mlp, pack, H, D,
+                                   rope_axes, base, eps, rows, store)
+    y1 = mo.mmdit_block_fwd(x, Wq, Wk, Wv, Wo, Wup, np.zeros_like(Wdown), mod_attn, mod_mlp, pack,
+                            H, D, rope_axes, base, eps, rows, store)
+    gate = np.asarray(mod_mlp)[pack["tok_sample"], pack["tok_mod"], 2]
+    branch = (full - y1) / np.where(gate == 0, 1.0, gate)
+    return y1 + gate * mo.gelu_tanh(branch)
+
+
+def _mmdit_mlp_uses_attn_mod(x, Wq, Wk, Wv, Wo, Wup, Wdown, mod_attn, mod_mlp, pack, H, D,
+                             rope_axes, base=10000.0, eps=1e-6, rows=None, store=mo.store_bf16):
+    return mo.mmdit_block_fwd(x, Wq, Wk, Wv, Wo, Wup, Wdown, mod_attn, mod_attn, pack, H, D,
+                              rope_axes, base, eps, rows, store)
+
+
 MUTANTS = [
     ("rope sign flip", lambda: pins.check_rope_relative(_rope_sign_flip) or
      pins.check_rope_textbook_1d(_rope_sign_flip)),
@@ -143,6 +171,12 @@ MUTANTS = [
     ("linear weights of the other modality",
      lambda: pins.check_linear_routing(_linear_modality_swapped)),
     ("linear weight not transposed", lambda: pins.check_linear_vs_brute(_linear_untransposed)),
+    ("GELU sigmoid form", lambda: pins.check_gelu(_gelu_sigmoid_form)),
+    ("GELU without the cubic term", lambda: pins.check_gelu(_gelu_no_cubic)),
+    ("block: GELU after the down projection",
+     lambda: pins.check_mmdit_vs_brute(_mmdit_gelu_after_down, oracle.pack_build)),
+    ("block: MLP branch modulated by the attention vectors",
+     lambda: pins.check_mmdit_branch_gates(_mmdit_mlp_uses_attn_mod, oracle.pack_build)),
 ]
 
 

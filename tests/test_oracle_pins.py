@@ -180,3 +180,38 @@ def test_linear_routing():
 def test_linear_modality_ids_match_pack_build():
     w, tm, _x, _W = pins._linear_case()
     assert np.array_equal(tm, oracle.pack_build(w.descs, 2)["tok_mod"])
+
+
+def test_gelu():
+    pins.check_gelu(oracle.gelu_tanh)
+
+
+def test_linear_gelu():
+    pins.check_linear_gelu(oracle.modality_linear, oracle.gelu_tanh)
+
+
+def test_mmdit_vs_brute():
+    pins.check_mmdit_vs_brute(oracle.mmdit_block_fwd, oracle.pack_build)
+
+
+def test_mmdit_zero_branches():
+    pins.check_mmdit_zero_branches(oracle.mmdit_block_fwd, oracle.pack_build)
+
+
+def test_mmdit_reduces_to_path():
+    pins.check_mmdit_reduces_to_path(oracle.mmdit_block_fwd, oracle.block_fwd,
+                                     oracle.adaln_modulate, oracle.pack_build)
+
+
+def test_mmdit_branch_gates():
+    pins.check_mmdit_branch_gates(oracle.mmdit_block_fwd, oracle.pack_build)
+
+
+def test_mmdit_rows_subset():
+    w, ws, mods = pins._mmdit_case(seed=74)
+    p = oracle.pack_build(w.descs, 2)
+    x = w.f32("x")
+    full = oracle.mmdit_block_fwd(x, **ws, **mods, pack=p, H=w.H, D=w.D, rope_axes=2)
+    rows = np.array([0, 5, 7, 13])
+    part = oracle.mmdit_block_fwd(x, **ws, **mods, pack=p, H=w.H, D=w.D, rope_axes=2, rows=rows)
+    assert np.array_equal(full[rows], part)
