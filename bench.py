@@ -498,14 +498,14 @@ def run_linear(args, rank, world, local_rank):
 
     clocks = ClockSampler(local_rank) if rank == 0 else None
     for _ in range(args.warmup):
-        mf.mf_modality_linear(x, W, tm, w.descs, K, N, out, stream)
+        mf.mf_modality_linear(x, W, tm, w.descs, K, N, out, 0, stream)
     barrier()
     torch.cuda.synchronize(dev)
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for _ in range(args.steps):
-        mf.mf_modality_linear(x, W, tm, w.descs, K, N, out, stream)
+        mf.mf_modality_linear(x, W, tm, w.descs, K, N, out, 0, stream)
     t1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
@@ -534,6 +534,94 @@ def run_linear(args, rank, world, local_rank):
         "gpu_launches": args.steps, "clocks": clk}), flush=True)
 
 
+def run_mmdit(args, rank, world, local_rank):
+    """`--op mmdit`: one whole NR-MMDiT block (adaLN, per-modality projections,
+    RoPE + packed attention, gated residuals, GELU MLP of width 4 hid) over the
+    workload's pack, random-init weights."""
+    import torch
+    import resolution_packed_diffusion_b200 as mf
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = make_workload(args.config, seed=rank_seed(args.config, rank))
+    T, H, D, hid, S = w.T, w.H, w.D, w.hid, w.S
+    F = 4 * hid
+    g = torch.Generator(device=dev)
+    g.manual_seed(rank_seed(args.config, rank))
+
+    def weight(n, k):
+        return (torch.randn((2, n, k), device=dev, generator=g) / k ** 0.5).to(torch.bfloat16)
+
+    Wq, Wk, Wv, Wo = (weight(hid, hid) for _ in range(4))
+    Wup, Wdown = weight(F, hid), weight(hid, F)
+    x = torch.from_numpy(np.ascontiguousarray(w.x_bits).view(np.int16)).to(dev).view(torch.bfloat16)
+    c = torch.from_numpy(w.c).to(dev)
+    Wm1 = torch.from_numpy(w.W).to(dev)
+    Wm2 = (torch.randn(Wm1.shape, device=dev, generator=g) * 0.02).contiguous()
+    mod_attn = torch.empty((S, 2, 3, hid), dtype=torch.float32, device=dev)
+    mod_mlp = torch.empty_like(mod_attn)
+    cu_d = torch.empty(S + 1, dtype=torch.int32, device=dev)
+    pos = torch.empty((T, 3), dtype=torch.int32, device=dev)
+    ts = torch.empty(T, dtype=torch.int32, device=dev)
+    tm = torch.empty(T, dtype=torch.uint8, device=dev)
+    y = torch.empty_like(x)
+    ws_bytes = mf.mf_mmdit_workspace_size(T, H, D, F)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        cu_h, _ = mf.mf_pack_build(w.descs, w.rope_axes, w.budget, cu_d, pos, ts, tm, stream)
+        mf.mf_adaln_params(c, Wm1, S, c.shape[1], hid, mod_attn, stream)
+        mf.mf_adaln_params(c, Wm2, S, c.shape[1], hid, mod_mlp, stream)
+        mf.mf_mmdit_block_fwd(x, Wq, Wk, Wv, Wo, Wup, Wdown, mod_attn, mod_mlp, w.descs, cu_d,
+                              cu_h, pos, ts, tm, S, H, D, F, w.rope_axes, w.base, w.eps, y, ws,
+                              ws_bytes, stream)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    clocks = ClockSampler(local_rank) if rank == 0 else None
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    torch.cuda.synchronize(dev)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop() if clocks else None
+    if mf.mf_get_error(stream) != mf.MF_OK:
+        raise RuntimeError("device error in the MMDiT block")
+    gemm_flops = 2.0 * T * hid * hid * 4 + 2.0 * T * hid * F * 2
+    flops = gemm_flops + useful_flops(w)
+    ms_step, flops_all = reduce_timing(t0.elapsed_time(t1) / args.steps, flops, world)
+    tokens_all = reduce_timing(0.0, float(real_tokens(w)), world)[1]
+    if rank != 0:
+        return
+    peaks, peak_src = load_peaks()
+    achieved = flops / (ms_step * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    print(json.dumps({
+        "metric": "NR-MMDiT block forward TFLOP/s (GEMMs + useful attention)", "op": "mmdit",
+        "value": flops_all / (ms_step * 1e-3) / 1e12, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic inputs, random-init weights",
+        "config": {"workload": w.name, "config_index": args.config, "T": T, "H": H, "D": D,
+                   "hid": hid, "mlp": F},
+        "block_tokens_per_s": tokens_all / (ms_step * 1e-3),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
+                     "frac": achieved / peak, "traffic": None,
+                     "peak_source": f"{peak_src} bf16_tflops (burst)"},
+        "gpu_launches": 15 * args.steps, "clocks": clk}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -542,9 +630,10 @@ def main():
     ap.add_argument("--config", type=int, default=DEFAULT_CONFIG, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--impl", default="mf", choices=["mf", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", default="block", choices=["block", "linear"],
+    ap.add_argument("--op", default="block", choices=["block", "linear", "mmdit"],
                     help="block: the packed joint-attention block (the default line); "
-                         "linear: the modality-specific linear layer as a QKV projection")
+                         "linear: the modality-specific linear layer as a QKV projection; "
+                         "mmdit: one whole NR-MMDiT block around the path")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -564,6 +653,8 @@ def main():
     try:
         if args.op == "linear":
             run_linear(args, rank, world, local_rank)
+        elif args.op == "mmdit":
+            run_mmdit(args, rank, world, local_rank)
         else:
             run_gpu(args, rank, world, local_rank)
     finally:

@@ -212,12 +212,42 @@ mf_status mf_cfg_combine(const mf_bf16* v, const mf_sample_desc* desc, int32_t S
  * features, image weights first); out: [T][N] bf16 (must not overlap x or W).
  * tok_mod: [T] device, from mf_pack_build of the same desc; desc: host, S
  * samples (they fix T and where each modality's rows lie). K % 64 == 0,
- * N % 256 == 0, T <= 131072 (else MF_ERR_UNSUPPORTED). tcgen05 tensor cores,
- * bf16 operands, fp32 accumulation over K, bf16 round-to-nearest-even output.
- * A row whose tok_mod is neither 0 nor 1 is left unwritten. */
+ * N % 256 == 0, T <= 131072 (else MF_ERR_UNSUPPORTED). act: MF_ACT_NONE, or
+ * MF_ACT_GELU for GELU in its tanh form, 0.5 y (1 + tanh(sqrt(2/pi)(y + 0.044715
+ * y^3))), on every output (the MLP's first layer). tcgen05 tensor cores, bf16
+ * operands, fp32 accumulation over K and activation, bf16 round-to-nearest-even
+ * output. A row whose tok_mod is neither 0 nor 1 is left unwritten. */
+#define MF_ACT_NONE 0
+#define MF_ACT_GELU 1
 mf_status mf_modality_linear(const mf_bf16* x, const mf_bf16* W, const uint8_t* tok_mod,
                              const mf_sample_desc* desc, int32_t S, int32_t K, int32_t N,
-                             mf_bf16* out, cudaStream_t stream);
+                             int32_t act, mf_bf16* out, cudaStream_t stream);
+
+/* One NR-MMDiT block forward around the joint-attention path [norm], [fuse]. The
+ * pages give the operations, not the block's wiring; this is the DiT-family block
+ * with two gated branches and modality-specific projections (m = tok_mod[t]):
+ *   x1 = adaLN(x; mod_attn); q, k, v = x1 W{q,k,v}[m]^T
+ *   o  = RoPE + block-diagonal attention (softmax scale 1/sqrt(D)) per sample
+ *   y1 = x + gate_attn * (o Wo[m]^T)
+ *   x2 = adaLN(y1; mod_mlp); y = y1 + gate_mlp * (GELU(x2 Wup[m]^T) Wdown[m]^T)
+ * x, y: [T][hid] bf16 (hid = H * D, a multiple of 256); Wq, Wk, Wv, Wo:
+ * [2][hid][hid]; Wup: [2][F][hid]; Wdown: [2][hid][F] (F % 256 == 0; image
+ * weights first); mod_attn, mod_mlp: [S][2][3][hid] fp32 (mf_adaln_params);
+ * desc, offsets and ids as for mf_block_fwd and mf_modality_linear. Every
+ * intermediate is stored in bf16 in the workspace (ws_bytes >=
+ * mf_mmdit_workspace_size(T, H, D, F)); the kernels are the library's own
+ * (adaLN, linear layers on tcgen05, RoPE, attention, gated residual). y must not
+ * overlap x. */
+mf_status mf_mmdit_block_fwd(const mf_bf16* x, const mf_bf16* Wq, const mf_bf16* Wk,
+                             const mf_bf16* Wv, const mf_bf16* Wo, const mf_bf16* Wup,
+                             const mf_bf16* Wdown, const float* mod_attn, const float* mod_mlp,
+                             const mf_sample_desc* desc, const int32_t* cu_seqlens_d,
+                             const int32_t* cu_seqlens_h, const int32_t* pos_ids,
+                             const int32_t* tok_sample, const uint8_t* tok_mod, int32_t S,
+                             int32_t H, int32_t D, int32_t F, int32_t rope_axes, float base,
+                             float eps, mf_bf16* y, void* workspace, size_t ws_bytes,
+                             cudaStream_t stream);
+size_t mf_mmdit_workspace_size(int32_t T, int32_t H, int32_t D, int32_t F);
 
 /* Bytes of workspace mf_varlen_attn_fwd / mf_block_fwd need (with_rope != 0:
  * room for the rotated Q and K). */

@@ -75,7 +75,10 @@ _SIGS = {
     "mf_block_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F,
                                   _F, _P, _P, _P]),
     "mf_cfg_combine": (_I, [_P, _P, _I, _P, _I, _I, _F, _P, _P]),
-    "mf_modality_linear": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _P]),
+    "mf_modality_linear": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P, _P]),
+    "mf_mmdit_block_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I,
+                                _I, _I, _I, _I, _F, _F, _P, _P, _SZ, _P]),
+    "mf_mmdit_workspace_size": (_SZ, [_I, _I, _I, _I]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -255,9 +258,31 @@ def mf_cfg_combine(v, descs, pairs, C: int, w: float, out, stream=None) -> None:
                               C, w, _ptr(out), _stream(stream)), "mf_cfg_combine")
 
 
-def mf_modality_linear(x, W, tok_mod, descs, K: int, N: int, out, stream=None) -> None:
-    """out[t] = x[t] W[tok_mod[t]]^T: W is [2][N][K] (image weights first)."""
+MF_ACT_NONE, MF_ACT_GELU = 0, 1
+
+
+def mf_modality_linear(x, W, tok_mod, descs, K: int, N: int, out, act: int = MF_ACT_NONE,
+                       stream=None) -> None:
+    """out[t] = act(x[t] W[tok_mod[t]]^T): W is [2][N][K] (image weights first)."""
     arr = make_descs(descs)
     S = len(list(descs))
     _check(lib.mf_modality_linear(_ptr(x), _ptr(W), _ptr(tok_mod), ctypes.cast(arr, _P), S, K, N,
-                                  _ptr(out), _stream(stream)), "mf_modality_linear")
+                                  act, _ptr(out), _stream(stream)), "mf_modality_linear")
+
+
+def mf_mmdit_workspace_size(T: int, H: int, D: int, F: int) -> int:
+    return int(lib.mf_mmdit_workspace_size(T, H, D, F))
+
+
+def mf_mmdit_block_fwd(x, Wq, Wk, Wv, Wo, Wup, Wdown, mod_attn, mod_mlp, descs, cu_seqlens_d,
+                       cu_seqlens_h: np.ndarray, pos_ids, tok_sample, tok_mod, S: int, H: int,
+                       D: int, F: int, rope_axes: int, base: float, eps: float, y, workspace,
+                       ws_bytes: int, stream=None) -> None:
+    arr = make_descs(descs)
+    cu_h = np.ascontiguousarray(cu_seqlens_h, dtype=np.int32)
+    _check(lib.mf_mmdit_block_fwd(_ptr(x), _ptr(Wq), _ptr(Wk), _ptr(Wv), _ptr(Wo), _ptr(Wup),
+                                  _ptr(Wdown), _ptr(mod_attn), _ptr(mod_mlp),
+                                  ctypes.cast(arr, _P), _ptr(cu_seqlens_d), cu_h.ctypes.data_as(_P),
+                                  _ptr(pos_ids), _ptr(tok_sample), _ptr(tok_mod), S, H, D, F,
+                                  rope_axes, base, eps, _ptr(y), _ptr(workspace), ws_bytes,
+                                  _stream(stream)), "mf_mmdit_block_fwd")

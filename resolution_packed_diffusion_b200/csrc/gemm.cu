@@ -66,6 +66,7 @@ struct GemmArgs {
   GemmJobs jobs;
   int32_t T, K, N;
   int32_t nb;  // column tiles per block of the traversal (divides N / GN)
+  int32_t act;  // 0: none, 1: GELU (tanh form)
   const uint8_t* tok_mod;
   mf_bf16* out;
   KernelCtl ctl;
@@ -100,6 +101,12 @@ __device__ __forceinline__ void unit_coords(int u, int n_jobs, int nb, int& job_
   const int r = u - b * per_block;
   job_idx = r / nb;
   nt = b * nb + (r - job_idx * nb);
+}
+
+// GELU, tanh form: 0.5 y (1 + tanh(sqrt(2/pi) (y + 0.044715 y^3))).
+__device__ __forceinline__ float gelu_tanh(float y) {
+  const float u = 0.7978845608028654f * fmaf(0.044715f * y, y * y, y);
+  return 0.5f * y * (1.f + tanhf(u));
 }
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const KernelCtl& ctl,
@@ -241,6 +248,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 32; ++e) asm volatile("" : "+r"(v[e]));
+        if (args.act == 1) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(gelu_tanh(__uint_as_float(v[e])));
+        }
         if (keep) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -340,7 +351,8 @@ bool build_gemm_jobs(const int32_t* mods_per_sample_img, const int32_t* mods_per
 
 cudaError_t launch_modality_linear(const mf_bf16* x, const mf_bf16* W, const uint8_t* tok_mod,
                                    const GemmJobs& jobs, int32_t T, int32_t K, int32_t N,
-                                   mf_bf16* out, const KernelCtl& ctl, cudaStream_t st) {
+                                   int32_t act, mf_bf16* out, const KernelCtl& ctl,
+                                   cudaStream_t st) {
   if (jobs.n == 0) return cudaSuccess;
   CUtensorMap mx, mw;
   if (!make_map(&mx, x, T, K, GM) || !make_map(&mw, W, 2LL * N, K, GN))
@@ -352,6 +364,7 @@ cudaError_t launch_modality_linear(const mf_bf16* x, const mf_bf16* W, const uin
   a.N = N;
   a.tok_mod = tok_mod;
   a.out = out;
+  a.act = act;
   // column-tile block: the largest divisor of N / GN that is at most 12
   const int nN = N / GN;
   a.nb = 1;

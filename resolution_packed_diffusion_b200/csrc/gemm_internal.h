@@ -28,6 +28,7 @@ bool build_gemm_jobs(const int32_t* n_img, const int32_t* n_txt, int32_t S, int3
 
 cudaError_t launch_modality_linear(const mf_bf16* x, const mf_bf16* W, const uint8_t* tok_mod,
                                    const GemmJobs& jobs, int32_t T, int32_t K, int32_t N,
-                                   mf_bf16* out, const KernelCtl& ctl, cudaStream_t st);
+                                   int32_t act, mf_bf16* out, const KernelCtl& ctl,
+                                   cudaStream_t st);
 
 }  // namespace mf

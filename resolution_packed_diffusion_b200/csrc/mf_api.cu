@@ -389,9 +389,9 @@ mf_status mf_cfg_combine(const mf_bf16* v, const mf_sample_desc* desc, int32_t S
 
 mf_status mf_modality_linear(const mf_bf16* x, const mf_bf16* W, const uint8_t* tok_mod,
                              const mf_sample_desc* desc, int32_t S, int32_t K, int32_t N,
-                             mf_bf16* out, cudaStream_t stream) {
+                             int32_t act, mf_bf16* out, cudaStream_t stream) {
   if (desc == nullptr || S < 1 || S > MF_MAX_SAMPLES || K < 64 || K % 64 != 0 || N < 256 ||
-      N % 256 != 0 || N > (1 << 20))
+      N % 256 != 0 || N > (1 << 20) || (act != MF_ACT_NONE && act != MF_ACT_GELU))
     return MF_ERR_INVALID;
   int32_t n_img[MF_MAX_SAMPLES], n_txt[MF_MAX_SAMPLES];
   int64_t T = 0;
@@ -417,7 +417,7 @@ mf_status mf_modality_linear(const mf_bf16* x, const mf_bf16* W, const uint8_t* 
   KernelCtl ctl;
   if (cudaError_t ge = get_ctl(&ctl); ge != cudaSuccess) return cuda_status(ge);
   return cuda_status(launch_modality_linear(x, W, tok_mod, jobs, static_cast<int32_t>(T), K, N,
-                                            out, ctl, stream));
+                                            act, out, ctl, stream));
 }
 
 mf_status mf_get_error(cudaStream_t stream) {

@@ -17,7 +17,7 @@ if not torch.cuda.is_available():
     pytest.skip("needs a CUDA device", allow_module_level=True)
 
 
-def _run(descs, K, N, seed):
+def _run(descs, K, N, seed, act=0):
     rng = np.random.default_rng(seed)
     pack = oracle.pack_build(descs, 2)
     T = pack["T"]
@@ -27,7 +27,7 @@ def _run(descs, K, N, seed):
     x, W = dev_bf16(x_bits), dev_bf16(w_bits)
     tm = torch.from_numpy(pack["tok_mod"]).cuda()
     out = torch.full((T, N), float("nan"), dtype=torch.bfloat16, device="cuda")
-    mf.mf_modality_linear(x, W, tm, descs, K, N, out)
+    mf.mf_modality_linear(x, W, tm, descs, K, N, out, act)
     assert mf.mf_get_error() == mf.MF_OK
     return pack, host_f32(x), host_f32(W), host_f32(out)
 
@@ -50,6 +50,15 @@ def test_linear_every_row(k):
     assert_bf16_close(out, ref, "linear out")
 
 
+@pytest.mark.parametrize("k", [0, 1])
+def test_linear_gelu_every_row(k):
+    descs, K, N = SMALL[k]
+    pack, x, W, out = _run(descs, K, N, 920 + k, act=mf.MF_ACT_GELU)
+    ref = oracle.modality_linear(x, W, pack["tok_mod"], "gelu")
+    assert np.isfinite(out).all()
+    assert_bf16_close(out, ref, "linear + GELU out")
+
+
 def test_linear_qkv_projection_of_the_training_pack():
     """Full size: the training pack's 16384 tokens through a 3072 -> 9216
     projection (the fused Q, K, V widths), rows sampled around every sample and
@@ -68,9 +77,9 @@ def test_linear_rejects_bad_shapes():
     W = torch.zeros((2, 256, 128), dtype=torch.bfloat16, device="cuda")
     tm = torch.zeros(19, dtype=torch.uint8, device="cuda")
     out = torch.zeros((19, 256), dtype=torch.bfloat16, device="cuda")
-    for K, N in ((96, 256), (128, 200)):
+    for K, N, act in ((96, 256, 0), (128, 200, 0), (128, 256, 2)):
         with pytest.raises(mf.MFError) as e:
-            mf.mf_modality_linear(x, W, tm, descs, K, N, out)
+            mf.mf_modality_linear(x, W, tm, descs, K, N, out, act)
         assert e.value.status == mf.MF_ERR_INVALID
     with pytest.raises(mf.MFError):
         mf.mf_modality_linear(x, W, tm, descs, 128, 256, x)  # out overlaps x
