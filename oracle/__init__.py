@@ -58,4 +58,5 @@ from .mf_oracle import (  # noqa: F401
     store_bf16,
     useful_attention_flops,
     varlen_attention,
+    varlen_attention_bwd,
 )

@@ -214,6 +214,47 @@ def varlen_attention(q, k, v, cu_seqlens, scale: Optional[float] = None,
 # ---------------------------------------------------------------------------
 # Gated residual  ([fuse])
 # ---------------------------------------------------------------------------
+def varlen_attention_bwd(q, k, v, d_o, cu_seqlens, scale: Optional[float] = None):
+    """Gradients of the packed joint attention with respect to q, k and v.
+
+    For sample s and head h, with S = scale Q K^T, P = softmax(S) (rows),
+    O = P V and the output gradient dO (chain rule, written out):
+        dV = P^T dO
+        dP = dO V^T
+        dS = P * (dP - rowsum(dO * O))      (the softmax Jacobian, row by row)
+        dQ = scale dS K,  dK = scale dS^T Q
+    Nothing flows across samples (block-diagonal, like the forward). q, k, v,
+    d_o: [T][H][D]. Returns float64 (dq, dk, dv), each [T][H][D].
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    d_o = np.asarray(d_o, dtype=np.float64)
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    T, H, D = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for s in range(len(cu) - 1):
+        lo, hi = int(cu[s]), int(cu[s + 1])
+        if hi == lo:
+            continue
+        for h in range(H):
+            Q, K, V, dO = q[lo:hi, h], k[lo:hi, h], v[lo:hi, h], d_o[lo:hi, h]
+            S = (Q @ K.T) * scale
+            P = np.exp(S - S.max(axis=1, keepdims=True))
+            P /= P.sum(axis=1, keepdims=True)
+            O = P @ V
+            dv[lo:hi, h] = P.T @ dO
+            dP = dO @ V.T
+            dS = P * (dP - (dO * O).sum(axis=1, keepdims=True))
+            dq[lo:hi, h] = scale * (dS @ K)
+            dk[lo:hi, h] = scale * (dS.T @ Q)
+    return dq, dk, dv
+
+
 def gated_residual(x, o, mod, tok_sample, tok_mod, rows=None):
     """``y[t] = x[t] + gate[s, m] * O[t]`` with O viewed as [T][H*D] (head-major
     columns). Reading: the gate multiplies the attention branch and is added to

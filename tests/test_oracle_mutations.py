@@ -152,6 +152,32 @@ def _mmdit_mlp_uses_attn_mod(x, Wq, Wk, Wv, Wo, Wup, Wdown, mod_attn, mod_mlp, p
                               rope_axes, base, eps, rows, store)
 
 
+def _attn_bwd_no_delta(q, k, v, d_o, cu_seqlens, scale=None):
+    # the softmax Jacobian without its rowsum(dO * O) term
+    q, k, v, d_o = (np.asarray(a, dtype=np.float64) for a in (q, k, v, d_o))
+    cu = np.asarray(cu_seqlens)
+    dq, dk, dv = (np.zeros_like(q) for _ in range(3))
+    sc = 1.0 / math.sqrt(q.shape[2])
+    for s in range(len(cu) - 1):
+        lo, hi = int(cu[s]), int(cu[s + 1])
+        if hi == lo:
+            continue
+        for h in range(q.shape[1]):
+            S = q[lo:hi, h] @ k[lo:hi, h].T * sc
+            P = np.exp(S - S.max(1, keepdims=True))
+            P /= P.sum(1, keepdims=True)
+            dv[lo:hi, h] = P.T @ d_o[lo:hi, h]
+            dS = P * (d_o[lo:hi, h] @ v[lo:hi, h].T)
+            dq[lo:hi, h] = sc * dS @ k[lo:hi, h]
+            dk[lo:hi, h] = sc * dS.T @ q[lo:hi, h]
+    return dq, dk, dv
+
+
+def _attn_bwd_unscaled_dk(q, k, v, d_o, cu_seqlens, scale=None):
+    dq, dk, dv = mo.varlen_attention_bwd(q, k, v, d_o, cu_seqlens, scale)
+    return dq, dk * math.sqrt(np.asarray(q).shape[2]), dv
+
+
 MUTANTS = [
     ("rope sign flip", lambda: pins.check_rope_relative(_rope_sign_flip) or
      pins.check_rope_textbook_1d(_rope_sign_flip)),
@@ -175,6 +201,10 @@ MUTANTS = [
     ("GELU without the cubic term", lambda: pins.check_gelu(_gelu_no_cubic)),
     ("block: GELU after the down projection",
      lambda: pins.check_mmdit_vs_brute(_mmdit_gelu_after_down, oracle.pack_build)),
+    ("attention backward without the rowsum term",
+     lambda: pins.check_attention_bwd_vs_autograd(_attn_bwd_no_delta)),
+    ("attention backward dK without the scale",
+     lambda: pins.check_attention_bwd_finite_diff(_attn_bwd_unscaled_dk, oracle.varlen_attention)),
     ("block: MLP branch modulated by the attention vectors",
      lambda: pins.check_mmdit_branch_gates(_mmdit_mlp_uses_attn_mod, oracle.pack_build)),
 ]

@@ -215,3 +215,11 @@ def test_mmdit_rows_subset():
     rows = np.array([0, 5, 7, 13])
     part = oracle.mmdit_block_fwd(x, **ws, **mods, pack=p, H=w.H, D=w.D, rope_axes=2, rows=rows)
     assert np.array_equal(full[rows], part)
+
+
+def test_attention_bwd_vs_autograd():
+    pins.check_attention_bwd_vs_autograd(oracle.varlen_attention_bwd)
+
+
+def test_attention_bwd_finite_diff():
+    pins.check_attention_bwd_finite_diff(oracle.varlen_attention_bwd, oracle.varlen_attention)
