@@ -24,6 +24,9 @@
  *          adaptive normalization / RoPE / gating in NR-MMDiT.
  *   [cfg]  picx.dev summary, Methodology > NR-MMDiT, "Packed CFG inference":
  *          the conditional and unconditional branches packed into one forward.
+ *   [train] picx.dev summary, Methodology > Training Infrastructure and
+ *          Table 4: the packed NR-MMDiT is trained (MFU and training speedup),
+ *          so each training step also runs the backward of the block.
  * Where the pages are silent the library follows one stated reading: RoPE
  * splits head_dim evenly across the axes in whole adjacent-channel pairs, base
  * 10000 by default, leftover channels unrotated; text token j of a sample sits
@@ -148,6 +151,27 @@ mf_status mf_varlen_attn_fwd(const mf_bf16* q, const mf_bf16* k, const mf_bf16* 
                              const int32_t* pos_ids, int32_t rope_axes, float base,
                              mf_bf16* o, float* lse, void* workspace, size_t ws_bytes,
                              cudaStream_t stream);
+
+/* Backward of mf_varlen_attn_fwd [pack], [train] (q and k as the attention saw
+ * them, i.e. already rotated): for every sample s and head h, with
+ * P = softmax(scale Q K^T) rebuilt from lse,
+ *   dV = P^T dO, dP = dO V^T, dS = P * (dP - rowsum(dO * O)),
+ *   dQ = scale dS K, dK = scale dS^T Q;
+ * nothing crosses a sample boundary. q, k, v, o, d_o: [T][H][D] bf16 (o the
+ * forward's output, d_o the loss gradient with respect to it); lse: [H][T] fp32,
+ * the forward's natural-log log-sum-exp. dq, dk, dv: [T][H][D] bf16 outputs,
+ * disjoint from every input and from each other. Offsets, S, H, D and
+ * softmax_scale as for the forward. workspace (fp32 dQ accumulator and row
+ * tables): ws_bytes >= mf_attn_bwd_workspace_size(T, S, H, D), disjoint from
+ * everything else. The five products run on tcgen05 tensor cores with bf16
+ * operands and fp32 accumulation; P and dS are rounded to bf16 as operands. */
+mf_status mf_varlen_attn_bwd(const mf_bf16* q, const mf_bf16* k, const mf_bf16* v,
+                             const mf_bf16* o, const mf_bf16* d_o, const float* lse,
+                             const int32_t* cu_seqlens_d, const int32_t* cu_seqlens_h,
+                             int32_t S, int32_t H, int32_t D, float softmax_scale,
+                             mf_bf16* dq, mf_bf16* dk, mf_bf16* dv, void* workspace,
+                             size_t ws_bytes, cudaStream_t stream);
+size_t mf_attn_bwd_workspace_size(int32_t T, int32_t S, int32_t H, int32_t D);
 
 /* Gated residual [fuse]: y[t] = x[t] + gate[s,m] * o[t], o viewed as [T][H*D].
  * x, o, y: [T][hid] bf16 (y may equal x). Same id checks as mf_adaln_modulate. */

@@ -12,6 +12,7 @@ from .configs import (  # noqa: F401
     SampleDesc,
     Workload,
     bf16_bits_to_f32,
+    draw_grad_bits,
     f32_to_bf16_bits,
     make_workload,
     make_random_pack,

@@ -130,6 +130,12 @@ def _draw_normal_bf16(rng: np.random.Generator, shape) -> np.ndarray:
     return f32_to_bf16_bits(rng.standard_normal(shape, dtype=np.float32))
 
 
+def draw_grad_bits(seed: int, shape) -> np.ndarray:
+    """Seeded standard-normal bf16 bits, the upstream gradient (dO) of the
+    backward tests and bench."""
+    return _draw_normal_bf16(np.random.default_rng(seed), shape)
+
+
 def fill_arrays(w: Workload, rng: np.random.Generator) -> Workload:
     T, H, D, hid, S = w.T, w.H, w.D, w.hid, w.S
     w.x_bits = _draw_normal_bf16(rng, (T, hid))

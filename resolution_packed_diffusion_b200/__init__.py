@@ -63,6 +63,9 @@ _SIGS = {
     "mf_rope_apply": (_I, [_P, _P, _P, _I, _I, _I, _I, _F, _P, _P, _P]),
     "mf_varlen_attn_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _F, _P, _I, _F, _P, _P, _P,
                                 _SZ, _P]),
+    "mf_varlen_attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _F, _P, _P, _P, _P,
+                                _SZ, _P]),
+    "mf_attn_bwd_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "mf_gated_residual": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P, _P]),
     "mf_block_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _F, _P,
                           _P, _P, _SZ, _P]),
@@ -181,6 +184,21 @@ def mf_varlen_attn_fwd(q, k, v, cu_seqlens_d, cu_seqlens_h: np.ndarray, S: int, 
                                   _ptr(pos_ids), rope_axes, base, _ptr(o), _ptr(lse),
                                   _ptr(workspace), ws_bytes, _stream(stream)),
            "mf_varlen_attn_fwd")
+
+
+def mf_varlen_attn_bwd(q, k, v, o, d_o, lse, cu_seqlens_d, cu_seqlens_h: np.ndarray, S: int,
+                       H: int, D: int, softmax_scale: float, dq, dk, dv, workspace,
+                       ws_bytes: int, stream=None) -> None:
+    cu_h = np.ascontiguousarray(cu_seqlens_h, dtype=np.int32)
+    _check(lib.mf_varlen_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(d_o), _ptr(lse),
+                                  _ptr(cu_seqlens_d), cu_h.ctypes.data_as(_P), S, H, D,
+                                  softmax_scale, _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
+                                  ws_bytes, _stream(stream)),
+           "mf_varlen_attn_bwd")
+
+
+def mf_attn_bwd_workspace_size(T: int, S: int, H: int, D: int) -> int:
+    return int(lib.mf_attn_bwd_workspace_size(T, S, H, D))
 
 
 def mf_gated_residual(x, o, mod, tok_sample, tok_mod, T: int, S: int, hid: int, y,

@@ -1,0 +1,780 @@
+// attn_bwd.cu -- backward of the block-diagonal variable-length attention on
+// sm_100a tensor cores (tcgen05 + TMEM, operands staged by TMA).
+//
+// What it computes (picx.dev "Mage-Flow" summary, Methodology > Native-
+// Resolution MMDiT: samples of a pack attend only inside their own token
+// range; Training Infrastructure: the packed model is trained, so this
+// attention is differentiated): for every sample s and head h, with
+// P = softmax(scale Q K^T) rebuilt from the forward's log-sum-exp,
+//   dV = P^T dO,  dP = dO V^T,  dS = P * (dP - rowsum(dO * O)),
+//   dQ = scale dS K,  dK = scale dS^T Q.
+// Nothing crosses a sample boundary.
+//
+// Three kernels:
+//   bwd_rows_kernel   per query row and head: rowsum(dO * O) and the
+//                     log-sum-exp in log2 units, written into tables laid out
+//                     per 128-row query tile of a sample (rows past the
+//                     sample's end get +inf, so their P is exactly 0); zeroes
+//                     the fp32 dQ accumulator.
+//   attn_bwd_kernel   one persistent CTA per SM, 12 warps. A work item is
+//                     (sample, head, 128-key tile j); it keeps K_j, V_j in
+//                     shared memory and dK_j, dV_j in TMEM while it walks every
+//                     128-row query tile i of the sample:
+//     warp 0      TMA producer: K_j and V_j, then Q_i and dO_i into a 2-stage
+//                 ring.
+//     warp 1      tcgen05 issuer, per query tile:
+//                   S^T  = K_j Q_i^T            -> TMEM S   (keys on lanes)
+//                   dP^T = V_j dO_i^T           -> TMEM dP
+//                   dV  += P^T dO_i             (P^T read from TMEM S)
+//                   S^T of the next tile        (S is free once dV is issued)
+//                   dK  += dS^T Q_i             (dS^T from shared memory)
+//                   dQ_i = dS K_j               -> TMEM dP (free once dS exists)
+//                   dP^T of the next tile, once dQ_i has been read out.
+//                 MMAs from one thread run in issue order, so an MMA that
+//                 overwrites a TMEM region never overtakes one reading it.
+//     warps 2..3  idle.
+//     warps 4..7  one key row per thread (its TMEM lane): P^T = 2^(S^T scale
+//                 log2 e - lse) packed to bf16 into TMEM for the dV MMA; then
+//                 dS^T = scale P^T (dP^T - delta), rounded to bf16 and stored
+//                 to shared memory in the 128-byte-swizzled layout that serves
+//                 both as the K-major A operand of dK and as the MN-major A
+//                 operand of dQ.
+//     warps 8..11 one query row per thread: dQ_i from TMEM added to the fp32
+//                 accumulator in global memory (vector reductions); at the end
+//                 of the item, dK_j and dV_j rounded to bf16 and stored.
+//   bwd_dq_kernel     the fp32 dQ accumulator rounded to bf16.
+// TMEM (512 columns): S/P | dP/dQ | dV | dK.
+//
+// Every wait is bounded (mbar_wait); on expiry the CTA records MF_ERR_TIMEOUT,
+// lets its in-flight copies and MMAs finish, frees TMEM and returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <vector>
+
+#include "attn_bwd_internal.h"
+#include "mf_internal.h"
+#include "mf_ptx.cuh"
+
+namespace mf {
+
+namespace {
+
+constexpr int BM = 128;            // query rows per tile
+constexpr int BN = 128;            // key rows per work item
+constexpr int NUM_THREADS = 384;   // TMA, MMA, 2 idle, 4 softmax / dS, 4 dQ / epilogue
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TM_S = 0;       // S^T (fp32), then P^T (bf16 pairs, first 64 columns)
+constexpr uint32_t TM_DP = 128;    // dP^T (fp32), then dQ (fp32, D columns)
+constexpr uint32_t TM_DV = 256;    // dV accumulator (D columns); dK follows at 256 + D
+constexpr int BOX_BYTES = 128 * 128;  // one TMA box: 128 rows x 64 bf16, 128-byte swizzle
+constexpr int NQD = 2;             // Q / dO ring stages
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D>
+struct BwdLayout {
+  static constexpr int kBoxes = D / 64;
+  static constexpr int TILE_BYTES = 128 * D * 2;
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + TILE_BYTES;
+  static constexpr int OFF_Q = OFF_V + TILE_BYTES;            // NQD stages
+  static constexpr int OFF_DO = OFF_Q + NQD * TILE_BYTES;     // NQD stages
+  static constexpr int OFF_DS = OFF_DO + NQD * TILE_BYTES;    // dS^T: 2 boxes of 64 queries
+  static constexpr int DS_BYTES = BN * BM * 2;
+  static constexpr int OFF_BAR = OFF_DS + DS_BYTES;
+  static constexpr int B_KV_FULL = 0, B_KV_EMPTY = 1;
+  static constexpr int B_QD_FULL = 2;                  // NQD
+  static constexpr int B_QD_EMPTY = B_QD_FULL + NQD;   // NQD
+  static constexpr int B_S_FULL = B_QD_EMPTY + NQD;
+  static constexpr int B_P_FULL = B_S_FULL + 1;        // one arrival per softmax warp
+  static constexpr int B_DP_FULL = B_P_FULL + 1;
+  static constexpr int B_DS_FULL = B_DP_FULL + 1;      // one arrival per softmax warp
+  static constexpr int B_DS_EMPTY = B_DS_FULL + 1;
+  static constexpr int B_DQ_FULL = B_DS_EMPTY + 1;
+  static constexpr int B_DQ_EMPTY = B_DQ_FULL + 1;     // one arrival per dQ warp
+  static constexpr int B_ACC_FULL = B_DQ_EMPTY + 1;
+  static constexpr int B_ACC_EMPTY = B_ACC_FULL + 1;   // one arrival per dQ warp
+  static constexpr int B_DRAIN = B_ACC_EMPTY + 1;
+  static constexpr int NUM_BARS = B_DRAIN + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;  // tmem slot, abort flag
+  static constexpr int END = OFF_MISC + 16;
+  // + alignment slack; at least 120 KB so that two CTAs never share an SM (each
+  // holds all 512 TMEM columns)
+  static constexpr int SMEM_BYTES = (END + 1024) > 120 * 1024 ? (END + 1024) : 120 * 1024;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget of one CTA");
+
+  __device__ static uint32_t arrivals(int i) {
+    return (i == B_P_FULL || i == B_DS_FULL || i == B_DQ_EMPTY || i == B_ACC_EMPTY) ? 4u : 1u;
+  }
+};
+
+// Pack geometry from the host offsets, passed by value (about 8 KB).
+struct BwdArgs {
+  mf_bf16* dk;              // [T][H][D]
+  mf_bf16* dv;              // [T][H][D]
+  float* dq_acc;            // [T][H][D] fp32, zeroed by bwd_rows_kernel
+  const float* lse_tab;     // [H][tiles][128] lse * log2(e); +inf past the sample's end
+  const float* delta_tab;   // [H][tiles][128] rowsum(dO * O); 0 past the sample's end
+  int32_t S, T, H, tiles, total_items;
+  float scale_log2;         // softmax_scale * log2(e)
+  float scale;
+  KernelCtl ctl;
+  int32_t cu[MF_MAX_SAMPLES + 1];
+  int32_t order[MF_MAX_SAMPLES];       // samples, longest first
+  int32_t istart[MF_MAX_SAMPLES + 1];  // first item of order[r]
+  int32_t tile0[MF_MAX_SAMPLES + 1];   // first query tile of sample s (pack order)
+};
+
+struct BwdItem {
+  int32_t s, h, j, kv0, n, nq;
+};
+
+__device__ __forceinline__ BwdItem decode_item(int w, const BwdArgs& a) {
+  int lo = 0, hi = a.S - 1;  // largest r with istart[r] <= w
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (a.istart[mid] <= w) lo = mid; else hi = mid - 1;
+  }
+  BwdItem it;
+  it.s = a.order[lo];
+  const int local = w - a.istart[lo];
+  it.kv0 = a.cu[it.s];
+  it.n = a.cu[it.s + 1] - it.kv0;
+  const int nk = (it.n + BN - 1) / BN;
+  it.h = local / nk;
+  it.j = local - it.h * nk;
+  it.nq = (it.n + BM - 1) / BM;
+  return it;
+}
+
+// k-th item of CTA b among G: rounds of G items in longest-first order, dealt
+// forwards in even rounds and backwards in odd ones.
+__device__ __forceinline__ int snake_item(int k, int b, int G) {
+  return k * G + ((k & 1) ? (G - 1 - b) : b);
+}
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const KernelCtl& ctl,
+                                          volatile int* abort_flag) {
+  const bool ok = mbar_wait(bar, parity, ctl, abort_flag);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Bounded wait used while winding down: ignores the abort flag.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > limit_ns) return;
+  }
+}
+
+// Four fp32 additions into global memory, no value returned.
+__device__ __forceinline__ void red_add_v4(float* dst, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a), "f"(b),
+               "f"(c), "f"(d)
+               : "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    attn_bwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                    const __grid_constant__ CUtensorMap tmap_k,
+                    const __grid_constant__ CUtensorMap tmap_v,
+                    const __grid_constant__ CUtensorMap tmap_do,
+                    const __grid_constant__ BwdArgs args) {
+  using L = BwdLayout<D>;
+  constexpr uint32_t TM_DK = TM_DV + D;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < L::NUM_BARS; ++i) mbar_init(&bars[i], L::arrivals(i));
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_map(&tmap_q);
+    tma_prefetch_map(&tmap_k);
+    tma_prefetch_map(&tmap_v);
+    tma_prefetch_map(&tmap_do);
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int total = args.total_items;
+  const KernelCtl& ctl = args.ctl;
+
+  uint8_t* sK = smem + L::OFF_K;
+  uint8_t* sV = smem + L::OFF_V;
+  uint8_t* sQ = smem + L::OFF_Q;
+  uint8_t* sDO = smem + L::OFF_DO;
+
+  if (warp == 0) {
+    // ============================================================ TMA producer
+    if (lane == 0) {
+      uint32_t kv_issued = 0, c = 0;  // K/V loads and Q/dO stages issued so far
+      bool ok = true;
+      for (int k = 0, w = snake_item(0, blockIdx.x, gridDim.x); w < total && ok;
+           w = snake_item(++k, blockIdx.x, gridDim.x)) {
+        const BwdItem it = decode_item(w, args);
+        if (!mbar_wait(&bars[L::B_KV_EMPTY], (kv_issued & 1) ^ 1, ctl, abort_flag)) break;
+        mbar_expect_tx(&bars[L::B_KV_FULL], 2 * L::TILE_BYTES);
+        const int krow = it.kv0 + it.j * BN;
+#pragma unroll
+        for (int b = 0; b < L::kBoxes; ++b) {
+          tma_load_2d(sK + b * BOX_BYTES, &tmap_k, &bars[L::B_KV_FULL], it.h * D + 64 * b, krow);
+          tma_load_2d(sV + b * BOX_BYTES, &tmap_v, &bars[L::B_KV_FULL], it.h * D + 64 * b, krow);
+        }
+        ++kv_issued;
+        for (int i = 0; i < it.nq; ++i) {
+          const int st = c % NQD;
+          if (!mbar_wait(&bars[L::B_QD_EMPTY + st], ((c / NQD) & 1) ^ 1, ctl, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(&bars[L::B_QD_FULL + st], 2 * L::TILE_BYTES);
+          const int qrow = it.kv0 + i * BM;
+#pragma unroll
+          for (int b = 0; b < L::kBoxes; ++b) {
+            tma_load_2d(sQ + st * L::TILE_BYTES + b * BOX_BYTES, &tmap_q, &bars[L::B_QD_FULL + st],
+                        it.h * D + 64 * b, qrow);
+            tma_load_2d(sDO + st * L::TILE_BYTES + b * BOX_BYTES, &tmap_do,
+                        &bars[L::B_QD_FULL + st], it.h * D + 64 * b, qrow);
+          }
+          ++c;
+        }
+      }
+      // Let every copy this thread started land before the CTA can exit.
+      const uint64_t lim = ctl.wait_limit_ns;
+      if (kv_issued > 0) drain_wait(&bars[L::B_KV_FULL], (kv_issued - 1) & 1, lim);
+      for (int st = 0; st < NQD; ++st)
+        if (c > static_cast<uint32_t>(st)) {
+          const uint32_t last = c - 1 - ((c - 1 - st) % NQD);
+          drain_wait(&bars[L::B_QD_FULL + st], (last / NQD) & 1, lim);
+        }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ============================================================ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC_T = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T
+      constexpr uint32_t IDESC_KV = idesc_bf16_f32(128, D, 0, 1);   // dV, dK
+      constexpr uint32_t IDESC_Q = idesc_bf16_f32(128, D, 1, 1);    // dQ
+      // K-major views (rows x 64-column boxes, a 16-element K step is 32 B inside
+      // a box) and MN-major views (LBO = distance between 64-column boxes, a
+      // 16-row K step is 2048 B) of the same tiles.
+      const uint64_t k_km = sdesc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t v_km = sdesc_sw128(smem_u32(sV), 16, 1024);
+      const uint64_t q_km = sdesc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t do_km = sdesc_sw128(smem_u32(sDO), 16, 1024);
+      const uint64_t k_mn = sdesc_sw128(smem_u32(sK), BOX_BYTES, 1024);
+      const uint64_t q_mn = sdesc_sw128(smem_u32(sQ), BOX_BYTES, 1024);
+      const uint64_t do_mn = sdesc_sw128(smem_u32(sDO), BOX_BYTES, 1024);
+      const uint64_t ds_km = sdesc_sw128(smem_u32(smem + L::OFF_DS), 16, 1024);
+      const uint64_t ds_mn = sdesc_sw128(smem_u32(smem + L::OFF_DS), BOX_BYTES, 1024);
+      auto stage_off = [](int st) -> uint64_t {
+        return static_cast<uint64_t>((st * L::TILE_BYTES) >> 4);
+      };
+      auto km_step = [](int kk) -> uint64_t {
+        return static_cast<uint64_t>(((kk >> 2) * BOX_BYTES + (kk & 3) * 32) >> 4);
+      };
+      auto mn_step = [](int kk) -> uint64_t { return static_cast<uint64_t>((kk * 2048) >> 4); };
+      // X^T = A B^T over the head dimension: A = K or V (keys), B = Q or dO.
+      auto issue_t = [&](uint32_t dcol, uint64_t a, uint64_t b) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_ss(tmem + dcol, a + km_step(kk), b + km_step(kk), IDESC_T, kk > 0 ? 1u : 0u);
+      };
+      auto wait = [&](int bar, uint32_t parity) -> bool {
+        return mbar_wait(&bars[bar], parity, ctl, abort_flag);
+      };
+      uint32_t c = 0;  // query tiles processed (global over items)
+      int n_item = 0;
+      bool ok = true;
+      for (int k = 0, w = snake_item(0, blockIdx.x, gridDim.x); w < total && ok;
+           w = snake_item(++k, blockIdx.x, gridDim.x), ++n_item) {
+        const BwdItem it = decode_item(w, args);
+        if (!wait(L::B_KV_FULL, n_item & 1)) break;
+        if (!wait(L::B_QD_FULL + c % NQD, (c / NQD) & 1)) break;
+        tc_fence_after();
+        issue_t(TM_S, k_km, q_km + stage_off(c % NQD));
+        umma_commit(&bars[L::B_S_FULL]);
+        // dP^T lands where the previous tile's dQ sits: wait until it is read out
+        if (!wait(L::B_DQ_EMPTY, (c & 1) ^ 1)) break;
+        tc_fence_after();
+        issue_t(TM_DP, v_km, do_km + stage_off(c % NQD));
+        umma_commit(&bars[L::B_DP_FULL]);
+        for (int i = 0; i < it.nq; ++i, ++c) {
+          const int st = c % NQD;
+          const bool more = i + 1 < it.nq;
+          if (!wait(L::B_P_FULL, c & 1)) { ok = false; break; }
+          // the previous item's dK / dV must have been stored before this item
+          // starts accumulating over them
+          if (i == 0 && !wait(L::B_ACC_EMPTY, (n_item & 1) ^ 1)) { ok = false; break; }
+          tc_fence_after();
+          // dV += P^T dO_i: A = P^T from TMEM (8 columns per 16 queries)
+#pragma unroll
+          for (int kk = 0; kk < BM / 16; ++kk)
+            umma_ts(tmem + TM_DV, tmem + TM_S + kk * 8, do_mn + stage_off(st) + mn_step(kk),
+                    IDESC_KV, (i > 0 || kk > 0) ? 1u : 0u);
+          if (more) {
+            if (!wait(L::B_QD_FULL + (c + 1) % NQD, ((c + 1) / NQD) & 1)) { ok = false; break; }
+            tc_fence_after();
+            issue_t(TM_S, k_km, q_km + stage_off((c + 1) % NQD));
+            umma_commit(&bars[L::B_S_FULL]);
+          }
+          if (!wait(L::B_DS_FULL, c & 1)) { ok = false; break; }
+          tc_fence_after();
+          // dK += dS^T Q_i (dS^T K-major); dQ_i = dS K_j (dS^T read MN-major)
+#pragma unroll
+          for (int kk = 0; kk < BM / 16; ++kk)
+            umma_ss(tmem + TM_DK, ds_km + km_step(kk), q_mn + stage_off(st) + mn_step(kk),
+                    IDESC_KV, (i > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk)
+            umma_ss(tmem + TM_DP, ds_mn + mn_step(kk), k_mn + mn_step(kk), IDESC_Q,
+                    kk > 0 ? 1u : 0u);
+          umma_commit(&bars[L::B_DQ_FULL]);
+          umma_commit(&bars[L::B_DS_EMPTY]);
+          umma_commit(&bars[L::B_QD_EMPTY + st]);
+          if (more) {
+            if (!wait(L::B_DQ_EMPTY, c & 1)) { ok = false; break; }
+            tc_fence_after();
+            issue_t(TM_DP, v_km, do_km + stage_off((c + 1) % NQD));
+            umma_commit(&bars[L::B_DP_FULL]);
+          }
+        }
+        if (!ok) break;
+        umma_commit(&bars[L::B_KV_EMPTY]);
+        umma_commit(&bars[L::B_ACC_FULL]);
+      }
+      // every MMA this thread issued completes before TMEM is released
+      umma_commit(&bars[L::B_DRAIN]);
+      drain_wait(&bars[L::B_DRAIN], 0, ctl.wait_limit_ns);
+    }
+    __syncwarp();
+  } else if (warp >= 4 && warp < 8) {
+    // ============================================================ P and dS
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;  // key row of the tile (TMEM lane)
+    const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t s_col = tmem + lane_base + TM_S;
+    const uint32_t dp_col = tmem + lane_base + TM_DP;
+    uint8_t* ds_row = smem + L::OFF_DS + r * 128;
+    const int sw = r & 7;
+    const float scale_log2 = args.scale_log2;
+    const float scale = args.scale;
+    uint32_t c = 0;
+    bool ok = true;
+    for (int k = 0, w = snake_item(0, blockIdx.x, gridDim.x); w < total && ok;
+         w = snake_item(++k, blockIdx.x, gridDim.x)) {
+      const BwdItem it = decode_item(w, args);
+      const bool key_valid = it.j * BN + r < it.n;
+      for (int i = 0; i < it.nq; ++i, ++c) {
+        const size_t tab = (static_cast<size_t>(it.h) * args.tiles + args.tile0[it.s] + i) * BM;
+        const float4* lt = reinterpret_cast<const float4*>(args.lse_tab + tab);
+        const float4* dt = reinterpret_cast<const float4*>(args.delta_tab + tab);
+        if (!warp_wait(&bars[L::B_S_FULL], c & 1, ctl, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        // P^T row: 2^(s * scale * log2 e - lse_log2[q]) for the tile's 128 queries
+        uint32_t pp[BM / 2];
+#pragma unroll
+        for (int cc = 0; cc < BM; cc += 32) {
+          uint32_t sr[32];
+          tmem_ld32(s_col + cc, sr);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const float4 lv = __ldg(lt + cc / 4 + e4);
+            const float p0 = ex2_approx(fmaf(__uint_as_float(sr[4 * e4 + 0]), scale_log2, -lv.x));
+            const float p1 = ex2_approx(fmaf(__uint_as_float(sr[4 * e4 + 1]), scale_log2, -lv.y));
+            const float p2 = ex2_approx(fmaf(__uint_as_float(sr[4 * e4 + 2]), scale_log2, -lv.z));
+            const float p3 = ex2_approx(fmaf(__uint_as_float(sr[4 * e4 + 3]), scale_log2, -lv.w));
+            pp[cc / 2 + 2 * e4] = pack_bf16x2(p0, p1);
+            pp[cc / 2 + 2 * e4 + 1] = pack_bf16x2(p2, p3);
+          }
+        }
+        if (!key_valid) {
+#pragma unroll
+          for (int e = 0; e < BM / 2; ++e) pp[e] = 0u;
+        }
+        tmem_st32(s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(&pp[0]));
+        tmem_st32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&pp[32]));
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[L::B_P_FULL]);
+        // dS^T row = scale * P^T * (dP^T - delta), once dP^T is in TMEM and the
+        // previous tile's dK / dQ MMAs have read the shared dS^T buffer
+        if (!warp_wait(&bars[L::B_DP_FULL], c & 1, ctl, abort_flag)) { ok = false; break; }
+        if (!warp_wait(&bars[L::B_DS_EMPTY], (c & 1) ^ 1, ctl, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int cc = 0; cc < BM; cc += 32) {
+          uint32_t dr[32];
+          tmem_ld32(dp_col + cc, dr);
+          tmem_ld_wait();
+          uint32_t packed[16];
+#pragma unroll
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const float4 dl = __ldg(dt + cc / 4 + e4);
+            const uint32_t pa = pp[cc / 2 + 2 * e4], pb = pp[cc / 2 + 2 * e4 + 1];
+            const float ds0 = __uint_as_float(pa << 16) * (__uint_as_float(dr[4 * e4 + 0]) - dl.x);
+            const float ds1 = __uint_as_float(pa & 0xFFFF0000u) * (__uint_as_float(dr[4 * e4 + 1]) - dl.y);
+            const float ds2 = __uint_as_float(pb << 16) * (__uint_as_float(dr[4 * e4 + 2]) - dl.z);
+            const float ds3 = __uint_as_float(pb & 0xFFFF0000u) * (__uint_as_float(dr[4 * e4 + 3]) - dl.w);
+            packed[2 * e4] = pack_bf16x2(ds0 * scale, ds1 * scale);
+            packed[2 * e4 + 1] = pack_bf16x2(ds2 * scale, ds3 * scale);
+          }
+          // queries cc..cc+31: box cc / 64, 16-byte chunks (cc % 64) / 8 + u,
+          // placed at chunk ^ (row % 8) by the 128-byte swizzle
+          uint8_t* box_row = ds_row + (cc / 64) * BOX_BYTES;
+          const int chunk0 = (cc % 64) / 8;
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            *reinterpret_cast<uint4*>(box_row + (((chunk0 + u) ^ sw) << 4)) =
+                make_uint4(packed[4 * u], packed[4 * u + 1], packed[4 * u + 2], packed[4 * u + 3]);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[L::B_DS_FULL]);
+      }
+    }
+  } else if (warp >= 8) {
+    // ============================================================ dQ, dK, dV out
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;  // TMEM lane: query row (dQ) or key row (dK, dV)
+    const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t dq_col = tmem + lane_base + TM_DP;
+    const uint32_t dv_col = tmem + lane_base + TM_DV;
+    const uint32_t dk_col = tmem + lane_base + TM_DK;
+    const int hid = args.H * D;
+    uint32_t c = 0;
+    int n_item = 0;
+    bool ok = true;
+    for (int k = 0, w = snake_item(0, blockIdx.x, gridDim.x); w < total && ok;
+         w = snake_item(++k, blockIdx.x, gridDim.x), ++n_item) {
+      const BwdItem it = decode_item(w, args);
+      for (int i = 0; i < it.nq; ++i, ++c) {
+        if (!warp_wait(&bars[L::B_DQ_FULL], c & 1, ctl, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const int qi = i * BM + row;
+        float* dst = args.dq_acc + static_cast<size_t>(it.kv0 + qi) * hid + it.h * D;
+#pragma unroll
+        for (int cc = 0; cc < D; cc += 32) {
+          uint32_t a[32];
+          tmem_ld32(dq_col + cc, a);
+          tmem_ld_wait();
+          if (cc + 32 == D) {
+            // the whole dQ row is in registers: hand the TMEM region back
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[L::B_DQ_EMPTY]);
+          }
+          if (qi < it.n) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+              red_add_v4(dst + cc + e, __uint_as_float(a[e]), __uint_as_float(a[e + 1]),
+                         __uint_as_float(a[e + 2]), __uint_as_float(a[e + 3]));
+          }
+        }
+      }
+      if (!ok) break;
+      if (!warp_wait(&bars[L::B_ACC_FULL], n_item & 1, ctl, abort_flag)) break;
+      tc_fence_after();
+      const int ki = it.j * BN + row;
+      const size_t off = static_cast<size_t>(it.kv0 + ki) * hid + it.h * D;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t col = which ? dk_col : dv_col;
+        mf_bf16* out = (which ? args.dk : args.dv) + off;
+#pragma unroll
+        for (int cc = 0; cc < D; cc += 32) {
+          uint32_t a[32];
+          tmem_ld32(col + cc, a);
+          tmem_ld_wait();
+          if (ki < it.n) {
+            uint4* o4 = reinterpret_cast<uint4*>(out + cc);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              o4[u] = make_uint4(
+                  pack_bf16x2(__uint_as_float(a[8 * u + 0]), __uint_as_float(a[8 * u + 1])),
+                  pack_bf16x2(__uint_as_float(a[8 * u + 2]), __uint_as_float(a[8 * u + 3])),
+                  pack_bf16x2(__uint_as_float(a[8 * u + 4]), __uint_as_float(a[8 * u + 5])),
+                  pack_bf16x2(__uint_as_float(a[8 * u + 6]), __uint_as_float(a[8 * u + 7])));
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[L::B_ACC_EMPTY]);
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+// Row tables of the backward and zeroing of the dQ accumulator.
+struct RowsArgs {
+  const mf_bf16* o;
+  const mf_bf16* d_o;
+  const float* lse;   // [H][T] natural log
+  float* lse_tab;
+  float* delta_tab;
+  float* dq_acc;
+  int32_t S, T, H, tiles;
+  int32_t cu[MF_MAX_SAMPLES + 1];
+  int32_t tile0[MF_MAX_SAMPLES + 1];
+};
+
+// Block (g, h): query tile g of the pack, head h; D / 8 threads per row, each
+// with 8 channels (one 16-byte load of dO and of O).
+template <int D>
+__global__ void __launch_bounds__(256) bwd_rows_kernel(const __grid_constant__ RowsArgs a) {
+  constexpr int kLanes = D / 8;
+  constexpr int kRowsPerPass = 256 / kLanes;
+  const int g = blockIdx.x, h = blockIdx.y;
+  int lo = 0, hi = a.S - 1;  // the sample holding tile g: largest s with tile0[s] <= g
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (a.tile0[mid] <= g) lo = mid; else hi = mid - 1;
+  }
+  const int s = lo;
+  const int n = a.cu[s + 1] - a.cu[s];
+  const int base = (g - a.tile0[s]) * BM;  // first row of the tile inside the sample
+  const int part = threadIdx.x % kLanes;
+  const int hid = a.H * D;
+  for (int q = threadIdx.x / kLanes; q < BM; q += kRowsPerPass) {
+    const bool valid = base + q < n;
+    const int t = a.cu[s] + base + q;
+    float dot = 0.f;
+    if (valid) {
+      const size_t off = static_cast<size_t>(t) * hid + h * D + part * 8;
+      const uint4 ov = __ldg(reinterpret_cast<const uint4*>(a.o + off));
+      const uint4 gv = __ldg(reinterpret_cast<const uint4*>(a.d_o + off));
+      const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w};
+      const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        dot = fmaf(__uint_as_float(ow[e] << 16), __uint_as_float(gw[e] << 16), dot);
+        dot = fmaf(__uint_as_float(ow[e] & 0xFFFF0000u), __uint_as_float(gw[e] & 0xFFFF0000u), dot);
+      }
+      float4* z = reinterpret_cast<float4*>(a.dq_acc + off);
+      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int m = kLanes / 2; m > 0; m >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, m);
+    if (part == 0) {
+      const size_t tab = (static_cast<size_t>(h) * a.tiles + g) * BM + q;
+      a.delta_tab[tab] = valid ? dot : 0.f;
+      a.lse_tab[tab] = valid ? __ldg(a.lse + static_cast<size_t>(h) * a.T + t) * kLog2e : INFINITY;
+    }
+  }
+}
+
+// dq[i] = bf16(dq_acc[i]), eight elements per thread and step.
+__global__ void __launch_bounds__(256) bwd_dq_kernel(const float* __restrict__ acc,
+                                                     mf_bf16* __restrict__ dq, size_t n8) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n8;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(acc) + 2 * i);
+    const float4 b = __ldg(reinterpret_cast<const float4*>(acc) + 2 * i + 1);
+    reinterpret_cast<uint4*>(dq)[i] = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w),
+                                                 pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
+  }
+}
+
+// ---------------------------------------------------------------- host side
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// [T][H*D] bf16 as a 2D tensor; box = 64 columns x 128 rows, 128-byte swizzle;
+// rows past T read as zeros.
+bool make_map(CUtensorMap* map, const void* base, int32_t T, int32_t cols) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(T)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+size_t round256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
+
+size_t tab_bytes(int32_t T, int32_t S, int32_t H) {
+  // sum over samples of ceil(n / 128) <= T / 128 + S
+  return round256(static_cast<size_t>(H) * (static_cast<size_t>(T) / BM + S + 1) * BM * 4);
+}
+
+template <int D>
+cudaError_t launch_main(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                        const CUtensorMap& mdo, const BwdArgs& a, int grid, cudaStream_t st) {
+  constexpr int smem = BwdLayout<D>::SMEM_BYTES;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(attn_bwd_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  attn_bwd_kernel<D><<<grid, NUM_THREADS, smem, st>>>(mq, mk, mv, mdo, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int32_t bwd_query_tiles(const int32_t* cu_h, int32_t S) {
+  int64_t n = 0;
+  for (int32_t s = 0; s < S; ++s) n += (static_cast<int64_t>(cu_h[s + 1] - cu_h[s]) + BM - 1) / BM;
+  return static_cast<int32_t>(n);
+}
+
+size_t attn_bwd_workspace_bytes(int32_t T, int32_t S, int32_t H, int32_t D) {
+  return round256(static_cast<size_t>(T) * H * D * 4) + 2 * tab_bytes(T, S, H) + 256;
+}
+
+cudaError_t launch_attention_bwd(const mf_bf16* q, const mf_bf16* k, const mf_bf16* v,
+                                 const mf_bf16* o, const mf_bf16* d_o, const float* lse,
+                                 const int32_t* cu_seqlens_d, const int32_t* cu_seqlens_h,
+                                 int32_t S, int32_t T, int32_t H, int32_t D, float softmax_scale,
+                                 mf_bf16* dq, mf_bf16* dk, mf_bf16* dv, void* workspace,
+                                 const KernelCtl& ctl, cudaStream_t st) {
+  (void)cu_seqlens_d;  // the kernels take the pack geometry from the host offsets
+  if (T == 0) return cudaSuccess;
+  const uintptr_t w0 = (reinterpret_cast<uintptr_t>(workspace) + 255) & ~static_cast<uintptr_t>(255);
+  float* dq_acc = reinterpret_cast<float*>(w0);
+  float* lse_tab = reinterpret_cast<float*>(w0 + round256(static_cast<size_t>(T) * H * D * 4));
+  float* delta_tab = reinterpret_cast<float*>(reinterpret_cast<uintptr_t>(lse_tab) + tab_bytes(T, S, H));
+  const int32_t tiles = bwd_query_tiles(cu_seqlens_h, S);
+
+  static thread_local RowsArgs ra;
+  ra.o = o;
+  ra.d_o = d_o;
+  ra.lse = lse;
+  ra.lse_tab = lse_tab;
+  ra.delta_tab = delta_tab;
+  ra.dq_acc = dq_acc;
+  ra.S = S;
+  ra.T = T;
+  ra.H = H;
+  ra.tiles = tiles;
+  int32_t acc = 0;
+  for (int32_t s = 0; s <= S; ++s) {
+    ra.cu[s] = cu_seqlens_h[s];
+    ra.tile0[s] = acc;
+    if (s < S) acc += (cu_seqlens_h[s + 1] - cu_seqlens_h[s] + BM - 1) / BM;
+  }
+  const dim3 rgrid(static_cast<unsigned>(tiles), static_cast<unsigned>(H));
+  if (D == 128) bwd_rows_kernel<128><<<rgrid, 256, 0, st>>>(ra);
+  else if (D == 64) bwd_rows_kernel<64><<<rgrid, 256, 0, st>>>(ra);
+  else return cudaErrorInvalidValue;
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+
+  CUtensorMap mq, mk, mv, mdo;
+  const int32_t cols = H * D;
+  if (!make_map(&mq, q, T, cols) || !make_map(&mk, k, T, cols) || !make_map(&mv, v, T, cols) ||
+      !make_map(&mdo, d_o, T, cols))
+    return cudaErrorInvalidValue;
+  static thread_local BwdArgs a;
+  a.dk = dk;
+  a.dv = dv;
+  a.dq_acc = dq_acc;
+  a.lse_tab = lse_tab;
+  a.delta_tab = delta_tab;
+  a.S = S;
+  a.T = T;
+  a.H = H;
+  a.tiles = tiles;
+  a.scale = softmax_scale;
+  a.scale_log2 = softmax_scale * kLog2e;
+  a.ctl = ctl;
+  std::vector<int32_t> order(S);
+  for (int32_t i = 0; i < S; ++i) order[i] = i;
+  std::stable_sort(order.begin(), order.end(), [&](int32_t x, int32_t y) {
+    return (cu_seqlens_h[x + 1] - cu_seqlens_h[x]) > (cu_seqlens_h[y + 1] - cu_seqlens_h[y]);
+  });
+  int32_t items = 0;
+  for (int32_t r = 0; r < S; ++r) {
+    a.order[r] = order[r];
+    a.istart[r] = items;
+    const int32_t n = cu_seqlens_h[order[r] + 1] - cu_seqlens_h[order[r]];
+    items += ((n + BN - 1) / BN) * H;
+  }
+  a.istart[S] = items;
+  for (int32_t s = 0; s <= S; ++s) {
+    a.cu[s] = ra.cu[s];
+    a.tile0[s] = ra.tile0[s];
+  }
+  a.total_items = items;
+  if (items > 0) {
+    const int sms = sm_count();
+    const int grid = items < sms ? items : sms;
+    e = D == 128 ? launch_main<128>(mq, mk, mv, mdo, a, grid, st)
+                 : launch_main<64>(mq, mk, mv, mdo, a, grid, st);
+    if (e != cudaSuccess) return e;
+  }
+  const size_t n8 = static_cast<size_t>(T) * H * D / 8;
+  const int sms = sm_count();
+  const size_t want = (n8 + 255) / 256;
+  const unsigned cgrid = static_cast<unsigned>(want < static_cast<size_t>(sms) * 8 ? want : sms * 8);
+  bwd_dq_kernel<<<cgrid, 256, 0, st>>>(dq_acc, dq, n8);
+  return cudaGetLastError();
+}
+
+}  // namespace mf

@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "mf.h"
+#include "attn_bwd_internal.h"
 #include "cfg_internal.h"
 #include "gemm_internal.h"
 #include "mf_internal.h"
@@ -276,6 +277,53 @@ mf_status mf_varlen_attn_fwd(const mf_bf16* q, const mf_bf16* k, const mf_bf16* 
   ep.lse = lse;
   return cuda_status(timed_attention(qa, ka, v, cu_seqlens_d, cu_seqlens_h, S, T, H, D, softmax_scale, ep,
                                      count_items(cu_seqlens_h, S, H), ctl, stream));
+}
+
+size_t mf_attn_bwd_workspace_size(int32_t T, int32_t S, int32_t H, int32_t D) {
+  if (T < 0 || S < 1 || H < 1 || D < 1) return 0;
+  return attn_bwd_workspace_bytes(T, S, H, D);
+}
+
+mf_status mf_varlen_attn_bwd(const mf_bf16* q, const mf_bf16* k, const mf_bf16* v,
+                             const mf_bf16* o, const mf_bf16* d_o, const float* lse,
+                             const int32_t* cu_seqlens_d, const int32_t* cu_seqlens_h, int32_t S,
+                             int32_t H, int32_t D, float softmax_scale, mf_bf16* dq, mf_bf16* dk,
+                             mf_bf16* dv, void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  if (S < 1 || S > MF_MAX_SAMPLES || H < 1 || H > 128 || !std::isfinite(softmax_scale) ||
+      !(softmax_scale > 0.f))
+    return MF_ERR_INVALID;
+  if (!valid_head_dim(D)) return MF_ERR_UNSUPPORTED;
+  int32_t T = 0;
+  if (!check_offsets(cu_seqlens_h, S, &T)) return MF_ERR_INVALID;
+  if (T == 0) return MF_OK;
+  const mf_bf16* ins[5] = {q, k, v, o, d_o};
+  mf_bf16* outs[3] = {dq, dk, dv};
+  for (const mf_bf16* p : ins)
+    if (p == nullptr || !aligned16(p)) return MF_ERR_INVALID;
+  for (mf_bf16* p : outs)
+    if (p == nullptr || !aligned16(p)) return MF_ERR_INVALID;
+  if (lse == nullptr || !aligned16(lse) || cu_seqlens_d == nullptr) return MF_ERR_INVALID;
+  if (workspace == nullptr || !aligned16(workspace) ||
+      ws_bytes < mf_attn_bwd_workspace_size(T, S, H, D))
+    return MF_ERR_INVALID;
+  const size_t bytes = static_cast<size_t>(T) * H * D * 2;
+  const size_t ws = mf_attn_bwd_workspace_size(T, S, H, D);
+  for (int i = 0; i < 3; ++i) {
+    for (const mf_bf16* p : ins)
+      if (overlap(outs[i], bytes, p, bytes)) return MF_ERR_INVALID;
+    for (int j = i + 1; j < 3; ++j)
+      if (overlap(outs[i], bytes, outs[j], bytes)) return MF_ERR_INVALID;
+    if (overlap(outs[i], bytes, workspace, ws) || overlap(outs[i], bytes, lse, static_cast<size_t>(T) * H * 4))
+      return MF_ERR_INVALID;
+  }
+  for (const mf_bf16* p : ins)
+    if (overlap(p, bytes, workspace, ws)) return MF_ERR_INVALID;
+  if (overlap(lse, static_cast<size_t>(T) * H * 4, workspace, ws)) return MF_ERR_INVALID;
+  KernelCtl ctl;
+  if (cudaError_t ge = get_ctl(&ctl); ge != cudaSuccess) return cuda_status(ge);
+  return cuda_status(launch_attention_bwd(q, k, v, o, d_o, lse, cu_seqlens_d, cu_seqlens_h, S, T,
+                                          H, D, softmax_scale, dq, dk, dv, workspace, ctl,
+                                          stream));
 }
 
 mf_status mf_gated_residual(const mf_bf16* x, const mf_bf16* o, const float* mod,
