@@ -16,7 +16,7 @@
 //                     per 128-row query tile of a sample (rows past the
 //                     sample's end get +inf, so their P is exactly 0); zeroes
 //                     the fp32 dQ accumulator.
-//   attn_bwd_kernel   one persistent CTA per SM, 12 warps. A work item is
+//   attn_bwd_kernel   one persistent CTA per SM, 16 warps. A work item is
 //                     (sample, head, 128-key tile j); it keeps K_j, V_j in
 //                     shared memory and dK_j, dV_j in TMEM while it walks every
 //                     128-row query tile i of the sample:
@@ -33,15 +33,18 @@
 //                 MMAs from one thread run in issue order, so an MMA that
 //                 overwrites a TMEM region never overtakes one reading it.
 //     warps 2..3  idle.
-//     warps 4..7  one key row per thread (its TMEM lane): P^T = 2^(S^T scale
-//                 log2 e - lse) packed to bf16 into TMEM for the dV MMA; then
-//                 dS^T = scale P^T (dP^T - delta), rounded to bf16 and stored
-//                 to shared memory in the 128-byte-swizzled layout that serves
-//                 both as the K-major A operand of dK and as the MN-major A
-//                 operand of dQ.
-//     warps 8..11 one query row per thread: dQ_i from TMEM added to the fp32
-//                 accumulator in global memory (vector reductions); at the end
-//                 of the item, dK_j and dV_j rounded to bf16 and stored.
+//     warps 4..11 one key row (its TMEM lane) and 64 of the tile's 128 query
+//                 columns per thread (warps 4..7 the first half, 8..11 the
+//                 second, so every SM sub-partition runs two of these warps):
+//                 P^T = 2^(S^T scale log2 e - lse) packed to bf16 into TMEM for
+//                 the dV MMA; then dS^T = scale P^T (dP^T - delta), rounded to
+//                 bf16 and stored to shared memory in the 128-byte-swizzled
+//                 layout that serves both as the K-major A operand of dK and as
+//                 the MN-major A operand of dQ.
+//     warps 12..15 one query row per thread: dQ_i from TMEM, regrouped across
+//                 lanes so that each vector reduction into the fp32 accumulator
+//                 in global memory covers whole 128-byte lines; at the end of
+//                 the item, dK_j and dV_j rounded to bf16 and stored.
 //   bwd_dq_kernel     the fp32 dQ accumulator rounded to bf16.
 // TMEM (512 columns): S/P | dP/dQ | dV | dK.
 //
@@ -64,9 +67,9 @@ namespace {
 
 constexpr int BM = 128;            // query rows per tile
 constexpr int BN = 128;            // key rows per work item
-constexpr int NUM_THREADS = 384;   // TMA, MMA, 2 idle, 4 softmax / dS, 4 dQ / epilogue
+constexpr int NUM_THREADS = 512;   // TMA, MMA, 2 idle, 8 softmax / dS, 4 dQ / epilogue
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TM_S = 0;       // S^T (fp32), then P^T (bf16 pairs, first 64 columns)
+constexpr uint32_t TM_S = 0;       // S^T (fp32), then P^T (bf16 pairs, columns 0-31, 64-95)
 constexpr uint32_t TM_DP = 128;    // dP^T (fp32), then dQ (fp32, D columns)
 constexpr uint32_t TM_DV = 256;    // dV accumulator (D columns); dK follows at 256 + D
 constexpr int BOX_BYTES = 128 * 128;  // one TMA box: 128 rows x 64 bf16, 128-byte swizzle
@@ -88,9 +91,9 @@ struct BwdLayout {
   static constexpr int B_QD_FULL = 2;                  // NQD
   static constexpr int B_QD_EMPTY = B_QD_FULL + NQD;   // NQD
   static constexpr int B_S_FULL = B_QD_EMPTY + NQD;
-  static constexpr int B_P_FULL = B_S_FULL + 1;        // one arrival per softmax warp
+  static constexpr int B_P_FULL = B_S_FULL + 1;        // one arrival per softmax warp (8)
   static constexpr int B_DP_FULL = B_P_FULL + 1;
-  static constexpr int B_DS_FULL = B_DP_FULL + 1;      // one arrival per softmax warp
+  static constexpr int B_DS_FULL = B_DP_FULL + 1;      // one arrival per softmax warp (8)
   static constexpr int B_DS_EMPTY = B_DS_FULL + 1;
   static constexpr int B_DQ_FULL = B_DS_EMPTY + 1;
   static constexpr int B_DQ_EMPTY = B_DQ_FULL + 1;     // one arrival per dQ warp
@@ -106,7 +109,8 @@ struct BwdLayout {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget of one CTA");
 
   __device__ static uint32_t arrivals(int i) {
-    return (i == B_P_FULL || i == B_DS_FULL || i == B_DQ_EMPTY || i == B_ACC_EMPTY) ? 4u : 1u;
+    if (i == B_P_FULL || i == B_DS_FULL) return 8u;
+    return (i == B_DQ_EMPTY || i == B_ACC_EMPTY) ? 4u : 1u;
   }
 };
 
@@ -174,6 +178,28 @@ __device__ __forceinline__ void red_add_v4(float* dst, float a, float b, float c
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a), "f"(b),
                "f"(c), "f"(d)
                : "memory");
+}
+
+// Transpose of 16-byte units inside each group of 8 lanes: on entry lane
+// 8g + u holds units 0..7 (a[4x .. 4x+3]) of its own row; on exit unit k is
+// unit u of lane 8g + k's row. Three xor-butterfly stages (lane masks 4, 2, 1),
+// each swapping the off-diagonal half of the units with the partner lane.
+__device__ __forceinline__ void transpose_units8(uint32_t (&a)[32], int lane) {
+#pragma unroll
+  for (int m = 4; m >= 1; m >>= 1) {
+    const bool upper = (lane & m) != 0;
+#pragma unroll
+    for (int x = 0; x < 8; ++x) {
+      if (x & m) continue;
+      const int y = x | m;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t send = upper ? a[4 * x + e] : a[4 * y + e];
+        const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, m);
+        if (upper) a[4 * x + e] = recv; else a[4 * y + e] = recv;
+      }
+    }
+  }
 }
 
 template <int D>
@@ -326,10 +352,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           // starts accumulating over them
           if (i == 0 && !wait(L::B_ACC_EMPTY, (n_item & 1) ^ 1)) { ok = false; break; }
           tc_fence_after();
-          // dV += P^T dO_i: A = P^T from TMEM (8 columns per 16 queries)
+          // dV += P^T dO_i: A = P^T from TMEM, 8 columns per 16 queries; queries
+          // 0..63 at columns 0..31, 64..127 at columns 64..95
 #pragma unroll
           for (int kk = 0; kk < BM / 16; ++kk)
-            umma_ts(tmem + TM_DV, tmem + TM_S + kk * 8, do_mn + stage_off(st) + mn_step(kk),
+            umma_ts(tmem + TM_DV, tmem + TM_S + (kk >> 2) * 64 + (kk & 3) * 8,
+                    do_mn + stage_off(st) + mn_step(kk),
                     IDESC_KV, (i > 0 || kk > 0) ? 1u : 0u);
           if (more) {
             if (!wait(L::B_QD_FULL + (c + 1) % NQD, ((c + 1) / NQD) & 1)) { ok = false; break; }
@@ -367,9 +395,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       drain_wait(&bars[L::B_DRAIN], 0, ctl.wait_limit_ns);
     }
     __syncwarp();
-  } else if (warp >= 4 && warp < 8) {
+  } else if (warp >= 4 && warp < 12) {
     // ============================================================ P and dS
     const int wq = warp & 3;
+    const int half = (warp - 4) >> 2;  // query columns [64 half, 64 half + 64)
+    const int c0 = 64 * half;
     const int r = wq * 32 + lane;  // key row of the tile (TMEM lane)
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t s_col = tmem + lane_base + TM_S;
@@ -390,10 +420,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const float4* dt = reinterpret_cast<const float4*>(args.delta_tab + tab);
         if (!warp_wait(&bars[L::B_S_FULL], c & 1, ctl, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        // P^T row: 2^(s * scale * log2 e - lse_log2[q]) for the tile's 128 queries
-        uint32_t pp[BM / 2];
+        // P^T row: 2^(s * scale * log2 e - lse_log2[q]) for this thread's 64 queries
+        uint32_t pp[32];
 #pragma unroll
-        for (int cc = 0; cc < BM; cc += 32) {
+        for (int cl = 0; cl < 64; cl += 32) {
+          const int cc = c0 + cl;
           uint32_t sr[32];
           tmem_ld32(s_col + cc, sr);
           tmem_ld_wait();
@@ -404,16 +435,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const float p1 = ex2_approx(fmaf(__uint_as_float(sr[4 * e4 + 1]), scale_log2, -lv.y));
             const float p2 = ex2_approx(fmaf(__uint_as_float(sr[4 * e4 + 2]), scale_log2, -lv.z));
             const float p3 = ex2_approx(fmaf(__uint_as_float(sr[4 * e4 + 3]), scale_log2, -lv.w));
-            pp[cc / 2 + 2 * e4] = pack_bf16x2(p0, p1);
-            pp[cc / 2 + 2 * e4 + 1] = pack_bf16x2(p2, p3);
+            pp[cl / 2 + 2 * e4] = pack_bf16x2(p0, p1);
+            pp[cl / 2 + 2 * e4 + 1] = pack_bf16x2(p2, p3);
           }
         }
         if (!key_valid) {
 #pragma unroll
-          for (int e = 0; e < BM / 2; ++e) pp[e] = 0u;
+          for (int e = 0; e < 32; ++e) pp[e] = 0u;
         }
-        tmem_st32(s_col + 0, *reinterpret_cast<uint32_t(*)[32]>(&pp[0]));
-        tmem_st32(s_col + 32, *reinterpret_cast<uint32_t(*)[32]>(&pp[32]));
+        // bf16 pairs of queries c0 .. c0+63 go to columns c0 .. c0+31: inside
+        // this half's own fp32 scores, which it has finished reading (the other
+        // half may still be reading its own)
+        tmem_st32(s_col + c0, pp);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -424,7 +457,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!warp_wait(&bars[L::B_DS_EMPTY], (c & 1) ^ 1, ctl, abort_flag)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
-        for (int cc = 0; cc < BM; cc += 32) {
+        for (int cl = 0; cl < 64; cl += 32) {
+          const int cc = c0 + cl;
           uint32_t dr[32];
           tmem_ld32(dp_col + cc, dr);
           tmem_ld_wait();
@@ -432,7 +466,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int e4 = 0; e4 < 8; ++e4) {
             const float4 dl = __ldg(dt + cc / 4 + e4);
-            const uint32_t pa = pp[cc / 2 + 2 * e4], pb = pp[cc / 2 + 2 * e4 + 1];
+            const uint32_t pa = pp[cl / 2 + 2 * e4], pb = pp[cl / 2 + 2 * e4 + 1];
             const float ds0 = __uint_as_float(pa << 16) * (__uint_as_float(dr[4 * e4 + 0]) - dl.x);
             const float ds1 = __uint_as_float(pa & 0xFFFF0000u) * (__uint_as_float(dr[4 * e4 + 1]) - dl.y);
             const float ds2 = __uint_as_float(pb << 16) * (__uint_as_float(dr[4 * e4 + 2]) - dl.z);
@@ -455,7 +489,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (lane == 0) mbar_arrive(&bars[L::B_DS_FULL]);
       }
     }
-  } else if (warp >= 8) {
+  } else if (warp >= 12) {
     // ============================================================ dQ, dK, dV out
     const int wq = warp & 3;
     const int row = wq * 32 + lane;  // TMEM lane: query row (dQ) or key row (dK, dV)
@@ -473,8 +507,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int i = 0; i < it.nq; ++i, ++c) {
         if (!warp_wait(&bars[L::B_DQ_FULL], c & 1, ctl, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const int qi = i * BM + row;
-        float* dst = args.dq_acc + static_cast<size_t>(it.kv0 + qi) * hid + it.h * D;
+        // 32 columns at a time: after transpose_units8, reduction k of lane
+        // 8g + u adds columns 4u..4u+3 of row 8g + k of the warp, so each
+        // instruction covers four rows x 128 contiguous bytes (4 lines rather
+        // than 32).
+        const int row_k0 = i * BM + wq * 32 + (lane & ~7);  // sample row of k = 0
+        float* dst0 = args.dq_acc + static_cast<size_t>(it.kv0 + row_k0) * hid + it.h * D +
+                      4 * (lane & 7);
 #pragma unroll
         for (int cc = 0; cc < D; cc += 32) {
           uint32_t a[32];
@@ -486,12 +525,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[L::B_DQ_EMPTY]);
           }
-          if (qi < it.n) {
+          transpose_units8(a, lane);
 #pragma unroll
-            for (int e = 0; e < 32; e += 4)
-              red_add_v4(dst + cc + e, __uint_as_float(a[e]), __uint_as_float(a[e + 1]),
-                         __uint_as_float(a[e + 2]), __uint_as_float(a[e + 3]));
-          }
+          for (int kk = 0; kk < 8; ++kk)
+            if (row_k0 + kk < it.n)
+              red_add_v4(dst0 + static_cast<size_t>(kk) * hid + cc, __uint_as_float(a[4 * kk]),
+                         __uint_as_float(a[4 * kk + 1]), __uint_as_float(a[4 * kk + 2]),
+                         __uint_as_float(a[4 * kk + 3]));
         }
       }
       if (!ok) break;
