@@ -622,6 +622,87 @@ def run_mmdit(args, rank, world, local_rank):
         "gpu_launches": 15 * args.steps, "clocks": clk}), flush=True)
 
 
+def run_attn_bwd(args, rank, world, local_rank):
+    """`--op attn_bwd`: the backward of the packed attention (mf_varlen_attn_bwd:
+    row tables, the tcgen05 pass, dQ rounding) over the workload's pack, with O
+    and the log-sum-exp from one forward before the timed region. Useful FLOPs:
+    10 * D * H * sum(n_s^2) over the real samples (the five n x n x D products,
+    S recomputed included)."""
+    import torch
+    import resolution_packed_diffusion_b200 as mf
+    from packgen import draw_grad_bits
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = make_workload(args.config, seed=rank_seed(args.config, rank))
+    T, H, D, S = w.T, w.H, w.D, w.S
+
+    def dbf16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    q, k, v = dbf16(w.q_bits), dbf16(w.k_bits), dbf16(w.v_bits)
+    d_o = dbf16(draw_grad_bits(rank_seed(args.config, rank), (T, H, D)))
+    cu_h, _ = mf.mf_pack_build(w.descs, w.rope_axes, w.budget)
+    cu_d = torch.from_numpy(np.ascontiguousarray(cu_h, dtype=np.int32)).to(dev)
+    scale = 1.0 / D ** 0.5
+    stream = torch.cuda.current_stream(dev)
+    o = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((H, T), dtype=torch.float32, device=dev)
+    mf.mf_varlen_attn_fwd(q, k, v, cu_d, cu_h, S, H, D, scale, None, 2, 10000.0, o, lse, None, 0,
+                          stream)
+    dq, dk, dv = (torch.empty((T, H, D), dtype=torch.bfloat16, device=dev) for _ in range(3))
+    ws_bytes = mf.mf_attn_bwd_workspace_size(T, S, H, D)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+
+    def step():
+        mf.mf_varlen_attn_bwd(q, k, v, o, d_o, lse, cu_d, cu_h, S, H, D, scale, dq, dk, dv, ws,
+                              ws_bytes, stream)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    clocks = ClockSampler(local_rank) if rank == 0 else None
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    torch.cuda.synchronize(dev)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop() if clocks else None
+    if mf.mf_get_error(stream) != mf.MF_OK:
+        raise RuntimeError("device error in the attention backward")
+    flops = 2.5 * useful_flops(w)
+    ms_step, flops_all = reduce_timing(t0.elapsed_time(t1) / args.steps, flops, world)
+    if rank != 0:
+        return
+    peaks, peak_src = load_peaks()
+    achieved = flops / (ms_step * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    in_mb = (6 * T * H * D * 2 + T * H * D * 4) >> 20
+    print(json.dumps({
+        "metric": "packed varlen attention backward useful TFLOP/s", "op": "attn_bwd",
+        "value": flops_all / (ms_step * 1e-3) / 1e12, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "config_index": args.config, "T": T, "H": H, "D": D,
+                   "l2": "q, k, v, O, dO, dq/dk/dv and the fp32 dQ accumulator total %d MB vs "
+                         "126 MB L2; no flush" % in_mb},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
+                     "frac": achieved / peak, "traffic": None,
+                     "kernel": "attn_bwd_kernel (timed with its two small companion launches)",
+                     "peak_source": f"{peak_src} bf16_tflops (burst)"},
+        "gpu_launches": 3 * args.steps, "clocks": clk}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -630,10 +711,11 @@ def main():
     ap.add_argument("--config", type=int, default=DEFAULT_CONFIG, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--impl", default="mf", choices=["mf", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", default="block", choices=["block", "linear", "mmdit"],
+    ap.add_argument("--op", default="block", choices=["block", "linear", "mmdit", "attn_bwd"],
                     help="block: the packed joint-attention block (the default line); "
                          "linear: the modality-specific linear layer as a QKV projection; "
-                         "mmdit: one whole NR-MMDiT block around the path")
+                         "mmdit: one whole NR-MMDiT block around the path; "
+                         "attn_bwd: the backward of the packed attention")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -655,6 +737,8 @@ def main():
             run_linear(args, rank, world, local_rank)
         elif args.op == "mmdit":
             run_mmdit(args, rank, world, local_rank)
+        elif args.op == "attn_bwd":
+            run_attn_bwd(args, rank, world, local_rank)
         else:
             run_gpu(args, rank, world, local_rank)
     finally:

@@ -32,7 +32,8 @@
 //                   dP^T of the next tile, once dQ_i has been read out.
 //                 MMAs from one thread run in issue order, so an MMA that
 //                 overwrites a TMEM region never overtakes one reading it.
-//     warps 2..3  idle.
+//     warps 2..3  idle (they complete the control warpgroup, which gives
+//                 registers to the dQ warpgroup with setmaxnreg).
 //     warps 4..11 one key row (its TMEM lane) and 64 of the tile's 128 query
 //                 columns per thread (warps 4..7 the first half, 8..11 the
 //                 second, so every SM sub-partition runs two of these warps):
@@ -75,6 +76,16 @@ constexpr uint32_t TM_DV = 256;    // dV accumulator (D columns); dK follows at 
 constexpr int BOX_BYTES = 128 * 128;  // one TMA box: 128 rows x 64 bf16, 128-byte swizzle
 constexpr int NQD = 2;             // Q / dO ring stages
 constexpr float kLog2e = 1.4426950408889634f;
+// Registers: launched at 128 per thread (512 x 128 = the SM's 65536); the
+// control warpgroup gives back down to kRegsControl and the dQ warpgroup takes
+// kRegsDq, enough to hold a whole fp32 dQ row while it hands TMEM back; the two
+// softmax warpgroups keep 128. 128 * (104 + 128 + 128 + 152) = 65536; 104 keeps
+// the fully unrolled MMA issue free of spills.
+constexpr int kLaunchRegs = 128;
+constexpr int kRegsControl = 104;
+constexpr int kRegsDq = 152;
+static_assert(128 * (kRegsControl + 2 * kLaunchRegs + kRegsDq) <= NUM_THREADS * kLaunchRegs,
+              "register split exceeds the launch allocation");
 
 template <int D>
 struct BwdLayout {
@@ -249,6 +260,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t* sQ = smem + L::OFF_Q;
   uint8_t* sDO = smem + L::OFF_DO;
 
+  // Each role sets its register budget inside its own branch: code after a join
+  // of differently budgeted paths is compiled for the smaller budget.
+  if (warp < 4) {
+  regs_dec<kRegsControl>();
   if (warp == 0) {
     // ============================================================ TMA producer
     if (lane == 0) {
@@ -367,16 +382,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           if (!wait(L::B_DS_FULL, c & 1)) { ok = false; break; }
           tc_fence_after();
-          // dK += dS^T Q_i (dS^T K-major); dQ_i = dS K_j (dS^T read MN-major)
-#pragma unroll
-          for (int kk = 0; kk < BM / 16; ++kk)
-            umma_ss(tmem + TM_DK, ds_km + km_step(kk), q_mn + stage_off(st) + mn_step(kk),
-                    IDESC_KV, (i > 0 || kk > 0) ? 1u : 0u);
+          // dQ_i = dS K_j (dS^T read MN-major) first, so that its drain overlaps
+          // dK += dS^T Q_i (dS^T K-major)
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk)
             umma_ss(tmem + TM_DP, ds_mn + mn_step(kk), k_mn + mn_step(kk), IDESC_Q,
                     kk > 0 ? 1u : 0u);
           umma_commit(&bars[L::B_DQ_FULL]);
+#pragma unroll
+          for (int kk = 0; kk < BM / 16; ++kk)
+            umma_ss(tmem + TM_DK, ds_km + km_step(kk), q_mn + stage_off(st) + mn_step(kk),
+                    IDESC_KV, (i > 0 || kk > 0) ? 1u : 0u);
           umma_commit(&bars[L::B_DS_EMPTY]);
           umma_commit(&bars[L::B_QD_EMPTY + st]);
           if (more) {
@@ -395,6 +411,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       drain_wait(&bars[L::B_DRAIN], 0, ctl.wait_limit_ns);
     }
     __syncwarp();
+  }
   } else if (warp >= 4 && warp < 12) {
     // ============================================================ P and dS
     const int wq = warp & 3;
@@ -490,6 +507,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
     }
   } else if (warp >= 12) {
+    regs_inc<kRegsDq>();
     // ============================================================ dQ, dK, dV out
     const int wq = warp & 3;
     const int row = wq * 32 + lane;  // TMEM lane: query row (dQ) or key row (dK, dV)
@@ -514,17 +532,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int row_k0 = i * BM + wq * 32 + (lane & ~7);  // sample row of k = 0
         float* dst0 = args.dq_acc + static_cast<size_t>(it.kv0 + row_k0) * hid + it.h * D +
                       4 * (lane & 7);
+        // the whole dQ row into registers, then hand the TMEM region back
+        uint32_t row_vals[D];
+#pragma unroll
+        for (int cc = 0; cc < D; cc += 32)
+          tmem_ld32(dq_col + cc, *reinterpret_cast<uint32_t(*)[32]>(&row_vals[cc]));
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[L::B_DQ_EMPTY]);
 #pragma unroll
         for (int cc = 0; cc < D; cc += 32) {
-          uint32_t a[32];
-          tmem_ld32(dq_col + cc, a);
-          tmem_ld_wait();
-          if (cc + 32 == D) {
-            // the whole dQ row is in registers: hand the TMEM region back
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[L::B_DQ_EMPTY]);
-          }
+          uint32_t(&a)[32] = *reinterpret_cast<uint32_t(*)[32]>(&row_vals[cc]);
           transpose_units8(a, lane);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
@@ -707,8 +726,15 @@ cudaError_t launch_main(const CUtensorMap& mq, const CUtensorMap& mk, const CUte
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(attn_bwd_kernel<D>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    // The setmaxnreg split assumes exactly kLaunchRegs registers per thread at
+    // launch; with fewer the dQ warpgroup's setmaxnreg.inc could never be
+    // satisfied, so refuse to launch.
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, attn_bwd_kernel<D>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
+    e = cudaFuncSetAttribute(attn_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
