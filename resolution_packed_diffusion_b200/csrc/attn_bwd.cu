@@ -20,8 +20,9 @@
 //                     (sample, head, 128-key tile j); it keeps K_j, V_j in
 //                     shared memory and dK_j, dV_j in TMEM while it walks every
 //                     128-row query tile i of the sample:
-//     warp 0      TMA producer: K_j and V_j, then Q_i and dO_i into a 2-stage
-//                 ring.
+//     warp 0      TMA producer: K_j and V_j, then Q_i into a 2-stage ring and
+//                 dO_i into a single buffer (its last reader, the dV MMA of the
+//                 previous tile, finishes long before dP^T needs the next one).
 //     warp 1      tcgen05 issuer, per query tile:
 //                   S^T  = K_j Q_i^T            -> TMEM S   (keys on lanes)
 //                   dP^T = V_j dO_i^T           -> TMEM dP
@@ -42,10 +43,13 @@
 //                 bf16 and stored to shared memory in the 128-byte-swizzled
 //                 layout that serves both as the K-major A operand of dK and as
 //                 the MN-major A operand of dQ.
-//     warps 12..15 one query row per thread: dQ_i from TMEM, regrouped across
-//                 lanes so that each vector reduction into the fp32 accumulator
-//                 in global memory covers whole 128-byte lines; at the end of
-//                 the item, dK_j and dV_j rounded to bf16 and stored.
+//     warps 12..15 one query row per thread: dQ_i from TMEM into registers
+//                 (TMEM handed back at once), then 32 columns at a time into a
+//                 two-stage shared-memory box that one thread adds into the
+//                 fp32 accumulator in global memory with a TMA reduction (the
+//                 adds happen in L2, issued by the TMA unit rather than as
+//                 per-thread atomics); at the end of the item, dK_j and dV_j
+//                 rounded to bf16 and stored.
 //   bwd_dq_kernel     the fp32 dQ accumulator rounded to bf16.
 // TMEM (512 columns): S/P | dP/dQ | dV | dK.
 //
@@ -74,7 +78,10 @@ constexpr uint32_t TM_S = 0;       // S^T (fp32), then P^T (bf16 pairs, columns 
 constexpr uint32_t TM_DP = 128;    // dP^T (fp32), then dQ (fp32, D columns)
 constexpr uint32_t TM_DV = 256;    // dV accumulator (D columns); dK follows at 256 + D
 constexpr int BOX_BYTES = 128 * 128;  // one TMA box: 128 rows x 64 bf16, 128-byte swizzle
-constexpr int NQD = 2;             // Q / dO ring stages
+constexpr int NQ = 2;              // Q ring stages (dO has one: its last reader, the dV MMA,
+                                   // finishes long before the next dP^T needs the next tile)
+constexpr int DQ_CHUNK = 32;       // dQ columns per TMA reduction (128 B of fp32 per row)
+constexpr int DQ_STAGE_BYTES = BM * DQ_CHUNK * 4;  // 16 KB, two stages
 constexpr float kLog2e = 1.4426950408889634f;
 // Registers: launched at 128 per thread (512 x 128 = the SM's 65536); the
 // control warpgroup gives back down to kRegsControl and the dQ warpgroup takes
@@ -93,15 +100,18 @@ struct BwdLayout {
   static constexpr int TILE_BYTES = 128 * D * 2;
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + TILE_BYTES;
-  static constexpr int OFF_Q = OFF_V + TILE_BYTES;            // NQD stages
-  static constexpr int OFF_DO = OFF_Q + NQD * TILE_BYTES;     // NQD stages
-  static constexpr int OFF_DS = OFF_DO + NQD * TILE_BYTES;    // dS^T: 2 boxes of 64 queries
+  static constexpr int OFF_Q = OFF_V + TILE_BYTES;            // NQ stages
+  static constexpr int OFF_DO = OFF_Q + NQ * TILE_BYTES;      // one stage
+  static constexpr int OFF_DS = OFF_DO + TILE_BYTES;          // dS^T: 2 boxes of 64 queries
   static constexpr int DS_BYTES = BN * BM * 2;
-  static constexpr int OFF_BAR = OFF_DS + DS_BYTES;
+  static constexpr int OFF_DQ = OFF_DS + DS_BYTES;            // dQ staging, 2 stages
+  static constexpr int OFF_BAR = OFF_DQ + 2 * DQ_STAGE_BYTES;
   static constexpr int B_KV_FULL = 0, B_KV_EMPTY = 1;
-  static constexpr int B_QD_FULL = 2;                  // NQD
-  static constexpr int B_QD_EMPTY = B_QD_FULL + NQD;   // NQD
-  static constexpr int B_S_FULL = B_QD_EMPTY + NQD;
+  static constexpr int B_Q_FULL = 2;                   // NQ
+  static constexpr int B_Q_EMPTY = B_Q_FULL + NQ;      // NQ
+  static constexpr int B_DO_FULL = B_Q_EMPTY + NQ;
+  static constexpr int B_DO_EMPTY = B_DO_FULL + 1;
+  static constexpr int B_S_FULL = B_DO_EMPTY + 1;
   static constexpr int B_P_FULL = B_S_FULL + 1;        // one arrival per softmax warp (8)
   static constexpr int B_DP_FULL = B_P_FULL + 1;
   static constexpr int B_DS_FULL = B_DP_FULL + 1;      // one arrival per softmax warp (8)
@@ -110,7 +120,9 @@ struct BwdLayout {
   static constexpr int B_DQ_EMPTY = B_DQ_FULL + 1;     // one arrival per dQ warp
   static constexpr int B_ACC_FULL = B_DQ_EMPTY + 1;
   static constexpr int B_ACC_EMPTY = B_ACC_FULL + 1;   // one arrival per dQ warp
-  static constexpr int B_DRAIN = B_ACC_EMPTY + 1;
+  static constexpr int B_DQS_FULL = B_ACC_EMPTY + 1;  // [2], one arrival per dQ warp
+  static constexpr int B_DQS_FREE = B_DQS_FULL + 2;   // [2]
+  static constexpr int B_DRAIN = B_DQS_FREE + 2;
   static constexpr int NUM_BARS = B_DRAIN + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;  // tmem slot, abort flag
   static constexpr int END = OFF_MISC + 16;
@@ -121,7 +133,8 @@ struct BwdLayout {
 
   __device__ static uint32_t arrivals(int i) {
     if (i == B_P_FULL || i == B_DS_FULL) return 8u;
-    return (i == B_DQ_EMPTY || i == B_ACC_EMPTY) ? 4u : 1u;
+    return (i == B_DQ_EMPTY || i == B_ACC_EMPTY || i == B_DQS_FULL || i == B_DQS_FULL + 1) ? 4u
+                                                                                           : 1u;
   }
 };
 
@@ -184,33 +197,27 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint6
   }
 }
 
-// Four fp32 additions into global memory, no value returned.
-__device__ __forceinline__ void red_add_v4(float* dst, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a), "f"(b),
-               "f"(c), "f"(d)
-               : "memory");
+// Element-wise add of a shared-memory box into a 2D tensor in global memory
+// (TMA, fp32 .add); completion is tracked by the issuing thread's bulk groups.
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, const void* src,
+                                                  int32_t x, int32_t y) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group"
+      " [%0, {%2, %3}], [%1];" ::"l"(reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(src)), "r"(x), "r"(y)
+      : "memory");
 }
-
-// Transpose of 16-byte units inside each group of 8 lanes: on entry lane
-// 8g + u holds units 0..7 (a[4x .. 4x+3]) of its own row; on exit unit k is
-// unit u of lane 8g + k's row. Three xor-butterfly stages (lane masks 4, 2, 1),
-// each swapping the off-diagonal half of the units with the partner lane.
-__device__ __forceinline__ void transpose_units8(uint32_t (&a)[32], int lane) {
-#pragma unroll
-  for (int m = 4; m >= 1; m >>= 1) {
-    const bool upper = (lane & m) != 0;
-#pragma unroll
-    for (int x = 0; x < 8; ++x) {
-      if (x & m) continue;
-      const int y = x | m;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const uint32_t send = upper ? a[4 * x + e] : a[4 * y + e];
-        const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, m);
-        if (upper) a[4 * x + e] = recv; else a[4 * y + e] = recv;
-      }
-    }
-  }
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// All but the newest N bulk groups of this thread have finished reading shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_group_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// All bulk groups of this thread have completed.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 template <int D>
@@ -219,6 +226,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     const __grid_constant__ CUtensorMap tmap_k,
                     const __grid_constant__ CUtensorMap tmap_v,
                     const __grid_constant__ CUtensorMap tmap_do,
+                    const __grid_constant__ CUtensorMap tmap_dq,
                     const __grid_constant__ BwdArgs args) {
   using L = BwdLayout<D>;
   constexpr uint32_t TM_DK = TM_DV + D;
@@ -242,6 +250,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_map(&tmap_k);
     tma_prefetch_map(&tmap_v);
     tma_prefetch_map(&tmap_do);
+    tma_prefetch_map(&tmap_dq);
   }
   __syncthreads();
   if (warp == 1) {
@@ -267,7 +276,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 0) {
     // ============================================================ TMA producer
     if (lane == 0) {
-      uint32_t kv_issued = 0, c = 0;  // K/V loads and Q/dO stages issued so far
+      uint32_t kv_issued = 0, c = 0, d_issued = 0;  // K/V, Q and dO loads issued so far
       bool ok = true;
       for (int k = 0, w = snake_item(0, blockIdx.x, gridDim.x); w < total && ok;
            w = snake_item(++k, blockIdx.x, gridDim.x)) {
@@ -282,30 +291,40 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         ++kv_issued;
         for (int i = 0; i < it.nq; ++i) {
-          const int st = c % NQD;
-          if (!mbar_wait(&bars[L::B_QD_EMPTY + st], ((c / NQD) & 1) ^ 1, ctl, abort_flag)) {
+          // Q_i into its ring stage, then dO_i into the single dO buffer (free
+          // once the previous tile's dV MMA has read it)
+          const int st = c % NQ;
+          const int qrow = it.kv0 + i * BM;
+          if (!mbar_wait(&bars[L::B_Q_EMPTY + st], ((c / NQ) & 1) ^ 1, ctl, abort_flag)) {
             ok = false;
             break;
           }
-          mbar_expect_tx(&bars[L::B_QD_FULL + st], 2 * L::TILE_BYTES);
-          const int qrow = it.kv0 + i * BM;
+          mbar_expect_tx(&bars[L::B_Q_FULL + st], L::TILE_BYTES);
 #pragma unroll
-          for (int b = 0; b < L::kBoxes; ++b) {
-            tma_load_2d(sQ + st * L::TILE_BYTES + b * BOX_BYTES, &tmap_q, &bars[L::B_QD_FULL + st],
+          for (int b = 0; b < L::kBoxes; ++b)
+            tma_load_2d(sQ + st * L::TILE_BYTES + b * BOX_BYTES, &tmap_q, &bars[L::B_Q_FULL + st],
                         it.h * D + 64 * b, qrow);
-            tma_load_2d(sDO + st * L::TILE_BYTES + b * BOX_BYTES, &tmap_do,
-                        &bars[L::B_QD_FULL + st], it.h * D + 64 * b, qrow);
-          }
           ++c;
+          if (!mbar_wait(&bars[L::B_DO_EMPTY], ((c - 1) & 1) ^ 1, ctl, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(&bars[L::B_DO_FULL], L::TILE_BYTES);
+#pragma unroll
+          for (int b = 0; b < L::kBoxes; ++b)
+            tma_load_2d(sDO + b * BOX_BYTES, &tmap_do, &bars[L::B_DO_FULL], it.h * D + 64 * b,
+                        qrow);
+          ++d_issued;
         }
       }
       // Let every copy this thread started land before the CTA can exit.
       const uint64_t lim = ctl.wait_limit_ns;
       if (kv_issued > 0) drain_wait(&bars[L::B_KV_FULL], (kv_issued - 1) & 1, lim);
-      for (int st = 0; st < NQD; ++st)
+      if (d_issued > 0) drain_wait(&bars[L::B_DO_FULL], (d_issued - 1) & 1, lim);
+      for (int st = 0; st < NQ; ++st)
         if (c > static_cast<uint32_t>(st)) {
-          const uint32_t last = c - 1 - ((c - 1 - st) % NQD);
-          drain_wait(&bars[L::B_QD_FULL + st], (last / NQD) & 1, lim);
+          const uint32_t last = c - 1 - ((c - 1 - st) % NQ);
+          drain_wait(&bars[L::B_Q_FULL + st], (last / NQ) & 1, lim);
         }
     }
     __syncwarp();
@@ -350,17 +369,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
            w = snake_item(++k, blockIdx.x, gridDim.x), ++n_item) {
         const BwdItem it = decode_item(w, args);
         if (!wait(L::B_KV_FULL, n_item & 1)) break;
-        if (!wait(L::B_QD_FULL + c % NQD, (c / NQD) & 1)) break;
+        if (!wait(L::B_Q_FULL + c % NQ, (c / NQ) & 1)) break;
         tc_fence_after();
-        issue_t(TM_S, k_km, q_km + stage_off(c % NQD));
+        issue_t(TM_S, k_km, q_km + stage_off(c % NQ));
         umma_commit(&bars[L::B_S_FULL]);
         // dP^T lands where the previous tile's dQ sits: wait until it is read out
         if (!wait(L::B_DQ_EMPTY, (c & 1) ^ 1)) break;
+        if (!wait(L::B_DO_FULL, c & 1)) break;
         tc_fence_after();
-        issue_t(TM_DP, v_km, do_km + stage_off(c % NQD));
+        issue_t(TM_DP, v_km, do_km);
         umma_commit(&bars[L::B_DP_FULL]);
         for (int i = 0; i < it.nq; ++i, ++c) {
-          const int st = c % NQD;
+          const int st = c % NQ;
           const bool more = i + 1 < it.nq;
           if (!wait(L::B_P_FULL, c & 1)) { ok = false; break; }
           // the previous item's dK / dV must have been stored before this item
@@ -372,12 +392,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < BM / 16; ++kk)
             umma_ts(tmem + TM_DV, tmem + TM_S + (kk >> 2) * 64 + (kk & 3) * 8,
-                    do_mn + stage_off(st) + mn_step(kk),
-                    IDESC_KV, (i > 0 || kk > 0) ? 1u : 0u);
+                    do_mn + mn_step(kk), IDESC_KV, (i > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(&bars[L::B_DO_EMPTY]);
           if (more) {
-            if (!wait(L::B_QD_FULL + (c + 1) % NQD, ((c + 1) / NQD) & 1)) { ok = false; break; }
+            if (!wait(L::B_Q_FULL + (c + 1) % NQ, ((c + 1) / NQ) & 1)) { ok = false; break; }
             tc_fence_after();
-            issue_t(TM_S, k_km, q_km + stage_off((c + 1) % NQD));
+            issue_t(TM_S, k_km, q_km + stage_off((c + 1) % NQ));
             umma_commit(&bars[L::B_S_FULL]);
           }
           if (!wait(L::B_DS_FULL, c & 1)) { ok = false; break; }
@@ -394,11 +414,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             umma_ss(tmem + TM_DK, ds_km + km_step(kk), q_mn + stage_off(st) + mn_step(kk),
                     IDESC_KV, (i > 0 || kk > 0) ? 1u : 0u);
           umma_commit(&bars[L::B_DS_EMPTY]);
-          umma_commit(&bars[L::B_QD_EMPTY + st]);
+          umma_commit(&bars[L::B_Q_EMPTY + st]);
           if (more) {
             if (!wait(L::B_DQ_EMPTY, c & 1)) { ok = false; break; }
+            if (!wait(L::B_DO_FULL, (c + 1) & 1)) { ok = false; break; }
             tc_fence_after();
-            issue_t(TM_DP, v_km, do_km + stage_off((c + 1) % NQD));
+            issue_t(TM_DP, v_km, do_km);
             umma_commit(&bars[L::B_DP_FULL]);
           }
         }
@@ -516,7 +537,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t dv_col = tmem + lane_base + TM_DV;
     const uint32_t dk_col = tmem + lane_base + TM_DK;
     const int hid = args.H * D;
+    const bool leader = warp == 12 && lane == 0;  // issues the dQ reductions
     uint32_t c = 0;
+    uint32_t g = 0;  // dQ staging boxes filled so far
     int n_item = 0;
     bool ok = true;
     for (int k = 0, w = snake_item(0, blockIdx.x, gridDim.x); w < total && ok;
@@ -525,13 +548,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int i = 0; i < it.nq; ++i, ++c) {
         if (!warp_wait(&bars[L::B_DQ_FULL], c & 1, ctl, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        // 32 columns at a time: after transpose_units8, reduction k of lane
-        // 8g + u adds columns 4u..4u+3 of row 8g + k of the warp, so each
-        // instruction covers four rows x 128 contiguous bytes (4 lines rather
-        // than 32).
-        const int row_k0 = i * BM + wq * 32 + (lane & ~7);  // sample row of k = 0
-        float* dst0 = args.dq_acc + static_cast<size_t>(it.kv0 + row_k0) * hid + it.h * D +
-                      4 * (lane & 7);
         // the whole dQ row into registers, then hand the TMEM region back
         uint32_t row_vals[D];
 #pragma unroll
@@ -541,17 +557,41 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[L::B_DQ_EMPTY]);
+        // 32 columns at a time: each thread writes its row's 128 bytes into a
+        // staging box (128-byte swizzle: 16-byte unit u of row r at u ^ (r % 8)),
+        // and one thread adds the box into the accumulator with a TMA
+        // reduction. Rows past the sample's end hold exactly 0 (their P is 0),
+        // so adding the whole 128-row box is exact; rows past T are clipped.
 #pragma unroll
-        for (int cc = 0; cc < D; cc += 32) {
-          uint32_t(&a)[32] = *reinterpret_cast<uint32_t(*)[32]>(&row_vals[cc]);
-          transpose_units8(a, lane);
+        for (int cc = 0; cc < D; cc += DQ_CHUNK, ++g) {
+          const int b = g & 1;
+          const uint32_t use = g >> 1;
+          uint8_t* box = smem + L::OFF_DQ + b * DQ_STAGE_BYTES;
+          if (!warp_wait(&bars[L::B_DQS_FREE + b], (use & 1) ^ 1, ctl, abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint8_t* rowp = box + row * 128;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            if (row_k0 + kk < it.n)
-              red_add_v4(dst0 + static_cast<size_t>(kk) * hid + cc, __uint_as_float(a[4 * kk]),
-                         __uint_as_float(a[4 * kk + 1]), __uint_as_float(a[4 * kk + 2]),
-                         __uint_as_float(a[4 * kk + 3]));
+          for (int u = 0; u < 8; ++u)
+            *reinterpret_cast<uint4*>(rowp + ((u ^ (row & 7)) << 4)) =
+                make_uint4(row_vals[cc + 4 * u], row_vals[cc + 4 * u + 1],
+                           row_vals[cc + 4 * u + 2], row_vals[cc + 4 * u + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars[L::B_DQS_FULL + b]);
+          if (leader) {
+            if (mbar_wait(&bars[L::B_DQS_FULL + b], use & 1, ctl, abort_flag)) {
+              tma_reduce_add_2d(&tmap_dq, box, it.h * D + cc, it.kv0 + i * BM);
+              bulk_commit_group();
+              // the previous box (the other stage) has been read: release it
+              bulk_wait_group_read<1>();
+              if (g > 0) mbar_arrive(&bars[L::B_DQS_FREE + (b ^ 1)]);
+            }
+          }
+          __syncwarp();
         }
+        if (!ok) break;
       }
       if (!ok) break;
       if (!warp_wait(&bars[L::B_ACC_FULL], n_item & 1, ctl, abort_flag)) break;
@@ -583,6 +623,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[L::B_ACC_EMPTY]);
     }
+    // every reduction this thread issued completes before the CTA exits
+    if (leader) bulk_wait_all();
   }
 
   // ---------------------------------------------------------------- teardown
@@ -697,6 +739,21 @@ bool make_map(CUtensorMap* map, const void* base, int32_t T, int32_t cols) {
          CUDA_SUCCESS;
 }
 
+// The fp32 dQ accumulator [T][H*D] as a 2D tensor for TMA reductions: box =
+// 32 columns (128 B) x 128 rows, 128-byte swizzle; rows past T are clipped.
+bool make_acc_map(CUtensorMap* map, void* base, int32_t T, int32_t cols) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(T)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 4};
+  const cuuint32_t box[2] = {DQ_CHUNK, BM};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 int sm_count() {
   static int cached[64] = {0};
   int dev = 0;
@@ -720,7 +777,8 @@ size_t tab_bytes(int32_t T, int32_t S, int32_t H) {
 
 template <int D>
 cudaError_t launch_main(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                        const CUtensorMap& mdo, const BwdArgs& a, int grid, cudaStream_t st) {
+                        const CUtensorMap& mdo, const CUtensorMap& mdq, const BwdArgs& a,
+                        int grid, cudaStream_t st) {
   constexpr int smem = BwdLayout<D>::SMEM_BYTES;
   static bool attr_set[64] = {false};
   int dev = 0;
@@ -738,7 +796,7 @@ cudaError_t launch_main(const CUtensorMap& mq, const CUtensorMap& mk, const CUte
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  attn_bwd_kernel<D><<<grid, NUM_THREADS, smem, st>>>(mq, mk, mv, mdo, a);
+  attn_bwd_kernel<D><<<grid, NUM_THREADS, smem, st>>>(mq, mk, mv, mdo, mdq, a);
   return cudaGetLastError();
 }
 
@@ -792,10 +850,10 @@ cudaError_t launch_attention_bwd(const mf_bf16* q, const mf_bf16* k, const mf_bf
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
-  CUtensorMap mq, mk, mv, mdo;
+  CUtensorMap mq, mk, mv, mdo, mdq;
   const int32_t cols = H * D;
   if (!make_map(&mq, q, T, cols) || !make_map(&mk, k, T, cols) || !make_map(&mv, v, T, cols) ||
-      !make_map(&mdo, d_o, T, cols))
+      !make_map(&mdo, d_o, T, cols) || !make_acc_map(&mdq, dq_acc, T, cols))
     return cudaErrorInvalidValue;
   static thread_local BwdArgs a;
   a.dk = dk;
@@ -831,8 +889,8 @@ cudaError_t launch_attention_bwd(const mf_bf16* q, const mf_bf16* k, const mf_bf
   if (items > 0) {
     const int sms = sm_count();
     const int grid = items < sms ? items : sms;
-    e = D == 128 ? launch_main<128>(mq, mk, mv, mdo, a, grid, st)
-                 : launch_main<64>(mq, mk, mv, mdo, a, grid, st);
+    e = D == 128 ? launch_main<128>(mq, mk, mv, mdo, mdq, a, grid, st)
+                 : launch_main<64>(mq, mk, mv, mdo, mdq, a, grid, st);
     if (e != cudaSuccess) return e;
   }
   const size_t n8 = static_cast<size_t>(T) * H * D / 8;
