@@ -43,16 +43,21 @@ from .mf_oracle import (  # noqa: F401
     MOD_IMG,
     MOD_TXT,
     adaln_modulate,
+    adaln_modulate_bwd,
     adaln_params,
+    adaln_params_bwd,
+    block_bwd,
     block_fwd,
     cfg_combine,
     gated_residual,
+    gated_residual_bwd,
     gelu_tanh,
     layer_norm_rows,
     mmdit_block_fwd,
     modality_linear,
     pack_build,
     rope_apply,
+    rope_bwd,
     rope_pair_angles,
     rope_split,
     store_bf16,

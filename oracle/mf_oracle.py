@@ -298,6 +298,93 @@ def block_fwd(x, q, k, v, mod, pack, rope_axes: int, base: float = 10000.0,
 
 
 # ---------------------------------------------------------------------------
+# Backward of the block  ([train]: the packed model is trained)
+# ---------------------------------------------------------------------------
+def gated_residual_bwd(dy, o, mod, tok_sample, tok_mod, S: int):
+    """Gradients of ``y = x + gate[s, m] * O`` (chain rule, written out):
+    dx = dy; dO = gate[s, m] * dy; dgate[s, m] = sum over the tokens t of sample
+    s and modality m of dy[t] * O[t]. O and dO are viewed as [T][H*D]. Returns
+    float64 (dx [T][hid], d_o [T][hid], dmod [S][2][3][hid] with only the GATE
+    slot non-zero)."""
+    dy = np.asarray(dy, dtype=np.float64)
+    o = np.asarray(o, dtype=np.float64).reshape(dy.shape[0], -1)
+    tok_sample = np.asarray(tok_sample).astype(np.int64)
+    tok_mod = np.asarray(tok_mod).astype(np.int64)
+    gate = mod[tok_sample, tok_mod, GATE]
+    dmod = np.zeros((S, 2, 3, dy.shape[1]), dtype=np.float64)
+    np.add.at(dmod, (tok_sample, tok_mod, GATE), dy * o)
+    return dy.copy(), gate * dy, dmod
+
+
+def adaln_modulate_bwd(dxm, x, mod, tok_sample, tok_mod, S: int, eps: float = 1e-6):
+    """Gradients of ``x_mod = xhat * (1 + scale[s, m]) + shift[s, m]`` with
+    ``xhat = (x - mean) / sqrt(var + eps)`` over each row (population variance):
+        dshift[s, m] = sum_t dx_mod[t],   dscale[s, m] = sum_t dx_mod[t] * xhat[t]
+        g = dx_mod * (1 + scale)
+        dx = (g - mean(g) - xhat * mean(g * xhat)) / sqrt(var + eps)
+    (sums over the tokens of sample s and modality m; means over the row).
+    Returns float64 (dx [T][hid], dmod [S][2][3][hid] with SHIFT and SCALE set)."""
+    dxm = np.asarray(dxm, dtype=np.float64)
+    x = np.asarray(x, dtype=np.float64)
+    tok_sample = np.asarray(tok_sample).astype(np.int64)
+    tok_mod = np.asarray(tok_mod).astype(np.int64)
+    mu = x.mean(axis=1, keepdims=True)
+    rstd = 1.0 / np.sqrt(np.mean((x - mu) ** 2, axis=1, keepdims=True) + eps)
+    xhat = (x - mu) * rstd
+    scale = mod[tok_sample, tok_mod, SCALE]
+    g = dxm * (1.0 + scale)
+    dx = (g - g.mean(axis=1, keepdims=True) - xhat * (g * xhat).mean(axis=1, keepdims=True)) * rstd
+    dmod = np.zeros((S, 2, 3, x.shape[1]), dtype=np.float64)
+    np.add.at(dmod, (tok_sample, tok_mod, SHIFT), dxm)
+    np.add.at(dmod, (tok_sample, tok_mod, SCALE), dxm * xhat)
+    return dx, dmod
+
+
+def rope_bwd(dx_r, pos_ids, rope_axes: int, base: float = 10000.0):
+    """Gradient of ``rope_apply``: every pair rotation is orthogonal, so the
+    gradient turns back by the same angle (the transpose):
+    ``a = c dx0' + s dx1'``, ``b = -s dx0' + c dx1'``. [T][H][D] -> float64."""
+    g = np.asarray(dx_r, dtype=np.float64)
+    D = g.shape[-1]
+    theta = rope_pair_angles(pos_ids, D, rope_axes, base)[:, None, :]
+    cos, sin = np.cos(theta), np.sin(theta)
+    g0, g1 = g[..., 0::2], g[..., 1::2]
+    out = np.empty_like(g)
+    out[..., 0::2] = g0 * cos + g1 * sin
+    out[..., 1::2] = -g0 * sin + g1 * cos
+    return out
+
+
+def adaln_params_bwd(dmod, c, W):
+    """Gradients of ``mod = c W`` (flattened to [S][6 hid]): dW = c^T dmod,
+    dc = dmod W^T. Returns float64 (dc [S][C], dW [C][6 hid])."""
+    c = np.asarray(c, dtype=np.float64)
+    W = np.asarray(W, dtype=np.float64)
+    dm = np.asarray(dmod, dtype=np.float64).reshape(c.shape[0], -1)
+    return dm @ W.T, c.T @ dm
+
+
+def block_bwd(dy, dx_mod, x, q, k, v, mod, pack, rope_axes: int, base: float = 10000.0,
+              eps: float = 1e-6):
+    """Backward of ``block_fwd`` for upstream gradients dy (of y) and dx_mod
+    (of x_mod): the gate, the attention (from the rotated q, k), RoPE and the
+    adaLN modulation in reverse order. Returns float64 (dx, dq, dk, dv, dmod);
+    dmod [S][2][3][hid] holds the shift, scale and gate gradients."""
+    S = len(pack["cu_seqlens"]) - 1
+    tok_sample, tok_mod = pack["tok_sample"], pack["tok_mod"]
+    q_r = rope_apply(q, pack["pos_ids"], rope_axes, base)
+    k_r = rope_apply(k, pack["pos_ids"], rope_axes, base)
+    o, _ = varlen_attention(q_r, k_r, v, pack["cu_seqlens"])
+    dx_res, d_o, dmod_gate = gated_residual_bwd(dy, o, mod, tok_sample, tok_mod, S)
+    T, H, D = np.asarray(q).shape
+    dq_r, dk_r, dv = varlen_attention_bwd(q_r, k_r, v, d_o.reshape(T, H, D), pack["cu_seqlens"])
+    dq = rope_bwd(dq_r, pack["pos_ids"], rope_axes, base)
+    dk = rope_bwd(dk_r, pack["pos_ids"], rope_axes, base)
+    dx_ln, dmod_ln = adaln_modulate_bwd(dx_mod, x, mod, tok_sample, tok_mod, S, eps)
+    return dx_res + dx_ln, dq, dk, dv, dmod_gate + dmod_ln
+
+
+# ---------------------------------------------------------------------------
 # Modality-specific linear layer  ([norm])
 # ---------------------------------------------------------------------------
 def gelu_tanh(x) -> np.ndarray:

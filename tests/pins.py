@@ -605,3 +605,106 @@ def check_attention_bwd_finite_diff(varlen_attention_bwd, varlen_attention):
         args_m[i] = args_m[i] - eps * u
         fd = (loss(*args_p) - loss(*args_m)) / (2 * eps)
         assert abs(fd - float((g * u).sum())) < 1e-6 * max(1.0, abs(fd)), (i, fd)
+
+
+def _bwd_case(seed: int, rope_axes: int, D: int = 8, H: int = 2):
+    """A small random pack with modulation vectors of order 0.3 (so that every
+    term of the block matters) and upstream gradients."""
+    w = make_random_pack(seed, S=3, H=H, D=D, rope_axes=rope_axes, max_grid=3, max_text=4)
+    from oracle.mf_oracle import pack_build as _pb
+    pack = _pb(w.descs, rope_axes)
+    rng = np.random.default_rng(seed + 1)
+    T, hid = w.T, H * D
+    x = w.f32("x").astype(np.float64)
+    q, k, v = (w.f32(n).astype(np.float64) for n in ("q", "k", "v"))
+    mod = 0.3 * rng.standard_normal((w.S, 2, 3, hid))
+    dy = rng.standard_normal((T, hid))
+    dxm = rng.standard_normal((T, hid))
+    return pack, x, q, k, v, mod, dy, dxm, rng
+
+
+def check_block_bwd_finite_diff(block_bwd, block_fwd):
+    """Directional derivatives of L = <dy, y> + <dx_mod, x_mod> by central
+    differences of the forward match <grad, direction> for x, q, k, v and the
+    modulation vectors (2D and 3D RoPE packs)."""
+    for seed, axes, D in ((90, 2, 8), (92, 3, 16)):
+        pack, x, q, k, v, mod, dy, dxm, rng = _bwd_case(seed, axes, D)
+        grads = block_bwd(dy, dxm, x, q, k, v, mod, pack, axes)
+
+        def loss(xx, qq, kk, vv, mm):
+            xm, y, _ = block_fwd(xx, qq, kk, vv, mm, pack, axes)
+            return float((y * dy).sum() + (xm * dxm).sum())
+
+        base = [x, q, k, v, mod]
+        eps = 1e-6
+        for i, g in enumerate(grads):
+            u = rng.standard_normal(base[i].shape)
+            plus = list(base)
+            minus = list(base)
+            plus[i] = base[i] + eps * u
+            minus[i] = base[i] - eps * u
+            fd = (loss(*plus) - loss(*minus)) / (2 * eps)
+            got = float((g * u).sum())
+            assert abs(fd - got) < 1e-5 * max(1.0, abs(fd)), (axes, i, fd, got)
+
+
+def check_adaln_bwd_vs_torch_layer_norm(adaln_modulate_bwd):
+    """torch autograd through its own layer_norm (a library routine) and the
+    per-token gather of shift / scale gives the same dx and the same per-sample,
+    per-modality sums of the shift and scale gradients."""
+    pack, x, q, k, v, mod, dy, dxm, rng = _bwd_case(94, 2)
+    S, hid = mod.shape[0], x.shape[1]
+    eps = 1e-6
+    dx, dmod = adaln_modulate_bwd(dxm, x, mod, pack["tok_sample"], pack["tok_mod"], S, eps)
+    xt = torch.tensor(x, requires_grad=True)
+    mt = torch.tensor(mod, requires_grad=True)
+    ts = torch.tensor(pack["tok_sample"].astype(np.int64))
+    tm = torch.tensor(pack["tok_mod"].astype(np.int64))
+    xhat = torch.nn.functional.layer_norm(xt, (hid,), eps=eps)
+    out = xhat * (1.0 + mt[ts, tm, 1]) + mt[ts, tm, 0]
+    out.backward(torch.tensor(dxm))
+    assert np.allclose(dx, xt.grad.numpy(), rtol=0, atol=1e-10)
+    assert np.allclose(dmod, mt.grad.numpy(), rtol=0, atol=1e-10)
+
+
+def check_adaln_bwd_invariants(adaln_modulate_bwd):
+    """LayerNorm ignores a constant added to a row, so each row of dx sums to 0;
+    with eps = 0 it also ignores a row's scale, so dx is orthogonal to the
+    centred row."""
+    pack, x, q, k, v, mod, dy, dxm, rng = _bwd_case(96, 2)
+    S = mod.shape[0]
+    dx, _ = adaln_modulate_bwd(dxm, x, mod, pack["tok_sample"], pack["tok_mod"], S, 1e-6)
+    assert np.abs(dx.sum(axis=1)).max() < 1e-10
+    dx0, _ = adaln_modulate_bwd(dxm, x, mod, pack["tok_sample"], pack["tok_mod"], S, 0.0)
+    xc = x - x.mean(axis=1, keepdims=True)
+    assert np.abs((dx0 * xc).sum(axis=1)).max() < 1e-9
+
+
+def check_rope_bwd_adjoint(rope_bwd, rope_apply):
+    """rope_bwd is the adjoint of rope_apply: <R x, y> = <x, R^T y> for random
+    x, y, and R^T R x = x (2D packs and 3D packs with unrotated leftover
+    channels)."""
+    for seed, axes, D in ((98, 2, 8), (99, 3, 16)):
+        pack, x, q, k, v, mod, dy, dxm, rng = _bwd_case(seed, axes, D)
+        a = rng.standard_normal(q.shape)
+        b = rng.standard_normal(q.shape)
+        lhs = float((rope_apply(a, pack["pos_ids"], axes) * b).sum())
+        rhs = float((a * rope_bwd(b, pack["pos_ids"], axes)).sum())
+        assert abs(lhs - rhs) < 1e-10 * max(1.0, abs(lhs))
+        back = rope_bwd(rope_apply(a, pack["pos_ids"], axes), pack["pos_ids"], axes)
+        assert np.abs(back - a).max() < 1e-12
+
+
+def check_adaln_params_bwd_adjoint(adaln_params_bwd, adaln_params):
+    """mod = c W is bilinear: <dmod, c' W> = <dc, c'> and <dmod, c W'> = <dW, W'>
+    for any directions c', W'."""
+    rng = np.random.default_rng(100)
+    S, C, hid = 3, 5, 4
+    c = rng.standard_normal((S, C))
+    W = rng.standard_normal((C, 6 * hid))
+    dmod = rng.standard_normal((S, 2, 3, hid))
+    dc, dW = adaln_params_bwd(dmod, c, W)
+    c2 = rng.standard_normal((S, C))
+    W2 = rng.standard_normal((C, 6 * hid))
+    assert abs(float((adaln_params(c2, W, hid) * dmod).sum()) - float((dc * c2).sum())) < 1e-10
+    assert abs(float((adaln_params(c, W2, hid) * dmod).sum()) - float((dW * W2).sum())) < 1e-10

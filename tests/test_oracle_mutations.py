@@ -178,6 +178,47 @@ def _attn_bwd_unscaled_dk(q, k, v, d_o, cu_seqlens, scale=None):
     return dq, dk * math.sqrt(np.asarray(q).shape[2]), dv
 
 
+def _adaln_bwd_no_xhat_term(dxm, x, mod, tok_sample, tok_mod, S, eps=1e-6):
+    # the LayerNorm gradient without its xhat * mean(g * xhat) projection
+    x = np.asarray(x, dtype=np.float64)
+    dxm = np.asarray(dxm, dtype=np.float64)
+    ts, tm = np.asarray(tok_sample).astype(np.int64), np.asarray(tok_mod).astype(np.int64)
+    mu = x.mean(axis=1, keepdims=True)
+    rstd = 1.0 / np.sqrt(np.mean((x - mu) ** 2, axis=1, keepdims=True) + eps)
+    g = dxm * (1.0 + mod[ts, tm, 1])
+    _, dmod = mo.adaln_modulate_bwd(dxm, x, mod, tok_sample, tok_mod, S, eps)
+    return (g - g.mean(axis=1, keepdims=True)) * rstd, dmod
+
+
+def _adaln_bwd_scale_ignored(dxm, x, mod, tok_sample, tok_mod, S, eps=1e-6):
+    # dx computed as if scale were 0
+    dx, dmod = mo.adaln_modulate_bwd(dxm, x, np.zeros_like(mod), tok_sample, tok_mod, S, eps)
+    _, dmod = mo.adaln_modulate_bwd(dxm, x, mod, tok_sample, tok_mod, S, eps)
+    return dx, dmod
+
+
+def _rope_bwd_forward_rotation(dx_r, pos_ids, rope_axes, base=10000.0):
+    # turns the gradient forwards instead of back
+    return mo.rope_apply(dx_r, pos_ids, rope_axes, base)
+
+
+def _block_bwd_sample_blind_gate(dy, dx_mod, x, q, k, v, mod, pack, rope_axes, base=10000.0,
+                                 eps=1e-6):
+    # every sample's gate gradient summed into sample 0
+    dx, dq, dk, dv, dmod = mo.block_bwd(dy, dx_mod, x, q, k, v, mod, pack, rope_axes, base, eps)
+    dmod = dmod.copy()
+    dmod[0, :, 2] = dmod[:, :, 2].sum(axis=0)
+    dmod[1:, :, 2] = 0.0
+    return dx, dq, dk, dv, dmod
+
+
+def _block_bwd_no_residual(dy, dx_mod, x, q, k, v, mod, pack, rope_axes, base=10000.0,
+                           eps=1e-6):
+    # dx loses the identity path of y = x + gate * O
+    dx, dq, dk, dv, dmod = mo.block_bwd(dy, dx_mod, x, q, k, v, mod, pack, rope_axes, base, eps)
+    return dx - np.asarray(dy, dtype=np.float64), dq, dk, dv, dmod
+
+
 MUTANTS = [
     ("rope sign flip", lambda: pins.check_rope_relative(_rope_sign_flip) or
      pins.check_rope_textbook_1d(_rope_sign_flip)),
@@ -205,6 +246,16 @@ MUTANTS = [
      lambda: pins.check_attention_bwd_vs_autograd(_attn_bwd_no_delta)),
     ("attention backward dK without the scale",
      lambda: pins.check_attention_bwd_finite_diff(_attn_bwd_unscaled_dk, oracle.varlen_attention)),
+    ("adaLN backward without the xhat projection",
+     lambda: pins.check_adaln_bwd_vs_torch_layer_norm(_adaln_bwd_no_xhat_term)),
+    ("adaLN backward ignoring the scale",
+     lambda: pins.check_adaln_bwd_vs_torch_layer_norm(_adaln_bwd_scale_ignored)),
+    ("RoPE backward turning forwards",
+     lambda: pins.check_rope_bwd_adjoint(_rope_bwd_forward_rotation, oracle.rope_apply)),
+    ("block backward with the gate gradient blind to samples",
+     lambda: pins.check_block_bwd_finite_diff(_block_bwd_sample_blind_gate, oracle.block_fwd)),
+    ("block backward without the residual path",
+     lambda: pins.check_block_bwd_finite_diff(_block_bwd_no_residual, oracle.block_fwd)),
     ("block: MLP branch modulated by the attention vectors",
      lambda: pins.check_mmdit_branch_gates(_mmdit_mlp_uses_attn_mod, oracle.pack_build)),
 ]

@@ -223,3 +223,23 @@ def test_attention_bwd_vs_autograd():
 
 def test_attention_bwd_finite_diff():
     pins.check_attention_bwd_finite_diff(oracle.varlen_attention_bwd, oracle.varlen_attention)
+
+
+def test_block_bwd_finite_diff():
+    pins.check_block_bwd_finite_diff(oracle.block_bwd, oracle.block_fwd)
+
+
+def test_adaln_bwd_vs_torch_layer_norm():
+    pins.check_adaln_bwd_vs_torch_layer_norm(oracle.adaln_modulate_bwd)
+
+
+def test_adaln_bwd_invariants():
+    pins.check_adaln_bwd_invariants(oracle.adaln_modulate_bwd)
+
+
+def test_rope_bwd_adjoint():
+    pins.check_rope_bwd_adjoint(oracle.rope_bwd, oracle.rope_apply)
+
+
+def test_adaln_params_bwd_adjoint():
+    pins.check_adaln_params_bwd_adjoint(oracle.adaln_params_bwd, oracle.adaln_params)
