@@ -134,6 +134,15 @@ mf_status mf_rope_apply(const mf_bf16* q, const mf_bf16* k, const int32_t* pos_i
                         int32_t T, int32_t H, int32_t D, int32_t rope_axes, float base,
                         mf_bf16* q_out, mf_bf16* k_out, cudaStream_t stream);
 
+/* Backward of mf_rope_apply [rope], [train]: every pair rotation is orthogonal,
+ * so the gradient turns back by the same angle (the transpose):
+ * dx0 = c g0 + s g1, dx1 = -s g0 + c g1 for the output gradient (g0, g1) of a
+ * pair; unrotated channels are copied. Same arguments, layout, aliasing and
+ * checks as mf_rope_apply (dq_r / dk_r in, dq / dk out). */
+mf_status mf_rope_bwd(const mf_bf16* dq_r, const mf_bf16* dk_r, const int32_t* pos_ids,
+                      int32_t T, int32_t H, int32_t D, int32_t rope_axes, float base,
+                      mf_bf16* dq, mf_bf16* dk, cudaStream_t stream);
+
 /* Block-diagonal varlen attention [pack], [norm]: for every sample s and head h,
  * O = softmax(Q K^T * softmax_scale) V over the sample's own tokens only.
  * q, k, v, o: [T][H][D] bf16 (o must not alias inputs). cu_seqlens_d and

@@ -61,6 +61,7 @@ _SIGS = {
     "mf_adaln_params": (_I, [_P, _P, _I, _I, _I, _P, _P]),
     "mf_adaln_modulate": (_I, [_P, _P, _P, _P, _I, _I, _I, _F, _P, _P]),
     "mf_rope_apply": (_I, [_P, _P, _P, _I, _I, _I, _I, _F, _P, _P, _P]),
+    "mf_rope_bwd": (_I, [_P, _P, _P, _I, _I, _I, _I, _F, _P, _P, _P]),
     "mf_varlen_attn_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _F, _P, _I, _F, _P, _P, _P,
                                 _SZ, _P]),
     "mf_varlen_attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _F, _P, _P, _P, _P,
@@ -173,6 +174,12 @@ def mf_rope_apply(q, k, pos_ids, T: int, H: int, D: int, rope_axes: int, base: f
                   k_out, stream=None) -> None:
     _check(lib.mf_rope_apply(_ptr(q), _ptr(k), _ptr(pos_ids), T, H, D, rope_axes, base,
                              _ptr(q_out), _ptr(k_out), _stream(stream)), "mf_rope_apply")
+
+
+def mf_rope_bwd(dq_r, dk_r, pos_ids, T: int, H: int, D: int, rope_axes: int, base: float, dq,
+                dk, stream=None) -> None:
+    _check(lib.mf_rope_bwd(_ptr(dq_r), _ptr(dk_r), _ptr(pos_ids), T, H, D, rope_axes, base,
+                           _ptr(dq), _ptr(dk), _stream(stream)), "mf_rope_bwd")
 
 
 def mf_varlen_attn_fwd(q, k, v, cu_seqlens_d, cu_seqlens_h: np.ndarray, S: int, H: int, D: int,

@@ -91,6 +91,35 @@ cudaError_t timed_attention(const mf_bf16* q, const mf_bf16* k, const mf_bf16* v
   return e;
 }
 
+// Shared by mf_rope_apply and mf_rope_bwd: the backward turns by the negated
+// angles (inverse frequencies negated in the table), which is the transpose
+// of each pair rotation.
+mf_status rope_call(const mf_bf16* q, const mf_bf16* k, const int32_t* pos_ids, int32_t T,
+                    int32_t H, int32_t D, int32_t rope_axes, float base, mf_bf16* q_out,
+                    mf_bf16* k_out, bool transpose, cudaStream_t stream) {
+  if (T < 0 || T > MF_MAX_TOKENS || H < 1 || H > 128 || (rope_axes != 2 && rope_axes != 3) ||
+      !(base > 0.f) || !std::isfinite(base))
+    return MF_ERR_INVALID;
+  if (!valid_head_dim(D)) return MF_ERR_UNSUPPORTED;
+  if (q == nullptr && k == nullptr) return MF_ERR_INVALID;
+  if ((q != nullptr) != (q_out != nullptr) || (k != nullptr) != (k_out != nullptr))
+    return MF_ERR_INVALID;
+  if (T == 0) return MF_OK;
+  if (pos_ids == nullptr || !aligned16(q) || !aligned16(k) || !aligned16(q_out) ||
+      !aligned16(k_out))
+    return MF_ERR_INVALID;
+  const size_t bytes = static_cast<size_t>(T) * H * D * 2;
+  // in place is allowed; a partial overlap is not
+  if (q && q != q_out && overlap(q, bytes, q_out, bytes)) return MF_ERR_INVALID;
+  if (k && k != k_out && overlap(k, bytes, k_out, bytes)) return MF_ERR_INVALID;
+  if (q_out && k_out && overlap(q_out, bytes, k_out, bytes)) return MF_ERR_INVALID;
+  RopeTable tab;
+  make_rope_table(D, rope_axes, base, &tab);
+  if (transpose)
+    for (float& f : tab.inv_freq) f = -f;
+  return cuda_status(launch_rope(q, k, pos_ids, T, H, D, tab, q_out, k_out, stream));
+}
+
 }  // namespace
 
 cudaError_t get_ctl(KernelCtl* ctl) {
@@ -203,28 +232,17 @@ mf_status mf_adaln_modulate(const mf_bf16* x, const float* mod, const int32_t* t
       launch_adaln_modulate(x, mod, tok_sample, tok_mod, T, S, hid, eps, x_mod, ctl, stream));
 }
 
+
 mf_status mf_rope_apply(const mf_bf16* q, const mf_bf16* k, const int32_t* pos_ids, int32_t T,
                         int32_t H, int32_t D, int32_t rope_axes, float base, mf_bf16* q_out,
                         mf_bf16* k_out, cudaStream_t stream) {
-  if (T < 0 || T > MF_MAX_TOKENS || H < 1 || H > 128 || (rope_axes != 2 && rope_axes != 3) ||
-      !(base > 0.f) || !std::isfinite(base))
-    return MF_ERR_INVALID;
-  if (!valid_head_dim(D)) return MF_ERR_UNSUPPORTED;
-  if (q == nullptr && k == nullptr) return MF_ERR_INVALID;
-  if ((q != nullptr) != (q_out != nullptr) || (k != nullptr) != (k_out != nullptr))
-    return MF_ERR_INVALID;
-  if (T == 0) return MF_OK;
-  if (pos_ids == nullptr || !aligned16(q) || !aligned16(k) || !aligned16(q_out) ||
-      !aligned16(k_out))
-    return MF_ERR_INVALID;
-  const size_t bytes = static_cast<size_t>(T) * H * D * 2;
-  // in place is allowed; a partial overlap is not
-  if (q && q != q_out && overlap(q, bytes, q_out, bytes)) return MF_ERR_INVALID;
-  if (k && k != k_out && overlap(k, bytes, k_out, bytes)) return MF_ERR_INVALID;
-  if (q_out && k_out && overlap(q_out, bytes, k_out, bytes)) return MF_ERR_INVALID;
-  RopeTable tab;
-  make_rope_table(D, rope_axes, base, &tab);
-  return cuda_status(launch_rope(q, k, pos_ids, T, H, D, tab, q_out, k_out, stream));
+  return mf::rope_call(q, k, pos_ids, T, H, D, rope_axes, base, q_out, k_out, false, stream);
+}
+
+mf_status mf_rope_bwd(const mf_bf16* dq_r, const mf_bf16* dk_r, const int32_t* pos_ids,
+                      int32_t T, int32_t H, int32_t D, int32_t rope_axes, float base,
+                      mf_bf16* dq, mf_bf16* dk, cudaStream_t stream) {
+  return mf::rope_call(dq_r, dk_r, pos_ids, T, H, D, rope_axes, base, dq, dk, true, stream);
 }
 
 size_t mf_workspace_size(int32_t T, int32_t H, int32_t D, int32_t with_rope) {

@@ -135,3 +135,38 @@ def test_cfg_combine_argument_checks_launch_nothing():
     assert call([(0, 2)], C=12) == mf.MF_ERR_INVALID
     assert call([(0, 2)], w=float("inf")) == mf.MF_ERR_INVALID
     assert call([]) == mf.MF_ERR_INVALID            # no pairs
+
+
+def test_backward_argument_checks_without_gpu():
+    """The backward entry points validate before touching the GPU."""
+    lib = mf.lib
+    P = ctypes.c_void_p
+    cu = np.array([0, 10], dtype=np.int32)
+    T, H, D = 10, 2, 64
+    ws = mf.mf_attn_bwd_workspace_size(T, 1, H, D)
+    assert ws >= T * H * D * 4
+    assert mf.mf_attn_bwd_workspace_size(2 * T, 1, H, D) > ws
+    MB = 1 << 20
+    q, k, v, o, do, lse = (P((i + 1) * MB) for i in range(6))
+    dq, dk, dv, w = (P((i + 10) * MB) for i in range(4))
+
+    def call(D=D, scale=0.125, dq=dq, dk=dk, dv=dv, w=w, ws=ws, cu=cu):
+        return lib.mf_varlen_attn_bwd(q, k, v, o, do, lse, P(16), cu.ctypes.data_as(P),
+                                      len(cu) - 1, H, D, scale, dq, dk, dv, w, ws, None)
+
+    assert call(D=96) == mf.MF_ERR_UNSUPPORTED
+    assert call(scale=0.0) == mf.MF_ERR_INVALID
+    assert call(dq=q) == mf.MF_ERR_INVALID            # an output aliases an input
+    assert call(dv=dk) == mf.MF_ERR_INVALID           # two outputs share a buffer
+    assert call(w=dq) == mf.MF_ERR_INVALID            # workspace overlaps an output
+    assert call(ws=ws - 256) == mf.MF_ERR_INVALID     # workspace too small
+    assert call(dq=P(10 * MB + 8)) == mf.MF_ERR_INVALID  # misaligned
+    assert call(cu=np.array([0, 10, 5], dtype=np.int32)) == mf.MF_ERR_INVALID
+    assert call(cu=np.array([0, 0], dtype=np.int32)) == mf.MF_OK  # empty pack: nothing to do
+    # RoPE backward: same checks as the forward rotation
+    assert lib.mf_rope_bwd(None, None, P(16), 4, 1, 64, 2, 10000.0, None, None, None) == \
+        mf.MF_ERR_INVALID
+    assert lib.mf_rope_bwd(q, None, P(16), 4, 1, 64, 4, 10000.0, dq, None, None) == \
+        mf.MF_ERR_INVALID
+    assert lib.mf_rope_bwd(q, None, P(16), 4, 1, 96, 2, 10000.0, dq, None, None) == \
+        mf.MF_ERR_UNSUPPORTED
