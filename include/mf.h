@@ -170,7 +170,9 @@ mf_status mf_varlen_attn_fwd(const mf_bf16* q, const mf_bf16* k, const mf_bf16* 
  * forward's output, d_o the loss gradient with respect to it); lse: [H][T] fp32,
  * the forward's natural-log log-sum-exp. dq, dk, dv: [T][H][D] bf16 outputs,
  * disjoint from every input and from each other. Offsets, S, H, D and
- * softmax_scale as for the forward. workspace (fp32 dQ accumulator and row
+ * softmax_scale as for the forward (cu_seqlens_d must hold the same offsets as
+ * cu_seqlens_h; the backward's kernels take the pack geometry from the host
+ * copy). workspace (fp32 dQ accumulator and row
  * tables): ws_bytes >= mf_attn_bwd_workspace_size(T, S, H, D), disjoint from
  * everything else. The five products run on tcgen05 tensor cores with bf16
  * operands and fp32 accumulation; P and dS are rounded to bf16 as operands. */
