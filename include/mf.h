@@ -190,6 +190,34 @@ mf_status mf_gated_residual(const mf_bf16* x, const mf_bf16* o, const float* mod
                             const int32_t* tok_sample, const uint8_t* tok_mod, int32_t T,
                             int32_t S, int32_t hid, mf_bf16* y, cudaStream_t stream);
 
+/* Backward of mf_gated_residual [fuse], [train]: for y = x + gate[s,m] * o,
+ * d_o = gate[s,m] * dy and dmod[s][m][gate][:] = the sum over the tokens of
+ * sample s and modality m of dy * o (dx = dy is the caller's identity path).
+ * dy, o, d_o: [T][hid] bf16 (d_o may equal dy; it must not overlap o). dmod:
+ * [S][2][3][hid] fp32; only its gate slots are written (overwritten, zero for a
+ * (sample, modality) without tokens). Sums use fp32 atomics (their order, and so
+ * the last bits, can vary between runs). Bad ids as for mf_gated_residual. */
+mf_status mf_gated_residual_bwd(const mf_bf16* dy, const mf_bf16* o, const float* mod,
+                                const int32_t* tok_sample, const uint8_t* tok_mod, int32_t T,
+                                int32_t S, int32_t hid, mf_bf16* d_o, float* dmod,
+                                cudaStream_t stream);
+
+/* Backward of mf_adaln_modulate [norm], [train]: with xhat = (x - mean) * rstd
+ * over each row, g = dx_mod * (1 + scale[s,m]):
+ *   dx = resid + (g - mean(g) - xhat * mean(g * xhat)) * rstd,
+ *   dmod[s][m][shift][:] = sum dx_mod, dmod[s][m][scale][:] = sum dx_mod * xhat
+ * (sums over the tokens of sample s and modality m). dx_mod, x, dx and resid:
+ * [T][hid] bf16; resid may be NULL (taken as 0) and dx may equal resid (in
+ * place); dx must not overlap x, dx_mod, dmod or the workspace. dmod: only its
+ * shift and scale slots are written (overwritten). eps as in the forward.
+ * workspace: ws_bytes >= mf_adaln_bwd_workspace_size(T) (row statistics). */
+mf_status mf_adaln_modulate_bwd(const mf_bf16* dx_mod, const mf_bf16* x, const float* mod,
+                                const int32_t* tok_sample, const uint8_t* tok_mod,
+                                const mf_bf16* resid, int32_t T, int32_t S, int32_t hid,
+                                float eps, mf_bf16* dx, float* dmod, void* workspace,
+                                size_t ws_bytes, cudaStream_t stream);
+size_t mf_adaln_bwd_workspace_size(int32_t T);
+
 /* The whole block [fuse]: x_mod = adaLN(x); then RoPE on q and k, varlen
  * attention with softmax scale 1/sqrt(D), and the gated residual fused into the
  * attention epilogue: y = x + gate * O (O never reaches memory).

@@ -68,6 +68,10 @@ _SIGS = {
                                 _SZ, _P]),
     "mf_attn_bwd_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "mf_gated_residual": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P, _P]),
+    "mf_gated_residual_bwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P]),
+    "mf_adaln_modulate_bwd": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _F, _P, _P, _P, _SZ,
+                                   _P]),
+    "mf_adaln_bwd_workspace_size": (_SZ, [_I]),
     "mf_block_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _F, _P,
                           _P, _P, _SZ, _P]),
     "mf_workspace_size": (_SZ, [_I, _I, _I, _I]),
@@ -206,6 +210,25 @@ def mf_varlen_attn_bwd(q, k, v, o, d_o, lse, cu_seqlens_d, cu_seqlens_h: np.ndar
 
 def mf_attn_bwd_workspace_size(T: int, S: int, H: int, D: int) -> int:
     return int(lib.mf_attn_bwd_workspace_size(T, S, H, D))
+
+
+def mf_gated_residual_bwd(dy, o, mod, tok_sample, tok_mod, T: int, S: int, hid: int, d_o, dmod,
+                          stream=None) -> None:
+    _check(lib.mf_gated_residual_bwd(_ptr(dy), _ptr(o), _ptr(mod), _ptr(tok_sample),
+                                     _ptr(tok_mod), T, S, hid, _ptr(d_o), _ptr(dmod),
+                                     _stream(stream)), "mf_gated_residual_bwd")
+
+
+def mf_adaln_bwd_workspace_size(T: int) -> int:
+    return int(lib.mf_adaln_bwd_workspace_size(T))
+
+
+def mf_adaln_modulate_bwd(dx_mod, x, mod, tok_sample, tok_mod, resid, T: int, S: int, hid: int,
+                          eps: float, dx, dmod, workspace, ws_bytes: int, stream=None) -> None:
+    _check(lib.mf_adaln_modulate_bwd(_ptr(dx_mod), _ptr(x), _ptr(mod), _ptr(tok_sample),
+                                     _ptr(tok_mod), _ptr(resid), T, S, hid, eps, _ptr(dx),
+                                     _ptr(dmod), _ptr(workspace), ws_bytes, _stream(stream)),
+           "mf_adaln_modulate_bwd")
 
 
 def mf_gated_residual(x, o, mod, tok_sample, tok_mod, T: int, S: int, hid: int, y,

@@ -10,6 +10,7 @@
 
 #include "mf.h"
 #include "attn_bwd_internal.h"
+#include "block_bwd_internal.h"
 #include "cfg_internal.h"
 #include "gemm_internal.h"
 #include "mf_internal.h"
@@ -342,6 +343,72 @@ mf_status mf_varlen_attn_bwd(const mf_bf16* q, const mf_bf16* k, const mf_bf16* 
   return cuda_status(launch_attention_bwd(q, k, v, o, d_o, lse, cu_seqlens_d, cu_seqlens_h, S, T,
                                           H, D, softmax_scale, dq, dk, dv, workspace, ctl,
                                           stream));
+}
+
+mf_status mf_gated_residual_bwd(const mf_bf16* dy, const mf_bf16* o, const float* mod,
+                                const int32_t* tok_sample, const uint8_t* tok_mod, int32_t T,
+                                int32_t S, int32_t hid, mf_bf16* d_o, float* dmod,
+                                cudaStream_t stream) {
+  if (T < 0 || T > MF_MAX_TOKENS || S < 1 || S > MF_MAX_SAMPLES || hid < 8 || hid % 8 != 0 ||
+      hid > 65536)
+    return MF_ERR_INVALID;
+  if (mod == nullptr || dmod == nullptr || !aligned16(mod) || !aligned16(dmod))
+    return MF_ERR_INVALID;
+  const size_t mod_bytes = static_cast<size_t>(S) * 6 * hid * 4;
+  if (overlap(mod, mod_bytes, dmod, mod_bytes)) return MF_ERR_INVALID;
+  if (T > 0) {
+    if (dy == nullptr || o == nullptr || d_o == nullptr || tok_sample == nullptr ||
+        tok_mod == nullptr || !aligned16(dy) || !aligned16(o) || !aligned16(d_o))
+      return MF_ERR_INVALID;
+    const size_t bytes = static_cast<size_t>(T) * hid * 2;
+    if (d_o != dy && overlap(d_o, bytes, dy, bytes)) return MF_ERR_INVALID;
+    if (overlap(d_o, bytes, o, bytes) || overlap(d_o, bytes, dmod, mod_bytes)) return MF_ERR_INVALID;
+  }
+  KernelCtl ctl;
+  if (cudaError_t ge = get_ctl(&ctl); ge != cudaSuccess) return cuda_status(ge);
+  return cuda_status(launch_gated_residual_bwd(dy, o, mod, tok_sample, tok_mod, T, S, hid, d_o,
+                                               dmod, ctl, stream));
+}
+
+size_t mf_adaln_bwd_workspace_size(int32_t T) {
+  if (T <= 0) return 0;
+  return round_up(static_cast<size_t>(T) * 8, 256) + 256;
+}
+
+mf_status mf_adaln_modulate_bwd(const mf_bf16* dx_mod, const mf_bf16* x, const float* mod,
+                                const int32_t* tok_sample, const uint8_t* tok_mod,
+                                const mf_bf16* resid, int32_t T, int32_t S, int32_t hid,
+                                float eps, mf_bf16* dx, float* dmod, void* workspace,
+                                size_t ws_bytes, cudaStream_t stream) {
+  if (T < 0 || T > MF_MAX_TOKENS || S < 1 || S > MF_MAX_SAMPLES || hid < 8 || hid % 8 != 0 ||
+      hid > 65536 || !(eps > 0.f) || !std::isfinite(eps))
+    return MF_ERR_INVALID;
+  if (mod == nullptr || dmod == nullptr || !aligned16(mod) || !aligned16(dmod))
+    return MF_ERR_INVALID;
+  const size_t mod_bytes = static_cast<size_t>(S) * 6 * hid * 4;
+  if (overlap(mod, mod_bytes, dmod, mod_bytes)) return MF_ERR_INVALID;
+  float* stats = nullptr;
+  if (T > 0) {
+    if (dx_mod == nullptr || x == nullptr || dx == nullptr || tok_sample == nullptr ||
+        tok_mod == nullptr || !aligned16(dx_mod) || !aligned16(x) || !aligned16(dx) ||
+        (resid != nullptr && !aligned16(resid)))
+      return MF_ERR_INVALID;
+    if (workspace == nullptr || !aligned16(workspace) || ws_bytes < mf_adaln_bwd_workspace_size(T))
+      return MF_ERR_INVALID;
+    const size_t bytes = static_cast<size_t>(T) * hid * 2;
+    const size_t ws = mf_adaln_bwd_workspace_size(T);
+    // dx may equal resid (in place); it must not touch x, dx_mod, dmod or the workspace
+    if (resid != nullptr && dx != resid && overlap(dx, bytes, resid, bytes)) return MF_ERR_INVALID;
+    if (overlap(dx, bytes, x, bytes) || overlap(dx, bytes, dx_mod, bytes) ||
+        overlap(dx, bytes, dmod, mod_bytes) || overlap(dx, bytes, workspace, ws) ||
+        overlap(dmod, mod_bytes, workspace, ws))
+      return MF_ERR_INVALID;
+    stats = reinterpret_cast<float*>(round_up(reinterpret_cast<uintptr_t>(workspace), 256));
+  }
+  KernelCtl ctl;
+  if (cudaError_t ge = get_ctl(&ctl); ge != cudaSuccess) return cuda_status(ge);
+  return cuda_status(launch_adaln_modulate_bwd(dx_mod, x, mod, tok_sample, tok_mod, resid, T, S,
+                                               hid, eps, dx, dmod, stats, ctl, stream));
 }
 
 mf_status mf_gated_residual(const mf_bf16* x, const mf_bf16* o, const float* mod,
