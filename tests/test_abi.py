@@ -170,3 +170,33 @@ def test_backward_argument_checks_without_gpu():
         mf.MF_ERR_INVALID
     assert lib.mf_rope_bwd(q, None, P(16), 4, 1, 96, 2, 10000.0, dq, None, None) == \
         mf.MF_ERR_UNSUPPORTED
+
+
+def test_gate_and_adaln_backward_argument_checks_without_gpu():
+    lib = mf.lib
+    P = ctypes.c_void_p
+    MB = 1 << 20
+    T, S, hid = 100, 2, 64
+    dy, o, mod, ts, tm, d_o, dmod = (P((i + 1) * MB) for i in range(7))
+    assert lib.mf_gated_residual_bwd(dy, o, mod, ts, tm, T, S, 60, d_o, dmod, None) == \
+        mf.MF_ERR_INVALID                                        # hid not a multiple of 8
+    assert lib.mf_gated_residual_bwd(dy, o, mod, ts, tm, T, S, hid, o, dmod, None) == \
+        mf.MF_ERR_INVALID                                        # d_o overlaps o
+    assert lib.mf_gated_residual_bwd(dy, o, mod, ts, tm, T, S, hid, d_o, mod, None) == \
+        mf.MF_ERR_INVALID                                        # dmod overlaps mod
+    assert lib.mf_gated_residual_bwd(dy, o, mod, ts, tm, T, 0, hid, d_o, dmod, None) == \
+        mf.MF_ERR_INVALID                                        # no samples
+    ws = mf.mf_adaln_bwd_workspace_size(T)
+    assert ws >= T * 8 and mf.mf_adaln_bwd_workspace_size(0) == 0
+    x, dxm, dx, w = P(20 * MB), P(21 * MB), P(22 * MB), P(23 * MB)
+
+    def ln(dx=dx, resid=None, eps=1e-6, w=w, ws=ws):
+        return lib.mf_adaln_modulate_bwd(dxm, x, mod, ts, tm, resid, T, S, hid, eps, dx, dmod, w,
+                                         ws, None)
+
+    assert ln(eps=0.0) == mf.MF_ERR_INVALID
+    assert ln(dx=x) == mf.MF_ERR_INVALID                         # dx overlaps x
+    assert ln(dx=dxm) == mf.MF_ERR_INVALID                       # dx overlaps dx_mod
+    assert ln(ws=ws - 1) == mf.MF_ERR_INVALID                    # workspace too small
+    assert ln(w=dx) == mf.MF_ERR_INVALID                         # workspace overlaps dx
+    assert ln(resid=P(22 * MB + 64)) == mf.MF_ERR_INVALID        # partial overlap with resid
