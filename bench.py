@@ -703,6 +703,112 @@ def run_attn_bwd(args, rank, world, local_rank):
         "gpu_launches": 3 * args.steps, "clocks": clk}), flush=True)
 
 
+def run_block_bwd(args, rank, world, local_rank):
+    """`--op block_bwd`: the backward of the path block over the workload's pack,
+    from upstream gradients dy (of y) and dx_mod (of x_mod): gate backward
+    (dO, dgate), attention backward (dq, dk, dv of the rotated q, k from O and
+    the log-sum-exp), RoPE backward, adaLN backward (dx = dy + the LayerNorm
+    path, dshift, dscale). The forward state (rotated q and k, O, LSE) is
+    computed once before the timed region. Useful FLOPs: the attention
+    backward's 10 * D * H * sum(n_s^2) over the real samples."""
+    import torch
+    import resolution_packed_diffusion_b200 as mf
+    from packgen import draw_grad_bits
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = make_workload(args.config, seed=rank_seed(args.config, rank))
+    T, H, D, S, hid = w.T, w.H, w.D, w.S, w.hid
+
+    def dbf16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    x = dbf16(w.x_bits.reshape(T, hid))
+    q, k, v = dbf16(w.q_bits), dbf16(w.k_bits), dbf16(w.v_bits)
+    seed = rank_seed(args.config, rank)
+    dy = dbf16(draw_grad_bits(seed, (T, hid)))
+    dxm = dbf16(draw_grad_bits(seed + 1, (T, hid)))
+    cu_d = torch.empty(S + 1, dtype=torch.int32, device=dev)
+    pos = torch.empty((T, 3), dtype=torch.int32, device=dev)
+    ts = torch.empty(T, dtype=torch.int32, device=dev)
+    tm = torch.empty(T, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    cu_h, _ = mf.mf_pack_build(w.descs, w.rope_axes, w.budget, cu_d, pos, ts, tm, stream)
+    c = torch.from_numpy(w.c).to(dev)
+    Wm = torch.from_numpy(w.W).to(dev)
+    mod = torch.empty((S, 2, 3, hid), dtype=torch.float32, device=dev)
+    mf.mf_adaln_params(c, Wm, S, c.shape[1], hid, mod, stream)
+    scale = 1.0 / D ** 0.5
+    q_r, k_r = torch.empty_like(q), torch.empty_like(k)
+    mf.mf_rope_apply(q, k, pos, T, H, D, w.rope_axes, w.base, q_r, k_r, stream)
+    o = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((H, T), dtype=torch.float32, device=dev)
+    mf.mf_varlen_attn_fwd(q_r, k_r, v, cu_d, cu_h, S, H, D, scale, None, w.rope_axes, w.base, o,
+                          lse, None, 0, stream)
+    d_o = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
+    dq_r, dk_r, dv = (torch.empty((T, H, D), dtype=torch.bfloat16, device=dev) for _ in range(3))
+    dq, dk = torch.empty_like(dq_r), torch.empty_like(dk_r)
+    dx = torch.empty_like(x)
+    dmod = torch.empty((S, 2, 3, hid), dtype=torch.float32, device=dev)
+    abw = mf.mf_attn_bwd_workspace_size(T, S, H, D)
+    aws = torch.empty(abw, dtype=torch.uint8, device=dev)
+    lbw = mf.mf_adaln_bwd_workspace_size(T)
+    lws = torch.empty(max(lbw, 16), dtype=torch.uint8, device=dev)
+
+    def step():
+        mf.mf_gated_residual_bwd(dy, o, mod, ts, tm, T, S, hid, d_o, dmod, stream)
+        mf.mf_varlen_attn_bwd(q_r, k_r, v, o, d_o, lse, cu_d, cu_h, S, H, D, scale, dq_r, dk_r, dv,
+                              aws, abw, stream)
+        mf.mf_rope_bwd(dq_r, dk_r, pos, T, H, D, w.rope_axes, w.base, dq, dk, stream)
+        mf.mf_adaln_modulate_bwd(dxm, x, mod, ts, tm, dy, T, S, hid, w.eps, dx, dmod, lws, lbw,
+                                 stream)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    clocks = ClockSampler(local_rank) if rank == 0 else None
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    torch.cuda.synchronize(dev)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop() if clocks else None
+    if mf.mf_get_error(stream) != mf.MF_OK:
+        raise RuntimeError("device error in the block backward")
+    flops = 2.5 * useful_flops(w)
+    ms_step, flops_all = reduce_timing(t0.elapsed_time(t1) / args.steps, flops, world)
+    tokens_all = reduce_timing(0.0, float(real_tokens(w)), world)[1]
+    if rank != 0:
+        return
+    peaks, peak_src = load_peaks()
+    achieved = flops / (ms_step * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    print(json.dumps({
+        "metric": "path block backward useful TFLOP/s (attention backward FLOPs)",
+        "op": "block_bwd",
+        "value": flops_all / (ms_step * 1e-3) / 1e12, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "config_index": args.config, "T": T, "H": H, "D": D,
+                   "hid": hid, "l2": "inputs and outputs far above the 126 MB L2; no flush"},
+        "block_bwd_tokens_per_s": tokens_all / (ms_step * 1e-3),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
+                     "frac": achieved / peak, "traffic": None,
+                     "kernel": "whole backward step (attn_bwd_kernel dominant)",
+                     "peak_source": f"{peak_src} bf16_tflops (burst)"},
+        "gpu_launches": 9 * args.steps, "clocks": clk}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -711,11 +817,13 @@ def main():
     ap.add_argument("--config", type=int, default=DEFAULT_CONFIG, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--impl", default="mf", choices=["mf", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", default="block", choices=["block", "linear", "mmdit", "attn_bwd"],
+    ap.add_argument("--op", default="block",
+                    choices=["block", "linear", "mmdit", "attn_bwd", "block_bwd"],
                     help="block: the packed joint-attention block (the default line); "
                          "linear: the modality-specific linear layer as a QKV projection; "
                          "mmdit: one whole NR-MMDiT block around the path; "
-                         "attn_bwd: the backward of the packed attention")
+                         "attn_bwd: the backward of the packed attention; "
+                         "block_bwd: the backward of the whole path block")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -739,6 +847,8 @@ def main():
             run_mmdit(args, rank, world, local_rank)
         elif args.op == "attn_bwd":
             run_attn_bwd(args, rank, world, local_rank)
+        elif args.op == "block_bwd":
+            run_block_bwd(args, rank, world, local_rank)
         else:
             run_gpu(args, rank, world, local_rank)
     finally:
