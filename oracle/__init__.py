@@ -52,9 +52,12 @@ from .mf_oracle import (  # noqa: F401
     gated_residual,
     gated_residual_bwd,
     gelu_tanh,
+    gelu_tanh_bwd,
     layer_norm_rows,
+    mmdit_block_bwd,
     mmdit_block_fwd,
     modality_linear,
+    modality_linear_bwd,
     pack_build,
     rope_apply,
     rope_bwd,

@@ -475,6 +475,82 @@ def mmdit_block_fwd(x, Wq, Wk, Wv, Wo, Wup, Wdown, mod_attn, mod_mlp, pack, H: i
     return gated_residual(y1, mlp, mod_mlp, ts[r], tm[r])
 
 
+def gelu_tanh_bwd(z, dh) -> np.ndarray:
+    """Gradient through ``gelu_tanh`` at pre-activation z: with
+    u = sqrt(2/pi) (z + 0.044715 z^3),
+    d gelu / dz = 0.5 (1 + tanh u) + 0.5 z (1 - tanh^2 u) sqrt(2/pi) (1 + 3 * 0.044715 z^2)."""
+    z = np.asarray(z, dtype=np.float64)
+    c = math.sqrt(2.0 / math.pi)
+    th = np.tanh(c * (z + 0.044715 * z ** 3))
+    return np.asarray(dh, dtype=np.float64) * (
+        0.5 * (1.0 + th) + 0.5 * z * (1.0 - th * th) * c * (1.0 + 3.0 * 0.044715 * z * z))
+
+
+def modality_linear_bwd(x, W, tok_mod, dout):
+    """Gradients of ``out[t] = x[t] @ W[m(t)].T`` (no activation):
+    dx[t] = dout[t] @ W[m(t)], dW[m] = sum over the tokens of modality m of
+    dout[t]^T x[t]. Returns float64 (dx [T][K], dW [2][N][K])."""
+    x = np.asarray(x, dtype=np.float64)
+    W = np.asarray(W, dtype=np.float64)
+    dout = np.asarray(dout, dtype=np.float64)
+    tok_mod = np.asarray(tok_mod)
+    dx = np.zeros_like(x)
+    dW = np.zeros_like(W)
+    for m in (MOD_IMG, MOD_TXT):
+        sel = tok_mod == m
+        dx[sel] = dout[sel] @ W[m]
+        dW[m] = dout[sel].T @ x[sel]
+    return dx, dW
+
+
+def mmdit_block_bwd(dy, x, Wq, Wk, Wv, Wo, Wup, Wdown, mod_attn, mod_mlp, pack, H: int, D: int,
+                    rope_axes: int, base: float = 10000.0, eps: float = 1e-6):
+    """Backward of ``mmdit_block_fwd`` without intermediate rounding (every
+    intermediate kept in float64), for the upstream gradient dy of y: the MLP
+    branch (gate, down projection, GELU, up projection, adaLN), then the
+    attention branch (gate, output projection, attention, RoPE, the three input
+    projections, adaLN), the residual path carrying dy through both. Returns a
+    dict of float64 gradients: x, Wq, Wk, Wv, Wo, Wup, Wdown, mod_attn, mod_mlp."""
+    x = np.asarray(x, dtype=np.float64)
+    T = x.shape[0]
+    S = len(pack["cu_seqlens"]) - 1
+    ts, tm = np.asarray(pack["tok_sample"]), np.asarray(pack["tok_mod"])
+    # forward, keeping what the backward needs
+    x1 = adaln_modulate(x, mod_attn, ts, tm, eps)
+    q = modality_linear(x1, Wq, tm).reshape(T, H, D)
+    k = modality_linear(x1, Wk, tm).reshape(T, H, D)
+    v = modality_linear(x1, Wv, tm).reshape(T, H, D)
+    q_r = rope_apply(q, pack["pos_ids"], rope_axes, base)
+    k_r = rope_apply(k, pack["pos_ids"], rope_axes, base)
+    o, _ = varlen_attention(q_r, k_r, v, pack["cu_seqlens"])
+    o = o.reshape(T, H * D)
+    a = modality_linear(o, Wo, tm)
+    y1 = gated_residual(x, a, mod_attn, ts, tm)
+    x2 = adaln_modulate(y1, mod_mlp, ts, tm, eps)
+    z = modality_linear(x2, Wup, tm)
+    h = gelu_tanh(z)
+    mlp = modality_linear(h, Wdown, tm)
+    # MLP branch
+    dy1, dmlp, dmod_mlp = gated_residual_bwd(dy, mlp, mod_mlp, ts, tm, S)
+    dh, dWdown = modality_linear_bwd(h, Wdown, tm, dmlp)
+    dx2, dWup = modality_linear_bwd(x2, Wup, tm, gelu_tanh_bwd(z, dh))
+    dy1_ln, dmod_mlp_ln = adaln_modulate_bwd(dx2, y1, mod_mlp, ts, tm, S, eps)
+    dy1 = dy1 + dy1_ln
+    dmod_mlp = dmod_mlp + dmod_mlp_ln
+    # attention branch
+    dx, da, dmod_attn = gated_residual_bwd(dy1, a, mod_attn, ts, tm, S)
+    do, dWo = modality_linear_bwd(o, Wo, tm, da)
+    dq_r, dk_r, dv = varlen_attention_bwd(q_r, k_r, v, do.reshape(T, H, D), pack["cu_seqlens"])
+    dq = rope_bwd(dq_r, pack["pos_ids"], rope_axes, base).reshape(T, H * D)
+    dk = rope_bwd(dk_r, pack["pos_ids"], rope_axes, base).reshape(T, H * D)
+    dx1q, dWq = modality_linear_bwd(x1, Wq, tm, dq)
+    dx1k, dWk = modality_linear_bwd(x1, Wk, tm, dk)
+    dx1v, dWv = modality_linear_bwd(x1, Wv, tm, dv.reshape(T, H * D))
+    dx_ln, dmod_attn_ln = adaln_modulate_bwd(dx1q + dx1k + dx1v, x, mod_attn, ts, tm, S, eps)
+    return dict(x=dx + dx_ln, Wq=dWq, Wk=dWk, Wv=dWv, Wo=dWo, Wup=dWup, Wdown=dWdown,
+                mod_attn=dmod_attn + dmod_attn_ln, mod_mlp=dmod_mlp)
+
+
 # ---------------------------------------------------------------------------
 # Packed classifier-free guidance  ([cfg])
 # ---------------------------------------------------------------------------

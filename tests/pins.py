@@ -708,3 +708,48 @@ def check_adaln_params_bwd_adjoint(adaln_params_bwd, adaln_params):
     W2 = rng.standard_normal((C, 6 * hid))
     assert abs(float((adaln_params(c2, W, hid) * dmod).sum()) - float((dc * c2).sum())) < 1e-10
     assert abs(float((adaln_params(c, W2, hid) * dmod).sum()) - float((dW * W2).sum())) < 1e-10
+
+
+def check_gelu_bwd_vs_torch(gelu_tanh_bwd):
+    """torch autograd through its own tanh-form GELU (a library routine) gives
+    the same derivative, over a range that covers both tails."""
+    z = np.linspace(-8.0, 8.0, 2001)
+    dh = np.random.default_rng(101).standard_normal(z.shape)
+    zt = torch.tensor(z, requires_grad=True)
+    torch.nn.functional.gelu(zt, approximate="tanh").backward(torch.tensor(dh))
+    assert np.allclose(gelu_tanh_bwd(z, dh), zt.grad.numpy(), rtol=0, atol=1e-12)
+
+
+def check_mmdit_bwd_finite_diff(mmdit_block_bwd, mmdit_block_fwd):
+    """Directional derivatives of L = <dy, y> of the unrounded whole block by
+    central differences match <grad, direction> for x, all six weight tensors
+    and both modulation maps."""
+    w = make_random_pack(102, S=2, H=2, D=8, rope_axes=2, max_grid=3, max_text=3)
+    from oracle.mf_oracle import pack_build as _pb
+    pack = _pb(w.descs, 2)
+    rng = np.random.default_rng(103)
+    T, hid = w.T, 16
+    F = 4 * hid
+    x = rng.standard_normal((T, hid))
+    Ws = {n: rng.standard_normal((2, hid, hid)) / 4 for n in ("Wq", "Wk", "Wv", "Wo")}
+    Ws["Wup"] = rng.standard_normal((2, F, hid)) / 4
+    Ws["Wdown"] = rng.standard_normal((2, hid, F)) / 8
+    mods = {n: 0.3 * rng.standard_normal((w.S, 2, 3, hid)) for n in ("mod_attn", "mod_mlp")}
+    dy = rng.standard_normal((T, hid))
+    args = dict(x=x, **Ws, **mods)
+    order = ("x", "Wq", "Wk", "Wv", "Wo", "Wup", "Wdown", "mod_attn", "mod_mlp")
+
+    def loss(a):
+        y = mmdit_block_fwd(*[a[n] for n in order], pack, 2, 8, 2, store=lambda t: t)
+        return float((y * dy).sum())
+
+    grads = mmdit_block_bwd(dy, *[args[n] for n in order], pack, 2, 8, 2)
+    eps = 1e-6
+    for n in order:
+        u = rng.standard_normal(args[n].shape)
+        plus, minus = dict(args), dict(args)
+        plus[n] = args[n] + eps * u
+        minus[n] = args[n] - eps * u
+        fd = (loss(plus) - loss(minus)) / (2 * eps)
+        got = float((grads[n] * u).sum())
+        assert abs(fd - got) < 1e-5 * max(1.0, abs(fd)), (n, fd, got)

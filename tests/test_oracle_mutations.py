@@ -219,6 +219,42 @@ def _block_bwd_no_residual(dy, dx_mod, x, q, k, v, mod, pack, rope_axes, base=10
     return dx - np.asarray(dy, dtype=np.float64), dq, dk, dv, dmod
 
 
+def _gelu_bwd_no_sech_term(z, dh):
+    # keeps 0.5 (1 + tanh u), drops the z * sech^2 part
+    z = np.asarray(z, dtype=np.float64)
+    th = np.tanh(math.sqrt(2.0 / math.pi) * (z + 0.044715 * z ** 3))
+    return np.asarray(dh, dtype=np.float64) * 0.5 * (1.0 + th)
+
+
+def _mmdit_bwd_swapped_weight_grads(*args, **kwargs):
+    # the image and text gradients of the up projection land in each other's slot
+    g = mo.mmdit_block_bwd(*args, **kwargs)
+    g = dict(g)
+    g["Wup"] = g["Wup"][::-1].copy()
+    return g
+
+
+def _mmdit_bwd_no_mlp_norm_path(dy, x, Wq, Wk, Wv, Wo, Wup, Wdown, mod_attn, mod_mlp, pack, H, D,
+                                rope_axes, base=10000.0, eps=1e-6):
+    # the attention branch sees only the identity path of the MLP branch
+    saved = mo.adaln_modulate_bwd
+    calls = []
+
+    def zero_first(*a, **k):
+        dx, dmod = saved(*a, **k)
+        if not calls:
+            calls.append(1)
+            dx = np.zeros_like(dx)
+        return dx, dmod
+
+    mo.adaln_modulate_bwd = zero_first
+    try:
+        return mo.mmdit_block_bwd(dy, x, Wq, Wk, Wv, Wo, Wup, Wdown, mod_attn, mod_mlp, pack, H,
+                                  D, rope_axes, base, eps)
+    finally:
+        mo.adaln_modulate_bwd = saved
+
+
 MUTANTS = [
     ("rope sign flip", lambda: pins.check_rope_relative(_rope_sign_flip) or
      pins.check_rope_textbook_1d(_rope_sign_flip)),
@@ -256,6 +292,14 @@ MUTANTS = [
      lambda: pins.check_block_bwd_finite_diff(_block_bwd_sample_blind_gate, oracle.block_fwd)),
     ("block backward without the residual path",
      lambda: pins.check_block_bwd_finite_diff(_block_bwd_no_residual, oracle.block_fwd)),
+    ("GELU backward without the sech^2 term",
+     lambda: pins.check_gelu_bwd_vs_torch(_gelu_bwd_no_sech_term)),
+    ("MMDiT backward with image and text weight gradients swapped",
+     lambda: pins.check_mmdit_bwd_finite_diff(_mmdit_bwd_swapped_weight_grads,
+                                              oracle.mmdit_block_fwd)),
+    ("MMDiT backward without the MLP branch's normalization path",
+     lambda: pins.check_mmdit_bwd_finite_diff(_mmdit_bwd_no_mlp_norm_path,
+                                              oracle.mmdit_block_fwd)),
     ("block: MLP branch modulated by the attention vectors",
      lambda: pins.check_mmdit_branch_gates(_mmdit_mlp_uses_attn_mod, oracle.pack_build)),
 ]

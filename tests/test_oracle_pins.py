@@ -243,3 +243,11 @@ def test_rope_bwd_adjoint():
 
 def test_adaln_params_bwd_adjoint():
     pins.check_adaln_params_bwd_adjoint(oracle.adaln_params_bwd, oracle.adaln_params)
+
+
+def test_gelu_bwd_vs_torch():
+    pins.check_gelu_bwd_vs_torch(oracle.gelu_tanh_bwd)
+
+
+def test_mmdit_bwd_finite_diff():
+    pins.check_mmdit_bwd_finite_diff(oracle.mmdit_block_bwd, oracle.mmdit_block_fwd)
