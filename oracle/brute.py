@@ -165,3 +165,38 @@ def brute_mmdit_block(x, Wq, Wk, Wv, Wo, Wup, Wdown, mod_attn, mod_mlp, descs, H
         m = brute_linear_row(hmid, Wdown[tm[t]])
         y.append(brute_gate_row(y1, m, mod_vec(mod_mlp, t, 2)))
     return y
+
+
+def brute_attention_bwd(q, k, v, d_o, cu, scale=None):
+    """dq, dk, dv of the per-sample attention by explicit loops: for each sample,
+    head and query row, the softmax row p, then dp_j = <dO_i, v_j>,
+    ds_j = p_j (dp_j - sum_l p_l dp_l), dq_i += scale ds_j k_j, dk_j += scale ds_j q_i,
+    dv_j += p_j dO_i. Nested lists [T][H][D] in and out."""
+    T = len(q)
+    H = len(q[0]) if T else 0
+    D = len(q[0][0]) if T else 0
+    if scale is None:
+        scale = 1.0 / math.sqrt(D) if D else 1.0
+    dq = [[[0.0] * D for _ in range(H)] for _ in range(T)]
+    dk = [[[0.0] * D for _ in range(H)] for _ in range(T)]
+    dv = [[[0.0] * D for _ in range(H)] for _ in range(T)]
+    for s in range(len(cu) - 1):
+        lo, hi = cu[s], cu[s + 1]
+        for h in range(H):
+            for i in range(lo, hi):
+                sc = [scale * sum(float(q[i][h][d]) * float(k[j][h][d]) for d in range(D))
+                      for j in range(lo, hi)]
+                mx = max(sc)
+                e = [math.exp(a - mx) for a in sc]
+                tot = sum(e)
+                p = [a / tot for a in e]
+                dp = [sum(float(d_o[i][h][d]) * float(v[j][h][d]) for d in range(D))
+                      for j in range(lo, hi)]
+                mean_dp = sum(pj * dpj for pj, dpj in zip(p, dp))
+                for jj, j in enumerate(range(lo, hi)):
+                    ds = p[jj] * (dp[jj] - mean_dp)
+                    for d in range(D):
+                        dq[i][h][d] += scale * ds * float(k[j][h][d])
+                        dk[j][h][d] += scale * ds * float(q[i][h][d])
+                        dv[j][h][d] += p[jj] * float(d_o[i][h][d])
+    return dq, dk, dv

@@ -280,6 +280,8 @@ MUTANTS = [
      lambda: pins.check_mmdit_vs_brute(_mmdit_gelu_after_down, oracle.pack_build)),
     ("attention backward without the rowsum term",
      lambda: pins.check_attention_bwd_vs_autograd(_attn_bwd_no_delta)),
+    ("attention backward without the rowsum term, against the scalar loops",
+     lambda: pins.check_attention_bwd_vs_brute(_attn_bwd_no_delta)),
     ("attention backward dK without the scale",
      lambda: pins.check_attention_bwd_finite_diff(_attn_bwd_unscaled_dk, oracle.varlen_attention)),
     ("adaLN backward without the xhat projection",

@@ -251,3 +251,7 @@ def test_gelu_bwd_vs_torch():
 
 def test_mmdit_bwd_finite_diff():
     pins.check_mmdit_bwd_finite_diff(oracle.mmdit_block_bwd, oracle.mmdit_block_fwd)
+
+
+def test_attention_bwd_vs_brute():
+    pins.check_attention_bwd_vs_brute(oracle.varlen_attention_bwd)
