@@ -362,7 +362,12 @@ mf_status mf_gated_residual_bwd(const mf_bf16* dy, const mf_bf16* o, const float
       return MF_ERR_INVALID;
     const size_t bytes = static_cast<size_t>(T) * hid * 2;
     if (d_o != dy && overlap(d_o, bytes, dy, bytes)) return MF_ERR_INVALID;
-    if (overlap(d_o, bytes, o, bytes) || overlap(d_o, bytes, dmod, mod_bytes)) return MF_ERR_INVALID;
+    if (overlap(d_o, bytes, o, bytes) || overlap(d_o, bytes, dmod, mod_bytes) ||
+        overlap(d_o, bytes, mod, mod_bytes))
+      return MF_ERR_INVALID;
+    // dmod is zeroed before dy and o are read: it must not overlap them
+    if (overlap(dmod, mod_bytes, dy, bytes) || overlap(dmod, mod_bytes, o, bytes))
+      return MF_ERR_INVALID;
   }
   KernelCtl ctl;
   if (cudaError_t ge = get_ctl(&ctl); ge != cudaSuccess) return cuda_status(ge);
@@ -401,7 +406,14 @@ mf_status mf_adaln_modulate_bwd(const mf_bf16* dx_mod, const mf_bf16* x, const f
     if (resid != nullptr && dx != resid && overlap(dx, bytes, resid, bytes)) return MF_ERR_INVALID;
     if (overlap(dx, bytes, x, bytes) || overlap(dx, bytes, dx_mod, bytes) ||
         overlap(dx, bytes, dmod, mod_bytes) || overlap(dx, bytes, workspace, ws) ||
-        overlap(dmod, mod_bytes, workspace, ws))
+        overlap(dx, bytes, mod, mod_bytes) || overlap(dmod, mod_bytes, workspace, ws))
+      return MF_ERR_INVALID;
+    // dmod is zeroed and the row statistics written before the inputs are read
+    if (overlap(dmod, mod_bytes, x, bytes) || overlap(dmod, mod_bytes, dx_mod, bytes) ||
+        (resid != nullptr && overlap(dmod, mod_bytes, resid, bytes)) ||
+        overlap(workspace, ws, x, bytes) || overlap(workspace, ws, dx_mod, bytes) ||
+        overlap(workspace, ws, mod, mod_bytes) ||
+        (resid != nullptr && overlap(workspace, ws, resid, bytes)))
       return MF_ERR_INVALID;
     stats = reinterpret_cast<float*>(round_up(reinterpret_cast<uintptr_t>(workspace), 256));
   }

@@ -200,3 +200,11 @@ def test_gate_and_adaln_backward_argument_checks_without_gpu():
     assert ln(ws=ws - 1) == mf.MF_ERR_INVALID                    # workspace too small
     assert ln(w=dx) == mf.MF_ERR_INVALID                         # workspace overlaps dx
     assert ln(resid=P(22 * MB + 64)) == mf.MF_ERR_INVALID        # partial overlap with resid
+
+    assert lib.mf_gated_residual_bwd(dy, o, mod, ts, tm, T, S, hid, d_o, dy, None) == \
+        mf.MF_ERR_INVALID                                        # dmod overlaps dy
+    assert lib.mf_gated_residual_bwd(dy, o, mod, ts, tm, T, S, hid, mod, dmod, None) == \
+        mf.MF_ERR_INVALID                                        # d_o overlaps mod
+    assert ln(w=x) == mf.MF_ERR_INVALID                          # workspace overlaps x
+    assert lib.mf_adaln_modulate_bwd(dxm, x, mod, ts, tm, None, T, S, hid, 1e-6, dx, x, w, ws,
+                                     None) == mf.MF_ERR_INVALID  # dmod overlaps x
