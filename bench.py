@@ -15,6 +15,8 @@ buffers (e2e) and the CPU oracle on a bounded sample (cpu_baseline).
 
 Multi-GPU: every rank runs its own replica pack (same shapes, its own seed); no
 data moves between ranks. Timing is the max over ranks of the CUDA-event time.
+Under torchrun the ranks come from the environment (RANK, WORLD_SIZE, ...);
+``--gpus N`` without them starts N replica processes itself, rank r on GPU r.
 ``--impl reference`` times the CPU oracle (the only reference this method has)
 on rank 0; other ranks exit without work.
 """
@@ -37,7 +39,7 @@ if ROOT not in sys.path:
 
 from packgen import make_workload  # noqa: E402
 
-DEFAULT_CONFIG = 2  # the 16384-token native-resolution training pack
+DEFAULT_CONFIG = 5  # the largest single-GPU pack: 2048^2 image plus three 4:1 images
 METRIC = "packed varlen attention useful TFLOP/s (% bf16 peak); block tokens/s at 1 B200"
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -809,6 +811,49 @@ def run_block_bwd(args, rank, world, local_rank):
         "gpu_launches": 9 * args.steps, "clocks": clk}), flush=True)
 
 
+ARMS = {"block": "run_gpu", "linear": "run_linear", "mmdit": "run_mmdit",
+        "attn_bwd": "run_attn_bwd", "block_bwd": "run_block_bwd"}
+
+
+def run_rank(args, rank, world, local_rank, backend="nccl", arm=None):
+    """One rank of the GPU arm: joins the process group when world > 1, runs
+    the arm (``arm`` or the one ``--op`` names), leaves the group."""
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        if backend == "nccl":
+            torch.cuda.set_device(local_rank)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    try:
+        (arm or globals()[ARMS[args.op]])(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+def _free_port() -> int:
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _replica_main(rank, world, port, args, backend, arm):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank), LOCAL_WORLD_SIZE=str(world))
+    run_rank(args, rank, world, rank, backend, arm)
+
+
+def launch_replicas(args, n: int, backend: str = "nccl", arm=None):
+    """``--gpus N`` outside torchrun: start N replica ranks in fresh (spawned)
+    processes, rank r on GPU r, rendezvous on 127.0.0.1, and wait for all of
+    them; a rank that fails makes the launch raise."""
+    import torch.multiprocessing as mp
+    mp.spawn(_replica_main, args=(n, _free_port(), args, backend, arm), nprocs=n, join=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -817,8 +862,7 @@ def main():
     ap.add_argument("--config", type=int, default=DEFAULT_CONFIG, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--impl", default="mf", choices=["mf", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", default="block",
-                    choices=["block", "linear", "mmdit", "attn_bwd", "block_bwd"],
+    ap.add_argument("--op", default="block", choices=sorted(ARMS),
                     help="block: the packed joint-attention block (the default line); "
                          "linear: the modality-specific linear layer as a QKV projection; "
                          "mmdit: one whole NR-MMDiT block around the path; "
@@ -827,34 +871,22 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be at least 1")
 
+    launched = "WORLD_SIZE" in os.environ
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if launched:
+        args.gpus = world  # the launcher's rank count is what runs
     if args.impl == "reference":
-        run_reference(args, rank)
+        run_reference(args, rank)  # rank 0 alone; no GPU and no process group
         return
-    if world > 1:
-        import datetime
-        import torch
-        import torch.distributed as dist
-        torch.cuda.set_device(local_rank)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    try:
-        if args.op == "linear":
-            run_linear(args, rank, world, local_rank)
-        elif args.op == "mmdit":
-            run_mmdit(args, rank, world, local_rank)
-        elif args.op == "attn_bwd":
-            run_attn_bwd(args, rank, world, local_rank)
-        elif args.op == "block_bwd":
-            run_block_bwd(args, rank, world, local_rank)
-        else:
-            run_gpu(args, rank, world, local_rank)
-    finally:
-        if world > 1:
-            import torch.distributed as dist
-            dist.destroy_process_group()
+    if not launched and args.gpus > 1:
+        launch_replicas(args, args.gpus)
+        return
+    run_rank(args, rank, world, local_rank)
 
 
 if __name__ == "__main__":

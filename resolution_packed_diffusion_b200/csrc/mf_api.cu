@@ -56,16 +56,6 @@ inline mf_status cuda_status(cudaError_t e) {
 
 bool valid_head_dim(int32_t D) { return D == 64 || D == 128; }
 
-// Checks host offsets: 0 = cu[0] <= cu[1] <= ... ; writes T.
-bool check_offsets(const int32_t* cu_h, int32_t S, int32_t* T) {
-  if (cu_h == nullptr || cu_h[0] != 0) return false;
-  for (int32_t s = 0; s < S; ++s)
-    if (cu_h[s + 1] < cu_h[s]) return false;
-  if (cu_h[S] > MF_MAX_TOKENS) return false;
-  *T = cu_h[S];
-  return true;
-}
-
 int32_t count_items(const int32_t* cu_h, int32_t S, int32_t H) {
   return attention_work_items(cu_h, S, H);
 }
@@ -122,6 +112,15 @@ mf_status rope_call(const mf_bf16* q, const mf_bf16* k, const int32_t* pos_ids, 
 }
 
 }  // namespace
+
+bool check_offsets(const int32_t* cu_h, int32_t S, int32_t* T) {
+  if (cu_h == nullptr || cu_h[0] != 0) return false;
+  for (int32_t s = 0; s < S; ++s)
+    if (cu_h[s + 1] < cu_h[s]) return false;
+  if (cu_h[S] > MF_MAX_TOKENS) return false;
+  *T = cu_h[S];
+  return true;
+}
 
 cudaError_t get_ctl(KernelCtl* ctl) {
   int dev = 0;
@@ -272,8 +271,6 @@ mf_status mf_varlen_attn_fwd(const mf_bf16* q, const mf_bf16* k, const mf_bf16* 
     return MF_ERR_INVALID;
   if (lse && (overlap(lse, static_cast<size_t>(T) * H * 4, o, bytes)))
     return MF_ERR_INVALID;
-  KernelCtl ctl;
-  if (cudaError_t ge = get_ctl(&ctl); ge != cudaSuccess) return cuda_status(ge);
   const mf_bf16* qa = q;
   const mf_bf16* ka = k;
   if (pos_ids != nullptr) {
@@ -281,15 +278,26 @@ mf_status mf_varlen_attn_fwd(const mf_bf16* q, const mf_bf16* k, const mf_bf16* 
       return MF_ERR_INVALID;
     if (workspace == nullptr || !aligned16(workspace) || ws_bytes < mf_workspace_size(T, H, D, 1))
       return MF_ERR_INVALID;
+    // the rotated Q and K are written while other CTAs still read q and k, and the
+    // attention reads them while it writes o and lse
+    const size_t ws = mf_workspace_size(T, H, D, 1);
+    if (overlap(workspace, ws, q, bytes) || overlap(workspace, ws, k, bytes) ||
+        overlap(workspace, ws, v, bytes) || overlap(workspace, ws, o, bytes) ||
+        overlap(workspace, ws, pos_ids, static_cast<size_t>(T) * 12) ||
+        (lse && overlap(workspace, ws, lse, static_cast<size_t>(T) * H * 4)))
+      return MF_ERR_INVALID;
     const uintptr_t w0 = round_up(reinterpret_cast<uintptr_t>(workspace), 256);
-    mf_bf16* wq = reinterpret_cast<mf_bf16*>(w0);
-    mf_bf16* wk = reinterpret_cast<mf_bf16*>(w0 + round_up(bytes, 256));
+    qa = reinterpret_cast<mf_bf16*>(w0);
+    ka = reinterpret_cast<mf_bf16*>(w0 + round_up(bytes, 256));
+  }
+  KernelCtl ctl;
+  if (cudaError_t ge = get_ctl(&ctl); ge != cudaSuccess) return cuda_status(ge);
+  if (pos_ids != nullptr) {
     RopeTable tab;
     make_rope_table(D, rope_axes, base, &tab);
-    cudaError_t e = launch_rope(q, k, pos_ids, T, H, D, tab, wq, wk, stream);
+    cudaError_t e = launch_rope(q, k, pos_ids, T, H, D, tab, const_cast<mf_bf16*>(qa),
+                                const_cast<mf_bf16*>(ka), stream);
     if (e != cudaSuccess) return cuda_status(e);
-    qa = wq;
-    ka = wk;
   }
   AttnEpilogue ep{};
   ep.o = o;
@@ -469,7 +477,17 @@ mf_status mf_block_fwd(const mf_bf16* x, const mf_bf16* q, const mf_bf16* k, con
   for (const void* in : ins)
     if (overlap(in, bytes, x_mod, bytes) || overlap(in, bytes, y, bytes)) return MF_ERR_INVALID;
   if (overlap(x_mod, bytes, y, bytes)) return MF_ERR_INVALID;
-  if (overlap(workspace, ws_bytes, x_mod, bytes) || overlap(workspace, ws_bytes, y, bytes))
+  // The rotated Q and K are written into the workspace while other CTAs still
+  // read q and k, and the fused epilogue reads x, v and mod while y is written:
+  // the workspace and the outputs must stay clear of every input.
+  const size_t ws = mf_workspace_size(T, H, D, 1);
+  const size_t mod_bytes = static_cast<size_t>(S) * 6 * hid * 4;
+  for (const void* in : ins)
+    if (overlap(workspace, ws, in, bytes)) return MF_ERR_INVALID;
+  if (overlap(workspace, ws, mod, mod_bytes) || overlap(workspace, ws, x_mod, bytes) ||
+      overlap(workspace, ws, y, bytes) || overlap(workspace, ws, pos_ids, static_cast<size_t>(T) * 12))
+    return MF_ERR_INVALID;
+  if (overlap(x_mod, bytes, mod, mod_bytes) || overlap(y, bytes, mod, mod_bytes))
     return MF_ERR_INVALID;
   KernelCtl ctl;
   if (cudaError_t ge = get_ctl(&ctl); ge != cudaSuccess) return cuda_status(ge);

@@ -61,8 +61,9 @@ extern "C" mf_status mf_block_fwd_noalloc(
     int32_t rope_axes, float base, float eps, mf_bf16* x_mod, mf_bf16* y, cudaStream_t stream) {
   if (cu_seqlens_h == nullptr || S < 1 || S > MF_MAX_SAMPLES || H < 1 || D < 1)
     return MF_ERR_INVALID;
-  const int32_t T = cu_seqlens_h[S];
-  if (T < 0) return MF_ERR_INVALID;
+  // a malformed pack is an argument error whatever its size
+  int32_t T = 0;
+  if (!mf::check_offsets(cu_seqlens_h, S, &T)) return MF_ERR_INVALID;
   const size_t need = mf_workspace_size(T, H, D, 1);
   if (need > MF_NOALLOC_SCRATCH_BYTES) return MF_ERR_UNSUPPORTED;  // pack too large
   void* scratch = nullptr;

@@ -21,6 +21,10 @@ from packgen import Workload, bf16_bits_to_f32
 
 MAX_ABS = 2e-2
 REL_RMS = 5e-3
+# gradients of the attention: relative to each tensor and sample (see
+# assert_grad_close)
+GRAD_REL_RMS = 5e-3
+GRAD_MAX_REL = 2.0 ** -5
 
 
 def dev_bf16(bits: np.ndarray) -> torch.Tensor:
@@ -119,3 +123,41 @@ def sample_rows(cu: np.ndarray, per_sample: int, seed: int) -> np.ndarray:
 
 def oracle_pack(w: Workload):
     return oracle.pack_build(w.descs, w.rope_axes)
+
+
+def zero_grad_bound(q, k, v, d_o, D: int) -> float:
+    """A one-token sample has P = 1, so dS = dP - rowsum(dO * O) = dO.v - dO.v is
+    exactly 0 and so are its dQ and dK. The kernel forms the two dot products in
+    fp32 in different orders (tensor-core dP against the row table's delta, from
+    O = v stored in bf16, which is exact), so their difference is bounded by the
+    fp32 summation bound of two D-term sums, 2 * D * 2^-24 * sum|dO v|; dQ and dK
+    are that times scale * max|k| (resp. |q|)."""
+    terms = np.abs(d_o.astype(np.float64) * v.astype(np.float64)).sum(axis=-1).max()
+    big = max(np.abs(q).max(), np.abs(k).max())
+    return float(2 * D * 2.0 ** -24 * terms / math.sqrt(D) * big)
+
+
+def assert_grad_close(gpu: np.ndarray, ref: np.ndarray, cu, name: str, zero_tol=0.0) -> list:
+    """Per sample: relative RMS <= GRAD_REL_RMS and max error <= GRAD_MAX_REL * max|ref|;
+    for dQ and dK (zero_tol > 0) a one-token sample, whose exact gradient is 0
+    (see zero_grad_bound), must stay within zero_tol."""
+    stats = []
+    assert np.isfinite(gpu).all(), f"{name}: non-finite gradient"
+    for s in range(len(cu) - 1):
+        lo, hi = int(cu[s]), int(cu[s + 1])
+        if hi == lo:
+            continue
+        g, r = gpu[lo:hi].astype(np.float64), ref[lo:hi]
+        if hi - lo == 1 and zero_tol > 0:  # dQ, dK of a one-token sample: exactly 0
+            worst = float(np.abs(g).max())
+            stats.append((name, s, hi - lo, 0.0, worst))
+            assert worst <= zero_tol, f"{name} sample {s}: exact zero, got {worst:.3g} > {zero_tol:.3g}"
+            continue
+        scale = float(np.abs(r).max())
+        err = np.abs(g - r)
+        rr = float(np.linalg.norm(g - r) / max(np.linalg.norm(r), 1e-300))
+        mr = float(err.max() / max(scale, 1e-300))
+        stats.append((name, s, hi - lo, rr, mr))
+        assert rr <= GRAD_REL_RMS, f"{name} sample {s}: relative RMS {rr:.3g} > {GRAD_REL_RMS}"
+        assert mr <= GRAD_MAX_REL, f"{name} sample {s}: max error {mr:.3g} of max|ref| > {GRAD_MAX_REL}"
+    return stats

@@ -208,3 +208,57 @@ def test_gate_and_adaln_backward_argument_checks_without_gpu():
     assert ln(w=x) == mf.MF_ERR_INVALID                          # workspace overlaps x
     assert lib.mf_adaln_modulate_bwd(dxm, x, mod, ts, tm, None, T, S, hid, 1e-6, dx, x, w, ws,
                                      None) == mf.MF_ERR_INVALID  # dmod overlaps x
+
+
+def test_forward_workspace_and_output_overlap_checks_without_gpu():
+    """The forward entry points refuse a workspace that overlaps an input or an
+    output, and outputs that overlap the modulation vectors: the rotated Q and K
+    are written while other CTAs still read q and k, and the fused epilogue
+    reads x, v and mod while y is written."""
+    lib = mf.lib
+    P = ctypes.c_void_p
+    MB = 1 << 20
+    T, H, D = 128, 2, 64
+    cu = np.array([0, T], dtype=np.int32)
+    x, q, k, v, mod, xm, y, ws, pos = (P((i + 1) * MB) for i in range(9))
+    wsb = mf.mf_workspace_size(T, H, D, 1)
+
+    def blk(ws=ws, xm=xm, y=y, mod=mod, pos=pos):
+        return lib.mf_block_fwd(x, q, k, v, mod, P(16), cu.ctypes.data_as(P), pos, P(16), P(16),
+                                1, H, D, 2, 10000.0, 1e-6, xm, y, ws, wsb, None)
+
+    for bad in (x, q, k, v, mod, xm, y, pos):
+        assert blk(ws=bad) == mf.MF_ERR_INVALID
+    assert blk(ws=P(q.value + 4096)) == mf.MF_ERR_INVALID   # partial overlap
+    assert blk(xm=mod) == mf.MF_ERR_INVALID
+    assert blk(y=P(mod.value + 256)) == mf.MF_ERR_INVALID
+
+    def attn(ws=ws, o=y, lse=None):
+        return lib.mf_varlen_attn_fwd(q, k, v, P(16), cu.ctypes.data_as(P), 1, H, D, 0.125, pos,
+                                      2, 10000.0, o, lse, ws, wsb, None)
+
+    for bad in (q, k, v, y, pos):
+        assert attn(ws=bad) == mf.MF_ERR_INVALID
+    assert attn(lse=ws) == mf.MF_ERR_INVALID
+
+
+@pytest.mark.parametrize("offsets", [[5, 100], [0, 50000, 40000, 9000000],
+                                     [0, (1 << 24) + 64]])
+def test_noalloc_rejects_malformed_offsets_as_invalid(offsets):
+    """A malformed pack is an argument error whatever its last offset (the size
+    test against the fixed array comes after the offsets are validated)."""
+    P = ctypes.c_void_p
+    cu = np.array(offsets, dtype=np.int32)
+    st = mf.lib.mf_block_fwd_noalloc(P(16), P(16), P(16), P(16), P(16), P(16),
+                                     cu.ctypes.data_as(P), P(16), P(16), P(16), len(cu) - 1, 24,
+                                     128, 2, 10000.0, 1e-6, P(16), P(16), None)
+    assert st == mf.MF_ERR_INVALID
+
+
+def test_noalloc_size_limit_without_gpu():
+    P = ctypes.c_void_p
+    cu = np.array([0, 16384], dtype=np.int32)  # 2 x 16384 x 3072 bf16 = 201 MB of rotated Q, K
+    st = mf.lib.mf_block_fwd_noalloc(P(16), P(16), P(16), P(16), P(16), P(16),
+                                     cu.ctypes.data_as(P), P(16), P(16), P(16), 1, 24, 128, 2,
+                                     10000.0, 1e-6, P(16), P(16), None)
+    assert st == mf.MF_ERR_UNSUPPORTED

@@ -4,17 +4,19 @@ ABI) against the float64 oracle on the same seeded inputs.
 The GPU side runs the library's own forward for O and the log-sum-exp, then
 the backward; the oracle differentiates the same bf16 q, k, v and dO in float64
 (its own forward inside). Small packs are compared in full (ragged tiles, empty
-samples, both head sizes, several query and key tiles per sample); the training
-and packed-CFG packs at full size on two heads (the oracle works head by head,
-so a head subset is the same computation).
+samples, both head sizes, several query and key tiles per sample); the
+training, packed-CFG, edit and large packs at full size on two heads (the oracle
+works head by head, so a head subset is the same computation).
 
-Tolerance, from the arithmetic: P and dS are rounded to bf16 before their
-products (relative error up to 2^-9 each), O enters rowsum(dO * O) as bf16,
-and each output is stored as bf16 (half an ulp). Every output element is a sum
-of many such terms with independent rounding, so the error relative to the
-tensor's own scale stays a small multiple of 2^-9: the test asks for a relative
-RMS error <= 1e-2 per tensor and per sample, and a largest error <= 2^-5 of the
-largest reference magnitude of that tensor and sample.
+Tolerance: the stated one for bf16-in / fp32-accumulate outputs, relative RMS
+error <= 5e-3, taken per tensor and per sample (the gradients' scale varies
+from sample to sample), and a largest error <= 2^-5 of the largest reference
+magnitude of that tensor and sample in place of the absolute 2e-2 (|dq| is of
+the order of 1e-2 at these shapes, so an absolute bound would not test it).
+Sources of error: P and dS are rounded to bf16 before their products (relative
+error up to 2^-9 each), O enters rowsum(dO * O) as bf16, and each output is
+stored as bf16; every output element is a sum of many such terms with
+independent rounding.
 """
 
 from __future__ import annotations
@@ -34,10 +36,8 @@ if not torch.cuda.is_available():
     pytest.skip("needs a CUDA device", allow_module_level=True)
 
 import resolution_packed_diffusion_b200 as mf  # noqa: E402
-from gpu_util import DevicePack, dev_bf16, host_f32, oracle_pack  # noqa: E402
-
-REL_RMS = 1e-2
-MAX_REL = 2.0 ** -5
+from gpu_util import (DevicePack, assert_grad_close, dev_bf16, host_f32, oracle_pack,  # noqa: E402
+                      zero_grad_bound)
 
 
 def gpu_backward(dp: DevicePack, d_o: torch.Tensor, heads=None):
@@ -62,44 +62,6 @@ def gpu_backward(dp: DevicePack, d_o: torch.Tensor, heads=None):
                           ws, ws_bytes)
     assert mf.mf_get_error() == mf.MF_OK
     return host_f32(dq), host_f32(dk), host_f32(dv)
-
-
-def zero_grad_bound(q, k, v, d_o, D: int) -> float:
-    """A one-token sample has P = 1, so dS = dP - rowsum(dO * O) = dO.v - dO.v is
-    exactly 0 and so are its dQ and dK. The kernel forms the two dot products in
-    fp32 in different orders (tensor-core dP against the row table's delta, from
-    O = v stored in bf16, which is exact), so their difference is bounded by the
-    fp32 summation bound of two D-term sums, 2 * D * 2^-24 * sum|dO v|; dQ and dK
-    are that times scale * max|k| (resp. |q|)."""
-    terms = np.abs(d_o.astype(np.float64) * v.astype(np.float64)).sum(axis=-1).max()
-    big = max(np.abs(q).max(), np.abs(k).max())
-    return float(2 * D * 2.0 ** -24 * terms / math.sqrt(D) * big)
-
-
-def assert_grad_close(gpu: np.ndarray, ref: np.ndarray, cu, name: str, zero_tol=0.0) -> list:
-    """Per sample: relative RMS <= REL_RMS and max error <= MAX_REL * max|ref|;
-    for dQ and dK (zero_tol > 0) a one-token sample, whose exact gradient is 0
-    (see zero_grad_bound), must stay within zero_tol."""
-    stats = []
-    assert np.isfinite(gpu).all(), f"{name}: non-finite gradient"
-    for s in range(len(cu) - 1):
-        lo, hi = int(cu[s]), int(cu[s + 1])
-        if hi == lo:
-            continue
-        g, r = gpu[lo:hi].astype(np.float64), ref[lo:hi]
-        if hi - lo == 1 and zero_tol > 0:  # dQ, dK of a one-token sample: exactly 0
-            worst = float(np.abs(g).max())
-            stats.append((name, s, hi - lo, 0.0, worst))
-            assert worst <= zero_tol, f"{name} sample {s}: exact zero, got {worst:.3g} > {zero_tol:.3g}"
-            continue
-        scale = float(np.abs(r).max())
-        err = np.abs(g - r)
-        rr = float(np.linalg.norm(g - r) / max(np.linalg.norm(r), 1e-300))
-        mr = float(err.max() / max(scale, 1e-300))
-        stats.append((name, s, hi - lo, rr, mr))
-        assert rr <= REL_RMS, f"{name} sample {s}: relative RMS {rr:.3g} > {REL_RMS}"
-        assert mr <= MAX_REL, f"{name} sample {s}: max error {mr:.3g} of max|ref| > {MAX_REL}"
-    return stats
 
 
 def check(w, heads=None, seed=0):
@@ -139,10 +101,23 @@ def test_backward_small_packs_full_compare(k):
     check(w, seed=900 + k)
 
 
-@pytest.mark.parametrize("idx", [2, 3], ids=["training_pack", "cfg_pack"])
+@pytest.mark.parametrize("idx", [2, 3, 4, 5],
+                         ids=["training_pack", "cfg_pack", "edit_pack", "large_pack"])
 def test_backward_full_size_two_heads(idx):
     """The workloads at full size; heads 0 and H-1 are compared (the oracle's
-    cost grows with n^2 per head)."""
+    cost grows with n^2 per head). The large pack's 16896-token sample is the
+    longest key walk of the kernel and the most dQ reductions per query tile;
+    the oracle holds its n x n score, probability and gradient matrices in
+    float64 (about 2.3 GB each)."""
+    need_gb = {2: 4, 3: 4, 4: 12, 5: 16}[idx]
+    try:
+        import psutil
+        free_gb = psutil.virtual_memory().available / 2 ** 30
+    except ImportError:
+        free_gb = float("inf")
+    if free_gb < 2 * need_gb:
+        pytest.skip(f"the float64 oracle needs about {need_gb} GB of host memory "
+                    f"({free_gb:.0f} GB available)")
     w = make_workload(idx)
     check(w, heads=[0, w.H - 1], seed=idx)
 

@@ -137,13 +137,9 @@ def test_block_fwd(case):
                                         case.pack, w.rope_axes, rows=rows)
     assert_bf16_close(host_f32(x_mod)[rows], ref_xm, "block x_mod")
     assert_bf16_close(host_f32(y)[rows], ref_y, "block y")
-    # the attention branch alone, recovered from y: gate * O = y - x
-    gate = case.mod[case.pack["tok_sample"][rows], case.pack["tok_mod"][rows], 2]
-    x = w.f32("x")[rows].astype(np.float64)
     # deterministic: a second run gives the same bits
     x_mod2, y2 = dp.block()
     assert torch.equal(x_mod, x_mod2) and torch.equal(y, y2)
-    assert gate.shape == x.shape
 
 
 # ------------------------------------------------------------------ edge cases

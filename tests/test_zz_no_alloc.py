@@ -4,14 +4,16 @@ caller that must not make a call which can synchronise the device). It keeps the
 rotated Q and K in the library's own fixed device array instead of a
 caller-provided workspace.
 
-Checked through the C ABI against mf_block_fwd (which takes a workspace) on two
-calls in a row, with the tolerance the parity tests use. This file is collected
-last on purpose and needs nothing from the other test files."""
+Checked through the C ABI on two calls in a row against mf_block_fwd (which
+takes a workspace) and against the float64 oracle, with the tolerance the parity
+tests use. This file is collected last on purpose and needs nothing from the
+other test files."""
 
 import numpy as np
 import pytest
 import torch
 
+import oracle
 from packgen import SampleDesc, make_random_pack, make_workload
 
 pytestmark = pytest.mark.gpu
@@ -20,7 +22,7 @@ if not torch.cuda.is_available():
     pytest.skip("needs a CUDA device", allow_module_level=True)
 
 import resolution_packed_diffusion_b200 as mf  # noqa: E402
-from gpu_util import DevicePack, assert_bf16_close, host_f32  # noqa: E402
+from gpu_util import DevicePack, assert_bf16_close, host_f32, oracle_pack  # noqa: E402
 
 
 def _noalloc(dp):
@@ -45,15 +47,22 @@ PACKS = [
 
 @pytest.mark.parametrize("name,make", PACKS, ids=[p[0] for p in PACKS])
 def test_noalloc_matches_workspace_entry_point_twice(name, make):
-    dp = DevicePack(make())
+    w = make()
+    dp = DevicePack(w)
     ref_xm, ref_y = dp.block()
     assert mf.mf_get_error() == mf.MF_OK
     ref_xm, ref_y = host_f32(ref_xm), host_f32(ref_y)
+    mod = oracle.adaln_params(w.c, w.W, w.hid)
+    o_xm, o_y, _ = oracle.block_fwd(w.f32("x"), w.f32("q"), w.f32("k"), w.f32("v"), mod,
+                                    oracle_pack(w), w.rope_axes, w.base, w.eps)
     for call in range(2):  # the array keeps the previous call's contents
         x_mod, y = _noalloc(dp)
         assert mf.mf_get_error() == mf.MF_OK
-        assert_bf16_close(host_f32(x_mod), ref_xm, f"{name}: x_mod, call {call}")
-        assert_bf16_close(host_f32(y), ref_y, f"{name}: y, call {call}")
+        x_mod, y = host_f32(x_mod), host_f32(y)
+        assert_bf16_close(x_mod, ref_xm, f"{name}: x_mod vs mf_block_fwd, call {call}")
+        assert_bf16_close(y, ref_y, f"{name}: y vs mf_block_fwd, call {call}")
+        assert_bf16_close(x_mod, o_xm, f"{name}: x_mod vs oracle, call {call}")
+        assert_bf16_close(y, o_y, f"{name}: y vs oracle, call {call}")
 
 
 def test_noalloc_rejects_a_pack_beyond_its_array():
