@@ -710,7 +710,8 @@ def run_block_bwd(args, rank, world, local_rank):
     from upstream gradients dy (of y) and dx_mod (of x_mod): gate backward
     (dO, dgate), attention backward (dq, dk, dv of the rotated q, k from O and
     the log-sum-exp), RoPE backward, adaLN backward (dx = dy + the LayerNorm
-    path, dshift, dscale). The forward state (rotated q and k, O, LSE) is
+    path, dshift, dscale) and the modulation map's backward (dc, dW). The
+    forward state (rotated q and k, O, LSE) is
     computed once before the timed region. Useful FLOPs: the attention
     backward's 10 * D * H * sum(n_s^2) over the real samples."""
     import torch
@@ -756,6 +757,8 @@ def run_block_bwd(args, rank, world, local_rank):
     aws = torch.empty(abw, dtype=torch.uint8, device=dev)
     lbw = mf.mf_adaln_bwd_workspace_size(T)
     lws = torch.empty(max(lbw, 16), dtype=torch.uint8, device=dev)
+    dc = torch.empty_like(c)
+    dWm = torch.empty_like(Wm)
 
     def step():
         mf.mf_gated_residual_bwd(dy, o, mod, ts, tm, T, S, hid, d_o, dmod, stream)
@@ -764,6 +767,7 @@ def run_block_bwd(args, rank, world, local_rank):
         mf.mf_rope_bwd(dq_r, dk_r, pos, T, H, D, w.rope_axes, w.base, dq, dk, stream)
         mf.mf_adaln_modulate_bwd(dxm, x, mod, ts, tm, dy, T, S, hid, w.eps, dx, dmod, lws, lbw,
                                  stream)
+        mf.mf_adaln_params_bwd(dmod, c, Wm, S, c.shape[1], hid, dc, dWm, stream)
 
     def barrier():
         if world > 1:
@@ -808,7 +812,7 @@ def run_block_bwd(args, rank, world, local_rank):
                      "frac": achieved / peak, "traffic": None,
                      "kernel": "whole backward step (attn_bwd_kernel dominant)",
                      "peak_source": f"{peak_src} bf16_tflops (burst)"},
-        "gpu_launches": 9 * args.steps, "clocks": clk}), flush=True)
+        "gpu_launches": 11 * args.steps, "clocks": clk}), flush=True)
 
 
 ARMS = {"block": "run_gpu", "linear": "run_linear", "mmdit": "run_mmdit",

@@ -184,6 +184,18 @@ mf_status mf_varlen_attn_bwd(const mf_bf16* q, const mf_bf16* k, const mf_bf16* 
                              size_t ws_bytes, cudaStream_t stream);
 size_t mf_attn_bwd_workspace_size(int32_t T, int32_t S, int32_t H, int32_t D);
 
+/* Backward of mf_adaln_params [norm], [train]: with mod = c W (mod flattened to
+ * [S][6*hid]), dW = c^T dmod and dc = dmod W^T. dmod: [S][2][3][hid] fp32, the
+ * gradient of the modulation vectors (the shift, scale and gate slots that
+ * mf_adaln_modulate_bwd and mf_gated_residual_bwd write); c: [S][C] and
+ * W: [C][6*hid] fp32 as in the forward. Outputs, either of which may be NULL
+ * (not both): dc [S][C] fp32 and dW [C][6*hid] fp32, overwritten, disjoint from
+ * every input and from each other. Same shape limits as mf_adaln_params. fp32
+ * arithmetic; every sum is taken in a fixed order (no atomics), so repeated
+ * calls give the same bits. */
+mf_status mf_adaln_params_bwd(const float* dmod, const float* c, const float* W, int32_t S,
+                              int32_t C, int32_t hid, float* dc, float* dW, cudaStream_t stream);
+
 /* Gated residual [fuse]: y[t] = x[t] + gate[s,m] * o[t], o viewed as [T][H*D].
  * x, o, y: [T][hid] bf16 (y may equal x). Same id checks as mf_adaln_modulate. */
 mf_status mf_gated_residual(const mf_bf16* x, const mf_bf16* o, const float* mod,
@@ -235,10 +247,11 @@ mf_status mf_block_fwd(const mf_bf16* x, const mf_bf16* q, const mf_bf16* k, con
  * device memory and gives it no allocator, or a caller that must not make a call
  * which can synchronise the device). The paper has no counterpart: this is a
  * library convenience. Arguments and results are those of mf_block_fwd; the
- * rotated Q and K go to a file-scope device array of MF_NOALLOC_SCRATCH_BYTES
- * that every GPU loading the library holds until exit, so a pack needs
- * mf_workspace_size(T, H, D, 1) <= MF_NOALLOC_SCRATCH_BYTES (about 5400 tokens at
- * H*D = 3072); a larger pack returns MF_ERR_UNSUPPORTED and launches nothing.
+ * workspace mf_block_fwd would take (the fused RoPE's (cos, sin) table and the
+ * rotated k) is a file-scope device array of MF_NOALLOC_SCRATCH_BYTES that every
+ * GPU loading the library holds until exit, so a pack needs
+ * mf_workspace_size(T, H, D, 1) <= MF_NOALLOC_SCRATCH_BYTES (about 10400 tokens
+ * at H*D = 3072); a larger pack returns MF_ERR_UNSUPPORTED and launches nothing.
  * The function allocates nothing. Its first call on a device looks up the array's
  * device address (cudaGetSymbolAddress) with that device current; make that
  * first call before any stream capture. All calls share the array: calls that
@@ -313,7 +326,8 @@ mf_status mf_mmdit_block_fwd(const mf_bf16* x, const mf_bf16* Wq, const mf_bf16*
 size_t mf_mmdit_workspace_size(int32_t T, int32_t H, int32_t D, int32_t F);
 
 /* Bytes of workspace mf_varlen_attn_fwd / mf_block_fwd need (with_rope != 0:
- * room for the rotated Q and K). */
+ * room for the fused RoPE's (cos, sin) table, T x D/4 float2, and the rotated
+ * k, T x H x D bf16; q is turned inside the attention's load prologue). */
 size_t mf_workspace_size(int32_t T, int32_t H, int32_t D, int32_t with_rope);
 
 /* Synchronises `stream`, returns and clears the device error word of the

@@ -60,6 +60,7 @@ _SIGS = {
     "mf_pack_build": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
     "mf_adaln_params": (_I, [_P, _P, _I, _I, _I, _P, _P]),
     "mf_adaln_modulate": (_I, [_P, _P, _P, _P, _I, _I, _I, _F, _P, _P]),
+    "mf_adaln_params_bwd": (_I, [_P, _P, _P, _I, _I, _I, _P, _P, _P]),
     "mf_rope_apply": (_I, [_P, _P, _P, _I, _I, _I, _I, _F, _P, _P, _P]),
     "mf_rope_bwd": (_I, [_P, _P, _P, _I, _I, _I, _I, _F, _P, _P, _P]),
     "mf_varlen_attn_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _F, _P, _I, _F, _P, _P, _P,
@@ -166,6 +167,11 @@ def mf_pack_build(descs, rope_axes: int, budget: int = 0, cu_seqlens_d=None, pos
 def mf_adaln_params(c, W, S: int, C: int, hid: int, mod, stream=None) -> None:
     _check(lib.mf_adaln_params(_ptr(c), _ptr(W), S, C, hid, _ptr(mod), _stream(stream)),
            "mf_adaln_params")
+
+
+def mf_adaln_params_bwd(dmod, c, W, S: int, C: int, hid: int, dc, dW, stream=None) -> None:
+    _check(lib.mf_adaln_params_bwd(_ptr(dmod), _ptr(c), _ptr(W), S, C, hid, _ptr(dc), _ptr(dW),
+                                   _stream(stream)), "mf_adaln_params_bwd")
 
 
 def mf_adaln_modulate(x, mod, tok_sample, tok_mod, T: int, S: int, hid: int, eps: float, x_mod,

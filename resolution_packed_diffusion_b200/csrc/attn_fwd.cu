@@ -31,8 +31,21 @@
 //               tile's row sum stays below 2^32 (which bounds every P); only
 //               then is the reference moved to the tile max, O rescaled in TMEM
 //               and the tile redone (exact after the final 1/l: a stale
-//               reference scales numerator and denominator alike). P is packed to bf16 into the first 64
-//               columns of the tile's S region.
+//               reference scales numerator and denominator alike). P is packed
+//               to bf16 into the first 64 columns of the tile's S region. With
+//               RoPE fused, each thread first turns its own query row of the
+//               item's Q tile in shared memory.
+// RoPE in the load prologue ([rope]: per-sample 2D / 3D rotary embeddings; the
+// pages name it among the fused operations of the block): q is read unrotated
+// and every pair of a Q tile's row turns in shared memory by (cos, sin) looked
+// up for the token's position in a small per-position table (one set of
+// columns serves every axis), so no rotated copy of q reaches memory. The next
+// item's Q tiles land in shared memory as the item's last S MMAs complete; the
+// softmax warps turn them right after the item's last P if they have landed
+// (else after the epilogue). K arrives
+// rotated by a RoPE pass over k: a K tile is visited by every query block of
+// its sample and head, and turning it at each visit (8192 pair rotations per
+// tile by the two idle warps) measured 1.6x slower than the pass.
 // TMEM (512 columns): S_A/P_A | S_B/P_B | O_A | O_B.
 // Work items are ordered longest sample first and, inside a sample, the query
 // blocks of one head next to each other so that concurrently running CTAs stream
@@ -99,9 +112,11 @@ struct Layout {
   static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
   static constexpr int OFF_V = OFF_K + NK * TILE_BYTES;
   static constexpr int OFF_BAR = OFF_V + NV * TILE_BYTES;
-  // barriers (arrival count 1 unless arrivals() says one per softmax warp)
-  static constexpr int B_Q_FULL = 0, B_Q_EMPTY = 1;
-  static constexpr int B_K_FULL = 2;                 // NK
+  // barriers (arrival count 1 unless arrivals() says otherwise)
+  static constexpr int B_Q_FULL = 0;                 // [tile]
+  static constexpr int B_Q_EMPTY = B_Q_FULL + 2;     // [tile]
+  static constexpr int B_Q_ROT = B_Q_EMPTY + 2;      // [tile], one arrival per softmax warp
+  static constexpr int B_K_FULL = B_Q_ROT + 2;       // NK
   static constexpr int B_K_EMPTY = B_K_FULL + NK;    // NK
   static constexpr int B_V_FULL = B_K_EMPTY + NK;    // NV
   static constexpr int B_V_EMPTY = B_V_FULL + NV;    // NV
@@ -122,9 +137,10 @@ struct Layout {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget of one CTA");
 
   __device__ static uint32_t arrivals(int i) {
-    return (i == B_P_FULL || i == B_P_FULL + 1 || i == B_O_EMPTY || i == B_O_EMPTY + 1)
-               ? kSoftmaxWarpsPerTile
-               : 1u;
+    if (i == B_P_FULL || i == B_P_FULL + 1 || i == B_O_EMPTY || i == B_O_EMPTY + 1 ||
+        i == B_Q_ROT || i == B_Q_ROT + 1)
+      return kSoftmaxWarpsPerTile;
+    return 1u;
   }
 };
 
@@ -141,12 +157,24 @@ struct Schedule {
   int32_t ids[kMaxSchedItems + kMaxSchedCtas];  // items plus one end mark per CTA
 };
 
+// RoPE fused into the load prologue: pair i of axis a turns by the (cos, sin)
+// at tab[pos_a][i] (one row of D / (2 axes) pairs per position; every axis
+// uses the same frequencies).
+struct AttnRope {
+  const int32_t* pos_ids;  // [T][3] (f, h, w)
+  const float2* tab;       // [P][D / (2 axes)]
+  int32_t P;
+};
+
+
+
 struct AttnArgs {
   Schedule sched;
   const int32_t* cu_seqlens;
   int32_t S, T, H;
   float scale_log2;  // softmax_scale * log2(e)
   AttnEpilogue ep;
+  AttnRope rope;
   KernelCtl ctl;
 };
 
@@ -199,7 +227,87 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint6
   }
 }
 
-template <int D, bool GATED>
+// Rotates one row of a 128-row tile in shared memory (TMA layout: D / 64 boxes
+// of 128 rows x 128 bytes, 16-byte chunks swizzled by row & 7) by the RoPE of
+// the token at position (p0, p1, p2) = (f, h, w): pair (2i, 2i+1) turns by
+// the angle whose (cos, sin) the table holds for the position on the pair's axis. The pair -> (axis, column) map
+// is fixed by D and the axis count: every axis owns NPA = D / (2 AXES)
+// consecutive pairs, in axis order (h, w) or (f, h, w); pairs past them stay.
+// fp32 arithmetic, bf16 result, the same rounding as the standalone RoPE pass.
+// G chunks (4G pairs) at a time: their shared-memory words and table entries
+// are all requested before any is used. A position outside the table is
+// recorded as MF_ERR_INVALID and leaves the row as it is.
+template <int D, int AXES, int G>
+__device__ __forceinline__ void rope_row_smem(uint8_t* tile, int row, int p0, int p1, int p2,
+                                              const float2* tab, int P, const KernelCtl& ctl) {
+  static_assert(AXES == 0 || AXES == 2 || AXES == 3, "RoPE axis count");
+  if constexpr (AXES == 0) return;  // no RoPE: nothing to turn
+  constexpr int NPA = D / (2 * (AXES == 0 ? 1 : AXES));  // pairs per axis (= table columns)
+  constexpr int NCH = D / 8;           // 16-byte chunks per row
+  static_assert(NCH % G == 0, "chunks per batch");
+  if (static_cast<unsigned>(p0) >= static_cast<unsigned>(P) ||
+      static_cast<unsigned>(p1) >= static_cast<unsigned>(P) ||
+      static_cast<unsigned>(p2) >= static_cast<unsigned>(P)) {
+    atomicCAS(ctl.err, 0, static_cast<int>(MF_ERR_INVALID));
+    return;
+  }
+  // table rows of the axes in pair order: (h, w) for 2D, (f, h, w) for 3D
+  const float2* rt[3] = {tab + static_cast<size_t>(AXES == 2 ? p1 : p0) * NPA,
+                         tab + static_cast<size_t>(AXES == 2 ? p2 : p1) * NPA,
+                         tab + static_cast<size_t>(p2) * NPA};
+  uint8_t* rbase = tile + row * 128;
+#pragma unroll
+  for (int c0 = 0; c0 < NCH; c0 += G) {
+    uint4* ptr[G];
+    uint4 v[G];
+    float2 cs[G][4];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const int c = c0 + g;  // chunk in the head row: box c / 8, chunk c % 8 of the box
+      ptr[g] = reinterpret_cast<uint4*>(rbase + (c >> 3) * BOX_BYTES +
+                                        (((c & 7) ^ (row & 7)) << 4));
+      v[g] = *ptr[g];
+      if constexpr (NPA % 4 == 0) {
+        // the chunk's four pairs share one axis and are four consecutive columns
+        const int a = (4 * c) / NPA;
+        if (a < AXES) {
+          const float4* src = reinterpret_cast<const float4*>(rt[a] + (4 * c - a * NPA));
+          const float4 lo = __ldg(src), hi = __ldg(src + 1);
+          cs[g][0] = make_float2(lo.x, lo.y);
+          cs[g][1] = make_float2(lo.z, lo.w);
+          cs[g][2] = make_float2(hi.x, hi.y);
+          cs[g][3] = make_float2(hi.z, hi.w);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int pr = 4 * c + e;
+          const int a = pr / NPA;
+          if (a < AXES) cs[g][e] = __ldg(rt[a] + (pr - a * NPA));
+        }
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const int c = c0 + g;
+      uint32_t w[4] = {v[g].x, v[g].y, v[g].z, v[g].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int pr = 4 * c + e;
+        if (pr / NPA < AXES) {
+          const float x0 = __uint_as_float(w[e] << 16);
+          const float x1 = __uint_as_float(w[e] & 0xFFFF0000u);
+          w[e] = pack_bf16x2(x0 * cs[g][e].x - x1 * cs[g][e].y, x0 * cs[g][e].y + x1 * cs[g][e].x);
+        }
+      }
+      *ptr[g] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+}
+
+// AXES: 0 = q and k arrive rotated; 2 or 3 = RoPE with that many axes fused
+// into the Q load prologue (k arrives rotated).
+template <int D, bool GATED, int AXES>
 // Registers are split per SM sub-partition: with 12 warps each sub-partition
 // holds three, which caps a thread at 16384 / (3 * 32) = 170 -> 168 at launch.
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -208,6 +316,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                        const __grid_constant__ CUtensorMap tmap_v,
                        const __grid_constant__ AttnArgs args) {
   using L = Layout<D>;
+  constexpr bool ROPE = AXES != 0;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the 128-byte-swizzled TMA / UMMA tiles
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -293,7 +402,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // consumes S(j+1) before PV_B(j), so K runs one tile ahead of V.
     if (lane == 0) {
       uint32_t kc = 0, vc = 0;  // K / V tiles issued so far (global over items)
-      int n_item = 0;
+      uint32_t nq[2] = {0, 0};  // Q tiles issued per tile slot
       bool ok = true;
       auto load_k = [&](const WorkItem& wi, int j) -> bool {
         const int st = kc % NK;
@@ -317,16 +426,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ++vc;
         return true;
       };
-      for (int k = 0, w = item_k(0); w < total_items && ok; w = item_k(++k), ++n_item) {
+      for (int k = 0, w = item_k(0); w < total_items && ok; w = item_k(++k)) {
         const WorkItem wi = decode_item(w, S, s_cu, s_order, s_istart);
-        if (!mbar_wait(&bars[L::B_Q_EMPTY], (n_item & 1) ^ 1, args.ctl, abort_flag)) break;
         const int ntiles = wi.has_b ? 2 : 1;
-        mbar_expect_tx(&bars[L::B_Q_FULL], ntiles * L::TILE_BYTES);
-        for (int x = 0; x < ntiles; ++x)
+        // each query tile has its own full / empty barriers, so the warps of
+        // tile B only ever see the phases of items that hold a tile B
+        for (int x = 0; x < ntiles && ok; ++x) {
+          if (!mbar_wait(&bars[L::B_Q_EMPTY + x], (nq[x] & 1) ^ 1, args.ctl, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(&bars[L::B_Q_FULL + x], L::TILE_BYTES);
 #pragma unroll
           for (int b = 0; b < L::kBoxes; ++b)
-            tma_load_2d(sQ + x * L::TILE_BYTES + b * BOX_BYTES, &tmap_q, &bars[L::B_Q_FULL],
+            tma_load_2d(sQ + x * L::TILE_BYTES + b * BOX_BYTES, &tmap_q, &bars[L::B_Q_FULL + x],
                         wi.h * D + 64 * b, wi.row0 + x * BM);
+          ++nq[x];
+        }
+        if (!ok) break;
         if (!load_k(wi, 0)) break;
         for (int j = 0; j < wi.nkv; ++j) {
           if (j + 1 < wi.nkv && !load_k(wi, j + 1)) { ok = false; break; }
@@ -335,7 +452,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       // Let every copy this thread started land before the CTA can exit.
       const uint64_t lim = args.ctl.wait_limit_ns;
-      if (n_item > 0) drain_wait(&bars[L::B_Q_FULL], (n_item - 1) & 1, lim);
+      for (int x = 0; x < 2; ++x)
+        if (nq[x] > 0) drain_wait(&bars[L::B_Q_FULL + x], (nq[x] - 1) & 1, lim);
       for (int st = 0; st < NK; ++st)
         if (kc > static_cast<uint32_t>(st)) {
           const uint32_t last = kc - 1 - ((kc - 1 - st) % NK);
@@ -357,8 +475,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t kv = 0;           // key tiles consumed so far (global over items)
       uint32_t itx[2] = {0, 0};  // tiles processed per query tile slot (global)
       int nit[2] = {0, 0};       // items processed per query tile slot
-      int n_item = 0;
       bool ok = true;
+      // with RoPE fused, a Q tile is ready once its softmax warps have turned
+      // it; otherwise once its copy has landed (K always arrives rotated)
+      constexpr int kQReady = ROPE ? L::B_Q_ROT : L::B_Q_FULL;
+      constexpr int kKReady = L::B_K_FULL;
       // Shared-memory descriptors are built once per operand base; a byte offset
       // o inside shared memory moves the start-address field by o >> 4 (the
       // field cannot carry: shared addresses stay below 256 KB).
@@ -391,21 +512,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       auto wait = [&](int bar, uint32_t parity) -> bool {
         return mbar_wait(&bars[bar], parity, args.ctl, abort_flag);
       };
-      for (int k = 0, w = item_k(0); w < total_items && ok; w = item_k(++k), ++n_item) {
+      for (int k = 0, w = item_k(0); w < total_items && ok; w = item_k(++k)) {
         const WorkItem wi = decode_item(w, S, s_cu, s_order, s_istart);
         const int ntiles = wi.has_b ? 2 : 1;
-        if (!wait(L::B_Q_FULL, n_item & 1)) break;
         // prologue: S_A(0), S_B(0)
-        if (!wait(L::B_K_FULL + kv % NK, (kv / NK) & 1)) break;
-        tc_fence_after();
-        for (int x = 0; x < ntiles; ++x) issue_s(x, kv);
+        if (!wait(kKReady + kv % NK, (kv / NK) & 1)) break;
+        for (int x = 0; x < ntiles && ok; ++x) {
+          if (!wait(kQReady + x, nit[x] & 1)) { ok = false; break; }
+          tc_fence_after();
+          issue_s(x, kv);
+        }
+        if (!ok) break;
         umma_commit(&bars[L::B_K_EMPTY + kv % NK]);
-        if (wi.nkv == 1) umma_commit(&bars[L::B_Q_EMPTY]);
+        if (wi.nkv == 1)
+          for (int x = 0; x < ntiles; ++x) umma_commit(&bars[L::B_Q_EMPTY + x]);
         for (int j = 0; j < wi.nkv && ok; ++j) {
           const uint32_t c = kv + j;
           const bool more = j + 1 < wi.nkv;
           if (!wait(L::B_V_FULL + c % NV, (c / NV) & 1)) { ok = false; break; }
-          if (more && !wait(L::B_K_FULL + (c + 1) % NK, ((c + 1) / NK) & 1)) { ok = false; break; }
+          if (more && !wait(kKReady + (c + 1) % NK, ((c + 1) / NK) & 1)) { ok = false; break; }
           for (int x = 0; x < ntiles; ++x) {
             // PV_X(j) once softmax X has written P_X(j) (and, on the item's first
             // tile, once the previous item's epilogue has read O_X)
@@ -419,7 +544,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           umma_commit(&bars[L::B_V_EMPTY + c % NV]);
           if (more) {
             umma_commit(&bars[L::B_K_EMPTY + (c + 1) % NK]);
-            if (j + 2 == wi.nkv) umma_commit(&bars[L::B_Q_EMPTY]);
+            if (j + 2 == wi.nkv)
+              for (int x = 0; x < ntiles; ++x) umma_commit(&bars[L::B_Q_EMPTY + x]);
           }
         }
         if (!ok) break;
@@ -449,9 +575,31 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t it = 0;  // tiles of this query tile slot processed (global)
     int n_item = 0;   // items with this tile present
     bool ok = true;
+    bool q_turned = false;  // this warp has already turned its rows of the item's Q tile
+    // RoPE in the load prologue: this thread's query row of tile X, turned in
+    // place once its copy has landed; the MMA warp issues S_X(0) once all four
+    // warps of the tile have arrived on Q_ROT[X]
+    auto turn_q = [&](const WorkItem& q_it) {
+      const int rr = q_it.qb * QB + x * BM + row;  // row in the sample
+      if (rr < q_it.n) {
+        const int32_t* pp = args.rope.pos_ids + 3 * static_cast<size_t>(q_it.kv0 + rr);
+        rope_row_smem<D, AXES, 8>(sQ + x * L::TILE_BYTES, row, __ldg(pp), __ldg(pp + 1),
+                                  __ldg(pp + 2), args.rope.tab, args.rope.P, args.ctl);
+      }
+      fence_proxy_async_smem();  // the MMA reads the tile through the async proxy
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[L::B_Q_ROT + x]);
+    };
     for (int k = 0, w = item_k(0); w < total_items && ok; w = item_k(++k)) {
       const WorkItem wi = decode_item(w, S, s_cu, s_order, s_istart);
       if (x == 1 && !wi.has_b) continue;
+      if constexpr (ROPE) {
+        if (!q_turned) {
+          if (!warp_wait(&bars[L::B_Q_FULL + x], n_item & 1, args.ctl, abort_flag)) break;
+          turn_q(wi);
+        }
+        q_turned = false;
+      }
       const int last_cols = wi.n - (wi.nkv - 1) * BN;  // valid keys in the last tile
       float m_ref = 0.f;  // reference max (scaled, log2 units)
       float l = 0.f;
@@ -564,6 +712,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (lane == 0) mbar_arrive(&bars[L::B_P_FULL + x]);
       }
       if (!ok) break;
+      if constexpr (ROPE) {
+        // The next item's Q tile was requested when S_X(last) completed and has
+        // often landed by now: turn it while PV_X(last) runs, so that S_X(0) of
+        // the next item is computed during this epilogue rather than after it.
+        // Only when the next item of this CTA holds tile X (then its copy is the
+        // next phase of Q_FULL[X]), and only if every lane of the warp sees the
+        // copy complete (each lane then has its own acquire); otherwise the tile
+        // is turned after the epilogue.
+        const int wn = item_k(k + 1);
+        if (wn < total_items) {
+          const WorkItem nx = decode_item(wn, S, s_cu, s_order, s_istart);
+          if ((x == 0 || nx.has_b) &&
+              __all_sync(0xffffffffu, mbar_try_wait(&bars[L::B_Q_FULL + x], (n_item + 1) & 1))) {
+            turn_q(nx);
+            q_turned = true;
+          }
+        }
+      }
       // ---------------------------------------------------------- epilogue
       // O row in chunks of 32 columns: normalise by 1/l and write (y = x + gate
       // * O in the fused block, else O); then release O_X to the next item.
@@ -679,7 +845,7 @@ bool make_tile_map(CUtensorMap* map, const void* base, int32_t T, int32_t cols) 
          CUDA_SUCCESS;
 }
 
-template <int D, bool GATED>
+template <int D, bool GATED, int AXES>
 cudaError_t launch_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                      const AttnArgs& a, int grid, cudaStream_t st) {
   constexpr int smem = Layout<D>::SMEM_BYTES;
@@ -691,15 +857,15 @@ cudaError_t launch_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
     // kLaunchRegs registers per thread; with fewer the softmax warpgroups'
     // setmaxnreg.inc could never be satisfied, so refuse to launch.
     cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, varlen_attn_kernel<D, GATED>);
+    cudaError_t e = cudaFuncGetAttributes(&fa, varlen_attn_kernel<D, GATED, AXES>);
     if (e != cudaSuccess) return e;
     if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
-    e = cudaFuncSetAttribute(varlen_attn_kernel<D, GATED>,
+    e = cudaFuncSetAttribute(varlen_attn_kernel<D, GATED, AXES>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  varlen_attn_kernel<D, GATED><<<grid, NUM_THREADS, smem, st>>>(mq, mk, mv, a);
+  varlen_attn_kernel<D, GATED, AXES><<<grid, NUM_THREADS, smem, st>>>(mq, mk, mv, a);
   return cudaGetLastError();
 }
 
@@ -784,8 +950,8 @@ int32_t attention_work_items(const int32_t* cu_h, int32_t S, int32_t H) {
 cudaError_t launch_attention(const mf_bf16* q, const mf_bf16* k, const mf_bf16* v,
                              const int32_t* cu_seqlens_d, const int32_t* cu_seqlens_h, int32_t S,
                              int32_t T, int32_t H, int32_t D, float softmax_scale,
-                             const AttnEpilogue& ep, int32_t num_items, const KernelCtl& ctl,
-                             cudaStream_t st) {
+                             const AttnEpilogue& ep, const AttnRopeParams* rope,
+                             int32_t num_items, const KernelCtl& ctl, cudaStream_t st) {
   if (num_items <= 0) return cudaSuccess;
   CUtensorMap mq, mk, mv;
   const int32_t cols = H * D;
@@ -800,18 +966,32 @@ cudaError_t launch_attention(const mf_bf16* q, const mf_bf16* k, const mf_bf16* 
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
   a.ep = ep;
   a.ctl = ctl;
+  a.rope = AttnRope{};
+  if (rope != nullptr) {
+    if (rope->axes != 2 && rope->axes != 3) return cudaErrorInvalidValue;
+    a.rope.pos_ids = rope->pos_ids;
+    a.rope.tab = reinterpret_cast<const float2*>(rope->tab);
+    a.rope.P = rope->P;
+  }
   const int sms = sm_count_dev();
   const int grid = num_items < sms ? num_items : sms;
   build_schedule(cu_seqlens_h, S, H, grid, &a.sched);
   const bool gated = ep.y != nullptr;
-  if (D == 128) {
-    return gated ? launch_t<128, true>(mq, mk, mv, a, grid, st)
-                 : launch_t<128, false>(mq, mk, mv, a, grid, st);
+  // the fused gated residual is only used by the block, which always rotates
+  if (gated && rope == nullptr) return cudaErrorInvalidValue;
+  const int axes = rope ? rope->axes : 0;
+#define MF_ATTN_CASE(DD)                                                                   \
+  if (D == DD) {                                                                           \
+    if (axes == 0) return launch_t<DD, false, 0>(mq, mk, mv, a, grid, st);                 \
+    if (axes == 2)                                                                         \
+      return gated ? launch_t<DD, true, 2>(mq, mk, mv, a, grid, st)                        \
+                   : launch_t<DD, false, 2>(mq, mk, mv, a, grid, st);                      \
+    return gated ? launch_t<DD, true, 3>(mq, mk, mv, a, grid, st)                          \
+                 : launch_t<DD, false, 3>(mq, mk, mv, a, grid, st);                        \
   }
-  if (D == 64) {
-    return gated ? launch_t<64, true>(mq, mk, mv, a, grid, st)
-                 : launch_t<64, false>(mq, mk, mv, a, grid, st);
-  }
+  MF_ATTN_CASE(128)
+  MF_ATTN_CASE(64)
+#undef MF_ATTN_CASE
   return cudaErrorInvalidValue;
 }
 

@@ -25,6 +25,15 @@
 //                          x, dx_mod and the row statistics).
 // 16-byte vector accesses throughout; bad sample / modality ids are recorded
 // as MF_ERR_INVALID and their rows skipped.
+//
+// The modulation map mod = c W (no bias, no activation; [S][C] x [C][6 hid]) has
+// the backward dW = c^T dmod and dc = dmod W^T:
+//   params_dw_kernel       one thread per (4 columns, 16 rows of W): the S-term
+//                          sums for its 16 x 4 outputs, samples in order.
+//   params_dc_kernel       one CTA per conditioning channel: the dot products
+//                          of W's row with every sample's dmod row, 16-byte
+//                          loads, partial sums reduced in a fixed order.
+// Neither uses atomics, so both are deterministic.
 #include <cuda_bf16.h>
 
 #include <cmath>
@@ -268,6 +277,91 @@ __global__ void __launch_bounds__(kColThreads) ln_bwd_cols_kernel(
   if (cs >= 0) flush();
 }
 
+// ------------------------------------------------ modulation-map backward
+constexpr int kDwRows = 16;      // rows of dW per thread
+constexpr int kDwSamples = 8;    // samples staged per pass
+constexpr int kDwThreads = 128;
+constexpr int kDcThreads = 256;
+constexpr int kDcSamples = 8;    // dot products per pass over W's row
+
+// dW[r][n] = sum_s c[s][r] * dmod[s][n]. grid: (N4 / kDwThreads, C / kDwRows).
+__global__ void __launch_bounds__(kDwThreads) params_dw_kernel(
+    const float4* __restrict__ dmod4, const float* __restrict__ c, int S, int C, int N4,
+    float4* __restrict__ dW4) {
+  __shared__ float s_c[kDwSamples][kDwRows];
+  const int n4 = blockIdx.x * kDwThreads + threadIdx.x;
+  const int r0 = blockIdx.y * kDwRows;
+  float4 acc[kDwRows];
+#pragma unroll
+  for (int r = 0; r < kDwRows; ++r) acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s0 = 0; s0 < S; s0 += kDwSamples) {
+    const int ns = min(kDwSamples, S - s0);
+    __syncthreads();
+    for (int i = threadIdx.x; i < kDwSamples * kDwRows; i += kDwThreads) {
+      const int u = i / kDwRows, r = i % kDwRows;
+      s_c[u][r] = (u < ns && r0 + r < C) ? c[static_cast<size_t>(s0 + u) * C + r0 + r] : 0.f;
+    }
+    __syncthreads();
+    if (n4 < N4) {
+      for (int u = 0; u < ns; ++u) {
+        const float4 d = __ldg(dmod4 + static_cast<size_t>(s0 + u) * N4 + n4);
+#pragma unroll
+        for (int r = 0; r < kDwRows; ++r) {
+          const float cv = s_c[u][r];
+          acc[r].x = fmaf(cv, d.x, acc[r].x);
+          acc[r].y = fmaf(cv, d.y, acc[r].y);
+          acc[r].z = fmaf(cv, d.z, acc[r].z);
+          acc[r].w = fmaf(cv, d.w, acc[r].w);
+        }
+      }
+    }
+  }
+  if (n4 < N4) {
+#pragma unroll
+    for (int r = 0; r < kDwRows; ++r)
+      if (r0 + r < C) dW4[static_cast<size_t>(r0 + r) * N4 + n4] = acc[r];
+  }
+}
+
+// dc[s][r] = sum_n dmod[s][n] * W[r][n]. grid: C CTAs (one row of W each).
+__global__ void __launch_bounds__(kDcThreads) params_dc_kernel(
+    const float4* __restrict__ dmod4, const float4* __restrict__ W4, int S, int C, int N4,
+    float* __restrict__ dc) {
+  __shared__ float s_part[kDcThreads / 32][kDcSamples];
+  const int r = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const float4* wrow = W4 + static_cast<size_t>(r) * N4;
+  for (int s0 = 0; s0 < S; s0 += kDcSamples) {
+    const int ns = min(kDcSamples, S - s0);
+    float acc[kDcSamples];
+#pragma unroll
+    for (int u = 0; u < kDcSamples; ++u) acc[u] = 0.f;
+    for (int n4 = threadIdx.x; n4 < N4; n4 += kDcThreads) {
+      const float4 wv = __ldg(wrow + n4);
+#pragma unroll
+      for (int u = 0; u < kDcSamples; ++u) {
+        if (u < ns) {
+          const float4 d = __ldg(dmod4 + static_cast<size_t>(s0 + u) * N4 + n4);
+          acc[u] = fmaf(d.x, wv.x, fmaf(d.y, wv.y, fmaf(d.z, wv.z, fmaf(d.w, wv.w, acc[u]))));
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kDcSamples; ++u) acc[u] = warp_sum(acc[u]);
+    __syncthreads();  // the previous pass has read s_part
+    if (lane == 0)
+#pragma unroll
+      for (int u = 0; u < kDcSamples; ++u) s_part[warp][u] = acc[u];
+    __syncthreads();
+    if (threadIdx.x < ns) {
+      float v = 0.f;
+#pragma unroll
+      for (int wi = 0; wi < kDcThreads / 32; ++wi) v += s_part[wi][threadIdx.x];
+      dc[static_cast<size_t>(s0 + threadIdx.x) * C + r] = v;
+    }
+  }
+}
+
 cudaError_t zero_slots(float* dmod, int32_t S, int32_t hid, int slot_mask, cudaStream_t st) {
   const long long n = static_cast<long long>(S) * 6 * hid;
   long long blocks = (n + 255) / 256;
@@ -295,6 +389,26 @@ cudaError_t launch_gated_residual_bwd(const mf_bf16* dy, const mf_bf16* o, const
       reinterpret_cast<const uint4*>(dy), reinterpret_cast<const uint4*>(o), mod, tok_sample,
       tok_mod, T, S, hid, reinterpret_cast<uint4*>(d_o), dmod, ctl);
   return cudaGetLastError();
+}
+
+cudaError_t launch_adaln_params_bwd(const float* dmod, const float* c, const float* W,
+                                    int32_t S, int32_t C, int32_t hid, float* dc, float* dW,
+                                    cudaStream_t st) {
+  const int N4 = 6 * hid / 4;
+  auto D4 = reinterpret_cast<const float4*>(dmod);
+  if (dW != nullptr) {
+    const dim3 grid(static_cast<unsigned>((N4 + kDwThreads - 1) / kDwThreads),
+                    static_cast<unsigned>((C + kDwRows - 1) / kDwRows));
+    params_dw_kernel<<<grid, kDwThreads, 0, st>>>(D4, c, S, C, N4, reinterpret_cast<float4*>(dW));
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (dc != nullptr) {
+    params_dc_kernel<<<C, kDcThreads, 0, st>>>(D4, reinterpret_cast<const float4*>(W), S, C, N4,
+                                               dc);
+    return cudaGetLastError();
+  }
+  return cudaSuccess;
 }
 
 cudaError_t launch_adaln_modulate_bwd(const mf_bf16* dx_mod, const mf_bf16* x, const float* mod,

@@ -25,4 +25,10 @@ cudaError_t launch_adaln_modulate_bwd(const mf_bf16* dx_mod, const mf_bf16* x, c
                                       float eps, mf_bf16* dx, float* dmod, float* stats,
                                       const KernelCtl& ctl, cudaStream_t st);
 
+// Backward of mod = c W: dW = c^T dmod ([C][6 hid]) and dc = dmod W^T ([S][C]);
+// either output may be NULL.
+cudaError_t launch_adaln_params_bwd(const float* dmod, const float* c, const float* W,
+                                    int32_t S, int32_t C, int32_t hid, float* dc, float* dW,
+                                    cudaStream_t st);
+
 }  // namespace mf

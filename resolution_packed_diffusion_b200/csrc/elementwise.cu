@@ -494,6 +494,40 @@ cudaError_t launch_selftest_wait(uint64_t limit_ns, const KernelCtl& ctl, cudaSt
   return cudaGetLastError();
 }
 
+namespace {
+
+// (cos, sin) of p * inv_freq[j] for every position p < P and pair column j <
+// npa; the angle is the same fp32 product the RoPE pass forms.
+__global__ void __launch_bounds__(256) rope_table_kernel(float2* __restrict__ tab, int P, int npa,
+                                                         const RopeTable rt) {
+  const long long n = static_cast<long long>(P) * npa;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int p = static_cast<int>(i / npa);
+    const int j = static_cast<int>(i - static_cast<long long>(p) * npa);
+    float sn, cs;
+    sincosf(static_cast<float>(p) * rt.inv_freq[j], &sn, &cs);
+    tab[i] = make_float2(cs, sn);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_rope_table(int32_t D, int32_t rope_axes, float base, int32_t P, void* tab,
+                              AttnRopeParams* r, cudaStream_t st) {
+  RopeTable rt;
+  make_rope_table(D, rope_axes, base, &rt);
+  const int npa = D / (2 * rope_axes);
+  r->tab = tab;
+  r->P = P;
+  r->axes = rope_axes;
+  const long long n = static_cast<long long>(P) * npa;
+  if (n == 0) return cudaSuccess;
+  const int grid = grid_for(n, 256, 4);
+  rope_table_kernel<<<grid, 256, 0, st>>>(static_cast<float2*>(tab), P, npa, rt);
+  return cudaGetLastError();
+}
+
 void make_rope_table(int32_t D, int32_t rope_axes, float base, RopeTable* tab) {
   const int d_a = 2 * (D / (2 * rope_axes));
   for (int p = 0; p < 64; ++p) {

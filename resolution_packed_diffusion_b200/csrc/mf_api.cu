@@ -64,7 +64,8 @@ int32_t count_items(const int32_t* cu_h, int32_t S, int32_t H) {
 cudaError_t timed_attention(const mf_bf16* q, const mf_bf16* k, const mf_bf16* v,
                             const int32_t* cu_d, const int32_t* cu_h, int32_t S, int32_t T,
                             int32_t H, int32_t D, float scale, const AttnEpilogue& ep,
-                            int32_t items, const KernelCtl& ctl, cudaStream_t st) {
+                            const AttnRopeParams* rope, int32_t items, const KernelCtl& ctl,
+                            cudaStream_t st) {
   cudaEvent_t e0 = nullptr, e1 = nullptr;
   int dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDevices) {
@@ -76,7 +77,8 @@ cudaError_t timed_attention(const mf_bf16* q, const mf_bf16* k, const mf_bf16* v
     cudaError_t e = cudaEventRecord(e0, st);
     if (e != cudaSuccess) return e;
   }
-  cudaError_t e = launch_attention(q, k, v, cu_d, cu_h, S, T, H, D, scale, ep, items, ctl, st);
+  cudaError_t e =
+      launch_attention(q, k, v, cu_d, cu_h, S, T, H, D, scale, ep, rope, items, ctl, st);
   if (e != cudaSuccess) return e;
   if (e1 != nullptr) e = cudaEventRecord(e1, st);
   return e;
@@ -109,6 +111,24 @@ mf_status rope_call(const mf_bf16* q, const mf_bf16* k, const int32_t* pos_ids, 
   if (transpose)
     for (float& f : tab.inv_freq) f = -f;
   return cuda_status(launch_rope(q, k, pos_ids, T, H, D, tab, q_out, k_out, stream));
+}
+
+// Carves the fused RoPE's workspace: the (cos, sin) table the attention turns
+// Q tiles with, and the rotated k, written by the RoPE pass over k (the
+// attention turns Q in its load prologue, K arrives rotated). Returns the k the
+// attention reads.
+cudaError_t prepare_fused_rope(const mf_bf16* k, const int32_t* pos_ids, int32_t T, int32_t H,
+                               int32_t D, int32_t rope_axes, float base, void* workspace,
+                               AttnRopeParams* rope, const mf_bf16** k_att, cudaStream_t st) {
+  const uintptr_t w0 = round_up(reinterpret_cast<uintptr_t>(workspace), 256);
+  rope->pos_ids = pos_ids;
+  cudaError_t e = launch_rope_table(D, rope_axes, base, T, reinterpret_cast<void*>(w0), rope, st);
+  if (e != cudaSuccess) return e;
+  mf_bf16* kr = reinterpret_cast<mf_bf16*>(w0 + round_up(static_cast<size_t>(T) * (D / 4) * 8, 256));
+  RopeTable tab;
+  make_rope_table(D, rope_axes, base, &tab);
+  *k_att = kr;
+  return launch_rope(nullptr, k, pos_ids, T, H, D, tab, nullptr, kr, st);
 }
 
 }  // namespace
@@ -213,6 +233,26 @@ mf_status mf_adaln_params(const float* c, const float* W, int32_t S, int32_t C, 
   return cuda_status(launch_adaln_params(c, W, S, C, hid, mod, stream));
 }
 
+mf_status mf_adaln_params_bwd(const float* dmod, const float* c, const float* W, int32_t S,
+                              int32_t C, int32_t hid, float* dc, float* dW, cudaStream_t stream) {
+  if (dmod == nullptr || c == nullptr || W == nullptr || (dc == nullptr && dW == nullptr) ||
+      S < 1 || S > MF_MAX_SAMPLES || C < 1 || C > 1024 || hid < 8 || hid % 8 != 0 ||
+      hid > 16384)
+    return MF_ERR_INVALID;
+  if (!aligned16(dmod) || !aligned16(c) || !aligned16(W) || !aligned16(dc) || !aligned16(dW))
+    return MF_ERR_INVALID;
+  const size_t mb = static_cast<size_t>(S) * 6 * hid * 4, cb = static_cast<size_t>(S) * C * 4,
+               wb = static_cast<size_t>(C) * 6 * hid * 4;
+  const void* ins[3] = {dmod, c, W};
+  const size_t in_bytes[3] = {mb, cb, wb};
+  for (int i = 0; i < 3; ++i) {
+    if (dc && overlap(dc, cb, ins[i], in_bytes[i])) return MF_ERR_INVALID;
+    if (dW && overlap(dW, wb, ins[i], in_bytes[i])) return MF_ERR_INVALID;
+  }
+  if (dc && dW && overlap(dc, cb, dW, wb)) return MF_ERR_INVALID;
+  return cuda_status(launch_adaln_params_bwd(dmod, c, W, S, C, hid, dc, dW, stream));
+}
+
 mf_status mf_adaln_modulate(const mf_bf16* x, const float* mod, const int32_t* tok_sample,
                             const uint8_t* tok_mod, int32_t T, int32_t S, int32_t hid, float eps,
                             mf_bf16* x_mod, cudaStream_t stream) {
@@ -245,10 +285,17 @@ mf_status mf_rope_bwd(const mf_bf16* dq_r, const mf_bf16* dk_r, const int32_t* p
   return mf::rope_call(dq_r, dk_r, pos_ids, T, H, D, rope_axes, base, dq, dk, true, stream);
 }
 
+// The workspace of the fused RoPE holds its (cos, sin) table, one row of
+// D / (2 * rope_axes) <= D / 4 float2 per position, positions 0 .. T-1 (every
+// position of a pack is below T: a sample's positions stay below its length),
+// then the rotated k.
 size_t mf_workspace_size(int32_t T, int32_t H, int32_t D, int32_t with_rope) {
   if (T <= 0 || H <= 0 || D <= 0 || !with_rope) return 0;
-  return 2 * round_up(static_cast<size_t>(T) * H * D * 2, 256) + 256;
+  return round_up(static_cast<size_t>(T) * (D / 4) * 8, 256) +
+         round_up(static_cast<size_t>(T) * H * D * 2, 256) + 256;
 }
+
+
 
 mf_status mf_varlen_attn_fwd(const mf_bf16* q, const mf_bf16* k, const mf_bf16* v,
                              const int32_t* cu_seqlens_d, const int32_t* cu_seqlens_h, int32_t S,
@@ -271,38 +318,35 @@ mf_status mf_varlen_attn_fwd(const mf_bf16* q, const mf_bf16* k, const mf_bf16* 
     return MF_ERR_INVALID;
   if (lse && (overlap(lse, static_cast<size_t>(T) * H * 4, o, bytes)))
     return MF_ERR_INVALID;
-  const mf_bf16* qa = q;
-  const mf_bf16* ka = k;
   if (pos_ids != nullptr) {
-    if ((rope_axes != 2 && rope_axes != 3) || !(base > 0.f) || !std::isfinite(base))
+    if ((rope_axes != 2 && rope_axes != 3) || !(base > 0.f) || !std::isfinite(base) ||
+        !aligned16(pos_ids))
       return MF_ERR_INVALID;
     if (workspace == nullptr || !aligned16(workspace) || ws_bytes < mf_workspace_size(T, H, D, 1))
       return MF_ERR_INVALID;
-    // the rotated Q and K are written while other CTAs still read q and k, and the
-    // attention reads them while it writes o and lse
+    // the (cos, sin) table is written before the attention reads q, k, v and
+    // pos_ids, and read while it writes o and lse
     const size_t ws = mf_workspace_size(T, H, D, 1);
     if (overlap(workspace, ws, q, bytes) || overlap(workspace, ws, k, bytes) ||
         overlap(workspace, ws, v, bytes) || overlap(workspace, ws, o, bytes) ||
         overlap(workspace, ws, pos_ids, static_cast<size_t>(T) * 12) ||
         (lse && overlap(workspace, ws, lse, static_cast<size_t>(T) * H * 4)))
       return MF_ERR_INVALID;
-    const uintptr_t w0 = round_up(reinterpret_cast<uintptr_t>(workspace), 256);
-    qa = reinterpret_cast<mf_bf16*>(w0);
-    ka = reinterpret_cast<mf_bf16*>(w0 + round_up(bytes, 256));
   }
   KernelCtl ctl;
   if (cudaError_t ge = get_ctl(&ctl); ge != cudaSuccess) return cuda_status(ge);
+  AttnRopeParams rope{};
+  const mf_bf16* ka = k;
   if (pos_ids != nullptr) {
-    RopeTable tab;
-    make_rope_table(D, rope_axes, base, &tab);
-    cudaError_t e = launch_rope(q, k, pos_ids, T, H, D, tab, const_cast<mf_bf16*>(qa),
-                                const_cast<mf_bf16*>(ka), stream);
+    cudaError_t e = prepare_fused_rope(k, pos_ids, T, H, D, rope_axes, base, workspace, &rope,
+                                       &ka, stream);
     if (e != cudaSuccess) return cuda_status(e);
   }
   AttnEpilogue ep{};
   ep.o = o;
   ep.lse = lse;
-  return cuda_status(timed_attention(qa, ka, v, cu_seqlens_d, cu_seqlens_h, S, T, H, D, softmax_scale, ep,
+  return cuda_status(timed_attention(q, ka, v, cu_seqlens_d, cu_seqlens_h, S, T, H, D,
+                                     softmax_scale, ep, pos_ids != nullptr ? &rope : nullptr,
                                      count_items(cu_seqlens_h, S, H), ctl, stream));
 }
 
@@ -469,7 +513,8 @@ mf_status mf_block_fwd(const mf_bf16* x, const mf_bf16* q, const mf_bf16* k, con
       tok_mod == nullptr || x_mod == nullptr || y == nullptr || workspace == nullptr)
     return MF_ERR_INVALID;
   if (!aligned16(x) || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(mod) ||
-      !aligned16(cu_seqlens_d) || !aligned16(x_mod) || !aligned16(y) || !aligned16(workspace))
+      !aligned16(cu_seqlens_d) || !aligned16(x_mod) || !aligned16(y) || !aligned16(workspace) ||
+      !aligned16(pos_ids))
     return MF_ERR_INVALID;
   if (ws_bytes < mf_workspace_size(T, H, D, 1)) return MF_ERR_INVALID;
   const size_t bytes = static_cast<size_t>(T) * hid * 2;
@@ -477,9 +522,9 @@ mf_status mf_block_fwd(const mf_bf16* x, const mf_bf16* q, const mf_bf16* k, con
   for (const void* in : ins)
     if (overlap(in, bytes, x_mod, bytes) || overlap(in, bytes, y, bytes)) return MF_ERR_INVALID;
   if (overlap(x_mod, bytes, y, bytes)) return MF_ERR_INVALID;
-  // The rotated Q and K are written into the workspace while other CTAs still
-  // read q and k, and the fused epilogue reads x, v and mod while y is written:
-  // the workspace and the outputs must stay clear of every input.
+  // The (cos, sin) table is written into the workspace before the attention
+  // reads q, k, v and pos_ids, and the fused epilogue reads x and mod while y
+  // is written: the workspace and the outputs must stay clear of every input.
   const size_t ws = mf_workspace_size(T, H, D, 1);
   const size_t mod_bytes = static_cast<size_t>(S) * 6 * hid * 4;
   for (const void* in : ins)
@@ -494,20 +539,19 @@ mf_status mf_block_fwd(const mf_bf16* x, const mf_bf16* q, const mf_bf16* k, con
   cudaError_t e =
       launch_adaln_modulate(x, mod, tok_sample, tok_mod, T, S, hid, eps, x_mod, ctl, stream);
   if (e != cudaSuccess) return cuda_status(e);
-  const uintptr_t w0 = round_up(reinterpret_cast<uintptr_t>(workspace), 256);
-  mf_bf16* wq = reinterpret_cast<mf_bf16*>(w0);
-  mf_bf16* wk = reinterpret_cast<mf_bf16*>(w0 + round_up(bytes, 256));
-  RopeTable tab;
-  make_rope_table(D, rope_axes, base, &tab);
-  e = launch_rope(q, k, pos_ids, T, H, D, tab, wq, wk, stream);
+  // RoPE in the attention's load prologue: Q and K tiles are turned in shared
+  // memory with (cos, sin) from a per-position table in the workspace
+  AttnRopeParams rope{};
+  const mf_bf16* ka = k;
+  e = prepare_fused_rope(k, pos_ids, T, H, D, rope_axes, base, workspace, &rope, &ka, stream);
   if (e != cudaSuccess) return cuda_status(e);
   AttnEpilogue ep{};
   ep.x = x;
   ep.mod = mod;
   ep.tok_mod = tok_mod;
   ep.y = y;
-  return cuda_status(timed_attention(wq, wk, v, cu_seqlens_d, cu_seqlens_h, S, T, H, D,
-                                     1.0f / std::sqrt(static_cast<float>(D)), ep,
+  return cuda_status(timed_attention(q, ka, v, cu_seqlens_d, cu_seqlens_h, S, T, H, D,
+                                     1.0f / std::sqrt(static_cast<float>(D)), ep, &rope,
                                      count_items(cu_seqlens_h, S, H), ctl, stream));
 }
 

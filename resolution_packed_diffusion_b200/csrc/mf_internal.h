@@ -70,14 +70,34 @@ struct AttnEpilogue {
   mf_bf16* y;             // gated residual output [T][H*D], or NULL
 };
 
+// RoPE fused into the attention's load prologue: q is read unrotated and each
+// Q tile is turned in shared memory before its first MMA (k arrives rotated by
+// a RoPE pass over k alone), with (cos, sin) from a table of P positions x
+// D / (2 axes) pair columns (one column set serves every axis: all axes use the
+// same frequencies).
+struct AttnRopeParams {
+  const int32_t* pos_ids;  // [T][3]
+  const void* tab;         // float2 [P][D / (2 axes)], from launch_rope_table
+  int32_t P, axes;
+};
+
+// Writes the (cos, sin) table of P positions for head_dim D and rope_axes into
+// tab (P * D / (2 rope_axes) float2) and fills r's tab, P and axes; the angles
+// are computed as the standalone RoPE pass computes them.
+cudaError_t launch_rope_table(int32_t D, int32_t rope_axes, float base, int32_t P, void* tab,
+                              AttnRopeParams* r, cudaStream_t st);
+
+
 // Work items (sample, head, 256-row query block) of a pack, from host offsets.
 int32_t attention_work_items(const int32_t* cu_h, int32_t S, int32_t H);
 
+// rope == nullptr: q and k are already rotated. The gated epilogue (ep.y set)
+// needs rope.
 cudaError_t launch_attention(const mf_bf16* q, const mf_bf16* k, const mf_bf16* v,
                              const int32_t* cu_seqlens_d, const int32_t* cu_seqlens_h, int32_t S,
                              int32_t T, int32_t H, int32_t D, float softmax_scale,
-                             const AttnEpilogue& ep, int32_t num_items, const KernelCtl& ctl,
-                             cudaStream_t st);
+                             const AttnEpilogue& ep, const AttnRopeParams* rope,
+                             int32_t num_items, const KernelCtl& ctl, cudaStream_t st);
 
 cudaError_t launch_selftest_exp2(const float* x, float* y, int32_t n, cudaStream_t st);
 cudaError_t launch_selftest_wait(uint64_t limit_ns, const KernelCtl& ctl, cudaStream_t st);

@@ -5,14 +5,14 @@
 // a host application which owns all device memory and hands its plugins no
 // allocator, or a caller on a latency-critical path that must not make a call
 // which can synchronise the device. Such callers cannot supply the workspace
-// mf_block_fwd needs for the rotated Q and K. This entry point takes that
-// workspace from a file-scope device array instead, so the caller passes only
-// inputs and outputs.
+// mf_block_fwd needs for its fused RoPE (the (cos, sin) table and the rotated
+// k). This entry point takes that workspace from a file-scope device array
+// instead, so the caller passes only inputs and outputs.
 //
 // The array is part of the library's device image: every GPU that loads the
 // library holds MF_NOALLOC_SCRATCH_BYTES for it until the process exits. Every
 // call shares it and it keeps the last call's contents; nothing in it needs to
-// start at zero (each call rewrites all of the rotated Q and K it reads).
+// start at zero (each call rewrites all of the table and rotated k it reads).
 // Calls that overlap on the GPU (on different streams, or from different host
 // threads) race on the array and must be serialised by the caller.
 #include <cuda_runtime_api.h>

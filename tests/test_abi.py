@@ -70,10 +70,14 @@ def test_pack_rejects_too_many_samples():
 
 
 def test_workspace_size():
+    """The fused RoPE's workspace: its (cos, sin) table, T positions x D/4 pair
+    columns of two floats (the 2D split has D/4 pairs per axis, the 3D one
+    fewer), and the rotated k, T x H x D bf16."""
     assert mf.mf_workspace_size(0, 24, 128, 1) == 0
     assert mf.mf_workspace_size(100, 24, 128, 0) == 0
-    n = 100 * 24 * 128 * 2
-    assert mf.mf_workspace_size(100, 24, 128, 1) >= 2 * n
+    for D in (64, 128):
+        need = 100 * (D // 4) * 8 + 100 * 24 * D * 2
+        assert need <= mf.mf_workspace_size(100, 24, D, 1) <= need + 768
 
 
 def test_host_argument_checks_without_gpu():
@@ -257,8 +261,26 @@ def test_noalloc_rejects_malformed_offsets_as_invalid(offsets):
 
 def test_noalloc_size_limit_without_gpu():
     P = ctypes.c_void_p
-    cu = np.array([0, 16384], dtype=np.int32)  # 2 x 16384 x 3072 bf16 = 201 MB of rotated Q, K
+    cu = np.array([0, 16384], dtype=np.int32)  # 16384 x 3072 rotated k plus table: ~105 MB
     st = mf.lib.mf_block_fwd_noalloc(P(16), P(16), P(16), P(16), P(16), P(16),
                                      cu.ctypes.data_as(P), P(16), P(16), P(16), 1, 24, 128, 2,
                                      10000.0, 1e-6, P(16), P(16), None)
     assert st == mf.MF_ERR_UNSUPPORTED
+
+
+def test_adaln_params_bwd_argument_checks_without_gpu():
+    lib = mf.lib
+    P = ctypes.c_void_p
+    MB = 1 << 20
+    dmod, c, W, dc, dW = (P((i + 1) * 16 * MB) for i in range(5))
+
+    def call(dc=dc, dW=dW, S=3, C=128, hid=3072):
+        return lib.mf_adaln_params_bwd(dmod, c, W, S, C, hid, dc, dW, None)
+
+    assert call(dc=None, dW=None) == mf.MF_ERR_INVALID           # nothing to compute
+    assert call(hid=3076) == mf.MF_ERR_INVALID                   # hid not a multiple of 8
+    assert call(S=0) == mf.MF_ERR_INVALID
+    assert call(dc=W) == mf.MF_ERR_INVALID                       # dc overlaps W
+    assert call(dW=P(dmod.value + 64)) == mf.MF_ERR_INVALID      # dW overlaps dmod
+    assert call(dW=P(dc.value)) == mf.MF_ERR_INVALID             # the outputs overlap
+    assert call(dc=P(dc.value + 8)) == mf.MF_ERR_INVALID         # misaligned
