@@ -4,8 +4,8 @@
 
 One step is one pass of the whole path over one synthetic pack: pack metadata
 (mf_pack_build), modulation vectors (mf_adaln_params) and the fused block
-(mf_block_fwd: adaLN modulation, RoPE, tcgen05 varlen attention with the gated
-residual epilogue). Inputs are resident in HBM when the timed region starts.
+(mf_block_fwd: adaLN modulation, RoPE (Q in the attention's load prologue, K by
+a pass), tcgen05 varlen attention with the gated residual epilogue). Inputs are resident in HBM when the timed region starts.
 
 Metric: useful attention TFLOP/s of the whole step, where useful FLOPs are
 4 * D * H * sum(n_s^2) over the real samples (the padding segment is computed but
@@ -301,7 +301,9 @@ def run_gpu(args, rank, world, local_rank):
         mf.mf_block_fwd(bx, bq, bk, bv, mod, cu_d, cu_h, pos, ts, tm, S, H, D, w.rope_axes, w.base,
                         w.eps, bxm, by, ws, ws_bytes, stream)
 
-    launches_per_step = 5  # pack ids, adaLN params, adaLN modulate, RoPE, attention
+    # pack ids, adaLN params, adaLN modulate, RoPE (cos, sin) table, RoPE pass over k,
+    # attention (Q turned in its load prologue)
+    launches_per_step = 6
 
     def barrier():
         if world > 1:
@@ -452,7 +454,7 @@ def run_gpu(args, rank, world, local_rank):
         "pct_bf16_peak": 100.0 * value / (peak * world),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
                      "frac": achieved / peak, "traffic": attn_traffic_bytes(T),
-                     "kernel": "varlen_attn_kernel<128, gated>",
+                     "kernel": "varlen_attn_kernel<128, gated, 2D RoPE in the Q prologue>",
                      "peak_source": f"{peak_src} bf16_tflops (burst)",
                      "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
                      "attn_ms": attn_avg},
