@@ -264,6 +264,7 @@ def workload_config(w, args):
             "hid": w.hid, "real_tokens": real_tokens(w),
             "samples": [list(d.as_tuple()) for d in w.descs], "rope_axes": w.rope_axes,
             "parallelism": f"replicas x{args.gpus}",
+            "attention_cta_pairs": getattr(args, "cta_pair", None),
             "l2": ("inputs larger than L2: x, q, k, v total "
                    f"{4 * w.T * w.hid * 2 / 1e6:.0f} MB vs 126 MB L2; no flush")}
 
@@ -824,6 +825,11 @@ ARMS = {"block": "run_gpu", "linear": "run_linear", "mmdit": "run_mmdit",
 def run_rank(args, rank, world, local_rank, backend="nccl", arm=None):
     """One rank of the GPU arm: joins the process group when world > 1, runs
     the arm (``arm`` or the one ``--op`` names), leaves the group."""
+    if getattr(args, "cta_pair", None) is not None and arm is None:
+        import torch
+        import resolution_packed_diffusion_b200 as mf
+        torch.cuda.set_device(local_rank)
+        mf.mf_set_attn_cta_pair(args.cta_pair)
     if world > 1:
         import datetime
         import torch
@@ -868,6 +874,9 @@ def main():
     ap.add_argument("--config", type=int, default=DEFAULT_CONFIG, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--impl", default="mf", choices=["mf", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cta-pair", type=int, default=None, choices=[0, 1],
+                    help="attention on CTA pairs (1) or one CTA per SM (0); default: the "
+                         "library's default")
     ap.add_argument("--op", default="block", choices=sorted(ARMS),
                     help="block: the packed joint-attention block (the default line); "
                          "linear: the modality-specific linear layer as a QKV projection; "

@@ -339,6 +339,18 @@ mf_status mf_get_error(cudaStream_t stream);
  * and the kernel winds down and returns. */
 mf_status mf_set_wait_limit_ns(uint64_t ns);
 
+/* Attention kernel of later calls of mf_varlen_attn_fwd, mf_block_fwd and
+ * mf_mmdit_block_fwd on the current device, for head_dim 128 (head_dim 64
+ * always runs the one-CTA kernel): enable = 0, one CTA per SM, each running
+ * two 128-row query tiles; enable = 1, CTA pairs (thread-block clusters of two
+ * on two SMs) running each QK^T and PV product as one M = 256 tcgen05 MMA
+ * (cta_group::2): each CTA holds its own 128 rows of the two 256-row query tiles,
+ * half the keys of every K tile and half the head dims of every V tile, so each
+ * SM loads and reads half of the K / V bytes per FLOP. The same products, the
+ * same online softmax and epilogue, the same results up to the order of
+ * floating-point sums [pack]. Default 0. enable must be 0 or 1. */
+mf_status mf_set_attn_cta_pair(int32_t enable);
+
 /* Instrumentation: while both events are non-NULL, every later call of
  * mf_varlen_attn_fwd / mf_block_fwd on the current device records `start` on its
  * stream right before the attention kernel and `stop` right after it, so the

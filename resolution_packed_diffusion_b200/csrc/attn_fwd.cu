@@ -104,23 +104,39 @@ constexpr int kPolyPairsOf8 = 2;
 constexpr float kRedoSum = 4294967296.f;  // 2^32
 
 
-template <int D>
+// Shared-memory layout. PAIR: the CTA is one of a cluster pair that runs M = 256
+// MMAs together; it keeps its own 128 rows of each Q tile, half of each K tile's
+// keys (64 rows) and half of each V tile's head dims (64 columns), and the
+// smaller stages buy deeper K / V rings.
+template <int D, bool PAIR>
 struct Layout {
-  static constexpr int kBoxes = D / 64;  // 64-column boxes per 128-row tile
-  static constexpr int TILE_BYTES = BM * D * 2;
+  static_assert(!PAIR || D == 128, "CTA pairs take head_dim 128 (a V half is one 128-byte box)");
+  static constexpr int kBoxes = D / 64;  // 64-column boxes per Q / K row
+  static constexpr int TILE_BYTES = BM * D * 2;           // one Q tile (this CTA's rows)
+  static constexpr int NKS = PAIR ? 4 : NK;               // K ring stages
+  static constexpr int NVS = PAIR ? 4 : NV;               // V ring stages
+  static constexpr int K_ROWS = PAIR ? BN / 2 : BN;       // keys of a K tile held here
+  static constexpr int K_BOX = K_ROWS * 128;              // one 64-column box of a K stage
+  static constexpr int K_STAGE = K_ROWS * D * 2;
+  static constexpr int V_COLS = PAIR ? D / 2 : D;         // head dims of a V tile held here
+  static constexpr int V_STAGE = BN * V_COLS * 2;
+  static constexpr uint32_t kPeers = PAIR ? 2 : 1;        // CTAs whose softmax warps arrive
   static constexpr int OFF_Q = 0;  // Q_A, Q_B
   static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
-  static constexpr int OFF_V = OFF_K + NK * TILE_BYTES;
-  static constexpr int OFF_BAR = OFF_V + NV * TILE_BYTES;
-  // barriers (arrival count 1 unless arrivals() says otherwise)
+  static constexpr int OFF_V = OFF_K + NKS * K_STAGE;
+  static constexpr int OFF_BAR = OFF_V + NVS * V_STAGE;
+  // barriers (arrival count 1 unless arrivals() says otherwise). With PAIR the
+  // leader's FULL barriers of K and V count both CTAs' bytes, its Q_ROT, P_FULL
+  // and O_EMPTY both CTAs' softmax warps; EMPTY, S_FULL and O_FULL arrive in
+  // both CTAs from the leader's multicast commits.
   static constexpr int B_Q_FULL = 0;                 // [tile]
   static constexpr int B_Q_EMPTY = B_Q_FULL + 2;     // [tile]
   static constexpr int B_Q_ROT = B_Q_EMPTY + 2;      // [tile], one arrival per softmax warp
-  static constexpr int B_K_FULL = B_Q_ROT + 2;       // NK
-  static constexpr int B_K_EMPTY = B_K_FULL + NK;    // NK
-  static constexpr int B_V_FULL = B_K_EMPTY + NK;    // NV
-  static constexpr int B_V_EMPTY = B_V_FULL + NV;    // NV
-  static constexpr int B_S_FULL = B_V_EMPTY + NV;    // [tile]
+  static constexpr int B_K_FULL = B_Q_ROT + 2;       // NKS
+  static constexpr int B_K_EMPTY = B_K_FULL + NKS;   // NKS
+  static constexpr int B_V_FULL = B_K_EMPTY + NKS;   // NVS
+  static constexpr int B_V_EMPTY = B_V_FULL + NVS;   // NVS
+  static constexpr int B_S_FULL = B_V_EMPTY + NVS;   // [tile]
   static constexpr int B_P_FULL = B_S_FULL + 2;      // [tile], one arrival per softmax warp
   static constexpr int B_O_FULL = B_P_FULL + 2;      // [tile]
   static constexpr int B_O_EMPTY = B_O_FULL + 2;     // [tile], one arrival per softmax warp
@@ -139,7 +155,7 @@ struct Layout {
   __device__ static uint32_t arrivals(int i) {
     if (i == B_P_FULL || i == B_P_FULL + 1 || i == B_O_EMPTY || i == B_O_EMPTY + 1 ||
         i == B_Q_ROT || i == B_Q_ROT + 1)
-      return kSoftmaxWarpsPerTile;
+      return kSoftmaxWarpsPerTile * kPeers;
     return 1u;
   }
 };
@@ -183,6 +199,10 @@ struct WorkItem {
   bool has_b;  // tile B holds at least one row of the sample
 };
 
+// A work item covers IQ query rows of one (sample, head): tiles A and B of
+// IQ / 2 rows each (IQ = 256 for one CTA, 512 for a CTA pair, whose CTAs hold
+// 128 rows of each tile).
+template <int IQ>
 __device__ __forceinline__ WorkItem decode_item(int w, int S, const int32_t* s_cu,
                                                 const int32_t* s_order, const int32_t* s_istart) {
   int lo = 0, hi = S - 1;  // largest r with istart[r] <= w
@@ -195,12 +215,12 @@ __device__ __forceinline__ WorkItem decode_item(int w, int S, const int32_t* s_c
   const int local = w - s_istart[lo];
   it.kv0 = s_cu[it.s];
   it.n = s_cu[it.s + 1] - it.kv0;
-  const int nq = (it.n + QB - 1) / QB;
+  const int nq = (it.n + IQ - 1) / IQ;
   it.h = local / nq;
   it.qb = local - it.h * nq;
-  it.row0 = it.kv0 + it.qb * QB;
+  it.row0 = it.kv0 + it.qb * IQ;
   it.nkv = (it.n + BN - 1) / BN;
-  it.has_b = (it.n - it.qb * QB) > BM;
+  it.has_b = (it.n - it.qb * IQ) > IQ / 2;
   return it;
 }
 
@@ -307,16 +327,20 @@ __device__ __forceinline__ void rope_row_smem(uint8_t* tile, int row, int p0, in
 
 // AXES: 0 = q and k arrive rotated; 2 or 3 = RoPE with that many axes fused
 // into the Q load prologue (k arrives rotated).
-template <int D, bool GATED, int AXES>
+template <int D, bool GATED, int AXES, bool PAIR>
 // Registers are split per SM sub-partition: with 12 warps each sub-partition
 // holds three, which caps a thread at 16384 / (3 * 32) = 170 -> 168 at launch.
+// PAIR: launched in clusters of two CTAs (see Layout and the issuer below).
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     varlen_attn_kernel(const __grid_constant__ CUtensorMap tmap_q,
                        const __grid_constant__ CUtensorMap tmap_k,
                        const __grid_constant__ CUtensorMap tmap_v,
                        const __grid_constant__ AttnArgs args) {
-  using L = Layout<D>;
+  using L = Layout<D, PAIR>;
   constexpr bool ROPE = AXES != 0;
+  constexpr int IQ = PAIR ? 2 * QB : QB;  // query rows per work item
+  constexpr int TQ = IQ / 2;              // rows per query tile (A or B), over the pair
+  constexpr uint16_t kBoth = 3;           // multicast mask: both CTAs of the pair
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the 128-byte-swizzled TMA / UMMA tiles
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -363,8 +387,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
   __syncwarp();
   if (warp == 1) {
-    tmem_alloc(tmem_slot, TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      // both CTAs' warp 1, the same slot offset: the pair's TMEM at one address
+      tmem_alloc_pair(tmem_slot, TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -374,18 +404,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int r = 0; r < S; ++r) {
       s_istart[r] = acc;
       const int n = s_cu[s_order[r] + 1] - s_cu[s_order[r]];
-      acc += ((n + QB - 1) / QB) * H;
+      acc += ((n + IQ - 1) / IQ) * H;
     }
     s_istart[S] = acc;
     if (*bad_flag) atomicCAS(args.ctl.err, 0, static_cast<int>(MF_ERR_INVALID));
   }
   __syncthreads();
+  // Both CTAs' barriers are initialised before either CTA's arrivals, commits
+  // or copies can reach the other's.
+  if constexpr (PAIR) cluster_sync();
   const uint32_t tmem = *tmem_slot;
   const int total_items = *bad_flag ? 0 : s_istart[S];
-  // k-th work item of this CTA (at least total_items once the list is exhausted)
+  // With PAIR the pair is the scheduling unit and rank 1 takes the second
+  // 128 rows of every tile; the leader (rank 0) issues the MMAs.
+  const int rank = PAIR ? static_cast<int>(cluster_ctarank()) : 0;
+  const int unit = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int n_units = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  // k-th work item of this unit (at least total_items once the list is exhausted)
   auto item_k = [&](int k) -> int {
-    return args.sched.valid ? args.sched.ids[args.sched.start[blockIdx.x] + k]
-                            : snake_item(k, blockIdx.x, gridDim.x);
+    return args.sched.valid ? args.sched.ids[args.sched.start[unit] + k]
+                            : snake_item(k, unit, n_units);
+  };
+  auto decode = [&](int w) { return decode_item<IQ>(w, S, s_cu, s_order, s_istart); };
+  // Arrival of a softmax warp on a barrier the MMA thread waits on: the
+  // leader's, across the cluster for rank 1.
+  auto arrive_to_issuer = [&](int b) {
+    if constexpr (PAIR)
+      mbar_arrive_cluster(cluster_addr(&bars[b], 0));
+    else
+      mbar_arrive(&bars[b]);
   };
 
   uint8_t* sQ = smem + L::OFF_Q;
@@ -404,30 +451,53 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t kc = 0, vc = 0;  // K / V tiles issued so far (global over items)
       uint32_t nq[2] = {0, 0};  // Q tiles issued per tile slot
       bool ok = true;
+      // With PAIR this CTA copies its half of each K tile (keys rank * 64 ..
+      // +64) and of each V tile (head dims rank * 64 .. +64); both halves
+      // complete on the leader's FULL barrier, which the leader's producer
+      // arms for both CTAs' bytes (a copy that lands first only takes the
+      // barrier's byte count below zero for a while).
       auto load_k = [&](const WorkItem& wi, int j) -> bool {
-        const int st = kc % NK;
-        if (!mbar_wait(&bars[L::B_K_EMPTY + st], ((kc / NK) & 1) ^ 1, args.ctl, abort_flag)) return false;
-        mbar_expect_tx(&bars[L::B_K_FULL + st], L::TILE_BYTES);
+        const int st = kc % L::NKS;
+        if (!mbar_wait(&bars[L::B_K_EMPTY + st], ((kc / L::NKS) & 1) ^ 1, args.ctl, abort_flag))
+          return false;
+        uint8_t* dst = sK + st * L::K_STAGE;
+        const int y = wi.kv0 + j * BN + rank * L::K_ROWS;
+        if constexpr (PAIR) {
+          if (rank == 0) mbar_expect_tx(&bars[L::B_K_FULL + st], 2 * L::K_STAGE);
+          const uint32_t lb = cluster_addr(&bars[L::B_K_FULL + st], 0);
 #pragma unroll
-        for (int b = 0; b < L::kBoxes; ++b)
-          tma_load_2d(sK + st * L::TILE_BYTES + b * BOX_BYTES, &tmap_k, &bars[L::B_K_FULL + st],
-                      wi.h * D + 64 * b, wi.kv0 + j * BN);
+          for (int b = 0; b < L::kBoxes; ++b)
+            tma_load_2d_pair(dst + b * L::K_BOX, &tmap_k, lb, wi.h * D + 64 * b, y);
+        } else {
+          mbar_expect_tx(&bars[L::B_K_FULL + st], L::K_STAGE);
+#pragma unroll
+          for (int b = 0; b < L::kBoxes; ++b)
+            tma_load_2d(dst + b * L::K_BOX, &tmap_k, &bars[L::B_K_FULL + st], wi.h * D + 64 * b, y);
+        }
         ++kc;
         return true;
       };
       auto load_v = [&](const WorkItem& wi, int j) -> bool {
-        const int st = vc % NV;
-        if (!mbar_wait(&bars[L::B_V_EMPTY + st], ((vc / NV) & 1) ^ 1, args.ctl, abort_flag)) return false;
-        mbar_expect_tx(&bars[L::B_V_FULL + st], L::TILE_BYTES);
+        const int st = vc % L::NVS;
+        if (!mbar_wait(&bars[L::B_V_EMPTY + st], ((vc / L::NVS) & 1) ^ 1, args.ctl, abort_flag))
+          return false;
+        uint8_t* dst = sV + st * L::V_STAGE;
+        const int y = wi.kv0 + j * BN;
+        if constexpr (PAIR) {
+          if (rank == 0) mbar_expect_tx(&bars[L::B_V_FULL + st], 2 * L::V_STAGE);
+          tma_load_2d_pair(dst, &tmap_v, cluster_addr(&bars[L::B_V_FULL + st], 0),
+                           wi.h * D + rank * L::V_COLS, y);
+        } else {
+          mbar_expect_tx(&bars[L::B_V_FULL + st], L::V_STAGE);
 #pragma unroll
-        for (int b = 0; b < L::kBoxes; ++b)
-          tma_load_2d(sV + st * L::TILE_BYTES + b * BOX_BYTES, &tmap_v, &bars[L::B_V_FULL + st],
-                      wi.h * D + 64 * b, wi.kv0 + j * BN);
+          for (int b = 0; b < L::kBoxes; ++b)
+            tma_load_2d(dst + b * BOX_BYTES, &tmap_v, &bars[L::B_V_FULL + st], wi.h * D + 64 * b, y);
+        }
         ++vc;
         return true;
       };
       for (int k = 0, w = item_k(0); w < total_items && ok; w = item_k(++k)) {
-        const WorkItem wi = decode_item(w, S, s_cu, s_order, s_istart);
+        const WorkItem wi = decode(w);
         const int ntiles = wi.has_b ? 2 : 1;
         // each query tile has its own full / empty barriers, so the warps of
         // tile B only ever see the phases of items that hold a tile B
@@ -436,11 +506,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ok = false;
             break;
           }
+          // this CTA's own 128 rows of the tile, on its own barrier
           mbar_expect_tx(&bars[L::B_Q_FULL + x], L::TILE_BYTES);
 #pragma unroll
           for (int b = 0; b < L::kBoxes; ++b)
             tma_load_2d(sQ + x * L::TILE_BYTES + b * BOX_BYTES, &tmap_q, &bars[L::B_Q_FULL + x],
-                        wi.h * D + 64 * b, wi.row0 + x * BM);
+                        wi.h * D + 64 * b, wi.row0 + x * TQ + rank * BM);
           ++nq[x];
         }
         if (!ok) break;
@@ -450,36 +521,53 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (!load_v(wi, j)) { ok = false; break; }
         }
       }
-      // Let every copy this thread started land before the CTA can exit.
+      // Let every copy this thread started land before the CTA can exit. With
+      // PAIR, K and V copies complete on the leader's barriers: the leader
+      // drains them for both CTAs, and the pair's closing cluster barrier keeps
+      // rank 1 alive until then.
       const uint64_t lim = args.ctl.wait_limit_ns;
       for (int x = 0; x < 2; ++x)
         if (nq[x] > 0) drain_wait(&bars[L::B_Q_FULL + x], (nq[x] - 1) & 1, lim);
-      for (int st = 0; st < NK; ++st)
-        if (kc > static_cast<uint32_t>(st)) {
-          const uint32_t last = kc - 1 - ((kc - 1 - st) % NK);
-          drain_wait(&bars[L::B_K_FULL + st], (last / NK) & 1, lim);
-        }
-      for (int st = 0; st < NV; ++st)
-        if (vc > static_cast<uint32_t>(st)) {
-          const uint32_t last = vc - 1 - ((vc - 1 - st) % NV);
-          drain_wait(&bars[L::B_V_FULL + st], (last / NV) & 1, lim);
-        }
+      if (rank == 0) {
+        for (int st = 0; st < L::NKS; ++st)
+          if (kc > static_cast<uint32_t>(st)) {
+            const uint32_t last = kc - 1 - ((kc - 1 - st) % L::NKS);
+            drain_wait(&bars[L::B_K_FULL + st], (last / L::NKS) & 1, lim);
+          }
+        for (int st = 0; st < L::NVS; ++st)
+          if (vc > static_cast<uint32_t>(st)) {
+            const uint32_t last = vc - 1 - ((vc - 1 - st) % L::NVS);
+            drain_wait(&bars[L::B_V_FULL + st], (last / L::NVS) & 1, lim);
+          }
+      }
     }
     __syncwarp();
   } else if (warp == 1) {
     // ============================================================ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, 0, 0);
-      constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, 0, 1);
+    // With PAIR only the leader issues: every MMA is M = 256 over the pair
+    // (rank 0's 128 query rows, then rank 1's), B taken half from each CTA's
+    // shared memory (S: 64 keys each; PV: 64 head dims each), and every commit
+    // that a CTA's producer or softmax warps wait on is multicast to both.
+    if (lane == 0 && rank == 0) {
+      constexpr int MM = PAIR ? 2 * BM : BM;
+      constexpr uint32_t IDESC_S = idesc_bf16_f32(MM, BN, 0, 0);
+      constexpr uint32_t IDESC_PV = idesc_bf16_f32(MM, D, 0, 1);
       const uint32_t qaddr = smem_u32(sQ), kaddr = smem_u32(sK), vaddr = smem_u32(sV);
       uint32_t kv = 0;           // key tiles consumed so far (global over items)
       uint32_t itx[2] = {0, 0};  // tiles processed per query tile slot (global)
       int nit[2] = {0, 0};       // items processed per query tile slot
       bool ok = true;
       // with RoPE fused, a Q tile is ready once its softmax warps have turned
-      // it; otherwise once its copy has landed (K always arrives rotated)
-      constexpr int kQReady = ROPE ? L::B_Q_ROT : L::B_Q_FULL;
+      // it, and with PAIR once both CTAs' softmax warps have seen their rows
+      // land; otherwise once its copy has landed (K always arrives rotated)
+      constexpr int kQReady = (ROPE || PAIR) ? L::B_Q_ROT : L::B_Q_FULL;
       constexpr int kKReady = L::B_K_FULL;
+      auto commit = [&](int b) {
+        if constexpr (PAIR)
+          umma_commit_pair(&bars[b], kBoth);
+        else
+          umma_commit(&bars[b]);
+      };
       // Shared-memory descriptors are built once per operand base; a byte offset
       // o inside shared memory moves the start-address field by o >> 4 (the
       // field cannot carry: shared addresses stay below 256 KB).
@@ -490,47 +578,59 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // 16-element K step is a 32-byte advance inside a 64-column box.
       auto issue_s = [&](int x, uint32_t c) {
         const uint64_t a0 = qdesc + static_cast<uint64_t>((x * L::TILE_BYTES) >> 4);
-        const uint64_t b0 = kdesc + static_cast<uint64_t>(((c % NK) * L::TILE_BYTES) >> 4);
+        const uint64_t b0 = kdesc + static_cast<uint64_t>(((c % L::NKS) * L::K_STAGE) >> 4);
         const uint32_t d = tmem + tm_s(x);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t koff = ((kk >> 2) * BOX_BYTES + (kk & 3) * 32) >> 4;
-          umma_ss(d, a0 + koff, b0 + koff, IDESC_S, kk > 0 ? 1u : 0u);
+          const uint32_t aoff = ((kk >> 2) * BOX_BYTES + (kk & 3) * 32) >> 4;
+          const uint32_t boff = ((kk >> 2) * L::K_BOX + (kk & 3) * 32) >> 4;
+          if constexpr (PAIR)
+            umma_ss_pair(d, a0 + aoff, b0 + boff, IDESC_S, kk > 0 ? 1u : 0u);
+          else
+            umma_ss(d, a0 + aoff, b0 + boff, IDESC_S, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&bars[L::B_S_FULL + x]);
+        commit(L::B_S_FULL + x);
       };
       // O_X += P_X V_c; V is MN-major (LBO = distance between 64-column boxes,
       // SBO = 8 rows of 128 B); P_X comes from TMEM, 8 columns per 16 keys.
       auto issue_pv = [&](int x, uint32_t c, bool first) {
-        const uint64_t b0 = vdesc + static_cast<uint64_t>(((c % NV) * L::TILE_BYTES) >> 4);
+        const uint64_t b0 = vdesc + static_cast<uint64_t>(((c % L::NVS) * L::V_STAGE) >> 4);
         const uint32_t d = tmem + tm_o(x);
         const uint32_t a = tmem + tm_s(x);
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          umma_ts(d, a + kk * 8, b0 + ((kk * 16 * 128) >> 4), IDESC_PV, (first && kk == 0) ? 0u : 1u);
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint32_t acc = (first && kk == 0) ? 0u : 1u;
+          if constexpr (PAIR)
+            umma_ts_pair(d, a + kk * 8, b0 + ((kk * 16 * 128) >> 4), IDESC_PV, acc);
+          else
+            umma_ts(d, a + kk * 8, b0 + ((kk * 16 * 128) >> 4), IDESC_PV, acc);
+        }
       };
       auto wait = [&](int bar, uint32_t parity) -> bool {
         return mbar_wait(&bars[bar], parity, args.ctl, abort_flag);
       };
       for (int k = 0, w = item_k(0); w < total_items && ok; w = item_k(++k)) {
-        const WorkItem wi = decode_item(w, S, s_cu, s_order, s_istart);
+        const WorkItem wi = decode(w);
         const int ntiles = wi.has_b ? 2 : 1;
         // prologue: S_A(0), S_B(0)
-        if (!wait(kKReady + kv % NK, (kv / NK) & 1)) break;
+        if (!wait(kKReady + kv % L::NKS, (kv / L::NKS) & 1)) break;
         for (int x = 0; x < ntiles && ok; ++x) {
           if (!wait(kQReady + x, nit[x] & 1)) { ok = false; break; }
           tc_fence_after();
           issue_s(x, kv);
         }
         if (!ok) break;
-        umma_commit(&bars[L::B_K_EMPTY + kv % NK]);
+        commit(L::B_K_EMPTY + kv % L::NKS);
         if (wi.nkv == 1)
-          for (int x = 0; x < ntiles; ++x) umma_commit(&bars[L::B_Q_EMPTY + x]);
+          for (int x = 0; x < ntiles; ++x) commit(L::B_Q_EMPTY + x);
         for (int j = 0; j < wi.nkv && ok; ++j) {
           const uint32_t c = kv + j;
           const bool more = j + 1 < wi.nkv;
-          if (!wait(L::B_V_FULL + c % NV, (c / NV) & 1)) { ok = false; break; }
-          if (more && !wait(kKReady + (c + 1) % NK, ((c + 1) / NK) & 1)) { ok = false; break; }
+          if (!wait(L::B_V_FULL + c % L::NVS, (c / L::NVS) & 1)) { ok = false; break; }
+          if (more && !wait(kKReady + (c + 1) % L::NKS, ((c + 1) / L::NKS) & 1)) {
+            ok = false;
+            break;
+          }
           for (int x = 0; x < ntiles; ++x) {
             // PV_X(j) once softmax X has written P_X(j) (and, on the item's first
             // tile, once the previous item's epilogue has read O_X)
@@ -541,23 +641,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (more) issue_s(x, c + 1);
           }
           if (!ok) break;
-          umma_commit(&bars[L::B_V_EMPTY + c % NV]);
+          commit(L::B_V_EMPTY + c % L::NVS);
           if (more) {
-            umma_commit(&bars[L::B_K_EMPTY + (c + 1) % NK]);
+            commit(L::B_K_EMPTY + (c + 1) % L::NKS);
             if (j + 2 == wi.nkv)
-              for (int x = 0; x < ntiles; ++x) umma_commit(&bars[L::B_Q_EMPTY + x]);
+              for (int x = 0; x < ntiles; ++x) commit(L::B_Q_EMPTY + x);
           }
         }
         if (!ok) break;
         for (int x = 0; x < ntiles; ++x) {
-          umma_commit(&bars[L::B_O_FULL + x]);
+          commit(L::B_O_FULL + x);
           itx[x] += wi.nkv;
           ++nit[x];
         }
         kv += wi.nkv;
       }
       // every MMA this thread issued completes before TMEM is released
-      umma_commit(&bars[L::B_DRAIN]);
+      if constexpr (PAIR)
+        umma_commit_pair(&bars[L::B_DRAIN], 1);  // the leader's own barrier
+      else
+        umma_commit(&bars[L::B_DRAIN]);
       drain_wait(&bars[L::B_DRAIN], 0, args.ctl.wait_limit_ns);
     }
     __syncwarp();
@@ -579,21 +682,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // RoPE in the load prologue: this thread's query row of tile X, turned in
     // place once its copy has landed; the MMA warp issues S_X(0) once all four
     // warps of the tile have arrived on Q_ROT[X]
+    // With PAIR (no RoPE) the same path only reports the landed copy: the
+    // leader's MMA thread cannot see rank 1's copy barrier.
     auto turn_q = [&](const WorkItem& q_it) {
-      const int rr = q_it.qb * QB + x * BM + row;  // row in the sample
-      if (rr < q_it.n) {
-        const int32_t* pp = args.rope.pos_ids + 3 * static_cast<size_t>(q_it.kv0 + rr);
-        rope_row_smem<D, AXES, 8>(sQ + x * L::TILE_BYTES, row, __ldg(pp), __ldg(pp + 1),
-                                  __ldg(pp + 2), args.rope.tab, args.rope.P, args.ctl);
+      if constexpr (ROPE) {
+        const int rr = q_it.qb * IQ + x * TQ + rank * BM + row;  // row in the sample
+        if (rr < q_it.n) {
+          const int32_t* pp = args.rope.pos_ids + 3 * static_cast<size_t>(q_it.kv0 + rr);
+          rope_row_smem<D, AXES, 8>(sQ + x * L::TILE_BYTES, row, __ldg(pp), __ldg(pp + 1),
+                                    __ldg(pp + 2), args.rope.tab, args.rope.P, args.ctl);
+        }
+        fence_proxy_async_smem();  // the MMA reads the tile through the async proxy
       }
-      fence_proxy_async_smem();  // the MMA reads the tile through the async proxy
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[L::B_Q_ROT + x]);
+      if (lane == 0) arrive_to_issuer(L::B_Q_ROT + x);
     };
     for (int k = 0, w = item_k(0); w < total_items && ok; w = item_k(++k)) {
-      const WorkItem wi = decode_item(w, S, s_cu, s_order, s_istart);
+      const WorkItem wi = decode(w);
       if (x == 1 && !wi.has_b) continue;
-      if constexpr (ROPE) {
+      if constexpr (ROPE || PAIR) {
         if (!q_turned) {
           if (!warp_wait(&bars[L::B_Q_FULL + x], n_item & 1, args.ctl, abort_flag)) break;
           turn_q(wi);
@@ -709,10 +816,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[L::B_P_FULL + x]);
+        if (lane == 0) arrive_to_issuer(L::B_P_FULL + x);
       }
       if (!ok) break;
-      if constexpr (ROPE) {
+      if constexpr (ROPE || PAIR) {
         // The next item's Q tile was requested when S_X(last) completed and has
         // often landed by now: turn it while PV_X(last) runs, so that S_X(0) of
         // the next item is computed during this epilogue rather than after it.
@@ -722,7 +829,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // is turned after the epilogue.
         const int wn = item_k(k + 1);
         if (wn < total_items) {
-          const WorkItem nx = decode_item(wn, S, s_cu, s_order, s_istart);
+          const WorkItem nx = decode(wn);
           if ((x == 0 || nx.has_b) &&
               __all_sync(0xffffffffu, mbar_try_wait(&bars[L::B_Q_FULL + x], (n_item + 1) & 1))) {
             turn_q(nx);
@@ -733,8 +840,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // ---------------------------------------------------------- epilogue
       // O row in chunks of 32 columns: normalise by 1/l and write (y = x + gate
       // * O in the fused block, else O); then release O_X to the next item.
-      const int r_in_sample = wi.qb * QB + x * BM + row;
-      const int t = wi.row0 + x * BM + row;
+      const int r_in_sample = wi.qb * IQ + x * TQ + rank * BM + row;
+      const int t = wi.row0 + x * TQ + rank * BM + row;
       const bool row_valid = r_in_sample < wi.n;
       const int col0 = wi.h * D;  // first column of this head in [T][H*D]
       const int hid = H * D;
@@ -795,7 +902,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[L::B_O_EMPTY + x]);
+      if (lane == 0) arrive_to_issuer(L::B_O_EMPTY + x);
       ++n_item;
       if (row_valid && args.ep.lse != nullptr)
         args.ep.lse[static_cast<size_t>(wi.h) * args.T + t] =
@@ -807,7 +914,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
+  if constexpr (PAIR) {
+    // The leader has drained its MMAs (which write rank 1's TMEM) and the
+    // copies that complete on its barriers; neither CTA frees TMEM or leaves
+    // before both are here.
+    cluster_sync();
+    if (warp == 1) tmem_dealloc_pair(tmem, TMEM_COLS);
+  } else {
+    if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
+  }
 }
 
 // Host-side tensor-map creation through the driver entry point (no link-time
@@ -830,14 +945,15 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// [T][H*D] bf16 viewed as a 2D tensor; box = 64 columns x 128 rows, 128-byte
-// swizzle; rows past T read as zeros.
-bool make_tile_map(CUtensorMap* map, const void* base, int32_t T, int32_t cols) {
+// [T][H*D] bf16 viewed as a 2D tensor; box = 64 columns x box_rows rows,
+// 128-byte swizzle; rows past T read as zeros.
+bool make_tile_map(CUtensorMap* map, const void* base, int32_t T, int32_t cols,
+                   uint32_t box_rows = 128) {
   EncodeTiledFn enc = get_encode_fn();
   if (enc == nullptr) return false;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(T)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
-  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t box[2] = {64, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -845,28 +961,87 @@ bool make_tile_map(CUtensorMap* map, const void* base, int32_t T, int32_t cols) 
          CUDA_SUCCESS;
 }
 
-template <int D, bool GATED, int AXES>
-cudaError_t launch_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                     const AttnArgs& a, int grid, cudaStream_t st) {
-  constexpr int smem = Layout<D>::SMEM_BYTES;
+template <int D, bool GATED, int AXES, bool PAIR>
+bool kernel_ready(int dev) {
   static bool attr_set[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+  if (dev < 0 || dev >= 64) return false;
+  if (!attr_set[dev]) {
     // The setmaxnreg split assumes the kernel was built with exactly
     // kLaunchRegs registers per thread; with fewer the softmax warpgroups'
     // setmaxnreg.inc could never be satisfied, so refuse to launch.
     cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, varlen_attn_kernel<D, GATED, AXES>);
-    if (e != cudaSuccess) return e;
-    if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
-    e = cudaFuncSetAttribute(varlen_attn_kernel<D, GATED, AXES>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
+    if (cudaFuncGetAttributes(&fa, varlen_attn_kernel<D, GATED, AXES, PAIR>) != cudaSuccess ||
+        fa.numRegs != kLaunchRegs)
+      return false;
+    if (cudaFuncSetAttribute(varlen_attn_kernel<D, GATED, AXES, PAIR>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Layout<D, PAIR>::SMEM_BYTES) != cudaSuccess)
+      return false;
     attr_set[dev] = true;
   }
-  varlen_attn_kernel<D, GATED, AXES><<<grid, NUM_THREADS, smem, st>>>(mq, mk, mv, a);
+  return true;
+}
+
+template <int D, bool GATED, int AXES>
+cudaError_t launch_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                     const AttnArgs& a, int grid, cudaStream_t st) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!kernel_ready<D, GATED, AXES, false>(dev)) return cudaErrorInvalidConfiguration;
+  varlen_attn_kernel<D, GATED, AXES, false>
+      <<<grid, NUM_THREADS, Layout<D, false>::SMEM_BYTES, st>>>(mq, mk, mv, a);
   return cudaGetLastError();
+}
+
+// CTA pairs: clusters of two, `pairs` of them (grid = 2 * pairs).
+template <int D, bool GATED, int AXES>
+cudaError_t launch_pair_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                          const AttnArgs& a, int pairs, cudaStream_t st) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!kernel_ready<D, GATED, AXES, true>(dev)) return cudaErrorInvalidConfiguration;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = Layout<D, true>::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, varlen_attn_kernel<D, GATED, AXES, true>, mq, mk, mv, a);
+}
+
+// How many CTA pairs of the pair kernel can be resident at once (one CTA per
+// SM, both CTAs of a pair in one GPC); cached per device.
+template <bool GATED, int AXES>
+int max_pairs(int dev) {
+  static int cached[64] = {0};
+  if (dev < 0 || dev >= 64) return 0;
+  if (cached[dev] == 0) {
+    if (!kernel_ready<128, GATED, AXES, true>(dev)) return 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2);
+    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.dynamicSmemBytes = Layout<128, true>::SMEM_BYTES;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, varlen_attn_kernel<128, GATED, AXES, true>, &cfg) !=
+            cudaSuccess ||
+        n <= 0)
+      return 0;
+    cached[dev] = n;
+  }
+  return cached[dev];
 }
 
 int sm_count_dev() {
@@ -893,7 +1068,7 @@ int sm_count_dev() {
 // tie (equal items, or one item per CTA) the snake order measured a little
 // faster. Leaves s->valid = 0 for the snake order, and when the table cannot
 // hold the items.
-void build_schedule(const int32_t* cu_h, int32_t S, int32_t H, int grid, Schedule* s) {
+void build_schedule(const int32_t* cu_h, int32_t S, int32_t H, int grid, int iq, Schedule* s) {
   s->valid = 0;
   std::vector<int> order(S);
   for (int i = 0; i < S; ++i) order[i] = i;
@@ -901,7 +1076,7 @@ void build_schedule(const int32_t* cu_h, int32_t S, int32_t H, int grid, Schedul
     return (cu_h[a + 1] - cu_h[a]) > (cu_h[b + 1] - cu_h[b]);
   });
   int64_t total = 0;
-  for (int i = 0; i < S; ++i) total += static_cast<int64_t>((cu_h[i + 1] - cu_h[i] + QB - 1) / QB) * H;
+  for (int i = 0; i < S; ++i) total += static_cast<int64_t>((cu_h[i + 1] - cu_h[i] + iq - 1) / iq) * H;
   if (total > kMaxSchedItems || grid > kMaxSchedCtas || grid <= 0) return;
   std::vector<std::vector<int32_t>> lists(grid);
   std::vector<int64_t> snake_load(grid, 0);
@@ -912,7 +1087,7 @@ void build_schedule(const int32_t* cu_h, int32_t S, int32_t H, int grid, Schedul
   int32_t id = 0;
   for (int r = 0; r < S; ++r) {
     const int n = cu_h[order[r] + 1] - cu_h[order[r]];
-    const int nq = (n + QB - 1) / QB;
+    const int nq = (n + iq - 1) / iq;
     const int64_t nkv = (n + BN - 1) / BN;
     for (int h = 0; h < H; ++h) {
       for (int qb = 0; qb < nq; ++qb, ++id) {
@@ -941,21 +1116,25 @@ void build_schedule(const int32_t* cu_h, int32_t S, int32_t H, int grid, Schedul
 
 }  // namespace
 
-int32_t attention_work_items(const int32_t* cu_h, int32_t S, int32_t H) {
+int32_t attention_work_items(const int32_t* cu_h, int32_t S, int32_t H, bool pair) {
+  const int64_t iq = pair ? 2 * QB : QB;
   int64_t n = 0;
-  for (int32_t s = 0; s < S; ++s) n += (static_cast<int64_t>(cu_h[s + 1] - cu_h[s]) + QB - 1) / QB;
+  for (int32_t s = 0; s < S; ++s) n += (static_cast<int64_t>(cu_h[s + 1] - cu_h[s]) + iq - 1) / iq;
   return static_cast<int32_t>(n * H);
 }
 
 cudaError_t launch_attention(const mf_bf16* q, const mf_bf16* k, const mf_bf16* v,
                              const int32_t* cu_seqlens_d, const int32_t* cu_seqlens_h, int32_t S,
                              int32_t T, int32_t H, int32_t D, float softmax_scale,
-                             const AttnEpilogue& ep, const AttnRopeParams* rope,
-                             int32_t num_items, const KernelCtl& ctl, cudaStream_t st) {
+                             const AttnEpilogue& ep, const AttnRopeParams* rope, bool pair,
+                             const KernelCtl& ctl, cudaStream_t st) {
+  const bool use_pair = pair && D == 128;  // CTA pairs take head_dim 128 only
+  const int32_t num_items = attention_work_items(cu_seqlens_h, S, H, use_pair);
   if (num_items <= 0) return cudaSuccess;
   CUtensorMap mq, mk, mv;
   const int32_t cols = H * D;
-  if (!make_tile_map(&mq, q, T, cols) || !make_tile_map(&mk, k, T, cols) ||
+  // a CTA of a pair copies 64 keys of each K tile
+  if (!make_tile_map(&mq, q, T, cols) || !make_tile_map(&mk, k, T, cols, use_pair ? 64 : 128) ||
       !make_tile_map(&mv, v, T, cols))
     return cudaErrorInvalidValue;
   static thread_local AttnArgs a;  // ~17 KB: kept off the host stack
@@ -973,13 +1152,30 @@ cudaError_t launch_attention(const mf_bf16* q, const mf_bf16* k, const mf_bf16* 
     a.rope.tab = reinterpret_cast<const float2*>(rope->tab);
     a.rope.P = rope->P;
   }
-  const int sms = sm_count_dev();
-  const int grid = num_items < sms ? num_items : sms;
-  build_schedule(cu_seqlens_h, S, H, grid, &a.sched);
   const bool gated = ep.y != nullptr;
   // the fused gated residual is only used by the block, which always rotates
   if (gated && rope == nullptr) return cudaErrorInvalidValue;
   const int axes = rope ? rope->axes : 0;
+  if (use_pair) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int mp = 0;
+    if (axes == 0) mp = max_pairs<false, 0>(dev);
+    else if (axes == 2) mp = gated ? max_pairs<true, 2>(dev) : max_pairs<false, 2>(dev);
+    else mp = gated ? max_pairs<true, 3>(dev) : max_pairs<false, 3>(dev);
+    if (mp <= 0) return cudaErrorInvalidConfiguration;
+    const int pairs = num_items < mp ? num_items : mp;
+    build_schedule(cu_seqlens_h, S, H, pairs, 2 * QB, &a.sched);
+    if (axes == 0) return launch_pair_t<128, false, 0>(mq, mk, mv, a, pairs, st);
+    if (axes == 2)
+      return gated ? launch_pair_t<128, true, 2>(mq, mk, mv, a, pairs, st)
+                   : launch_pair_t<128, false, 2>(mq, mk, mv, a, pairs, st);
+    return gated ? launch_pair_t<128, true, 3>(mq, mk, mv, a, pairs, st)
+                 : launch_pair_t<128, false, 3>(mq, mk, mv, a, pairs, st);
+  }
+  const int sms = sm_count_dev();
+  const int grid = num_items < sms ? num_items : sms;
+  build_schedule(cu_seqlens_h, S, H, grid, QB, &a.sched);
 #define MF_ATTN_CASE(DD)                                                                   \
   if (D == DD) {                                                                           \
     if (axes == 0) return launch_t<DD, false, 0>(mq, mk, mv, a, grid, st);                 \

@@ -31,6 +31,7 @@ struct DeviceState {
   uint64_t wait_limit_ns = kDefaultWaitLimitNs;
   cudaEvent_t attn_start = nullptr;  // instrumentation (mf_set_attn_timing_events)
   cudaEvent_t attn_stop = nullptr;
+  bool attn_pair = false;            // mf_set_attn_cta_pair
 };
 
 DeviceState g_state[kMaxDevices];
@@ -56,29 +57,28 @@ inline mf_status cuda_status(cudaError_t e) {
 
 bool valid_head_dim(int32_t D) { return D == 64 || D == 128; }
 
-int32_t count_items(const int32_t* cu_h, int32_t S, int32_t H) {
-  return attention_work_items(cu_h, S, H);
-}
-
 // Runs the attention launcher between the caller's timing events, if any.
+// Runs the attention launcher (on CTA pairs when this device is set to) between
+// the caller's timing events, if any.
 cudaError_t timed_attention(const mf_bf16* q, const mf_bf16* k, const mf_bf16* v,
                             const int32_t* cu_d, const int32_t* cu_h, int32_t S, int32_t T,
                             int32_t H, int32_t D, float scale, const AttnEpilogue& ep,
-                            const AttnRopeParams* rope, int32_t items, const KernelCtl& ctl,
-                            cudaStream_t st) {
+                            const AttnRopeParams* rope, const KernelCtl& ctl, cudaStream_t st) {
   cudaEvent_t e0 = nullptr, e1 = nullptr;
+  bool pair = false;
   int dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDevices) {
     std::lock_guard<std::mutex> lock(g_mutex);
     e0 = g_state[dev].attn_start;
     e1 = g_state[dev].attn_stop;
+    pair = g_state[dev].attn_pair;
   }
   if (e0 != nullptr) {
     cudaError_t e = cudaEventRecord(e0, st);
     if (e != cudaSuccess) return e;
   }
   cudaError_t e =
-      launch_attention(q, k, v, cu_d, cu_h, S, T, H, D, scale, ep, rope, items, ctl, st);
+      launch_attention(q, k, v, cu_d, cu_h, S, T, H, D, scale, ep, rope, pair, ctl, st);
   if (e != cudaSuccess) return e;
   if (e1 != nullptr) e = cudaEventRecord(e1, st);
   return e;
@@ -347,7 +347,7 @@ mf_status mf_varlen_attn_fwd(const mf_bf16* q, const mf_bf16* k, const mf_bf16* 
   ep.lse = lse;
   return cuda_status(timed_attention(q, ka, v, cu_seqlens_d, cu_seqlens_h, S, T, H, D,
                                      softmax_scale, ep, pos_ids != nullptr ? &rope : nullptr,
-                                     count_items(cu_seqlens_h, S, H), ctl, stream));
+                                     ctl, stream));
 }
 
 size_t mf_attn_bwd_workspace_size(int32_t T, int32_t S, int32_t H, int32_t D) {
@@ -552,7 +552,7 @@ mf_status mf_block_fwd(const mf_bf16* x, const mf_bf16* q, const mf_bf16* k, con
   ep.y = y;
   return cuda_status(timed_attention(q, ka, v, cu_seqlens_d, cu_seqlens_h, S, T, H, D,
                                      1.0f / std::sqrt(static_cast<float>(D)), ep, &rope,
-                                     count_items(cu_seqlens_h, S, H), ctl, stream));
+                                     ctl, stream));
 }
 
 mf_status mf_cfg_combine(const mf_bf16* v, const mf_sample_desc* desc, int32_t S,
@@ -646,6 +646,16 @@ mf_status mf_set_wait_limit_ns(uint64_t ns) {
   if (dev < 0 || dev >= 64) return MF_ERR_INVALID;
   std::lock_guard<std::mutex> lock(g_mutex);
   g_state[dev].wait_limit_ns = ns;
+  return MF_OK;
+}
+
+mf_status mf_set_attn_cta_pair(int32_t enable) {
+  if (enable != 0 && enable != 1) return MF_ERR_INVALID;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MF_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MF_ERR_INVALID;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  g_state[dev].attn_pair = enable != 0;
   return MF_OK;
 }
 

@@ -88,16 +88,17 @@ cudaError_t launch_rope_table(int32_t D, int32_t rope_axes, float base, int32_t 
                               AttnRopeParams* r, cudaStream_t st);
 
 
-// Work items (sample, head, 256-row query block) of a pack, from host offsets.
-int32_t attention_work_items(const int32_t* cu_h, int32_t S, int32_t H);
+// Work items of a pack, from host offsets: (sample, head, 256-row query block),
+// or 512-row blocks for CTA pairs.
+int32_t attention_work_items(const int32_t* cu_h, int32_t S, int32_t H, bool pair);
 
 // rope == nullptr: q and k are already rotated. The gated epilogue (ep.y set)
-// needs rope.
+// needs rope. pair: run head_dim 128 on CTA pairs (cta_group::2, M = 256).
 cudaError_t launch_attention(const mf_bf16* q, const mf_bf16* k, const mf_bf16* v,
                              const int32_t* cu_seqlens_d, const int32_t* cu_seqlens_h, int32_t S,
                              int32_t T, int32_t H, int32_t D, float softmax_scale,
-                             const AttnEpilogue& ep, const AttnRopeParams* rope,
-                             int32_t num_items, const KernelCtl& ctl, cudaStream_t st);
+                             const AttnEpilogue& ep, const AttnRopeParams* rope, bool pair,
+                             const KernelCtl& ctl, cudaStream_t st);
 
 cudaError_t launch_selftest_exp2(const float* x, float* y, int32_t n, cudaStream_t st);
 cudaError_t launch_selftest_wait(uint64_t limit_ns, const KernelCtl& ctl, cudaStream_t st);
