@@ -26,6 +26,9 @@ every step of this path:
           chain in NR-MMDiT is adaptive normalization / RoPE / gating.
   [cfg]   picx.dev summary, Methodology > NR-MMDiT, bullet "Packed CFG
           inference": conditional and unconditional branches in one forward.
+  [vae], [vfuse] (``vae_oracle``) picx.dev summary, Methodology > Mage-VAE and
+          > Training Infrastructure: the fully convolutional VAE's repeated
+          blocks and their fused normalization - activation - residual chains.
 
 Where the pages are silent the oracle takes one stated reading (RoPE split and
 base, text positions, LayerNorm eps, modulation form); each reading is named at
@@ -67,4 +70,12 @@ from .mf_oracle import (  # noqa: F401
     useful_attention_flops,
     varlen_attention,
     varlen_attention_bwd,
+)
+from .vae_oracle import (  # noqa: F401
+    conv3x3,
+    group_norm,
+    group_norm_silu,
+    silu,
+    vae_block_flops,
+    vae_res_block,
 )

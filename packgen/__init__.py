@@ -18,3 +18,4 @@ from .configs import (  # noqa: F401
     make_random_pack,
     token_count,
 )
+from .vae import VAE_CONFIGS, VaeBlockInputs, make_vae_block  # noqa: F401,E402
