@@ -818,8 +818,82 @@ def run_block_bwd(args, rank, world, local_rank):
         "gpu_launches": 11 * args.steps, "clocks": clk}), flush=True)
 
 
+def run_vae(args, rank, world, local_rank):
+    """`--op vae_block`: one Mage-VAE conv block (SiLU(GroupNorm) -> 3x3 conv ->
+    SiLU(GroupNorm) -> 3x3 conv + the input) at a decoder-stage size, seeded
+    synthetic activations and random-init weights. FLOPs: the two convolutions,
+    2 x 2 x 9 x C^2 per pixel."""
+    import torch
+    import resolution_packed_diffusion_b200 as mf
+    from packgen import VAE_CONFIGS, make_vae_block
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    v = make_vae_block(args.vae_config, seed=rank_seed(len(VAE_CONFIGS), rank) + 17)
+    N, H, W, C, G = v.N, v.H, v.W, v.C, v.G
+
+    def dbf16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    x, W1, W2 = dbf16(v.x_bits), dbf16(v.W1_bits), dbf16(v.W2_bits)
+    f = {k: torch.from_numpy(getattr(v, k)).to(dev)
+         for k in ("gamma1", "beta1", "gamma2", "beta2", "c1", "c2")}
+    y = torch.empty_like(x)
+    ws_bytes = mf.mf_vae_block_workspace_size(N, H, W, C, G)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        mf.mf_vae_res_block(x, f["gamma1"], f["beta1"], W1, f["c1"], f["gamma2"], f["beta2"], W2,
+                            f["c2"], N, H, W, C, G, v.eps, y, ws, ws_bytes, stream)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    clocks = ClockSampler(local_rank) if rank == 0 else None
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    torch.cuda.synchronize(dev)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop() if clocks else None
+    if mf.mf_get_error(stream) != mf.MF_OK:
+        raise RuntimeError("device error in the VAE block")
+    flops = 4.0 * 9.0 * C * C * N * H * W
+    ms_step, flops_all = reduce_timing(t0.elapsed_time(t1) / args.steps, flops, world)
+    if rank != 0:
+        return
+    peaks, peak_src = load_peaks()
+    achieved = flops / (ms_step * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    act_mb = N * H * W * C * 2 / 1e6
+    print(json.dumps({
+        "metric": "Mage-VAE conv block TFLOP/s (two 3x3 convolutions)", "op": "vae_block",
+        "value": flops_all / (ms_step * 1e-3) / 1e12, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic activations, random-init weights",
+        "config": {"workload": f"VAE block {args.vae_config}", "N": N, "H": H, "W": W, "C": C,
+                   "G": G, "l2": "activations %.0f MB each, weights %.1f MB; no flush"
+                   % (act_mb, 2 * C * 9 * C * 2 / 1e6)},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
+                     "frac": achieved / peak, "traffic": None,
+                     "kernel": "whole block (conv3x3_kernel dominant)",
+                     "peak_source": f"{peak_src} bf16_tflops (burst)"},
+        "gpu_launches": 8 * args.steps, "clocks": clk}), flush=True)
+
+
 ARMS = {"block": "run_gpu", "linear": "run_linear", "mmdit": "run_mmdit",
-        "attn_bwd": "run_attn_bwd", "block_bwd": "run_block_bwd"}
+        "attn_bwd": "run_attn_bwd", "block_bwd": "run_block_bwd", "vae_block": "run_vae"}
 
 
 def run_rank(args, rank, world, local_rank, backend="nccl", arm=None):
@@ -882,7 +956,10 @@ def main():
                          "linear: the modality-specific linear layer as a QKV projection; "
                          "mmdit: one whole NR-MMDiT block around the path; "
                          "attn_bwd: the backward of the packed attention; "
-                         "block_bwd: the backward of the whole path block")
+                         "block_bwd: the backward of the whole path block; "
+                         "vae_block: one Mage-VAE conv block")
+    ap.add_argument("--vae-config", default="stage_1_8", choices=["tiny", "stage_1_8", "stage_1_4"],
+                    help="shape of the --op vae_block workload")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

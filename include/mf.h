@@ -27,6 +27,12 @@
  *   [train] picx.dev summary, Methodology > Training Infrastructure and
  *          Table 4: the packed NR-MMDiT is trained (MFU and training speedup),
  *          so each training step also runs the backward of the block.
+ *   [vae]  picx.dev summary, Methodology > Mage-VAE, "Architecture": a fully
+ *          convolutional one-step diffusion decoder (and its dual encoder) of
+ *          stacked convolutional blocks; 16x downsampled, 128-channel latents.
+ *   [vfuse] picx.dev summary, Methodology > Training Infrastructure: the
+ *          normalization - activation - residual chains of the VAE's repeated
+ *          blocks run as fused CUDA kernels.
  * Where the pages are silent the library follows one stated reading: RoPE
  * splits head_dim evenly across the axes in whole adjacent-channel pairs, base
  * 10000 by default, leftover channels unrotated; text token j of a sample sits
@@ -324,6 +330,50 @@ mf_status mf_mmdit_block_fwd(const mf_bf16* x, const mf_bf16* Wq, const mf_bf16*
                              float eps, mf_bf16* y, void* workspace, size_t ws_bytes,
                              cudaStream_t stream);
 size_t mf_mmdit_workspace_size(int32_t T, int32_t H, int32_t D, int32_t F);
+
+/* Mage-VAE conv block [vae], [vfuse]: the fully convolutional VAE's repeated
+ * blocks and their fused normalization - activation - residual chains. The
+ * pages give neither the wiring nor the widths; the library takes the diffusion
+ * conv nets' residual block
+ *   y = x + conv3x3(SiLU(GN(h; gamma2, beta2)); W2, c2),
+ *   h = conv3x3(SiLU(GN(x; gamma1, beta1)); W1, c1).
+ * Tensors are NHWC bf16 ([N][H][W][C], channels innermost); conv weights
+ * [Cout][3][3][Cin] bf16 (tap (dy, dx) reads pixel (h + dy - 1, w + dx - 1),
+ * zero outside the image); GroupNorm gamma / beta and conv biases fp32 [C].
+ * Supported: C (and Cin, Cout) in {64, 128, 256, 512, 1024, 2048}; C / G a
+ * multiple of 8; N * H * W < 2^31; else MF_ERR_UNSUPPORTED.
+ *
+ * SiLU(GroupNorm(x)) [vfuse]: each sample's channels in G consecutive groups of
+ * C / G, normalised over (H, W, C / G) with the population variance and eps,
+ * then y = SiLU(xhat * gamma[c] + beta[c]) in one pass over x (statistics by a
+ * first pass, merged in a fixed order: repeated calls give the same bits).
+ * y must not overlap x. workspace: ws_bytes >= mf_gn_workspace_size(N, H, W, G),
+ * disjoint from x and y. */
+mf_status mf_group_norm_silu(const mf_bf16* x, const float* gamma, const float* beta, int32_t N,
+                             int32_t H, int32_t W, int32_t C, int32_t G, float eps, mf_bf16* y,
+                             void* workspace, size_t ws_bytes, cudaStream_t stream);
+size_t mf_gn_workspace_size(int32_t N, int32_t H, int32_t W, int32_t G);
+
+/* 3x3 convolution, stride 1, zero padding 1 [vae], as an implicit GEMM on tcgen05
+ * tensor cores (bf16 operands, fp32 accumulation): y[n, h, w, o] = sum over taps
+ * and input channels of x * Wt, + bias[o] (NULL: none) + residual[n, h, w, o]
+ * (NULL: none) added in the epilogue [vfuse], rounded to bf16. x: [N][H][W][Cin];
+ * y, residual: [N][H][W][Cout]. y must not overlap x, Wt or bias; residual may
+ * equal y (in place) but not overlap it otherwise. */
+mf_status mf_conv3x3(const mf_bf16* x, const mf_bf16* Wt, const float* bias,
+                     const mf_bf16* residual, int32_t N, int32_t H, int32_t W, int32_t Cin,
+                     int32_t Cout, mf_bf16* y, cudaStream_t stream);
+
+/* The whole block: SiLU(GN) -> conv (+ c1) -> SiLU(GN) -> conv (+ c2 + x). Every
+ * intermediate is stored in bf16 in the workspace (ws_bytes >=
+ * mf_vae_block_workspace_size(N, H, W, C, G)); y must not overlap x, the
+ * weights or the workspace. C = Cin = Cout. */
+mf_status mf_vae_res_block(const mf_bf16* x, const float* gamma1, const float* beta1,
+                           const mf_bf16* W1, const float* c1, const float* gamma2,
+                           const float* beta2, const mf_bf16* W2, const float* c2, int32_t N,
+                           int32_t H, int32_t W, int32_t C, int32_t G, float eps, mf_bf16* y,
+                           void* workspace, size_t ws_bytes, cudaStream_t stream);
+size_t mf_vae_block_workspace_size(int32_t N, int32_t H, int32_t W, int32_t C, int32_t G);
 
 /* Bytes of workspace mf_varlen_attn_fwd / mf_block_fwd need (with_rope != 0:
  * room for the fused RoPE's (cos, sin) table, T x D/4 float2, and the rotated

@@ -4,8 +4,8 @@ activation - residual chains).
 The report gives the VAE's latent geometry (16x downsampling, 128 latent
 channels) but not its stage widths; the shapes below are readings: decoder
 stages of a 1024 x 1024 image at 1/8 resolution (128 x 128 pixels, 256
-channels) and at 1/4 (256 x 256, 128 channels), 32 groups, plus a small ragged
-case for parity. Every array is drawn from ``numpy.random.default_rng(seed)``
+channels, 32 groups) and at 1/4 (256 x 256, 128 channels, 16 groups: eight
+channels a group), plus a small ragged case for parity. Every array is drawn from ``numpy.random.default_rng(seed)``
 in this order: x ~ N(0, 1) (bf16), W1 and W2 ~ N(0, 1) / sqrt(9 C) (bf16,
 [C][3][3][C]), gamma1, beta1, gamma2, beta2 (fp32: 1 + 0.1 N(0,1) and
 0.1 N(0,1)), c1 and c2 ~ 0.02 N(0, 1) (fp32). No arithmetic of the block lives
@@ -23,7 +23,7 @@ from .configs import bf16_bits_to_f32, f32_to_bf16_bits
 VAE_CONFIGS = {
     "tiny": dict(N=2, H=9, W=13, C=64, G=8),
     "stage_1_8": dict(N=1, H=128, W=128, C=256, G=32),
-    "stage_1_4": dict(N=1, H=256, W=256, C=128, G=32),
+    "stage_1_4": dict(N=1, H=256, W=256, C=128, G=16),
 }
 
 

@@ -89,6 +89,12 @@ _SIGS = {
     "mf_mmdit_block_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I,
                                 _I, _I, _I, _I, _F, _F, _P, _P, _SZ, _P]),
     "mf_mmdit_workspace_size": (_SZ, [_I, _I, _I, _I]),
+    "mf_group_norm_silu": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _P, _SZ, _P]),
+    "mf_gn_workspace_size": (_SZ, [_I, _I, _I, _I]),
+    "mf_conv3x3": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
+    "mf_vae_res_block": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _P,
+                              _SZ, _P]),
+    "mf_vae_block_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -345,3 +351,33 @@ def mf_mmdit_block_fwd(x, Wq, Wk, Wv, Wo, Wup, Wdown, mod_attn, mod_mlp, descs, 
                                   _ptr(pos_ids), _ptr(tok_sample), _ptr(tok_mod), S, H, D, F,
                                   rope_axes, base, eps, _ptr(y), _ptr(workspace), ws_bytes,
                                   _stream(stream)), "mf_mmdit_block_fwd")
+
+
+def mf_gn_workspace_size(N: int, H: int, W: int, G: int) -> int:
+    return int(lib.mf_gn_workspace_size(N, H, W, G))
+
+
+def mf_group_norm_silu(x, gamma, beta, N: int, H: int, W: int, C: int, G: int, eps: float, y,
+                       workspace, ws_bytes: int, stream=None) -> None:
+    _check(lib.mf_group_norm_silu(_ptr(x), _ptr(gamma), _ptr(beta), N, H, W, C, G, eps, _ptr(y),
+                                  _ptr(workspace), ws_bytes, _stream(stream)),
+           "mf_group_norm_silu")
+
+
+def mf_conv3x3(x, Wt, bias, residual, N: int, H: int, W: int, Cin: int, Cout: int, y,
+               stream=None) -> None:
+    _check(lib.mf_conv3x3(_ptr(x), _ptr(Wt), _ptr(bias), _ptr(residual), N, H, W, Cin, Cout,
+                          _ptr(y), _stream(stream)), "mf_conv3x3")
+
+
+def mf_vae_block_workspace_size(N: int, H: int, W: int, C: int, G: int) -> int:
+    return int(lib.mf_vae_block_workspace_size(N, H, W, C, G))
+
+
+def mf_vae_res_block(x, gamma1, beta1, W1, c1, gamma2, beta2, W2, c2, N: int, H: int, W: int,
+                     C: int, G: int, eps: float, y, workspace, ws_bytes: int,
+                     stream=None) -> None:
+    _check(lib.mf_vae_res_block(_ptr(x), _ptr(gamma1), _ptr(beta1), _ptr(W1), _ptr(c1),
+                                _ptr(gamma2), _ptr(beta2), _ptr(W2), _ptr(c2), N, H, W, C, G,
+                                eps, _ptr(y), _ptr(workspace), ws_bytes, _stream(stream)),
+           "mf_vae_res_block")

@@ -14,6 +14,7 @@
 #include "cfg_internal.h"
 #include "gemm_internal.h"
 #include "mf_internal.h"
+#include "vae_internal.h"
 
 namespace mf {
 
@@ -625,6 +626,109 @@ mf_status mf_modality_linear(const mf_bf16* x, const mf_bf16* W, const uint8_t* 
   if (cudaError_t ge = get_ctl(&ctl); ge != cudaSuccess) return cuda_status(ge);
   return cuda_status(launch_modality_linear(x, W, tok_mod, jobs, static_cast<int32_t>(T), K, N,
                                             act, out, ctl, stream));
+}
+
+namespace {
+// Channel counts the VAE kernels take: a multiple of 64 (one 128-byte K atom of
+// the conv) whose 8-channel vector count divides 256 (the statistics pass).
+bool vae_channels_ok(int32_t C) {
+  return C >= 64 && C <= 2048 && (C & (C - 1)) == 0;
+}
+bool vae_shape_ok(int32_t N, int32_t H, int32_t W) {
+  return N >= 1 && H >= 1 && W >= 1 && static_cast<int64_t>(N) * H * W < (int64_t{1} << 31) &&
+         H <= (1 << 20) && W <= (1 << 20);
+}
+}  // namespace
+
+size_t mf_gn_workspace_size(int32_t N, int32_t H, int32_t W, int32_t G) {
+  if (!vae_shape_ok(N, H, W) || G < 1) return 0;
+  return gn_workspace_bytes(N, H, W, G) + 256;
+}
+
+mf_status mf_group_norm_silu(const mf_bf16* x, const float* gamma, const float* beta, int32_t N,
+                             int32_t H, int32_t W, int32_t C, int32_t G, float eps, mf_bf16* y,
+                             void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  if (x == nullptr || gamma == nullptr || beta == nullptr || y == nullptr ||
+      workspace == nullptr || G < 1 || !(eps >= 0.f) || !std::isfinite(eps))
+    return MF_ERR_INVALID;
+  if (!vae_shape_ok(N, H, W)) return MF_ERR_INVALID;
+  if (!vae_channels_ok(C) || C % G != 0 || (C / G) % 8 != 0) return MF_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(gamma) || !aligned16(beta) || !aligned16(y) ||
+      !aligned16(workspace))
+    return MF_ERR_INVALID;
+  const size_t ws = mf_gn_workspace_size(N, H, W, G);
+  if (ws_bytes < ws) return MF_ERR_INVALID;
+  const size_t bytes = static_cast<size_t>(N) * H * W * C * 2;
+  if (overlap(x, bytes, y, bytes) || overlap(workspace, ws, x, bytes) ||
+      overlap(workspace, ws, y, bytes) || overlap(y, bytes, gamma, C * 4) ||
+      overlap(y, bytes, beta, C * 4))
+    return MF_ERR_INVALID;
+  void* w0 = reinterpret_cast<void*>(round_up(reinterpret_cast<uintptr_t>(workspace), 256));
+  return cuda_status(launch_group_norm_silu(x, gamma, beta, N, H, W, C, G, eps, y, w0, stream));
+}
+
+mf_status mf_conv3x3(const mf_bf16* x, const mf_bf16* Wt, const float* bias,
+                     const mf_bf16* residual, int32_t N, int32_t H, int32_t W, int32_t Cin,
+                     int32_t Cout, mf_bf16* y, cudaStream_t stream) {
+  if (x == nullptr || Wt == nullptr || y == nullptr) return MF_ERR_INVALID;
+  if (!vae_shape_ok(N, H, W)) return MF_ERR_INVALID;
+  if (!vae_channels_ok(Cin) || !vae_channels_ok(Cout)) return MF_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(Wt) || !aligned16(y) || !aligned16(bias) ||
+      !aligned16(residual))
+    return MF_ERR_INVALID;
+  const size_t xb = static_cast<size_t>(N) * H * W * Cin * 2;
+  const size_t yb = static_cast<size_t>(N) * H * W * Cout * 2;
+  const size_t wb = static_cast<size_t>(Cout) * 9 * Cin * 2;
+  if (overlap(y, yb, x, xb) || overlap(y, yb, Wt, wb) || (bias && overlap(y, yb, bias, Cout * 4)))
+    return MF_ERR_INVALID;
+  if (residual != nullptr && residual != y && overlap(residual, yb, y, yb)) return MF_ERR_INVALID;
+  KernelCtl ctl;
+  if (cudaError_t ge = get_ctl(&ctl); ge != cudaSuccess) return cuda_status(ge);
+  return cuda_status(launch_conv3x3(x, Wt, bias, residual, N, H, W, Cin, Cout, y, ctl, stream));
+}
+
+size_t mf_vae_block_workspace_size(int32_t N, int32_t H, int32_t W, int32_t C, int32_t G) {
+  if (!vae_shape_ok(N, H, W) || C < 1 || G < 1) return 0;
+  const size_t act = round_up(static_cast<size_t>(N) * H * W * C * 2, 256);
+  return 2 * act + mf_gn_workspace_size(N, H, W, G) + 256;
+}
+
+mf_status mf_vae_res_block(const mf_bf16* x, const float* gamma1, const float* beta1,
+                           const mf_bf16* W1, const float* c1, const float* gamma2,
+                           const float* beta2, const mf_bf16* W2, const float* c2, int32_t N,
+                           int32_t H, int32_t W, int32_t C, int32_t G, float eps, mf_bf16* y,
+                           void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  if (x == nullptr || gamma1 == nullptr || beta1 == nullptr || W1 == nullptr ||
+      gamma2 == nullptr || beta2 == nullptr || W2 == nullptr || y == nullptr ||
+      workspace == nullptr || G < 1 || !(eps >= 0.f) || !std::isfinite(eps))
+    return MF_ERR_INVALID;
+  if (!vae_shape_ok(N, H, W)) return MF_ERR_INVALID;
+  if (!vae_channels_ok(C) || C % G != 0 || (C / G) % 8 != 0) return MF_ERR_UNSUPPORTED;
+  const void* ptrs[10] = {x, gamma1, beta1, W1, c1, gamma2, beta2, W2, c2, y};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return MF_ERR_INVALID;
+  if (!aligned16(workspace)) return MF_ERR_INVALID;
+  const size_t ws = mf_vae_block_workspace_size(N, H, W, C, G);
+  if (ws_bytes < ws) return MF_ERR_INVALID;
+  const size_t ab = static_cast<size_t>(N) * H * W * C * 2;
+  const size_t wb = static_cast<size_t>(C) * 9 * C * 2;
+  if (overlap(y, ab, x, ab) || overlap(y, ab, W1, wb) || overlap(y, ab, W2, wb) ||
+      overlap(y, ab, workspace, ws) || overlap(workspace, ws, x, ab) ||
+      overlap(workspace, ws, W1, wb) || overlap(workspace, ws, W2, wb))
+    return MF_ERR_INVALID;
+  KernelCtl ctl;
+  if (cudaError_t ge = get_ctl(&ctl); ge != cudaSuccess) return cuda_status(ge);
+  const uintptr_t w0 = round_up(reinterpret_cast<uintptr_t>(workspace), 256);
+  mf_bf16* a = reinterpret_cast<mf_bf16*>(w0);                       // SiLU(GN(.)), reused
+  mf_bf16* h = reinterpret_cast<mf_bf16*>(w0 + round_up(ab, 256));   // first conv's output
+  void* gws = reinterpret_cast<void*>(w0 + 2 * round_up(ab, 256));   // GroupNorm statistics
+  cudaError_t e = launch_group_norm_silu(x, gamma1, beta1, N, H, W, C, G, eps, a, gws, stream);
+  if (e != cudaSuccess) return cuda_status(e);
+  e = launch_conv3x3(a, W1, c1, nullptr, N, H, W, C, C, h, ctl, stream);
+  if (e != cudaSuccess) return cuda_status(e);
+  e = launch_group_norm_silu(h, gamma2, beta2, N, H, W, C, G, eps, a, gws, stream);
+  if (e != cudaSuccess) return cuda_status(e);
+  return cuda_status(launch_conv3x3(a, W2, c2, x, N, H, W, C, C, y, ctl, stream));
 }
 
 mf_status mf_get_error(cudaStream_t stream) {

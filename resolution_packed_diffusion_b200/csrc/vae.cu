@@ -1,0 +1,601 @@
+// vae.cu -- the Mage-VAE conv block's fused chains on sm_100a: GroupNorm + SiLU
+// as one normalise-and-activate pass, and the 3x3 convolution as an implicit
+// GEMM on tcgen05 tensor cores with the bias and the residual fused into its
+// epilogue.
+//
+// Sources (page title, section): picx.dev "Mage-Flow" summary, Methodology >
+// Mage-VAE, "Architecture" (a fully convolutional one-step diffusion decoder
+// of stacked convolutional blocks, no global attention; 16x downsampled,
+// 128-channel latents) and Methodology > Training Infrastructure (the stack's
+// CUDA kernels fuse the normalization - activation - residual chains of the
+// VAE's repeated blocks). The block's wiring is not on the pages; the library
+// takes the diffusion conv nets' residual block:
+//   y = x + conv3x3(SiLU(GN(h)); W2, c2),  h = conv3x3(SiLU(GN(x)); W1, c1).
+// Layout NHWC bf16 (channels innermost); conv weights [Cout][3][3][Cin] bf16;
+// GroupNorm affine parameters and conv biases fp32.
+//
+// Kernels:
+//   gn_partial_kernel   per (pixel chunk, sample): each thread folds its
+//                       8-channel vectors into (count, mean, M2) (Chan's
+//                       pairwise update); the CTA merges them per group in a
+//                       fixed order and writes one partial per group.
+//   gn_finalize_kernel  one CTA per (sample, group): merges the chunks'
+//                       partials in a fixed tree -> (mean, rstd). Deterministic.
+//   gn_silu_kernel      y = SiLU((x - mean) rstd gamma + beta), 16-byte vectors.
+//   conv3x3_kernel<GN>  one persistent CTA per SM, 8 warps: output tiles of 128
+//                       pixels (a BH x BW block of one image) x GN output
+//                       channels (256, else 128, else 64: the widest that
+//                       divides Cout); K runs over 9 taps x Cin / 64 channel blocks.
+//                       warp 0 loads, per K step, the 128 input pixels the tap
+//                       reads (a 4D TMA box {64 channels, BW, BH, 1} at
+//                       (c, w0 + dx - 1, h0 + dy - 1, n): coordinates outside
+//                       the image read as zeros, which is the zero padding) and
+//                       the tap's GN x 64 weight slice, into a 4-stage ring;
+//                       warp 1 issues M = 128, N = GN, K = 16 MMAs into one of
+//                       two TMEM accumulators; warps 4..7 add the bias and the
+//                       residual and store bf16 rows of valid pixels.
+// Every wait is bounded; a CTA whose wait runs out records MF_ERR_TIMEOUT and
+// winds down.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include <cstdint>
+
+#include "mf_internal.h"
+#include "mf_ptx.cuh"
+#include "vae_internal.h"
+
+namespace mf {
+
+namespace {
+
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+__device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+// ------------------------------------------------------------ GroupNorm
+// (count, mean, M2) of a set of values; merge() is Chan et al.'s pairwise
+// update, exact in real arithmetic and stable in floating point.
+struct Moments {
+  float n, mean, m2;
+};
+__device__ __forceinline__ Moments merge(const Moments& a, const Moments& b) {
+  const float n = a.n + b.n;
+  if (n == 0.f) return a;
+  const float d = b.mean - a.mean;
+  const float wb = b.n / n;
+  return {n, fmaf(d, wb, a.mean), a.m2 + b.m2 + d * d * a.n * wb};
+}
+
+constexpr int kGnThreads = 256;
+
+// grid (chunks, N); partial[(n * chunks + chunk) * G + g] = moments of group g
+// over the chunk's pixels. VP = C / 8 vectors per pixel divides 256.
+__global__ void __launch_bounds__(kGnThreads) gn_partial_kernel(
+    const uint4* __restrict__ x, int HW, int C, int G, int chunk_px, float4* __restrict__ partial) {
+  __shared__ Moments s_m[kGnThreads];
+  const int VP = C >> 3;
+  const int rows = kGnThreads / VP;  // pixels in flight per CTA step
+  const int v = threadIdx.x % VP;    // this thread's 8-channel vector
+  const int r = threadIdx.x / VP;
+  const int n = blockIdx.y;
+  const int p0 = blockIdx.x * chunk_px;
+  const int p1 = min(HW, p0 + chunk_px);
+  Moments m = {0.f, 0.f, 0.f};
+  const uint4* xs = x + static_cast<size_t>(n) * HW * VP;
+  for (int p = p0 + r; p < p1; p += rows) {
+    float f[8];
+    unpack8(__ldg(xs + static_cast<size_t>(p) * VP + v), f);
+    float s = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) s += f[e];
+    const float bm = s * 0.125f;
+    float b2 = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) b2 = fmaf(f[e] - bm, f[e] - bm, b2);
+    m = merge(m, Moments{8.f, bm, b2});
+  }
+  s_m[threadIdx.x] = m;
+  __syncthreads();
+  // per vector: merge the rows in order; then per group: its vectors in order
+  if (threadIdx.x < VP) {
+    Moments a = s_m[threadIdx.x];
+    for (int rr = 1; rr < rows; ++rr) a = merge(a, s_m[rr * VP + threadIdx.x]);
+    s_m[threadIdx.x] = a;
+  }
+  __syncthreads();
+  const int vpg = VP / G;  // vectors per group
+  for (int g = threadIdx.x; g < G; g += kGnThreads) {
+    Moments a = s_m[g * vpg];
+    for (int u = 1; u < vpg; ++u) a = merge(a, s_m[g * vpg + u]);
+    partial[(static_cast<size_t>(n) * gridDim.x + blockIdx.x) * G + g] =
+        make_float4(a.n, a.mean, a.m2, 0.f);
+  }
+}
+
+// one CTA per (sample, group): each thread merges the chunks t, t + 256, ...
+// in order, then the CTA merges the threads' moments pairwise in a fixed tree
+// -> stats[n * G + g] = (mean, rstd). The same order every call.
+__global__ void __launch_bounds__(kGnThreads) gn_finalize_kernel(const float4* __restrict__ partial,
+                                                                 int G, int chunks, float eps,
+                                                                 float2* __restrict__ stats) {
+  __shared__ Moments s_m[kGnThreads];
+  const int n = blockIdx.x / G, g = blockIdx.x - n * G;
+  Moments a = {0.f, 0.f, 0.f};
+  for (int c = threadIdx.x; c < chunks; c += kGnThreads) {
+    const float4 p = __ldg(partial + (static_cast<size_t>(n) * chunks + c) * G + g);
+    a = merge(a, Moments{p.x, p.y, p.z});
+  }
+  s_m[threadIdx.x] = a;
+  __syncthreads();
+  for (int half = kGnThreads / 2; half > 0; half >>= 1) {
+    if (threadIdx.x < half) s_m[threadIdx.x] = merge(s_m[threadIdx.x], s_m[threadIdx.x + half]);
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    const Moments m = s_m[0];
+    const float var = m.n > 0.f ? m.m2 / m.n : 0.f;
+    stats[blockIdx.x] = make_float2(m.mean, rsqrtf(var + eps));
+  }
+}
+
+// y = SiLU((x - mean) * rstd * gamma + beta), one 8-channel vector per step
+__global__ void __launch_bounds__(256) gn_silu_kernel(const uint4* __restrict__ x,
+                                                      const float* __restrict__ gamma,
+                                                      const float* __restrict__ beta,
+                                                      const float2* __restrict__ stats,
+                                                      long long total, int HW, int C, int G,
+                                                      uint4* __restrict__ y) {
+  const int VP = C >> 3;
+  const int cg = C / G;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int v = static_cast<int>(i % VP);
+    const int n = static_cast<int>(i / (static_cast<long long>(HW) * VP));
+    const int c0 = 8 * v;
+    const float2 st = __ldg(stats + n * G + c0 / cg);  // a vector never straddles groups
+    const float4 g0 = __ldg(reinterpret_cast<const float4*>(gamma + c0));
+    const float4 g1 = __ldg(reinterpret_cast<const float4*>(gamma + c0 + 4));
+    const float4 b0 = __ldg(reinterpret_cast<const float4*>(beta + c0));
+    const float4 b1 = __ldg(reinterpret_cast<const float4*>(beta + c0 + 4));
+    const float gm[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+    const float bt[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+    float f[8];
+    unpack8(__ldcs(x + i), f);
+    uint32_t o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float a0 = fmaf((f[2 * e] - st.x) * st.y, gm[2 * e], bt[2 * e]);
+      float a1 = fmaf((f[2 * e + 1] - st.x) * st.y, gm[2 * e + 1], bt[2 * e + 1]);
+      a0 = __fdividef(a0, 1.f + __expf(-a0));
+      a1 = __fdividef(a1, 1.f + __expf(-a1));
+      o[e] = pack_bf16x2(a0, a1);
+    }
+    __stcs(y + i, make_uint4(o[0], o[1], o[2], o[3]));
+  }
+}
+
+// ------------------------------------------------------------ conv3x3
+constexpr int CM = 128;            // output pixels per tile (MMA M)
+constexpr int CK = 64;             // input channels per K step (one 128-byte atom)
+constexpr int kConvStages = 4;
+constexpr int kConvThreads = 256;
+constexpr int CA_BYTES = CM * CK * 2;  // A stage: 128 pixels x 64 channels
+
+template <int GN>
+struct ConvLayout {
+  static constexpr int B_BYTES = GN * CK * 2;
+  static constexpr int STAGE = CA_BYTES + B_BYTES;
+  static constexpr int OFF_BAR = kConvStages * STAGE;
+  static constexpr int B_FULL = 0;                       // [stages]
+  static constexpr int B_EMPTY = B_FULL + kConvStages;   // [stages]
+  static constexpr int B_ACC_FULL = B_EMPTY + kConvStages;  // [2]
+  static constexpr int B_ACC_EMPTY = B_ACC_FULL + 2;        // [2], one arrival per epilogue warp
+  static constexpr int B_DRAIN = B_ACC_EMPTY + 2;
+  static constexpr int NUM_BARS = B_DRAIN + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget of one CTA");
+};
+
+struct ConvArgs {
+  int32_t N, H, W, Cin, Cout;
+  int32_t BH, BW;          // pixel tile: BH rows x BW columns of one image (BH * BW = 128)
+  int32_t tiles_h, tiles_w;
+  const float* bias;       // [Cout] or NULL
+  const mf_bf16* residual; // [N][H][W][Cout] or NULL
+  mf_bf16* y;              // [N][H][W][Cout]
+  KernelCtl ctl;
+};
+
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int32_t c, int32_t w, int32_t h, int32_t n) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c), "r"(w), "r"(h), "r"(n)
+      : "memory");
+}
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const KernelCtl& ctl,
+                                          volatile int* abort_flag) {
+  const bool ok = mbar_wait(bar, parity, ctl, abort_flag);
+  return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > limit_ns) return;
+  }
+}
+
+// unit u -> (image n, tile row h0, tile column w0, output-channel tile nt):
+// the output-channel tiles of one pixel tile are consecutive, so they share
+// its input boxes in L2
+__device__ __forceinline__ void conv_unit(const ConvArgs& a, int nN, int u, int& n, int& h0,
+                                          int& w0, int& nt) {
+  nt = u % nN;
+  int t = u / nN;
+  const int tw = t % a.tiles_w;
+  t /= a.tiles_w;
+  const int th = t % a.tiles_h;
+  n = t / a.tiles_h;
+  h0 = th * a.BH;
+  w0 = tw * a.BW;
+}
+
+template <int GN>
+__global__ void __launch_bounds__(kConvThreads, 1)
+    conv3x3_kernel(const __grid_constant__ CUtensorMap tmap_x,
+                   const __grid_constant__ CUtensorMap tmap_w,
+                   const __grid_constant__ ConvArgs args) {
+  using L = ConvLayout<GN>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < L::NUM_BARS; ++i)
+      mbar_init(&bars[i], (i == L::B_ACC_EMPTY || i == L::B_ACC_EMPTY + 1) ? 4u : 1u);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_map(&tmap_x);
+    tma_prefetch_map(&tmap_w);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 2 * GN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int nN = args.Cout / GN;
+  const int units = args.N * args.tiles_h * args.tiles_w * nN;
+  const int ncb = args.Cin / CK;
+  const int nk = 9 * ncb;  // K steps per tile: taps x channel blocks
+
+  if (warp == 0) {
+    // ============================================================ TMA producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        int n, h0, w0, nt;
+        conv_unit(args, nN, u, n, h0, w0, nt);
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int st = it % kConvStages;
+          if (!mbar_wait(&bars[L::B_EMPTY + st], ((it / kConvStages) & 1) ^ 1, args.ctl,
+                         abort_flag)) {
+            ok = false;
+            break;
+          }
+          const int tap = kb / ncb, cb = kb - tap * ncb;
+          const int dy = tap / 3, dx = tap - dy * 3;
+          uint8_t* sa = smem + st * L::STAGE;
+          mbar_expect_tx(&bars[L::B_FULL + st], L::STAGE);
+          // channel coordinate cb * 64: a multiple of 64 elements (128 bytes)
+          tma_load_4d(sa, &tmap_x, &bars[L::B_FULL + st], cb * CK, w0 + dx - 1, h0 + dy - 1, n);
+          tma_load_2d(sa + CA_BYTES, &tmap_w, &bars[L::B_FULL + st], tap * args.Cin + cb * CK,
+                      nt * GN);
+        }
+      }
+      for (int st = 0; st < kConvStages; ++st)
+        if (it > static_cast<uint32_t>(st)) {
+          const uint32_t last = it - 1 - ((it - 1 - st) % kConvStages);
+          drain_wait(&bars[L::B_FULL + st], (last / kConvStages) & 1, args.ctl.wait_limit_ns);
+        }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ============================================================ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC = idesc_bf16_f32(CM, GN, 0, 0);
+      const uint64_t desc0 = sdesc_sw128(smem_u32(smem), 16, 1024);
+      uint32_t it = 0, ul = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++ul) {
+        const uint32_t acc = ul & 1;
+        if (!mbar_wait(&bars[L::B_ACC_EMPTY + acc], ((ul >> 1) & 1) ^ 1, args.ctl, abort_flag))
+          break;
+        tc_fence_after();
+        const uint32_t d = tmem + acc * GN;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int st = it % kConvStages;
+          if (!mbar_wait(&bars[L::B_FULL + st], (it / kConvStages) & 1, args.ctl, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t a0 = desc0 + static_cast<uint64_t>((st * L::STAGE) >> 4);
+          const uint64_t b0 = desc0 + static_cast<uint64_t>((st * L::STAGE + CA_BYTES) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < CK / 16; ++kk)  // a 16-element K step is 32 bytes in the atom
+            umma_ss(d, a0 + kk * 2, b0 + kk * 2, IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(&bars[L::B_EMPTY + st]);
+        }
+        if (!ok) break;
+        umma_commit(&bars[L::B_ACC_FULL + acc]);
+      }
+      umma_commit(&bars[L::B_DRAIN]);
+      drain_wait(&bars[L::B_DRAIN], 0, args.ctl.wait_limit_ns);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ============================================================ epilogue
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;  // pixel of the tile: (row / BW, row % BW)
+    const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+    const int Cout = args.Cout;
+    uint32_t ul = 0;
+    for (int u = blockIdx.x; u < units; u += gridDim.x, ++ul) {
+      int n, h0, w0, nt;
+      conv_unit(args, nN, u, n, h0, w0, nt);
+      const int h = h0 + row / args.BW, w = w0 + row % args.BW;
+      const bool valid = h < args.H && w < args.W;
+      const size_t pix = (static_cast<size_t>(n) * args.H + (valid ? h : 0)) * args.W +
+                         (valid ? w : 0);
+      const uint32_t acc = ul & 1;
+      if (!warp_wait(&bars[L::B_ACC_FULL + acc], (ul >> 1) & 1, args.ctl, abort_flag)) break;
+      tc_fence_after();
+      const int c_base = nt * GN;
+#pragma unroll 1
+      for (int cc = 0; cc < GN; cc += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_base + acc * GN + cc, v);
+        tmem_ld_wait();
+        if (valid) {
+          const size_t off = pix * Cout + c_base + cc;  // 32 channels: four 16-byte vectors
+          float r[32];
+          if (args.residual != nullptr) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              float f[8];
+              unpack8(__ldg(reinterpret_cast<const uint4*>(args.residual + off) + q), f);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) r[8 * q + e] = f[e];
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = 0.f;
+          }
+          if (args.bias != nullptr) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float4 b = __ldg(reinterpret_cast<const float4*>(args.bias + c_base + cc) + q);
+              r[4 * q] += b.x;
+              r[4 * q + 1] += b.y;
+              r[4 * q + 2] += b.z;
+              r[4 * q + 3] += b.w;
+            }
+          }
+          uint4* out = reinterpret_cast<uint4*>(args.y + off);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 o;
+            o.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]) + r[8 * q + 0],
+                              __uint_as_float(v[8 * q + 1]) + r[8 * q + 1]);
+            o.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]) + r[8 * q + 2],
+                              __uint_as_float(v[8 * q + 3]) + r[8 * q + 3]);
+            o.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]) + r[8 * q + 4],
+                              __uint_as_float(v[8 * q + 5]) + r[8 * q + 5]);
+            o.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]) + r[8 * q + 6],
+                              __uint_as_float(v[8 * q + 7]) + r[8 * q + 7]);
+            out[q] = o;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[L::B_ACC_EMPTY + acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 2 * GN);
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// NHWC input as a 4D tensor {C, W, H, N}; box {64 channels, BW, BH, 1}; 128-byte
+// swizzle (a box lands as BH * BW rows of 128 bytes: the K-major A operand);
+// coordinates outside the tensor read as zeros.
+bool make_input_map(CUtensorMap* map, const void* x, int N, int H, int W, int C, int BH, int BW) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(W),
+                              static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(N)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(C) * 2,
+                                 static_cast<cuuint64_t>(W) * C * 2,
+                                 static_cast<cuuint64_t>(H) * W * C * 2};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(CK), static_cast<cuuint32_t>(BW),
+                             static_cast<cuuint32_t>(BH), 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(x), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+// weights [Cout][9 * Cin] (tap-major K); box {64, rows}
+bool make_weight_map(CUtensorMap* map, const void* Wt, int Cout, int Cin, int rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(9) * Cin, static_cast<cuuint64_t>(Cout)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(9) * Cin * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(CK), static_cast<cuuint32_t>(rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(Wt), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+template <int GN>
+cudaError_t launch_conv_t(const CUtensorMap& mx, const CUtensorMap& mw, const ConvArgs& a,
+                          int grid, cudaStream_t st) {
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(
+        conv3x3_kernel<GN>, cudaFuncAttributeMaxDynamicSharedMemorySize, ConvLayout<GN>::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  conv3x3_kernel<GN><<<grid, kConvThreads, ConvLayout<GN>::SMEM_BYTES, st>>>(mx, mw, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int gn_chunks(int32_t N, int32_t H, int32_t W) {
+  // about four CTAs per SM over the whole tensor, at least 64 pixels a chunk
+  const long long HW = static_cast<long long>(H) * W;
+  long long c = (4LL * sm_count() + N - 1) / N;
+  const long long max_c = (HW + 63) / 64;
+  if (c > max_c) c = max_c;
+  return static_cast<int>(c < 1 ? 1 : c);
+}
+
+size_t gn_workspace_bytes(int32_t N, int32_t H, int32_t W, int32_t G) {
+  const size_t partial = static_cast<size_t>(N) * gn_chunks(N, H, W) * G * sizeof(float4);
+  const size_t stats = static_cast<size_t>(N) * G * sizeof(float2);
+  return ((partial + 255) / 256) * 256 + ((stats + 255) / 256) * 256;
+}
+
+cudaError_t launch_group_norm_silu(const mf_bf16* x, const float* gamma, const float* beta,
+                                   int32_t N, int32_t H, int32_t W, int32_t C, int32_t G,
+                                   float eps, mf_bf16* y, void* workspace, cudaStream_t st) {
+  const int chunks = gn_chunks(N, H, W);
+  const int HW = H * W;
+  const int chunk_px = (HW + chunks - 1) / chunks;
+  float4* partial = static_cast<float4*>(workspace);
+  const size_t pbytes = static_cast<size_t>(N) * chunks * G * sizeof(float4);
+  float2* stats = reinterpret_cast<float2*>(static_cast<uint8_t*>(workspace) +
+                                            ((pbytes + 255) / 256) * 256);
+  gn_partial_kernel<<<dim3(chunks, N), kGnThreads, 0, st>>>(reinterpret_cast<const uint4*>(x), HW,
+                                                            C, G, chunk_px, partial);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  gn_finalize_kernel<<<N * G, kGnThreads, 0, st>>>(partial, G, chunks, eps, stats);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const long long total = static_cast<long long>(N) * HW * (C / 8);
+  long long blocks = (total + 255) / 256;
+  const long long cap = 8LL * sm_count();
+  if (blocks > cap) blocks = cap;
+  gn_silu_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+      reinterpret_cast<const uint4*>(x), gamma, beta, stats, total, HW, C, G,
+      reinterpret_cast<uint4*>(y));
+  return cudaGetLastError();
+}
+
+void conv_pixel_tile(int32_t H, int32_t W, int32_t* BH, int32_t* BW) {
+  // the 128-pixel block (BH x BW, BW a power of two from 8 to 128) that
+  // covers the image with the fewest computed pixels; wider on ties
+  long long best = -1;
+  for (int bw = 128; bw >= 8; bw /= 2) {
+    const int bh = 128 / bw;
+    const long long cost = static_cast<long long>((H + bh - 1) / bh) * bh * ((W + bw - 1) / bw) * bw;
+    if (best < 0 || cost < best) {
+      best = cost;
+      *BH = bh;
+      *BW = bw;
+    }
+  }
+}
+
+cudaError_t launch_conv3x3(const mf_bf16* x, const mf_bf16* Wt, const float* bias,
+                           const mf_bf16* residual, int32_t N, int32_t H, int32_t W, int32_t Cin,
+                           int32_t Cout, mf_bf16* y, const KernelCtl& ctl, cudaStream_t st) {
+  static thread_local ConvArgs a;
+  a.N = N;
+  a.H = H;
+  a.W = W;
+  a.Cin = Cin;
+  a.Cout = Cout;
+  conv_pixel_tile(H, W, &a.BH, &a.BW);
+  a.tiles_h = (H + a.BH - 1) / a.BH;
+  a.tiles_w = (W + a.BW - 1) / a.BW;
+  a.bias = bias;
+  a.residual = residual;
+  a.y = y;
+  a.ctl = ctl;
+  const int gn = (Cout % 256 == 0) ? 256 : (Cout % 128 == 0 ? 128 : 64);
+  CUtensorMap mx, mw;
+  if (!make_input_map(&mx, x, N, H, W, Cin, a.BH, a.BW) || !make_weight_map(&mw, Wt, Cout, Cin, gn))
+    return cudaErrorInvalidValue;
+  const long long units = static_cast<long long>(N) * a.tiles_h * a.tiles_w * (Cout / gn);
+  const int grid = units < sm_count() ? static_cast<int>(units) : sm_count();
+  if (gn == 256) return launch_conv_t<256>(mx, mw, a, grid, st);
+  if (gn == 128) return launch_conv_t<128>(mx, mw, a, grid, st);
+  return launch_conv_t<64>(mx, mw, a, grid, st);
+}
+
+}  // namespace mf

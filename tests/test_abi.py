@@ -284,3 +284,37 @@ def test_adaln_params_bwd_argument_checks_without_gpu():
     assert call(dW=P(dmod.value + 64)) == mf.MF_ERR_INVALID      # dW overlaps dmod
     assert call(dW=P(dc.value)) == mf.MF_ERR_INVALID             # the outputs overlap
     assert call(dc=P(dc.value + 8)) == mf.MF_ERR_INVALID         # misaligned
+
+
+def test_vae_argument_checks_without_gpu():
+    """The VAE entry points validate shapes, alignment and overlaps before
+    touching the GPU; workspace sizes follow the documented layout."""
+    lib = mf.lib
+    P = ctypes.c_void_p
+    MB = 1 << 20
+    x, Wt, y, b, ws = (P((i + 1) * 64 * MB) for i in range(5))
+    assert lib.mf_conv3x3(x, Wt, None, None, 1, 8, 8, 96, 64, y, None) == mf.MF_ERR_UNSUPPORTED
+    assert lib.mf_conv3x3(x, Wt, None, None, 1, 8, 8, 64, 4096, y, None) == mf.MF_ERR_UNSUPPORTED
+    assert lib.mf_conv3x3(x, Wt, None, None, 0, 8, 8, 64, 64, y, None) == mf.MF_ERR_INVALID
+    assert lib.mf_conv3x3(x, Wt, None, None, 1, 8, 8, 64, 64, x, None) == mf.MF_ERR_INVALID
+    assert lib.mf_conv3x3(x, Wt, None, P(y.value + 256), 1, 8, 8, 64, 64, y, None) == \
+        mf.MF_ERR_INVALID                                      # residual partly over y
+    assert lib.mf_conv3x3(x, Wt, P(b.value + 4), None, 1, 8, 8, 64, 64, y, None) == \
+        mf.MF_ERR_INVALID                                      # misaligned bias
+    gws = mf.mf_gn_workspace_size(1, 8, 8, 8)
+    assert gws > 0 and mf.mf_gn_workspace_size(0, 8, 8, 8) == 0
+
+    def gn(C=64, G=8, y=y, ws=ws, wsb=gws, eps=1e-6):
+        return lib.mf_group_norm_silu(x, b, b, 1, 8, 8, C, G, eps, y, ws, wsb, None)
+
+    assert gn(G=16) == mf.MF_ERR_UNSUPPORTED                   # 4 channels a group
+    assert gn(C=96, G=12) == mf.MF_ERR_UNSUPPORTED
+    assert gn(y=x) == mf.MF_ERR_INVALID
+    assert gn(wsb=gws - 1) == mf.MF_ERR_INVALID
+    assert gn(ws=x) == mf.MF_ERR_INVALID
+    assert gn(eps=float("nan")) == mf.MF_ERR_INVALID
+    act = 1 * 8 * 8 * 64 * 2
+    assert mf.mf_vae_block_workspace_size(1, 8, 8, 64, 8) >= 2 * act + gws
+    assert lib.mf_vae_res_block(x, b, b, Wt, b, b, b, Wt, b, 1, 8, 8, 64, 8, 1e-6, y, x,
+                                mf.mf_vae_block_workspace_size(1, 8, 8, 64, 8), None) == \
+        mf.MF_ERR_INVALID                                      # workspace over x

@@ -10,31 +10,13 @@ import torch
 
 import oracle
 import resolution_packed_diffusion_b200 as mf
-from gpu_util import MAX_ABS, REL_RMS, dev_bf16, half_ulp_bf16, host_f32, sample_rows
+from gpu_util import assert_block_close, dev_bf16, host_f32, sample_rows
 from packgen import SampleDesc, f32_to_bf16_bits, make_random_pack, make_workload
 
 pytestmark = pytest.mark.gpu
 
 if not torch.cuda.is_available():
     pytest.skip("needs a CUDA device", allow_module_level=True)
-
-
-def assert_block_close(got, ref, name):
-    """The block's output adds a bf16-stored intermediate (y1) that the GPU and
-    the oracle round independently, from fp32 and fp64 values: one bf16 ulp of
-    it can separate them on top of the output's own rounding. The bound is
-    therefore max-abs 2e-2 plus one bf16 ulp at the value's magnitude, with the
-    relative RMS bound unchanged (5e-3)."""
-    got = np.asarray(got, dtype=np.float64)
-    ref = np.asarray(ref, dtype=np.float64)
-    assert got.shape == ref.shape and np.isfinite(got).all(), name
-    err = np.abs(got - ref)
-    tol = MAX_ABS + 2.0 * half_ulp_bf16(ref)
-    worst = int(np.argmax(err - tol))
-    assert (err <= tol).all(), (f"{name}: |err| {err.flat[worst]:.4g} > {tol.flat[worst]:.4g} at "
-                                f"{np.unravel_index(worst, err.shape)}")
-    rr = float(np.linalg.norm(got - ref) / np.linalg.norm(ref))
-    assert rr <= REL_RMS, f"{name}: relative RMS {rr:.3g}"
 
 
 def _weights(rng, hid, F):
