@@ -445,19 +445,32 @@ def run_gpu(args, rank, world, local_rank):
     peaks, peak_src = load_peaks()
     attn_avg = float(np.mean(attn_ms))
     achieved = flops / (attn_avg * 1e-3) / 1e12
-    peak = float(peaks["bf16_tflops"])
+    # The attention kernel is timed inside the loop of whole block steps. When
+    # that loop runs for a second or more, or the clocks show the power cap, the
+    # GPU has settled under its power limit and the denominator is the measured
+    # sustained bf16 rate; a shorter loop at full clocks takes the burst rate.
+    # Both fractions are reported.
+    burst = float(peaks["bf16_tflops"])
+    sustained = float(peaks.get("bf16_tflops_sustained", burst))
+    timed_s = ms_step * args.steps * 1e-3
+    capped = "sw_power_cap" in (clk or {}).get("reasons", [])
+    use_sustained = sustained != burst and (timed_s >= 1.0 or capped)
+    peak = sustained if use_sustained else burst
+    peak_why = (f"{peak_src} bf16_tflops_sustained (timed loop {timed_s:.2f} s"
+                f"{', sw_power_cap active' if capped else ''})" if use_sustained else
+                f"{peak_src} bf16_tflops (burst; timed loop {timed_s:.2f} s, no power cap seen)")
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": workload_config(w, args),
         "block_tokens_per_s": tokens_all / (ms_step * 1e-3),
-        "pct_bf16_peak": 100.0 * value / (peak * world),
+        "pct_bf16_peak": 100.0 * value / (burst * world),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
                      "frac": achieved / peak, "traffic": attn_traffic_bytes(T),
                      "kernel": "varlen_attn_kernel<128, gated, 2D RoPE in the Q prologue>",
-                     "peak_source": f"{peak_src} bf16_tflops (burst)",
-                     "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
+                     "peak_source": peak_why,
+                     "frac_of_burst": achieved / burst, "frac_of_sustained": achieved / sustained,
                      "attn_ms": attn_avg},
         "gpu_launches": launches_per_step * args.steps,
         "e2e": {"value": flops_all / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,

@@ -3,7 +3,8 @@ float64 oracle (``oracle/vae_oracle.py``) on the same seeded inputs: the 3x3
 convolution (implicit GEMM on tcgen05, bias and residual in the epilogue) on
 ragged images whose pixel tiles overhang the edges, both output-channel tile
 widths and a one-row image; SiLU(GroupNorm) (deterministic statistics); and
-the whole block in full on a small image and at a decoder-stage size.
+the whole block in full on a small image, at a decoder-stage size, with one
+group of 512 channels (wider than the conv's channel tile) and with two groups.
 
 Tolerances: a conv or GroupNorm output is one bf16 rounding of an fp32 result
 (max-abs 2e-2, relative RMS 5e-3, as for the attention path); the block adds
@@ -96,9 +97,16 @@ def _block(v):
     return host_f32(y)
 
 
-@pytest.mark.parametrize("name", ["tiny", "stage_1_8"])
-def test_vae_res_block(name):
-    v = make_vae_block(name)
+@pytest.mark.parametrize("name,shape", [
+    ("tiny", None),
+    ("stage_1_8", None),
+    # one group of 512 channels: wider than the conv's 256-channel tile
+    (None, dict(N=1, H=6, W=7, C=512, G=1)),
+    # two groups of 64 channels
+    (None, dict(N=2, H=11, W=5, C=128, G=2)),
+], ids=["tiny", "stage_1_8", "one_group_512ch", "two_groups"])
+def test_vae_res_block(name, shape):
+    v = make_vae_block(name, **(shape or {}))
     got = _block(v)
     ref = oracle.vae_res_block(v.f32("x"), v.gamma1, v.beta1, v.f32("W1"), v.c1, v.gamma2,
                                v.beta2, v.f32("W2"), v.c2, v.G, v.eps)
