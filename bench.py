@@ -544,6 +544,7 @@ def run_linear(args, rank, world, local_rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": w.name, "config_index": args.config, "T": T, "K": K, "N": N,
+                   "linear_cta_pairs": getattr(args, "linear_pair", None),
                    "l2": "x, W and out total %d MB vs 126 MB L2; no flush"
                          % ((T * K + 2 * N * K + T * N) * 2 >> 20)},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
@@ -632,7 +633,7 @@ def run_mmdit(args, rank, world, local_rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic inputs, random-init weights",
         "config": {"workload": w.name, "config_index": args.config, "T": T, "H": H, "D": D,
-                   "hid": hid, "mlp": F},
+                   "hid": hid, "mlp": F, "linear_cta_pairs": getattr(args, "linear_pair", None)},
         "block_tokens_per_s": tokens_all / (ms_step * 1e-3),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
                      "frac": achieved / peak, "traffic": None,
@@ -912,11 +913,15 @@ ARMS = {"block": "run_gpu", "linear": "run_linear", "mmdit": "run_mmdit",
 def run_rank(args, rank, world, local_rank, backend="nccl", arm=None):
     """One rank of the GPU arm: joins the process group when world > 1, runs
     the arm (``arm`` or the one ``--op`` names), leaves the group."""
-    if getattr(args, "cta_pair", None) is not None and arm is None:
+    if arm is None and (getattr(args, "cta_pair", None) is not None
+                        or getattr(args, "linear_pair", None) is not None):
         import torch
         import resolution_packed_diffusion_b200 as mf
         torch.cuda.set_device(local_rank)
-        mf.mf_set_attn_cta_pair(args.cta_pair)
+        if getattr(args, "cta_pair", None) is not None:
+            mf.mf_set_attn_cta_pair(args.cta_pair)
+        if getattr(args, "linear_pair", None) is not None:
+            mf.mf_set_linear_cta_pair(args.linear_pair)
     if world > 1:
         import datetime
         import torch
@@ -963,6 +968,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cta-pair", type=int, default=None, choices=[0, 1],
                     help="attention on CTA pairs (1) or one CTA per SM (0); default: the "
+                         "library's default")
+    ap.add_argument("--linear-pair", type=int, default=None, choices=[0, 1],
+                    help="linear layers on CTA pairs (1) or one CTA per SM (0); default: the "
                          "library's default")
     ap.add_argument("--op", default="block", choices=sorted(ARMS),
                     help="block: the packed joint-attention block (the default line); "

@@ -401,6 +401,16 @@ mf_status mf_set_wait_limit_ns(uint64_t ns);
  * floating-point sums [pack]. Default 0. enable must be 0 or 1. */
 mf_status mf_set_attn_cta_pair(int32_t enable);
 
+/* Kernel of later calls of mf_modality_linear (and so of mf_mmdit_block_fwd) on
+ * the current device: enable = 0, one CTA per SM, each computing 128-row x
+ * 256-column output tiles; enable = 1, CTA pairs (thread-block clusters of two on
+ * two SMs) computing 256-row x 256-column tiles as M = 256 tcgen05 MMAs
+ * (cta_group::2), each CTA loading its own 128 rows of x and half of each weight
+ * tile, so each SM loads a third fewer operand bytes per FLOP. The same products
+ * and rounding, the same results up to the order of floating-point sums [norm].
+ * Default 0. enable must be 0 or 1. */
+mf_status mf_set_linear_cta_pair(int32_t enable);
+
 /* Instrumentation: while both events are non-NULL, every later call of
  * mf_varlen_attn_fwd / mf_block_fwd on the current device records `start` on its
  * stream right before the attention kernel and `stop` right after it, so the

@@ -6,23 +6,32 @@
 // Native-Resolution MMDiT (an MMDiT with modality-specific normalization and
 // joint self-attention: the image and the text stream keep their own weights).
 //
-// Design (one persistent CTA per SM, 8 warps). The output is cut into 128-row x
-// 256-column tiles; a 128-row tile of the pack whose tokens are all of one
-// modality is one job per column tile; a tile that holds both modalities (at
+// Design (one persistent CTA per SM, 8 warps). The output is cut into R-row x
+// 256-column tiles; an R-row block of the pack whose tokens are all of one
+// modality is one job per column tile; a block that holds both modalities (at
 // an image / text boundary) is two jobs, each computed with its modality's
 // weights and writing only its own rows.
-//   warp 0      TMA producer: 128 x 64 slices of x and 256 x 64 slices of W
-//               (128-byte swizzle, no multicast) into a 4-stage ring.
-//   warp 1      tcgen05 issuer: D (fp32, TMEM) += A B^T with M = 128, N = 256,
-//               K = 16, both operands K-major in shared memory; two TMEM
-//               accumulators of 256 columns alternate between jobs so that a
-//               job's epilogue overlaps the next job's MMAs.
+//   warp 0      TMA producer: 128 x 64 slices of x and 64-wide K slices of W
+//               (128-byte swizzle, no multicast) into a ring of stages.
+//   warp 1      tcgen05 issuer: D (fp32, TMEM) += A B^T with N = 256, K = 16,
+//               both operands K-major in shared memory; two TMEM accumulators
+//               of 256 columns alternate between jobs so that a job's
+//               epilogue overlaps the next job's MMAs.
 //   warps 2..3  idle.
 //   warps 4..7  epilogue: one output row per thread (its TMEM lane), 32 columns
 //               at a time, rounded to bf16 and stored if the row exists and is
 //               of the job's modality.
+// Two forms:
+//   single  R = 128, M = 128: each CTA loads 128 x 64 of x and 256 x 64 of W
+//           per K step (48 KB, 4 stages).
+//   pair    R = 256 over a cluster of two CTAs on two SMs (cta_group::2): the
+//           leader issues M = 256 MMAs; each CTA loads its own 128 rows of x
+//           and half of the weight tile (128 output columns), 32 KB per K step
+//           (6 stages), and keeps its 128 rows of the accumulator in its own
+//           TMEM. Per SM the same MMA work needs a third fewer operand bytes
+//           from L2, the limit of the single form.
 // Units (job, column tile) are walked in column blocks of up to 12 tiles, every
-// row tile inside a block: a block of weights stays in L2 while x streams past
+// row block inside a block: a block of weights stays in L2 while x streams past
 // it once per block (see unit_coords). Every wait is bounded.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -38,22 +47,29 @@ namespace mf {
 
 namespace {
 
-constexpr int GM = 128;             // rows per tile (MMA M)
+constexpr int GM = 128;             // rows of x per CTA (MMA M of the single form)
 constexpr int GN = 256;             // output columns per tile (MMA N)
 constexpr int GK = 64;              // K per stage: one 128-byte swizzle atom
-constexpr int kStages = 4;
-constexpr int A_BYTES = GM * GK * 2;
-constexpr int B_BYTES = GN * GK * 2;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int kThreads = 256;
 constexpr uint32_t kTmemCols = 512;  // two accumulators of GN columns
 
+template <bool PAIR>
 struct GemmLayout {
+  static constexpr int ROWS = PAIR ? 2 * GM : GM;   // rows of a job
+  static constexpr int B_ROWS = PAIR ? GN / 2 : GN;  // weight rows this CTA loads
+  static constexpr int STAGES = PAIR ? 6 : 4;
+  static constexpr int A_BYTES = GM * GK * 2;
+  static constexpr int B_BYTES = B_ROWS * GK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr uint32_t kPeers = PAIR ? 2 : 1;  // CTAs whose epilogue warps arrive
   static constexpr int OFF_STAGES = 0;
-  static constexpr int OFF_BAR = kStages * STAGE_BYTES;
-  static constexpr int B_FULL = 0;                    // [kStages]
-  static constexpr int B_EMPTY = B_FULL + kStages;    // [kStages]
-  static constexpr int B_ACC_FULL = B_EMPTY + kStages;  // [2]
+  static constexpr int OFF_BAR = STAGES * STAGE_BYTES;
+  // With PAIR the leader's FULL barriers count both CTAs' bytes and its
+  // ACC_EMPTY both CTAs' epilogue warps; EMPTY and ACC_FULL arrive in both CTAs
+  // from the leader's multicast commits.
+  static constexpr int B_FULL = 0;                      // [STAGES]
+  static constexpr int B_EMPTY = B_FULL + STAGES;       // [STAGES]
+  static constexpr int B_ACC_FULL = B_EMPTY + STAGES;   // [2]
   static constexpr int B_ACC_EMPTY = B_ACC_FULL + 2;    // [2], one arrival per epilogue warp
   static constexpr int B_DRAIN = B_ACC_EMPTY + 2;
   static constexpr int NUM_BARS = B_DRAIN + 1;
@@ -90,6 +106,18 @@ __device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* m
       : "memory");
 }
 
+// The same into this CTA's shared memory, completing on the pair leader's
+// mbarrier (a cluster address). No multicast.
+__device__ __forceinline__ void tma_load_2d_pair_hint(void* dst, const CUtensorMap* map,
+                                                      uint32_t leader_bar, int32_t x, int32_t y,
+                                                      uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(leader_bar), "r"(x), "r"(y), "l"(policy)
+      : "memory");
+}
+
 // Unit u of the traversal -> (job, column tile): column tiles in blocks of nb;
 // inside a block every job (row tile) in turn, the block's column tiles of a
 // job back to back. The ~148 units in flight then cover about 148 / nb row
@@ -122,11 +150,13 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint6
   }
 }
 
+template <bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     modality_linear_kernel(const __grid_constant__ CUtensorMap tmap_x,
                            const __grid_constant__ CUtensorMap tmap_w,
                            const __grid_constant__ GemmArgs args) {
-  using L = GemmLayout;
+  using L = GemmLayout<PAIR>;
+  constexpr int kStages = L::STAGES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
@@ -138,7 +168,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::NUM_BARS; ++i)
-      mbar_init(&bars[i], (i == L::B_ACC_EMPTY || i == L::B_ACC_EMPTY + 1) ? 4u : 1u);
+      mbar_init(&bars[i], (i == L::B_ACC_EMPTY || i == L::B_ACC_EMPTY + 1) ? 4u * L::kPeers : 1u);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -147,16 +177,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_map(&tmap_w);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      // both CTAs' warp 1, the same slot offset: the pair's TMEM at one address
+      tmem_alloc_pair(tmem_slot, kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  // Both CTAs' barriers are initialised before either CTA's arrivals, commits
+  // or copies can reach the other's.
+  if constexpr (PAIR) cluster_sync();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int nN = args.N / GN;
   const int nK = args.K / GK;
   const int units = args.jobs.n * nN;
+  // With PAIR the pair is the scheduling unit; rank r holds rows r * 128 ..
+  // r * 128 + 127 of every job and output columns r * 128 .. of every tile's B.
+  const int rank = PAIR ? static_cast<int>(cluster_ctarank()) : 0;
+  const int unit0 = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int n_units = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (warp == 0) {
     // ============================================================ TMA producer
@@ -164,41 +208,64 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t keep = policy_evict_last();
       uint32_t it = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      for (int u = unit0; u < units && ok; u += n_units) {
         int ji, nt;
         unit_coords(u, args.jobs.n, args.nb, ji, nt);
         const int job = args.jobs.job[ji];
-        const int tile = job & 0x7fff, m = job >> 15;
+        const int blk = job & 0x7fff, m = job >> 15;
+        const int xr = blk * L::ROWS + rank * GM;
+        const int wr = m * args.N + nt * GN + rank * L::B_ROWS;
         for (int kb = 0; kb < nK; ++kb, ++it) {
           const int st = it % kStages;
           if (!mbar_wait(&bars[L::B_EMPTY + st], ((it / kStages) & 1) ^ 1, args.ctl, abort_flag)) {
             ok = false;
             break;
           }
-          uint8_t* sa = smem + L::OFF_STAGES + st * STAGE_BYTES;
-          mbar_expect_tx(&bars[L::B_FULL + st], STAGE_BYTES);
-          tma_load_2d(sa, &tmap_x, &bars[L::B_FULL + st], kb * GK, tile * GM);
-          tma_load_2d_hint(sa + A_BYTES, &tmap_w, &bars[L::B_FULL + st], kb * GK,
-                           m * args.N + nt * GN, keep);
+          uint8_t* sa = smem + L::OFF_STAGES + st * L::STAGE_BYTES;
+          if constexpr (PAIR) {
+            // both CTAs' halves complete on the leader's FULL barrier, which the
+            // leader's producer arms for both (a copy that lands first only takes
+            // the barrier's byte count below zero for a while)
+            if (rank == 0) mbar_expect_tx(&bars[L::B_FULL + st], 2 * L::STAGE_BYTES);
+            const uint32_t lb = cluster_addr(&bars[L::B_FULL + st], 0);
+            tma_load_2d_pair(sa, &tmap_x, lb, kb * GK, xr);
+            tma_load_2d_pair_hint(sa + L::A_BYTES, &tmap_w, lb, kb * GK, wr, keep);
+          } else {
+            mbar_expect_tx(&bars[L::B_FULL + st], L::STAGE_BYTES);
+            tma_load_2d(sa, &tmap_x, &bars[L::B_FULL + st], kb * GK, xr);
+            tma_load_2d_hint(sa + L::A_BYTES, &tmap_w, &bars[L::B_FULL + st], kb * GK, wr, keep);
+          }
         }
       }
-      // every copy this thread started lands before the CTA can exit
-      for (int st = 0; st < kStages; ++st)
-        if (it > static_cast<uint32_t>(st)) {
-          const uint32_t last = it - 1 - ((it - 1 - st) % kStages);
-          drain_wait(&bars[L::B_FULL + st], (last / kStages) & 1, args.ctl.wait_limit_ns);
-        }
+      // Every copy this thread started lands before the CTA can exit. With
+      // PAIR all copies complete on the leader's barriers: the leader drains
+      // them for both CTAs, and the closing cluster barrier keeps rank 1 alive
+      // until then.
+      if (rank == 0)
+        for (int st = 0; st < kStages; ++st)
+          if (it > static_cast<uint32_t>(st)) {
+            const uint32_t last = it - 1 - ((it - 1 - st) % kStages);
+            drain_wait(&bars[L::B_FULL + st], (last / kStages) & 1, args.ctl.wait_limit_ns);
+          }
     }
     __syncwarp();
   } else if (warp == 1) {
     // ============================================================ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t IDESC = idesc_bf16_f32(GM, GN, 0, 0);
+    // With PAIR only the leader issues; every commit that a CTA's producer or
+    // epilogue waits on is multicast to both CTAs.
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t IDESC = idesc_bf16_f32(L::ROWS, GN, 0, 0);
       const uint32_t base = smem_u32(smem + L::OFF_STAGES);
       const uint64_t desc0 = sdesc_sw128(base, 16, 1024);
+      auto commit = [&](int b) {
+        if constexpr (PAIR)
+          umma_commit_pair(&bars[b], 3);
+        else
+          umma_commit(&bars[b]);
+      };
       uint32_t it = 0, ul = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++ul) {
+      for (int u = unit0; u < units && ok; u += n_units, ++ul) {
         const uint32_t acc = ul & 1;
         if (!mbar_wait(&bars[L::B_ACC_EMPTY + acc], ((ul >> 1) & 1) ^ 1, args.ctl, abort_flag)) break;
         tc_fence_after();
@@ -210,17 +277,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint64_t a0 = desc0 + static_cast<uint64_t>((st * STAGE_BYTES) >> 4);
-          const uint64_t b0 = desc0 + static_cast<uint64_t>((st * STAGE_BYTES + A_BYTES) >> 4);
+          const uint64_t a0 = desc0 + static_cast<uint64_t>((st * L::STAGE_BYTES) >> 4);
+          const uint64_t b0 = desc0 + static_cast<uint64_t>((st * L::STAGE_BYTES + L::A_BYTES) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < GK / 16; ++kk)  // a 16-element K step is 32 bytes inside the atom
-            umma_ss(d, a0 + kk * 2, b0 + kk * 2, IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(&bars[L::B_EMPTY + st]);
+          for (int kk = 0; kk < GK / 16; ++kk) {  // a 16-element K step is 32 bytes inside the atom
+            if constexpr (PAIR)
+              umma_ss_pair(d, a0 + kk * 2, b0 + kk * 2, IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
+            else
+              umma_ss(d, a0 + kk * 2, b0 + kk * 2, IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          commit(L::B_EMPTY + st);
         }
         if (!ok) break;
-        umma_commit(&bars[L::B_ACC_FULL + acc]);
+        commit(L::B_ACC_FULL + acc);
       }
-      umma_commit(&bars[L::B_DRAIN]);
+      // every MMA this thread issued completes before TMEM is released
+      if constexpr (PAIR)
+        umma_commit_pair(&bars[L::B_DRAIN], 1);  // the leader's own barrier
+      else
+        umma_commit(&bars[L::B_DRAIN]);
       drain_wait(&bars[L::B_DRAIN], 0, args.ctl.wait_limit_ns);
     }
     __syncwarp();
@@ -230,15 +305,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = wq * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
     uint32_t ul = 0;
-    for (int u = blockIdx.x; u < units; u += gridDim.x, ++ul) {
+    for (int u = unit0; u < units; u += n_units, ++ul) {
       int ji, nt;
       unit_coords(u, args.jobs.n, args.nb, ji, nt);
       const int job = args.jobs.job[ji];
-      const int tile = job & 0x7fff, m = job >> 15;
+      const int blk = job & 0x7fff, m = job >> 15;
       const uint32_t acc = ul & 1;
       if (!warp_wait(&bars[L::B_ACC_FULL + acc], (ul >> 1) & 1, args.ctl, abort_flag)) break;
       tc_fence_after();
-      const int t = tile * GM + row;
+      const int t = blk * L::ROWS + rank * GM + row;
       const bool keep = t < args.T && __ldg(args.tok_mod + t) == m;
       uint4* orow = reinterpret_cast<uint4*>(args.out + static_cast<size_t>(t) * args.N + nt * GN);
 #pragma unroll 1
@@ -266,14 +341,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[L::B_ACC_EMPTY + acc]);
+      if (lane == 0) {
+        if constexpr (PAIR)
+          mbar_arrive_cluster(cluster_addr(&bars[L::B_ACC_EMPTY + acc], 0));
+        else
+          mbar_arrive(&bars[L::B_ACC_EMPTY + acc]);
+      }
     }
   }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+  if constexpr (PAIR) {
+    // The leader has drained its MMAs (which write rank 1's TMEM) and the
+    // copies that complete on its barriers; neither CTA frees TMEM or leaves
+    // before both are here.
+    cluster_sync();
+    if (warp == 1) tmem_dealloc_pair(tmem, kTmemCols);
+  } else {
+    if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+  }
 }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -323,11 +411,60 @@ int sms() {
   return cached[dev];
 }
 
+template <bool PAIR>
+bool kernel_ready(int dev) {
+  static bool attr_set[64] = {false};
+  if (dev < 0 || dev >= 64) return false;
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(modality_linear_kernel<PAIR>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             GemmLayout<PAIR>::SMEM_BYTES) != cudaSuccess)
+      return false;
+    attr_set[dev] = true;
+  }
+  return true;
+}
+
+cudaLaunchConfig_t pair_config(int clusters, cudaLaunchAttribute* attr, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = GemmLayout<true>::SMEM_BYTES;
+  cfg.stream = st;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cfg;
+}
+
+// Clusters of two that can be resident at once (0 if the pair form cannot run).
+int max_clusters(int dev) {
+  static int cached[64] = {0};
+  if (dev < 0 || dev >= 64) return 0;
+  if (cached[dev] == 0) {
+    if (!kernel_ready<true>(dev)) return 0;
+    cudaLaunchAttribute attr[1];
+    cudaLaunchConfig_t cfg = pair_config(1, attr, nullptr);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, modality_linear_kernel<true>, &cfg) != cudaSuccess ||
+        n <= 0)
+      return 0;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
 }  // namespace
 
+int gemm_job_rows(bool pair) { return pair ? 2 * GM : GM; }
+
 bool build_gemm_jobs(const int32_t* mods_per_sample_img, const int32_t* mods_per_sample_txt,
-                     int32_t S, int32_t T, GemmJobs* jobs) {
-  const int tiles = (T + GM - 1) / GM;
+                     int32_t S, int32_t T, int32_t rows, GemmJobs* jobs) {
+  if (rows != GM && rows != 2 * GM) return false;
+  const int tiles = (T + rows - 1) / rows;
   if (tiles > kMaxGemmTiles) return false;
   std::vector<uint8_t> has(static_cast<size_t>(tiles), 0);  // bit m: modality m present
   int64_t row = 0;
@@ -335,7 +472,7 @@ bool build_gemm_jobs(const int32_t* mods_per_sample_img, const int32_t* mods_per
     const int64_t runs[2] = {mods_per_sample_img[s], mods_per_sample_txt[s]};
     for (int m = 0; m < 2; ++m) {
       if (runs[m] > 0) {
-        for (int64_t tl = row / GM; tl <= (row + runs[m] - 1) / GM; ++tl) has[tl] |= 1u << m;
+        for (int64_t tl = row / rows; tl <= (row + runs[m] - 1) / rows; ++tl) has[tl] |= 1u << m;
         row += runs[m];
       }
     }
@@ -350,12 +487,13 @@ bool build_gemm_jobs(const int32_t* mods_per_sample_img, const int32_t* mods_per
 }
 
 cudaError_t launch_modality_linear(const mf_bf16* x, const mf_bf16* W, const uint8_t* tok_mod,
-                                   const GemmJobs& jobs, int32_t T, int32_t K, int32_t N,
-                                   int32_t act, mf_bf16* out, const KernelCtl& ctl,
+                                   const GemmJobs& jobs, bool pair, int32_t T, int32_t K,
+                                   int32_t N, int32_t act, mf_bf16* out, const KernelCtl& ctl,
                                    cudaStream_t st) {
   if (jobs.n == 0) return cudaSuccess;
   CUtensorMap mx, mw;
-  if (!make_map(&mx, x, T, K, GM) || !make_map(&mw, W, 2LL * N, K, GN))
+  const int b_rows = pair ? GemmLayout<true>::B_ROWS : GemmLayout<false>::B_ROWS;
+  if (!make_map(&mx, x, T, K, GM) || !make_map(&mw, W, 2LL * N, K, b_rows))
     return cudaErrorInvalidValue;
   static thread_local GemmArgs a;
   a.jobs = jobs;
@@ -371,18 +509,20 @@ cudaError_t launch_modality_linear(const mf_bf16* x, const mf_bf16* W, const uin
   for (int d = 1; d <= 12 && d <= nN; ++d)
     if (nN % d == 0) a.nb = d;
   a.ctl = ctl;
-  static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    const cudaError_t e = cudaFuncSetAttribute(
-        modality_linear_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GemmLayout::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
+  const int units = jobs.n * nN;
+  if (pair) {
+    const int mc = max_clusters(dev);
+    if (mc <= 0) return cudaErrorInvalidConfiguration;
+    const int clusters = units < mc ? units : mc;
+    cudaLaunchAttribute attr[1];
+    cudaLaunchConfig_t cfg = pair_config(clusters, attr, st);
+    return cudaLaunchKernelEx(&cfg, modality_linear_kernel<true>, mx, mw, a);
   }
-  const int units = jobs.n * (N / GN);
+  if (!kernel_ready<false>(dev)) return cudaErrorInvalidConfiguration;
   const int grid = units < sms() ? units : sms();
-  modality_linear_kernel<<<grid, kThreads, GemmLayout::SMEM_BYTES, st>>>(mx, mw, a);
+  modality_linear_kernel<false><<<grid, kThreads, GemmLayout<false>::SMEM_BYTES, st>>>(mx, mw, a);
   return cudaGetLastError();
 }
 

@@ -33,6 +33,7 @@ struct DeviceState {
   cudaEvent_t attn_start = nullptr;  // instrumentation (mf_set_attn_timing_events)
   cudaEvent_t attn_stop = nullptr;
   bool attn_pair = false;            // mf_set_attn_cta_pair
+  bool linear_pair = false;          // mf_set_linear_cta_pair
 };
 
 DeviceState g_state[kMaxDevices];
@@ -620,12 +621,16 @@ mf_status mf_modality_linear(const mf_bf16* x, const mf_bf16* W, const uint8_t* 
   const size_t xb = static_cast<size_t>(T) * K * 2, wb = static_cast<size_t>(2) * N * K * 2,
                ob = static_cast<size_t>(T) * N * 2;
   if (overlap(out, ob, x, xb) || overlap(out, ob, W, wb)) return MF_ERR_INVALID;
-  static thread_local GemmJobs jobs;
-  if (!build_gemm_jobs(n_img, n_txt, S, static_cast<int32_t>(T), &jobs)) return MF_ERR_UNSUPPORTED;
   KernelCtl ctl;
   if (cudaError_t ge = get_ctl(&ctl); ge != cudaSuccess) return cuda_status(ge);
-  return cuda_status(launch_modality_linear(x, W, tok_mod, jobs, static_cast<int32_t>(T), K, N,
-                                            act, out, ctl, stream));
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MF_ERR_CUDA;
+  const bool pair = g_state[dev].linear_pair;
+  static thread_local GemmJobs jobs;
+  if (!build_gemm_jobs(n_img, n_txt, S, static_cast<int32_t>(T), gemm_job_rows(pair), &jobs))
+    return MF_ERR_UNSUPPORTED;
+  return cuda_status(launch_modality_linear(x, W, tok_mod, jobs, pair, static_cast<int32_t>(T), K,
+                                            N, act, out, ctl, stream));
 }
 
 namespace {
@@ -760,6 +765,16 @@ mf_status mf_set_attn_cta_pair(int32_t enable) {
   if (dev < 0 || dev >= kMaxDevices) return MF_ERR_INVALID;
   std::lock_guard<std::mutex> lock(g_mutex);
   g_state[dev].attn_pair = enable != 0;
+  return MF_OK;
+}
+
+mf_status mf_set_linear_cta_pair(int32_t enable) {
+  if (enable != 0 && enable != 1) return MF_ERR_INVALID;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MF_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MF_ERR_INVALID;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  g_state[dev].linear_pair = enable != 0;
   return MF_OK;
 }
 

@@ -1,6 +1,9 @@
 """The modality-specific linear layer on the GPU (tcgen05), through the C ABI,
 against the oracle: every row of small packs whose 128-row tiles mix image and
-text tokens, and sampled rows of a full-size projection."""
+text tokens, and sampled rows of a full-size projection. Each case runs on both
+kernels: one CTA per 128-row tile, and CTA pairs (mf_set_linear_cta_pair(1),
+256-row tiles as M = 256 MMAs over two SMs, whose row blocks may hold a
+modality in one CTA's half only)."""
 
 import numpy as np
 import pytest
@@ -15,6 +18,13 @@ pytestmark = pytest.mark.gpu
 
 if not torch.cuda.is_available():
     pytest.skip("needs a CUDA device", allow_module_level=True)
+
+
+@pytest.fixture(params=[0, 1], ids=["one_cta", "cta_pair"], autouse=True)
+def cta_pair(request):
+    mf.mf_set_linear_cta_pair(request.param)
+    yield request.param
+    mf.mf_set_linear_cta_pair(0)
 
 
 def _run(descs, K, N, seed, act=0):
@@ -38,6 +48,9 @@ SMALL = [
     ([SampleDesc(1, 16, 16, 20), SampleDesc(1, 8, 32, 12)], 192, 512),   # the 544-token pack
     ([SampleDesc(1, 1, 1, 0)], 64, 256),                                  # one token
     ([SampleDesc(0, 0, 0, 300), SampleDesc(1, 11, 13, 0)], 320, 256),    # text-only sample
+    # a 256-row block whose first 128 rows are image and second 128 rows text:
+    # each modality lives in one CTA's half of the pair's block
+    ([SampleDesc(1, 8, 16, 128), SampleDesc(1, 16, 8, 128)], 128, 256),
 ]
 
 
@@ -69,6 +82,11 @@ def test_linear_qkv_projection_of_the_training_pack():
     ref = oracle.modality_linear(x[rows], W, pack["tok_mod"][rows])
     assert np.isfinite(out).all()
     assert_bf16_close(out[rows], ref, "projection rows")
+
+
+def test_linear_pair_setting_is_checked():
+    with pytest.raises(mf.MFError):
+        mf.mf_set_linear_cta_pair(2)
 
 
 def test_linear_rejects_bad_shapes():

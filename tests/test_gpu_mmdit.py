@@ -60,10 +60,15 @@ def _run(w, F, seed, rows=None):
     return got if rows is None else got[rows], ref
 
 
-def test_mmdit_block_small_pack_every_row():
+@pytest.mark.parametrize("linear_pair", [0, 1], ids=["one_cta", "linear_cta_pairs"])
+def test_mmdit_block_small_pack_every_row(linear_pair):
     descs = [SampleDesc(1, 9, 14, 5), SampleDesc(0, 0, 0, 33), SampleDesc(1, 11, 13, 2)]
     w = make_random_pack(970, S=3, H=2, D=128, rope_axes=2, descs=descs)
-    got, ref = _run(w, 512, 971)
+    mf.mf_set_linear_cta_pair(linear_pair)
+    try:
+        got, ref = _run(w, 512, 971)
+    finally:
+        mf.mf_set_linear_cta_pair(0)
     assert np.isfinite(got).all()
     assert_block_close(got, ref, "block y")
 
