@@ -408,7 +408,7 @@ mf_status mf_set_attn_cta_pair(int32_t enable);
  * (cta_group::2), each CTA loading its own 128 rows of x and half of each weight
  * tile, so each SM loads a third fewer operand bytes per FLOP. The same products
  * and rounding, the same results up to the order of floating-point sums [norm].
- * Default 0. enable must be 0 or 1. */
+ * Default 1 (measured faster on every pack). enable must be 0 or 1. */
 mf_status mf_set_linear_cta_pair(int32_t enable);
 
 /* Instrumentation: while both events are non-NULL, every later call of

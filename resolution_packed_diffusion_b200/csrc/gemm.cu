@@ -27,7 +27,7 @@
 //   pair    R = 256 over a cluster of two CTAs on two SMs (cta_group::2): the
 //           leader issues M = 256 MMAs; each CTA loads its own 128 rows of x
 //           and half of the weight tile (128 output columns), 32 KB per K step
-//           (6 stages), and keeps its 128 rows of the accumulator in its own
+//           (7 stages), and keeps its 128 rows of the accumulator in its own
 //           TMEM. Per SM the same MMA work needs a third fewer operand bytes
 //           from L2, the limit of the single form.
 // Units (job, column tile) are walked in column blocks of up to 12 tiles, every
@@ -57,7 +57,7 @@ template <bool PAIR>
 struct GemmLayout {
   static constexpr int ROWS = PAIR ? 2 * GM : GM;   // rows of a job
   static constexpr int B_ROWS = PAIR ? GN / 2 : GN;  // weight rows this CTA loads
-  static constexpr int STAGES = PAIR ? 6 : 4;
+  static constexpr int STAGES = PAIR ? 7 : 4;
   static constexpr int A_BYTES = GM * GK * 2;
   static constexpr int B_BYTES = B_ROWS * GK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;

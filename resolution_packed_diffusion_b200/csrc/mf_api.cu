@@ -33,7 +33,7 @@ struct DeviceState {
   cudaEvent_t attn_start = nullptr;  // instrumentation (mf_set_attn_timing_events)
   cudaEvent_t attn_stop = nullptr;
   bool attn_pair = false;            // mf_set_attn_cta_pair
-  bool linear_pair = false;          // mf_set_linear_cta_pair
+  bool linear_pair = true;           // mf_set_linear_cta_pair
 };
 
 DeviceState g_state[kMaxDevices];

@@ -24,7 +24,7 @@ if not torch.cuda.is_available():
 def cta_pair(request):
     mf.mf_set_linear_cta_pair(request.param)
     yield request.param
-    mf.mf_set_linear_cta_pair(0)
+    mf.mf_set_linear_cta_pair(1)  # the library's default
 
 
 def _run(descs, K, N, seed, act=0):
