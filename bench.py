@@ -897,7 +897,8 @@ def run_vae(args, rank, world, local_rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic activations, random-init weights",
         "config": {"workload": f"VAE block {args.vae_config}", "N": N, "H": H, "W": W, "C": C,
-                   "G": G, "l2": "activations %.0f MB each, weights %.1f MB; no flush"
+                   "G": G, "conv_cta_pairs": getattr(args, "conv_pair", None),
+                   "l2": "activations %.0f MB each, weights %.1f MB; no flush"
                    % (act_mb, 2 * C * 9 * C * 2 / 1e6)},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
                      "frac": achieved / peak, "traffic": None,
@@ -914,7 +915,8 @@ def run_rank(args, rank, world, local_rank, backend="nccl", arm=None):
     """One rank of the GPU arm: joins the process group when world > 1, runs
     the arm (``arm`` or the one ``--op`` names), leaves the group."""
     if arm is None and (getattr(args, "cta_pair", None) is not None
-                        or getattr(args, "linear_pair", None) is not None):
+                        or getattr(args, "linear_pair", None) is not None
+                        or getattr(args, "conv_pair", None) is not None):
         import torch
         import resolution_packed_diffusion_b200 as mf
         torch.cuda.set_device(local_rank)
@@ -922,6 +924,8 @@ def run_rank(args, rank, world, local_rank, backend="nccl", arm=None):
             mf.mf_set_attn_cta_pair(args.cta_pair)
         if getattr(args, "linear_pair", None) is not None:
             mf.mf_set_linear_cta_pair(args.linear_pair)
+        if getattr(args, "conv_pair", None) is not None:
+            mf.mf_set_conv_cta_pair(args.conv_pair)
     if world > 1:
         import datetime
         import torch
@@ -972,6 +976,9 @@ def main():
     ap.add_argument("--linear-pair", type=int, default=None, choices=[0, 1],
                     help="linear layers on CTA pairs (1) or one CTA per SM (0); default: the "
                          "library's default")
+    ap.add_argument("--conv-pair", type=int, default=None, choices=[0, 1],
+                    help="VAE convolutions on CTA pairs (1) or one CTA per SM (0); default: "
+                         "the library's default")
     ap.add_argument("--op", default="block", choices=sorted(ARMS),
                     help="block: the packed joint-attention block (the default line); "
                          "linear: the modality-specific linear layer as a QKV projection; "

@@ -411,6 +411,15 @@ mf_status mf_set_attn_cta_pair(int32_t enable);
  * Default 1 (measured faster on every pack). enable must be 0 or 1. */
 mf_status mf_set_linear_cta_pair(int32_t enable);
 
+/* Kernel of later calls of mf_conv3x3 and mf_vae_res_block on the current device:
+ * enable = 0, one CTA per SM, each computing 128-pixel x GN-channel output tiles;
+ * enable = 1, CTA pairs (thread-block clusters of two on two SMs) computing two
+ * vertically adjacent 128-pixel tiles as M = 256 tcgen05 MMAs (cta_group::2), each
+ * CTA loading its own tile's input boxes and half of each weight slice. The same
+ * products and rounding, the same results up to the order of floating-point sums
+ * [vfuse]. Default 0. enable must be 0 or 1. */
+mf_status mf_set_conv_cta_pair(int32_t enable);
+
 /* Instrumentation: while both events are non-NULL, every later call of
  * mf_varlen_attn_fwd / mf_block_fwd on the current device records `start` on its
  * stream right before the attention kernel and `stop` right after it, so the

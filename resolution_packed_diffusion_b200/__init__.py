@@ -83,6 +83,7 @@ _SIGS = {
     "mf_set_attn_timing_events": (_I, [_P, _P]),
     "mf_set_attn_cta_pair": (_I, [_I]),
     "mf_set_linear_cta_pair": (_I, [_I]),
+    "mf_set_conv_cta_pair": (_I, [_I]),
     "mf_block_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F,
                                   _F, _P, _P, _P]),
     "mf_cfg_combine": (_I, [_P, _P, _I, _P, _I, _I, _F, _P, _P]),
@@ -288,6 +289,10 @@ def mf_set_attn_cta_pair(enable: int) -> None:
 
 def mf_set_linear_cta_pair(enable: int) -> None:
     _check(lib.mf_set_linear_cta_pair(int(enable)), "mf_set_linear_cta_pair")
+
+
+def mf_set_conv_cta_pair(enable: int) -> None:
+    _check(lib.mf_set_conv_cta_pair(int(enable)), "mf_set_conv_cta_pair")
 
 
 def mf_set_attn_timing_events(start, stop) -> None:

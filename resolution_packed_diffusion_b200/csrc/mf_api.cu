@@ -34,6 +34,7 @@ struct DeviceState {
   cudaEvent_t attn_stop = nullptr;
   bool attn_pair = false;            // mf_set_attn_cta_pair
   bool linear_pair = true;           // mf_set_linear_cta_pair
+  bool conv_pair = false;            // mf_set_conv_cta_pair
 };
 
 DeviceState g_state[kMaxDevices];
@@ -643,6 +644,15 @@ bool vae_shape_ok(int32_t N, int32_t H, int32_t W) {
   return N >= 1 && H >= 1 && W >= 1 && static_cast<int64_t>(N) * H * W < (int64_t{1} << 31) &&
          H <= (1 << 20) && W <= (1 << 20);
 }
+
+// The conv kernel form chosen for the current device (mf_set_conv_cta_pair).
+bool conv_pair_setting(bool* pair) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  *pair = g_state[dev].conv_pair;
+  return true;
+}
 }  // namespace
 
 size_t mf_gn_workspace_size(int32_t N, int32_t H, int32_t W, int32_t G) {
@@ -689,7 +699,10 @@ mf_status mf_conv3x3(const mf_bf16* x, const mf_bf16* Wt, const float* bias,
   if (residual != nullptr && residual != y && overlap(residual, yb, y, yb)) return MF_ERR_INVALID;
   KernelCtl ctl;
   if (cudaError_t ge = get_ctl(&ctl); ge != cudaSuccess) return cuda_status(ge);
-  return cuda_status(launch_conv3x3(x, Wt, bias, residual, N, H, W, Cin, Cout, y, ctl, stream));
+  bool pair = false;
+  if (!conv_pair_setting(&pair)) return MF_ERR_CUDA;
+  return cuda_status(
+      launch_conv3x3(x, Wt, bias, residual, N, H, W, Cin, Cout, y, pair, ctl, stream));
 }
 
 size_t mf_vae_block_workspace_size(int32_t N, int32_t H, int32_t W, int32_t C, int32_t G) {
@@ -723,17 +736,19 @@ mf_status mf_vae_res_block(const mf_bf16* x, const float* gamma1, const float* b
     return MF_ERR_INVALID;
   KernelCtl ctl;
   if (cudaError_t ge = get_ctl(&ctl); ge != cudaSuccess) return cuda_status(ge);
+  bool pair = false;
+  if (!conv_pair_setting(&pair)) return MF_ERR_CUDA;
   const uintptr_t w0 = round_up(reinterpret_cast<uintptr_t>(workspace), 256);
   mf_bf16* a = reinterpret_cast<mf_bf16*>(w0);                       // SiLU(GN(.)), reused
   mf_bf16* h = reinterpret_cast<mf_bf16*>(w0 + round_up(ab, 256));   // first conv's output
   void* gws = reinterpret_cast<void*>(w0 + 2 * round_up(ab, 256));   // GroupNorm statistics
   cudaError_t e = launch_group_norm_silu(x, gamma1, beta1, N, H, W, C, G, eps, a, gws, stream);
   if (e != cudaSuccess) return cuda_status(e);
-  e = launch_conv3x3(a, W1, c1, nullptr, N, H, W, C, C, h, ctl, stream);
+  e = launch_conv3x3(a, W1, c1, nullptr, N, H, W, C, C, h, pair, ctl, stream);
   if (e != cudaSuccess) return cuda_status(e);
   e = launch_group_norm_silu(h, gamma2, beta2, N, H, W, C, G, eps, a, gws, stream);
   if (e != cudaSuccess) return cuda_status(e);
-  return cuda_status(launch_conv3x3(a, W2, c2, x, N, H, W, C, C, y, ctl, stream));
+  return cuda_status(launch_conv3x3(a, W2, c2, x, N, H, W, C, C, y, pair, ctl, stream));
 }
 
 mf_status mf_get_error(cudaStream_t stream) {
@@ -775,6 +790,16 @@ mf_status mf_set_linear_cta_pair(int32_t enable) {
   if (dev < 0 || dev >= kMaxDevices) return MF_ERR_INVALID;
   std::lock_guard<std::mutex> lock(g_mutex);
   g_state[dev].linear_pair = enable != 0;
+  return MF_OK;
+}
+
+mf_status mf_set_conv_cta_pair(int32_t enable) {
+  if (enable != 0 && enable != 1) return MF_ERR_INVALID;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MF_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MF_ERR_INVALID;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  g_state[dev].conv_pair = enable != 0;
   return MF_OK;
 }
 

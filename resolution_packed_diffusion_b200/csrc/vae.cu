@@ -34,6 +34,12 @@
 //                       warp 1 issues M = 128, N = GN, K = 16 MMAs into one of
 //                       two TMEM accumulators; warps 4..7 add the bias and the
 //                       residual and store bf16 rows of valid pixels.
+//                       With CTA pairs (cta_group::2) a cluster of two CTAs on
+//                       two SMs computes two vertically adjacent pixel tiles
+//                       (2 BH x BW) as M = 256 MMAs issued by the leader: each
+//                       CTA loads its own tile's input boxes and half of each
+//                       weight slice (GN / 2 rows), so each SM loads a quarter
+//                       to a third fewer operand bytes per FLOP.
 // Every wait is bounded; a CTA whose wait runs out records MF_ERR_TIMEOUT and
 // winds down.
 #include <cuda.h>
@@ -197,30 +203,37 @@ __global__ void __launch_bounds__(256) gn_silu_kernel(const uint4* __restrict__ 
 // ------------------------------------------------------------ conv3x3
 constexpr int CM = 128;            // output pixels per tile (MMA M)
 constexpr int CK = 64;             // input channels per K step (one 128-byte atom)
-constexpr int kConvStages = 4;
 constexpr int kConvThreads = 256;
 constexpr int CA_BYTES = CM * CK * 2;  // A stage: 128 pixels x 64 channels
 
-template <int GN>
+template <int GN, bool PAIR>
 struct ConvLayout {
-  static constexpr int B_BYTES = GN * CK * 2;
+  static constexpr int B_ROWS = PAIR ? GN / 2 : GN;  // weight rows this CTA loads
+  static constexpr int B_BYTES = B_ROWS * CK * 2;
   static constexpr int STAGE = CA_BYTES + B_BYTES;
-  static constexpr int OFF_BAR = kConvStages * STAGE;
-  static constexpr int B_FULL = 0;                       // [stages]
-  static constexpr int B_EMPTY = B_FULL + kConvStages;   // [stages]
-  static constexpr int B_ACC_FULL = B_EMPTY + kConvStages;  // [2]
-  static constexpr int B_ACC_EMPTY = B_ACC_FULL + 2;        // [2], one arrival per epilogue warp
+  static constexpr int STAGES = (200 * 1024 / STAGE) < 8 ? (200 * 1024 / STAGE) : 8;
+  static constexpr uint32_t kPeers = PAIR ? 2 : 1;  // CTAs whose epilogue warps arrive
+  static constexpr int OFF_BAR = STAGES * STAGE;
+  // With PAIR the leader's FULL barriers count both CTAs' bytes and its
+  // ACC_EMPTY both CTAs' epilogue warps; EMPTY and ACC_FULL arrive in both CTAs
+  // from the leader's multicast commits.
+  static constexpr int B_FULL = 0;                      // [stages]
+  static constexpr int B_EMPTY = B_FULL + STAGES;       // [stages]
+  static constexpr int B_ACC_FULL = B_EMPTY + STAGES;   // [2]
+  static constexpr int B_ACC_EMPTY = B_ACC_FULL + 2;    // [2], one arrival per epilogue warp
   static constexpr int B_DRAIN = B_ACC_EMPTY + 2;
   static constexpr int NUM_BARS = B_DRAIN + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static_assert(STAGE % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget of one CTA");
 };
 
 struct ConvArgs {
   int32_t N, H, W, Cin, Cout;
   int32_t BH, BW;          // pixel tile: BH rows x BW columns of one image (BH * BW = 128)
-  int32_t tiles_h, tiles_w;
+  int32_t UH;              // rows of a unit's pixel block: BH, or 2 BH with CTA pairs
+  int32_t tiles_h, tiles_w;  // unit blocks down and across an image
   const float* bias;       // [Cout] or NULL
   const mf_bf16* residual; // [N][H][W][Cout] or NULL
   mf_bf16* y;              // [N][H][W][Cout]
@@ -233,6 +246,18 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, u
       "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c), "r"(w), "r"(h), "r"(n)
+      : "memory");
+}
+
+// The same into this CTA's shared memory, completing on the pair leader's
+// mbarrier (a cluster address). No multicast.
+__device__ __forceinline__ void tma_load_4d_pair(void* dst, const CUtensorMap* map,
+                                                 uint32_t leader_bar, int32_t c, int32_t w,
+                                                 int32_t h, int32_t n) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(leader_bar), "r"(c), "r"(w), "r"(h), "r"(n)
       : "memory");
 }
 
@@ -260,16 +285,17 @@ __device__ __forceinline__ void conv_unit(const ConvArgs& a, int nN, int u, int&
   t /= a.tiles_w;
   const int th = t % a.tiles_h;
   n = t / a.tiles_h;
-  h0 = th * a.BH;
+  h0 = th * a.UH;
   w0 = tw * a.BW;
 }
 
-template <int GN>
+template <int GN, bool PAIR>
 __global__ void __launch_bounds__(kConvThreads, 1)
     conv3x3_kernel(const __grid_constant__ CUtensorMap tmap_x,
                    const __grid_constant__ CUtensorMap tmap_w,
                    const __grid_constant__ ConvArgs args) {
-  using L = ConvLayout<GN>;
+  using L = ConvLayout<GN, PAIR>;
+  constexpr int kConvStages = L::STAGES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
@@ -281,7 +307,7 @@ __global__ void __launch_bounds__(kConvThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::NUM_BARS; ++i)
-      mbar_init(&bars[i], (i == L::B_ACC_EMPTY || i == L::B_ACC_EMPTY + 1) ? 4u : 1u);
+      mbar_init(&bars[i], (i == L::B_ACC_EMPTY || i == L::B_ACC_EMPTY + 1) ? 4u * L::kPeers : 1u);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -290,26 +316,41 @@ __global__ void __launch_bounds__(kConvThreads, 1)
     tma_prefetch_map(&tmap_w);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 2 * GN);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      // both CTAs' warp 1, the same slot offset: the pair's TMEM at one address
+      tmem_alloc_pair(tmem_slot, 2 * GN);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, 2 * GN);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  // Both CTAs' barriers are initialised before either CTA's arrivals, commits
+  // or copies can reach the other's.
+  if constexpr (PAIR) cluster_sync();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int nN = args.Cout / GN;
   const int units = args.N * args.tiles_h * args.tiles_w * nN;
   const int ncb = args.Cin / CK;
   const int nk = 9 * ncb;  // K steps per tile: taps x channel blocks
+  // With PAIR the pair is the scheduling unit: rank r computes the pixel tile
+  // r * BH rows below the unit's origin and loads weight rows r * GN / 2 ..
+  const int rank = PAIR ? static_cast<int>(cluster_ctarank()) : 0;
+  const int unit0 = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int n_units = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (warp == 0) {
     // ============================================================ TMA producer
     if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      for (int u = unit0; u < units && ok; u += n_units) {
         int n, h0, w0, nt;
         conv_unit(args, nN, u, n, h0, w0, nt);
+        h0 += rank * args.BH;
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int st = it % kConvStages;
           if (!mbar_wait(&bars[L::B_EMPTY + st], ((it / kConvStages) & 1) ^ 1, args.ctl,
@@ -320,28 +361,52 @@ __global__ void __launch_bounds__(kConvThreads, 1)
           const int tap = kb / ncb, cb = kb - tap * ncb;
           const int dy = tap / 3, dx = tap - dy * 3;
           uint8_t* sa = smem + st * L::STAGE;
-          mbar_expect_tx(&bars[L::B_FULL + st], L::STAGE);
           // channel coordinate cb * 64: a multiple of 64 elements (128 bytes)
-          tma_load_4d(sa, &tmap_x, &bars[L::B_FULL + st], cb * CK, w0 + dx - 1, h0 + dy - 1, n);
-          tma_load_2d(sa + CA_BYTES, &tmap_w, &bars[L::B_FULL + st], tap * args.Cin + cb * CK,
-                      nt * GN);
+          const int wrow = nt * GN + rank * L::B_ROWS;
+          if constexpr (PAIR) {
+            // both CTAs' copies complete on the leader's FULL barrier, which the
+            // leader's producer arms for both (a copy that lands first only
+            // takes the barrier's byte count below zero for a while)
+            if (rank == 0) mbar_expect_tx(&bars[L::B_FULL + st], 2 * L::STAGE);
+            const uint32_t lb = cluster_addr(&bars[L::B_FULL + st], 0);
+            tma_load_4d_pair(sa, &tmap_x, lb, cb * CK, w0 + dx - 1, h0 + dy - 1, n);
+            tma_load_2d_pair(sa + CA_BYTES, &tmap_w, lb, tap * args.Cin + cb * CK, wrow);
+          } else {
+            mbar_expect_tx(&bars[L::B_FULL + st], L::STAGE);
+            tma_load_4d(sa, &tmap_x, &bars[L::B_FULL + st], cb * CK, w0 + dx - 1, h0 + dy - 1, n);
+            tma_load_2d(sa + CA_BYTES, &tmap_w, &bars[L::B_FULL + st], tap * args.Cin + cb * CK,
+                        wrow);
+          }
         }
       }
-      for (int st = 0; st < kConvStages; ++st)
-        if (it > static_cast<uint32_t>(st)) {
-          const uint32_t last = it - 1 - ((it - 1 - st) % kConvStages);
-          drain_wait(&bars[L::B_FULL + st], (last / kConvStages) & 1, args.ctl.wait_limit_ns);
-        }
+      // Every copy this thread started lands before the CTA can exit. With
+      // PAIR all copies complete on the leader's barriers: the leader drains
+      // them for both CTAs, and the closing cluster barrier keeps rank 1 alive
+      // until then.
+      if (rank == 0)
+        for (int st = 0; st < kConvStages; ++st)
+          if (it > static_cast<uint32_t>(st)) {
+            const uint32_t last = it - 1 - ((it - 1 - st) % kConvStages);
+            drain_wait(&bars[L::B_FULL + st], (last / kConvStages) & 1, args.ctl.wait_limit_ns);
+          }
     }
     __syncwarp();
   } else if (warp == 1) {
     // ============================================================ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t IDESC = idesc_bf16_f32(CM, GN, 0, 0);
+    // With PAIR only the leader issues; every commit that a CTA's producer or
+    // epilogue waits on is multicast to both CTAs.
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t IDESC = idesc_bf16_f32(PAIR ? 2 * CM : CM, GN, 0, 0);
       const uint64_t desc0 = sdesc_sw128(smem_u32(smem), 16, 1024);
+      auto commit = [&](int b) {
+        if constexpr (PAIR)
+          umma_commit_pair(&bars[b], 3);
+        else
+          umma_commit(&bars[b]);
+      };
       uint32_t it = 0, ul = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++ul) {
+      for (int u = unit0; u < units && ok; u += n_units, ++ul) {
         const uint32_t acc = ul & 1;
         if (!mbar_wait(&bars[L::B_ACC_EMPTY + acc], ((ul >> 1) & 1) ^ 1, args.ctl, abort_flag))
           break;
@@ -357,14 +422,22 @@ __global__ void __launch_bounds__(kConvThreads, 1)
           const uint64_t a0 = desc0 + static_cast<uint64_t>((st * L::STAGE) >> 4);
           const uint64_t b0 = desc0 + static_cast<uint64_t>((st * L::STAGE + CA_BYTES) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < CK / 16; ++kk)  // a 16-element K step is 32 bytes in the atom
-            umma_ss(d, a0 + kk * 2, b0 + kk * 2, IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(&bars[L::B_EMPTY + st]);
+          for (int kk = 0; kk < CK / 16; ++kk) {  // a 16-element K step is 32 bytes in the atom
+            if constexpr (PAIR)
+              umma_ss_pair(d, a0 + kk * 2, b0 + kk * 2, IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
+            else
+              umma_ss(d, a0 + kk * 2, b0 + kk * 2, IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          commit(L::B_EMPTY + st);
         }
         if (!ok) break;
-        umma_commit(&bars[L::B_ACC_FULL + acc]);
+        commit(L::B_ACC_FULL + acc);
       }
-      umma_commit(&bars[L::B_DRAIN]);
+      // every MMA this thread issued completes before TMEM is released
+      if constexpr (PAIR)
+        umma_commit_pair(&bars[L::B_DRAIN], 1);  // the leader's own barrier
+      else
+        umma_commit(&bars[L::B_DRAIN]);
       drain_wait(&bars[L::B_DRAIN], 0, args.ctl.wait_limit_ns);
     }
     __syncwarp();
@@ -375,10 +448,10 @@ __global__ void __launch_bounds__(kConvThreads, 1)
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
     const int Cout = args.Cout;
     uint32_t ul = 0;
-    for (int u = blockIdx.x; u < units; u += gridDim.x, ++ul) {
+    for (int u = unit0; u < units; u += n_units, ++ul) {
       int n, h0, w0, nt;
       conv_unit(args, nN, u, n, h0, w0, nt);
-      const int h = h0 + row / args.BW, w = w0 + row % args.BW;
+      const int h = h0 + rank * args.BH + row / args.BW, w = w0 + row % args.BW;
       const bool valid = h < args.H && w < args.W;
       const size_t pix = (static_cast<size_t>(n) * args.H + (valid ? h : 0)) * args.W +
                          (valid ? w : 0);
@@ -434,14 +507,27 @@ __global__ void __launch_bounds__(kConvThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[L::B_ACC_EMPTY + acc]);
+      if (lane == 0) {
+        if constexpr (PAIR)
+          mbar_arrive_cluster(cluster_addr(&bars[L::B_ACC_EMPTY + acc], 0));
+        else
+          mbar_arrive(&bars[L::B_ACC_EMPTY + acc]);
+      }
     }
   }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 2 * GN);
+  if constexpr (PAIR) {
+    // The leader has drained its MMAs (which write rank 1's TMEM) and the
+    // copies that complete on its barriers; neither CTA frees TMEM or leaves
+    // before both are here.
+    cluster_sync();
+    if (warp == 1) tmem_dealloc_pair(tmem, 2 * GN);
+  } else {
+    if (warp == 1) tmem_dealloc(tmem, 2 * GN);
+  }
 }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -496,19 +582,69 @@ bool make_weight_map(CUtensorMap* map, const void* Wt, int Cout, int Cin, int ro
          CUDA_SUCCESS;
 }
 
-template <int GN>
-cudaError_t launch_conv_t(const CUtensorMap& mx, const CUtensorMap& mw, const ConvArgs& a,
-                          int grid, cudaStream_t st) {
+template <int GN, bool PAIR>
+bool conv_ready(int dev) {
   static bool attr_set[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    const cudaError_t e = cudaFuncSetAttribute(
-        conv3x3_kernel<GN>, cudaFuncAttributeMaxDynamicSharedMemorySize, ConvLayout<GN>::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return false;
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(conv3x3_kernel<GN, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             ConvLayout<GN, PAIR>::SMEM_BYTES) != cudaSuccess)
+      return false;
     attr_set[dev] = true;
   }
-  conv3x3_kernel<GN><<<grid, kConvThreads, ConvLayout<GN>::SMEM_BYTES, st>>>(mx, mw, a);
+  return true;
+}
+
+template <int GN>
+cudaLaunchConfig_t conv_pair_config(int clusters, cudaLaunchAttribute* attr, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters);
+  cfg.blockDim = dim3(kConvThreads);
+  cfg.dynamicSmemBytes = ConvLayout<GN, true>::SMEM_BYTES;
+  cfg.stream = st;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cfg;
+}
+
+// Clusters of two that can be resident at once (0 if the pair form cannot run).
+template <int GN>
+int conv_max_clusters(int dev) {
+  static int cached[64] = {0};
+  if (dev < 0 || dev >= 64) return 0;
+  if (cached[dev] == 0) {
+    if (!conv_ready<GN, true>(dev)) return 0;
+    cudaLaunchAttribute attr[1];
+    cudaLaunchConfig_t cfg = conv_pair_config<GN>(1, attr, nullptr);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, conv3x3_kernel<GN, true>, &cfg) != cudaSuccess || n <= 0)
+      return 0;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+template <int GN>
+cudaError_t launch_conv_t(const CUtensorMap& mx, const CUtensorMap& mw, const ConvArgs& a,
+                          long long units, bool pair, cudaStream_t st) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (pair) {
+    const int mc = conv_max_clusters<GN>(dev);
+    if (mc <= 0) return cudaErrorInvalidConfiguration;
+    const int clusters = units < mc ? static_cast<int>(units) : mc;
+    cudaLaunchAttribute attr[1];
+    cudaLaunchConfig_t cfg = conv_pair_config<GN>(clusters, attr, st);
+    return cudaLaunchKernelEx(&cfg, conv3x3_kernel<GN, true>, mx, mw, a);
+  }
+  if (!conv_ready<GN, false>(dev)) return cudaErrorInvalidConfiguration;
+  const int grid = units < sm_count() ? static_cast<int>(units) : sm_count();
+  conv3x3_kernel<GN, false>
+      <<<grid, kConvThreads, ConvLayout<GN, false>::SMEM_BYTES, st>>>(mx, mw, a);
   return cudaGetLastError();
 }
 
@@ -573,7 +709,8 @@ void conv_pixel_tile(int32_t H, int32_t W, int32_t* BH, int32_t* BW) {
 
 cudaError_t launch_conv3x3(const mf_bf16* x, const mf_bf16* Wt, const float* bias,
                            const mf_bf16* residual, int32_t N, int32_t H, int32_t W, int32_t Cin,
-                           int32_t Cout, mf_bf16* y, const KernelCtl& ctl, cudaStream_t st) {
+                           int32_t Cout, mf_bf16* y, bool pair, const KernelCtl& ctl,
+                           cudaStream_t st) {
   static thread_local ConvArgs a;
   a.N = N;
   a.H = H;
@@ -581,7 +718,8 @@ cudaError_t launch_conv3x3(const mf_bf16* x, const mf_bf16* Wt, const float* bia
   a.Cin = Cin;
   a.Cout = Cout;
   conv_pixel_tile(H, W, &a.BH, &a.BW);
-  a.tiles_h = (H + a.BH - 1) / a.BH;
+  a.UH = pair ? 2 * a.BH : a.BH;
+  a.tiles_h = (H + a.UH - 1) / a.UH;
   a.tiles_w = (W + a.BW - 1) / a.BW;
   a.bias = bias;
   a.residual = residual;
@@ -589,13 +727,13 @@ cudaError_t launch_conv3x3(const mf_bf16* x, const mf_bf16* Wt, const float* bia
   a.ctl = ctl;
   const int gn = (Cout % 256 == 0) ? 256 : (Cout % 128 == 0 ? 128 : 64);
   CUtensorMap mx, mw;
-  if (!make_input_map(&mx, x, N, H, W, Cin, a.BH, a.BW) || !make_weight_map(&mw, Wt, Cout, Cin, gn))
+  if (!make_input_map(&mx, x, N, H, W, Cin, a.BH, a.BW) ||
+      !make_weight_map(&mw, Wt, Cout, Cin, pair ? gn / 2 : gn))
     return cudaErrorInvalidValue;
   const long long units = static_cast<long long>(N) * a.tiles_h * a.tiles_w * (Cout / gn);
-  const int grid = units < sm_count() ? static_cast<int>(units) : sm_count();
-  if (gn == 256) return launch_conv_t<256>(mx, mw, a, grid, st);
-  if (gn == 128) return launch_conv_t<128>(mx, mw, a, grid, st);
-  return launch_conv_t<64>(mx, mw, a, grid, st);
+  if (gn == 256) return launch_conv_t<256>(mx, mw, a, units, pair, st);
+  if (gn == 128) return launch_conv_t<128>(mx, mw, a, units, pair, st);
+  return launch_conv_t<64>(mx, mw, a, units, pair, st);
 }
 
 }  // namespace mf

@@ -24,9 +24,12 @@ cudaError_t launch_group_norm_silu(const mf_bf16* x, const float* gamma, const f
 // The 128-pixel block (BH x BW) the conv tiles an H x W image with.
 void conv_pixel_tile(int32_t H, int32_t W, int32_t* BH, int32_t* BW);
 
-// y = conv3x3(x; Wt) + bias + residual on NHWC bf16 (bias / residual may be NULL).
+// y = conv3x3(x; Wt) + bias + residual on NHWC bf16 (bias / residual may be NULL);
+// `pair`: on clusters of two CTAs (M = 256 MMAs over two vertically adjacent
+// pixel tiles).
 cudaError_t launch_conv3x3(const mf_bf16* x, const mf_bf16* Wt, const float* bias,
                            const mf_bf16* residual, int32_t N, int32_t H, int32_t W, int32_t Cin,
-                           int32_t Cout, mf_bf16* y, const KernelCtl& ctl, cudaStream_t st);
+                           int32_t Cout, mf_bf16* y, bool pair, const KernelCtl& ctl,
+                           cudaStream_t st);
 
 }  // namespace mf

@@ -27,6 +27,16 @@ import resolution_packed_diffusion_b200 as mf  # noqa: E402
 from gpu_util import assert_bf16_close, assert_block_close, dev_bf16, host_f32  # noqa: E402
 
 
+@pytest.fixture(params=[0, 1], ids=["one_cta", "cta_pair"])
+def conv_pair(request):
+    """Both conv kernels: one CTA per 128-pixel tile, and CTA pairs computing two
+    vertically adjacent tiles as M = 256 MMAs (the second tile may lie wholly
+    below the image)."""
+    mf.mf_set_conv_cta_pair(request.param)
+    yield request.param
+    mf.mf_set_conv_cta_pair(0)  # the library's default
+
+
 def _f32(a):
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()
 
@@ -58,6 +68,7 @@ def _conv_case(N, H, W, Cin, Cout, seed, bias=True, residual=True):
     (1, 1, 200, 64, 64, True, True),      # one image row: every tap above and below reads zeros
     (3, 40, 24, 256, 128, False, True),   # four channel blocks per tap
 ], ids=["ragged", "ragged_plain", "n256", "one_row", "cin256"])
+@pytest.mark.usefixtures("conv_pair")
 def test_conv3x3(N, H, W, Cin, Cout, bias, residual):
     got, ref = _conv_case(N, H, W, Cin, Cout, 5000 + H * W + Cin, bias, residual)
     assert_bf16_close(got, ref, "conv3x3")
@@ -105,12 +116,18 @@ def _block(v):
     # two groups of 64 channels
     (None, dict(N=2, H=11, W=5, C=128, G=2)),
 ], ids=["tiny", "stage_1_8", "one_group_512ch", "two_groups"])
+@pytest.mark.usefixtures("conv_pair")
 def test_vae_res_block(name, shape):
     v = make_vae_block(name, **(shape or {}))
     got = _block(v)
     ref = oracle.vae_res_block(v.f32("x"), v.gamma1, v.beta1, v.f32("W1"), v.c1, v.gamma2,
                                v.beta2, v.f32("W2"), v.c2, v.G, v.eps)
     assert_block_close(got, ref, f"VAE block ({name})")
+
+
+def test_conv_pair_setting_is_checked():
+    with pytest.raises(mf.MFError):
+        mf.mf_set_conv_cta_pair(2)
 
 
 def test_vae_entry_points_reject_bad_arguments():
