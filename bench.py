@@ -556,7 +556,12 @@ def run_linear(args, rank, world, local_rank):
 def run_mmdit(args, rank, world, local_rank):
     """`--op mmdit`: one whole NR-MMDiT block (adaLN, per-modality projections,
     RoPE + packed attention, gated residuals, GELU MLP of width 4 hid) over the
-    workload's pack, random-init weights."""
+    workload's pack, random-init weights. `--op mmdit_bwd`: the block's backward
+    (mf_mmdit_block_bwd: the forward recomputed, then every input, weight and
+    modulation gradient) for a random loss gradient; its FLOPs count the
+    recomputed forward and the backward (the linear layers' input and weight
+    products, the attention backward's five products)."""
+    bwd = args.op == "mmdit_bwd"
     import torch
     import resolution_packed_diffusion_b200 as mf
 
@@ -584,7 +589,14 @@ def run_mmdit(args, rank, world, local_rank):
     ts = torch.empty(T, dtype=torch.int32, device=dev)
     tm = torch.empty(T, dtype=torch.uint8, device=dev)
     y = torch.empty_like(x)
-    ws_bytes = mf.mf_mmdit_workspace_size(T, H, D, F)
+    if bwd:
+        dy = torch.randn(x.shape, device=dev, generator=g).to(torch.bfloat16)
+        grads = {n: torch.empty_like(W) for n, W in
+                 (("q", Wq), ("k", Wk), ("v", Wv), ("o", Wo), ("up", Wup), ("down", Wdown))}
+        dmod_attn, dmod_mlp = torch.empty_like(mod_attn), torch.empty_like(mod_mlp)
+        ws_bytes = mf.mf_mmdit_bwd_workspace_size(T, S, H, D, F)
+    else:
+        ws_bytes = mf.mf_mmdit_workspace_size(T, H, D, F)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -592,9 +604,15 @@ def run_mmdit(args, rank, world, local_rank):
         cu_h, _ = mf.mf_pack_build(w.descs, w.rope_axes, w.budget, cu_d, pos, ts, tm, stream)
         mf.mf_adaln_params(c, Wm1, S, c.shape[1], hid, mod_attn, stream)
         mf.mf_adaln_params(c, Wm2, S, c.shape[1], hid, mod_mlp, stream)
-        mf.mf_mmdit_block_fwd(x, Wq, Wk, Wv, Wo, Wup, Wdown, mod_attn, mod_mlp, w.descs, cu_d,
-                              cu_h, pos, ts, tm, S, H, D, F, w.rope_axes, w.base, w.eps, y, ws,
-                              ws_bytes, stream)
+        if bwd:
+            mf.mf_mmdit_block_bwd(dy, x, Wq, Wk, Wv, Wo, Wup, Wdown, mod_attn, mod_mlp, w.descs,
+                                  cu_d, cu_h, pos, ts, tm, S, H, D, F, w.rope_axes, w.base, w.eps,
+                                  y, grads["q"], grads["k"], grads["v"], grads["o"], grads["up"],
+                                  grads["down"], dmod_attn, dmod_mlp, ws, ws_bytes, stream)
+        else:
+            mf.mf_mmdit_block_fwd(x, Wq, Wk, Wv, Wo, Wup, Wdown, mod_attn, mod_mlp, w.descs, cu_d,
+                                  cu_h, pos, ts, tm, S, H, D, F, w.rope_axes, w.base, w.eps, y,
+                                  ws, ws_bytes, stream)
 
     def barrier():
         if world > 1:
@@ -619,6 +637,8 @@ def run_mmdit(args, rank, world, local_rank):
         raise RuntimeError("device error in the MMDiT block")
     gemm_flops = 2.0 * T * hid * hid * 4 + 2.0 * T * hid * F * 2
     flops = gemm_flops + useful_flops(w)
+    if bwd:  # recomputed forward + input and weight products + the attention's five products
+        flops = 3.0 * gemm_flops + 3.5 * useful_flops(w)
     ms_step, flops_all = reduce_timing(t0.elapsed_time(t1) / args.steps, flops, world)
     tokens_all = reduce_timing(0.0, float(real_tokens(w)), world)[1]
     if rank != 0:
@@ -626,8 +646,19 @@ def run_mmdit(args, rank, world, local_rank):
     peaks, peak_src = load_peaks()
     achieved = flops / (ms_step * 1e-3) / 1e12
     peak = float(peaks["bf16_tflops"])
+    # kernels per step: pack ids and two modulation maps, then the block: 13 for
+    # the forward (the attention's RoPE table and k pass included); for the
+    # backward 12 (recomputed forward) + 12 (weight transposes) + 8 (MLP branch)
+    # + 12 (attention branch) + 16 per modality with tokens (four input
+    # transposes, six gradient transposes, six products), 6 zero fills otherwise
+    mods_present = sum(1 for m in (0, 1) if any(
+        (d.frames * d.grid_h * d.grid_w if m == 0 else d.n_text) > 0 for d in w.descs))
+    launches = 3 + (44 + 16 * mods_present + 6 * (2 - mods_present) if bwd else 13)
     print(json.dumps({
-        "metric": "NR-MMDiT block forward TFLOP/s (GEMMs + useful attention)", "op": "mmdit",
+        "metric": ("NR-MMDiT block backward TFLOP/s (recomputed forward + backward, GEMMs + "
+                   "useful attention)" if bwd else
+                   "NR-MMDiT block forward TFLOP/s (GEMMs + useful attention)"),
+        "op": args.op,
         "value": flops_all / (ms_step * 1e-3) / 1e12, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
@@ -638,7 +669,7 @@ def run_mmdit(args, rank, world, local_rank):
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
                      "frac": achieved / peak, "traffic": None,
                      "peak_source": f"{peak_src} bf16_tflops (burst)"},
-        "gpu_launches": 15 * args.steps, "clocks": clk}), flush=True)
+        "gpu_launches": launches * args.steps, "clocks": clk}), flush=True)
 
 
 def run_attn_bwd(args, rank, world, local_rank):
@@ -907,7 +938,7 @@ def run_vae(args, rank, world, local_rank):
         "gpu_launches": 8 * args.steps, "clocks": clk}), flush=True)
 
 
-ARMS = {"block": "run_gpu", "linear": "run_linear", "mmdit": "run_mmdit",
+ARMS = {"block": "run_gpu", "linear": "run_linear", "mmdit": "run_mmdit", "mmdit_bwd": "run_mmdit",
         "attn_bwd": "run_attn_bwd", "block_bwd": "run_block_bwd", "vae_block": "run_vae"}
 
 
@@ -983,6 +1014,7 @@ def main():
                     help="block: the packed joint-attention block (the default line); "
                          "linear: the modality-specific linear layer as a QKV projection; "
                          "mmdit: one whole NR-MMDiT block around the path; "
+                         "mmdit_bwd: that block's backward; "
                          "attn_bwd: the backward of the packed attention; "
                          "block_bwd: the backward of the whole path block; "
                          "vae_block: one Mage-VAE conv block")

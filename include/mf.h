@@ -331,6 +331,38 @@ mf_status mf_mmdit_block_fwd(const mf_bf16* x, const mf_bf16* Wq, const mf_bf16*
                              cudaStream_t stream);
 size_t mf_mmdit_workspace_size(int32_t T, int32_t H, int32_t D, int32_t F);
 
+/* Backward of mf_mmdit_block_fwd [norm], [fuse], [train] for the loss gradient dy
+ * of y ([T][hid] bf16), with every other argument as in the forward. The
+ * forward's intermediates are recomputed into the workspace (bf16, as the
+ * forward stores them; z = x2 Wup^T is kept before the GELU), then the chain
+ * rule runs through the MLP branch (gate, down projection, GELU, up projection,
+ * adaLN) and the attention branch (gate, output projection, attention, RoPE,
+ * the three input projections, adaLN), the residual path carrying dy through
+ * both. A linear layer's input gradient d_in = d_out W[m] is the tcgen05 linear
+ * kernel on the transposed weights; its weight gradient dW[m] = sum over
+ * modality-m tokens of d_out^T in is the same kernel on transposes that gather
+ * the modality's tokens (a modality without tokens gets dW[m] = 0).
+ * Outputs: dx [T][hid] bf16; dWq, dWk, dWv, dWo [2][hid][hid], dWup [2][F][hid],
+ * dWdown [2][hid][F] bf16 (image weights first); dmod_attn, dmod_mlp
+ * [S][2][3][hid] fp32 (every slot written: shift and scale from the adaLN
+ * backward, gate from the gated residual's). Every output is disjoint from every
+ * input, from the other outputs and from the workspace (ws_bytes >=
+ * mf_mmdit_bwd_workspace_size(T, S, H, D, F)). desc must match the offsets.
+ * bf16 operands and intermediates, fp32 accumulation in every product and sum;
+ * the dmod sums use fp32 atomics (their last bits can vary between runs). */
+mf_status mf_mmdit_block_bwd(const mf_bf16* dy, const mf_bf16* x, const mf_bf16* Wq,
+                             const mf_bf16* Wk, const mf_bf16* Wv, const mf_bf16* Wo,
+                             const mf_bf16* Wup, const mf_bf16* Wdown, const float* mod_attn,
+                             const float* mod_mlp, const mf_sample_desc* desc,
+                             const int32_t* cu_seqlens_d, const int32_t* cu_seqlens_h,
+                             const int32_t* pos_ids, const int32_t* tok_sample,
+                             const uint8_t* tok_mod, int32_t S, int32_t H, int32_t D, int32_t F,
+                             int32_t rope_axes, float base, float eps, mf_bf16* dx, mf_bf16* dWq,
+                             mf_bf16* dWk, mf_bf16* dWv, mf_bf16* dWo, mf_bf16* dWup,
+                             mf_bf16* dWdown, float* dmod_attn, float* dmod_mlp,
+                             void* workspace, size_t ws_bytes, cudaStream_t stream);
+size_t mf_mmdit_bwd_workspace_size(int32_t T, int32_t S, int32_t H, int32_t D, int32_t F);
+
 /* Mage-VAE conv block [vae], [vfuse]: the fully convolutional VAE's repeated
  * blocks and their fused normalization - activation - residual chains. The
  * pages give neither the wiring nor the widths; the library takes the diffusion

@@ -91,6 +91,10 @@ _SIGS = {
     "mf_mmdit_block_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I,
                                 _I, _I, _I, _I, _F, _F, _P, _P, _SZ, _P]),
     "mf_mmdit_workspace_size": (_SZ, [_I, _I, _I, _I]),
+    "mf_mmdit_block_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                _I, _I, _I, _I, _I, _F, _F, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                _P, _SZ, _P]),
+    "mf_mmdit_bwd_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "mf_group_norm_silu": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _P, _SZ, _P]),
     "mf_gn_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "mf_conv3x3": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
@@ -361,6 +365,27 @@ def mf_mmdit_block_fwd(x, Wq, Wk, Wv, Wo, Wup, Wdown, mod_attn, mod_mlp, descs, 
                                   _ptr(pos_ids), _ptr(tok_sample), _ptr(tok_mod), S, H, D, F,
                                   rope_axes, base, eps, _ptr(y), _ptr(workspace), ws_bytes,
                                   _stream(stream)), "mf_mmdit_block_fwd")
+
+
+def mf_mmdit_bwd_workspace_size(T: int, S: int, H: int, D: int, F: int) -> int:
+    return int(lib.mf_mmdit_bwd_workspace_size(T, S, H, D, F))
+
+
+def mf_mmdit_block_bwd(dy, x, Wq, Wk, Wv, Wo, Wup, Wdown, mod_attn, mod_mlp, descs, cu_seqlens_d,
+                       cu_seqlens_h: np.ndarray, pos_ids, tok_sample, tok_mod, S: int, H: int,
+                       D: int, F: int, rope_axes: int, base: float, eps: float, dx, dWq, dWk,
+                       dWv, dWo, dWup, dWdown, dmod_attn, dmod_mlp, workspace, ws_bytes: int,
+                       stream=None) -> None:
+    arr = make_descs(descs)
+    cu_h = np.ascontiguousarray(cu_seqlens_h, dtype=np.int32)
+    _check(lib.mf_mmdit_block_bwd(_ptr(dy), _ptr(x), _ptr(Wq), _ptr(Wk), _ptr(Wv), _ptr(Wo),
+                                  _ptr(Wup), _ptr(Wdown), _ptr(mod_attn), _ptr(mod_mlp),
+                                  ctypes.cast(arr, _P), _ptr(cu_seqlens_d), cu_h.ctypes.data_as(_P),
+                                  _ptr(pos_ids), _ptr(tok_sample), _ptr(tok_mod), S, H, D, F,
+                                  rope_axes, base, eps, _ptr(dx), _ptr(dWq), _ptr(dWk), _ptr(dWv),
+                                  _ptr(dWo), _ptr(dWup), _ptr(dWdown), _ptr(dmod_attn),
+                                  _ptr(dmod_mlp), _ptr(workspace), ws_bytes, _stream(stream)),
+           "mf_mmdit_block_bwd")
 
 
 def mf_gn_workspace_size(N: int, H: int, W: int, G: int) -> int:

@@ -24,7 +24,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmf.so")
 
 SOURCES = ["mf_api.cu", "elementwise.cu", "attn_fwd.cu", "noalloc.cu", "gemm.cu", "mmdit.cu",
-           "attn_bwd.cu", "block_bwd.cu", "vae.cu"]
+           "attn_bwd.cu", "block_bwd.cu", "vae.cu", "mmdit_bwd.cu"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",

@@ -314,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!warp_wait(&bars[L::B_ACC_FULL + acc], (ul >> 1) & 1, args.ctl, abort_flag)) break;
       tc_fence_after();
       const int t = blk * L::ROWS + rank * GM + row;
-      const bool keep = t < args.T && __ldg(args.tok_mod + t) == m;
+      const bool keep = t < args.T && (args.tok_mod == nullptr || __ldg(args.tok_mod + t) == m);
       uint4* orow = reinterpret_cast<uint4*>(args.out + static_cast<size_t>(t) * args.N + nt * GN);
 #pragma unroll 1
       for (int cc = 0; cc < GN; cc += 32) {
@@ -486,14 +486,18 @@ bool build_gemm_jobs(const int32_t* mods_per_sample_img, const int32_t* mods_per
   return true;
 }
 
-cudaError_t launch_modality_linear(const mf_bf16* x, const mf_bf16* W, const uint8_t* tok_mod,
-                                   const GemmJobs& jobs, bool pair, int32_t T, int32_t K,
-                                   int32_t N, int32_t act, mf_bf16* out, const KernelCtl& ctl,
-                                   cudaStream_t st) {
+namespace {
+
+// w_sets: weight matrices stacked in W (2 for the per-modality form, 1 when
+// tok_mod is NULL and every row uses W[0]).
+cudaError_t launch_linear_impl(const mf_bf16* x, const mf_bf16* W, int w_sets,
+                               const uint8_t* tok_mod, const GemmJobs& jobs, bool pair, int32_t T,
+                               int32_t K, int32_t N, int32_t act, mf_bf16* out,
+                               const KernelCtl& ctl, cudaStream_t st) {
   if (jobs.n == 0) return cudaSuccess;
   CUtensorMap mx, mw;
   const int b_rows = pair ? GemmLayout<true>::B_ROWS : GemmLayout<false>::B_ROWS;
-  if (!make_map(&mx, x, T, K, GM) || !make_map(&mw, W, 2LL * N, K, b_rows))
+  if (!make_map(&mx, x, T, K, GM) || !make_map(&mw, W, static_cast<int64_t>(w_sets) * N, K, b_rows))
     return cudaErrorInvalidValue;
   static thread_local GemmArgs a;
   a.jobs = jobs;
@@ -524,6 +528,27 @@ cudaError_t launch_modality_linear(const mf_bf16* x, const mf_bf16* W, const uin
   const int grid = units < sms() ? units : sms();
   modality_linear_kernel<false><<<grid, kThreads, GemmLayout<false>::SMEM_BYTES, st>>>(mx, mw, a);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_modality_linear(const mf_bf16* x, const mf_bf16* W, const uint8_t* tok_mod,
+                                   const GemmJobs& jobs, bool pair, int32_t T, int32_t K,
+                                   int32_t N, int32_t act, mf_bf16* out, const KernelCtl& ctl,
+                                   cudaStream_t st) {
+  return launch_linear_impl(x, W, 2, tok_mod, jobs, pair, T, K, N, act, out, ctl, st);
+}
+
+cudaError_t launch_linear_plain(const mf_bf16* x, const mf_bf16* W, int32_t T, int32_t K,
+                                int32_t N, bool pair, mf_bf16* out, const KernelCtl& ctl,
+                                cudaStream_t st) {
+  static thread_local GemmJobs jobs;
+  const int rows = gemm_job_rows(pair);
+  const int blocks = (T + rows - 1) / rows;
+  if (blocks > kMaxGemmTiles) return cudaErrorInvalidValue;
+  for (int b = 0; b < blocks; ++b) jobs.job[b] = static_cast<uint16_t>(b);
+  jobs.n = blocks;
+  return launch_linear_impl(x, W, 1, nullptr, jobs, pair, T, K, N, 0, out, ctl, st);
 }
 
 }  // namespace mf

@@ -37,4 +37,11 @@ cudaError_t launch_modality_linear(const mf_bf16* x, const mf_bf16* W, const uin
                                    int32_t N, int32_t act, mf_bf16* out, const KernelCtl& ctl,
                                    cudaStream_t st);
 
+// out[t] = x[t] W^T for every row t < T with one weight matrix W [N][K] (no
+// modality split, no activation): the weight-gradient and transposed products
+// of the backward.
+cudaError_t launch_linear_plain(const mf_bf16* x, const mf_bf16* W, int32_t T, int32_t K,
+                                int32_t N, bool pair, mf_bf16* out, const KernelCtl& ctl,
+                                cudaStream_t st);
+
 }  // namespace mf

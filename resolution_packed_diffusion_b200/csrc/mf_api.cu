@@ -145,6 +145,14 @@ bool check_offsets(const int32_t* cu_h, int32_t S, int32_t* T) {
   return true;
 }
 
+bool linear_cta_pair(bool* pair) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  *pair = g_state[dev].linear_pair;
+  return true;
+}
+
 cudaError_t get_ctl(KernelCtl* ctl) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -624,9 +632,8 @@ mf_status mf_modality_linear(const mf_bf16* x, const mf_bf16* W, const uint8_t* 
   if (overlap(out, ob, x, xb) || overlap(out, ob, W, wb)) return MF_ERR_INVALID;
   KernelCtl ctl;
   if (cudaError_t ge = get_ctl(&ctl); ge != cudaSuccess) return cuda_status(ge);
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MF_ERR_CUDA;
-  const bool pair = g_state[dev].linear_pair;
+  bool pair = false;
+  if (!linear_cta_pair(&pair)) return MF_ERR_CUDA;
   static thread_local GemmJobs jobs;
   if (!build_gemm_jobs(n_img, n_txt, S, static_cast<int32_t>(T), gemm_job_rows(pair), &jobs))
     return MF_ERR_UNSUPPORTED;

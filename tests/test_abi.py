@@ -318,3 +318,37 @@ def test_vae_argument_checks_without_gpu():
     assert lib.mf_vae_res_block(x, b, b, Wt, b, b, b, Wt, b, 1, 8, 8, 64, 8, 1e-6, y, x,
                                 mf.mf_vae_block_workspace_size(1, 8, 8, 64, 8), None) == \
         mf.MF_ERR_INVALID                                      # workspace over x
+
+
+def test_mmdit_block_bwd_argument_checks_without_gpu():
+    """The block backward checks shapes, the descriptors against the offsets,
+    alignment, workspace size and overlaps before touching the GPU."""
+    lib = mf.lib
+    P = ctypes.c_void_p
+    MB = 1 << 20
+    descs = [SampleDesc(1, 4, 4, 3), SampleDesc(0, 0, 0, 5)]
+    arr = mf.make_descs(descs)
+    cu = np.array([0, 19, 24], dtype=np.int32)
+    S, H, D, F = 2, 2, 128, 512
+    T = 24
+    ws_size = mf.mf_mmdit_bwd_workspace_size(T, S, H, D, F)
+    assert ws_size > 0 and mf.mf_mmdit_bwd_workspace_size(T, 0, H, D, F) == 0
+    ptr = [P((i + 1) * 64 * MB) for i in range(22)]
+    (dy, x, Wq, Wk, Wv, Wo, Wup, Wdown, ma, mm, dx, dWq, dWk, dWv, dWo, dWup, dWdown, dma, dmm,
+     ws, pos, ids) = ptr
+
+    def call(H=H, D=D, F=F, cu=cu, dx=dx, dWq=dWq, ws=ws, ws_bytes=ws_size):
+        return lib.mf_mmdit_block_bwd(dy, x, Wq, Wk, Wv, Wo, Wup, Wdown, ma, mm,
+                                      ctypes.cast(arr, P), P(16), cu.ctypes.data_as(P), pos, ids,
+                                      ids, S, H, D, F, 2, 10000.0, 1e-6, dx, dWq, dWk, dWv, dWo,
+                                      dWup, dWdown, dma, dmm, ws, ws_bytes, None)
+
+    assert call(F=500) == mf.MF_ERR_INVALID                         # F not a multiple of 256
+    assert call(D=64) == mf.MF_ERR_UNSUPPORTED                      # hid 128
+    assert call(cu=np.array([0, 18, 24], dtype=np.int32)) == mf.MF_ERR_INVALID  # desc vs offsets
+    assert call(cu=np.array([0, 19, 18], dtype=np.int32)) == mf.MF_ERR_INVALID  # decreasing
+    assert call(dx=x) == mf.MF_ERR_INVALID                          # output over an input
+    assert call(dWq=P(dWk.value + 64)) == mf.MF_ERR_INVALID         # two outputs overlap
+    assert call(dWq=P(dWq.value + 8)) == mf.MF_ERR_INVALID          # misaligned
+    assert call(ws_bytes=ws_size - 1) == mf.MF_ERR_INVALID
+    assert call(ws=P(dx.value + 256)) == mf.MF_ERR_INVALID          # workspace over dx
