@@ -148,3 +148,12 @@ def test_mmdit_block_bwd_medium_pack():
     w = make_random_pack(984, S=3, H=2, D=128, rope_axes=2, descs=descs)
     got, ref, pack = _run(w, 1024, 985)
     _check_all(got, ref, pack, "medium")
+
+
+def test_mmdit_block_bwd_wide_layers():
+    """hid 1024 (8 heads x 128) and MLP width 4096: every linear product runs
+    over several 256-column tiles and K steps; ~660 tokens, 3D RoPE."""
+    descs = [SampleDesc(2, 12, 16, 40), SampleDesc(1, 14, 18, 6)]
+    w = make_random_pack(986, S=2, H=8, D=128, rope_axes=3, descs=descs)
+    got, ref, pack = _run(w, 4096, 987)
+    _check_all(got, ref, pack, "wide")
