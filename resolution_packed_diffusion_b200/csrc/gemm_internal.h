@@ -25,6 +25,10 @@ struct GemmJobs {
 // Rows of a job: 128, or 256 with CTA pairs.
 int gemm_job_rows(bool pair);
 
+// The linear-layer kernel form chosen for the current device
+// (mf_set_linear_cta_pair, mf_api.cu); false if the device cannot be read.
+bool linear_cta_pair(bool* pair);
+
 // Fills the job list from each sample's image and text token counts (image
 // tokens first in a sample) for row blocks of `rows` (gemm_job_rows); false if
 // the pack has too many blocks or `rows` is not a job size.

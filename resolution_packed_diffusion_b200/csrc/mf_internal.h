@@ -21,10 +21,6 @@ struct KernelCtl {
 // Per-device error word and wait limit (mf_api.cu).
 cudaError_t get_ctl(KernelCtl* ctl);
 
-// The linear-layer kernel form chosen for the current device
-// (mf_set_linear_cta_pair); false if the device cannot be read.
-bool linear_cta_pair(bool* pair);
-
 // Host offsets of a pack: true when 0 = cu_h[0] <= cu_h[1] <= ... <= cu_h[S]
 // <= MF_MAX_TOKENS; then *T = cu_h[S].
 bool check_offsets(const int32_t* cu_h, int32_t S, int32_t* T);
