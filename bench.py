@@ -43,7 +43,8 @@ DEFAULT_CONFIG = 5  # the largest single-GPU pack: 2048^2 image plus three 4:1 i
 METRIC = "packed varlen attention useful TFLOP/s (% bf16 peak); block tokens/s at 1 B200"
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-REF_ROW_STRIDE = 32  # reference arm: rows sampled per step (keeps a step near 0.3 s)
+REF_ROW_STRIDE = 32  # reference arm: rows sampled per step at most (a step near 0.7 s)
+REF_BUDGET_S = 300.0  # reference arm: the whole run's oracle time, about
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_fwd_traffic.txt")
 # the attention kernel's sources: the traffic summary applies while they are unchanged
 ATTN_SRC = [os.path.join(ROOT, "resolution_packed_diffusion_b200", "csrc", f)
@@ -232,12 +233,19 @@ def run_reference(args, rank):
     if rank != 0:
         return
     w = make_workload(args.config)
-    # warm-up and timed steps, each a one-head sample of the workload
-    for _ in range(args.warmup):
-        oracle_sample_step(w, [0], REF_ROW_STRIDE)
+    # warm-up and timed steps, each a one-head sample of the workload; the
+    # warm-up steps also size the sample (every stride-th row, the stride
+    # doubled while the remaining steps would overrun the time budget)
+    stride = REF_ROW_STRIDE
+    for i in range(args.warmup):
+        dt, _ = oracle_sample_step(w, [0], stride)
+        left = args.warmup - 1 - i + args.steps
+        while dt * left > REF_BUDGET_S and stride < w.T:  # the next step re-measures
+            stride *= 2
+            dt *= 0.5
     times, flops = [], 0.0
     for _ in range(args.steps):
-        dt, fl = oracle_sample_step(w, [0], REF_ROW_STRIDE)
+        dt, fl = oracle_sample_step(w, [0], stride)
         times.append(dt)
         flops += fl
     total = sum(times)
@@ -251,7 +259,7 @@ def run_reference(args, rank):
         "config": workload_config(w, args),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                          "sample": (f"each step: {w.name}, pack metadata, modulation vectors, "
-                                    f"then for every {REF_ROW_STRIDE}th token row adaLN and, "
+                                    f"then for every {stride}th token row adaLN and, "
                                     f"for head 0 of {w.H}, RoPE + attention over the row's "
                                     f"sample + gated residual; fp64 NumPy ({api})")},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
