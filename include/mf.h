@@ -348,6 +348,7 @@ size_t mf_mmdit_workspace_size(int32_t T, int32_t H, int32_t D, int32_t F);
  * backward, gate from the gated residual's). Every output is disjoint from every
  * input, from the other outputs and from the workspace (ws_bytes >=
  * mf_mmdit_bwd_workspace_size(T, S, H, D, F)). desc must match the offsets.
+ * T and F up to 131072 (else MF_ERR_UNSUPPORTED).
  * bf16 operands and intermediates, fp32 accumulation in every product and sum;
  * the dmod sums use fp32 atomics (their last bits can vary between runs). */
 mf_status mf_mmdit_block_bwd(const mf_bf16* dy, const mf_bf16* x, const mf_bf16* Wq,

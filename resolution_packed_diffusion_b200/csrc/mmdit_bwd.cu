@@ -281,6 +281,11 @@ mf_status mf_mmdit_block_bwd(const mf_bf16* dy, const mf_bf16* x, const mf_bf16*
   if (hid % 256 != 0) return MF_ERR_UNSUPPORTED;
   int32_t T = 0;
   if (!check_offsets(cu_seqlens_h, S, &T)) return MF_ERR_INVALID;
+  // the weight-gradient products run over F (or hid) rows as one job table, and
+  // the forward's over T rows: both within the linear layer's job limit
+  if (static_cast<int64_t>(F) > static_cast<int64_t>(kMaxGemmTiles) * 128 ||
+      static_cast<int64_t>(T) > static_cast<int64_t>(kMaxGemmTiles) * 128)
+    return MF_ERR_UNSUPPORTED;
   for (int32_t s = 0; s < S; ++s) {
     const mf_sample_desc& d = desc[s];
     if (d.frames < 0 || d.grid_h < 0 || d.grid_w < 0 || d.n_text < 0 ||

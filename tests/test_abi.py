@@ -344,6 +344,7 @@ def test_mmdit_block_bwd_argument_checks_without_gpu():
                                       dWup, dWdown, dma, dmm, ws, ws_bytes, None)
 
     assert call(F=500) == mf.MF_ERR_INVALID                         # F not a multiple of 256
+    assert call(F=131072 + 256) == mf.MF_ERR_UNSUPPORTED            # beyond the job table
     assert call(D=64) == mf.MF_ERR_UNSUPPORTED                      # hid 128
     assert call(cu=np.array([0, 18, 24], dtype=np.int32)) == mf.MF_ERR_INVALID  # desc vs offsets
     assert call(cu=np.array([0, 19, 18], dtype=np.int32)) == mf.MF_ERR_INVALID  # decreasing
