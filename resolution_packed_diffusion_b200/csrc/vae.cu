@@ -21,7 +21,8 @@
 //                       fixed order and writes one partial per group.
 //   gn_finalize_kernel  one CTA per (sample, group): merges the chunks'
 //                       partials in a fixed tree -> (mean, rstd). Deterministic.
-//   gn_silu_kernel      y = SiLU((x - mean) rstd gamma + beta), 16-byte vectors.
+//   gn_silu_kernel      y = SiLU((x - mean) rstd gamma + beta), 16-byte vectors;
+//                       a thread keeps one 8-channel vector over a run of pixels.
 //   conv3x3_kernel<GN>  one persistent CTA per SM, 8 warps: output tiles of 128
 //                       pixels (a BH x BW block of one image) x GN output
 //                       channels (256, else 128, else 64: the widest that
@@ -165,33 +166,52 @@ __global__ void __launch_bounds__(kGnThreads) gn_finalize_kernel(const float4* _
 }
 
 // y = SiLU((x - mean) * rstd * gamma + beta), one 8-channel vector per step
+// grid: (pixel chunks, samples). A thread keeps one 8-channel vector v of the
+// pixels and walks pixels p0 + r, p0 + r + rows, ... of its chunk, so its
+// group's (mean, rstd) and its channels' gamma and beta are loaded once.
 __global__ void __launch_bounds__(256) gn_silu_kernel(const uint4* __restrict__ x,
                                                       const float* __restrict__ gamma,
                                                       const float* __restrict__ beta,
-                                                      const float2* __restrict__ stats,
-                                                      long long total, int HW, int C, int G,
+                                                      const float2* __restrict__ stats, int HW,
+                                                      int C, int G, int chunk_px,
                                                       uint4* __restrict__ y) {
-  const int VP = C >> 3;
-  const int cg = C / G;
-  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
-       i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const int v = static_cast<int>(i % VP);
-    const int n = static_cast<int>(i / (static_cast<long long>(HW) * VP));
-    const int c0 = 8 * v;
-    const float2 st = __ldg(stats + n * G + c0 / cg);  // a vector never straddles groups
+  const int VP = C >> 3;          // a power of two <= 256, so it divides the block
+  const int rows = blockDim.x / VP;
+  const int v = threadIdx.x % VP, r = threadIdx.x / VP;
+  const int n = blockIdx.y;
+  const int c0 = 8 * v;
+  const float2 st = __ldg(stats + n * G + c0 / (C / G));  // a vector never straddles groups
+  float gm[8], bt[8];
+  {
     const float4 g0 = __ldg(reinterpret_cast<const float4*>(gamma + c0));
     const float4 g1 = __ldg(reinterpret_cast<const float4*>(gamma + c0 + 4));
     const float4 b0 = __ldg(reinterpret_cast<const float4*>(beta + c0));
     const float4 b1 = __ldg(reinterpret_cast<const float4*>(beta + c0 + 4));
-    const float gm[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-    const float bt[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+    gm[0] = g0.x; gm[1] = g0.y; gm[2] = g0.z; gm[3] = g0.w;
+    gm[4] = g1.x; gm[5] = g1.y; gm[6] = g1.z; gm[7] = g1.w;
+    bt[0] = b0.x; bt[1] = b0.y; bt[2] = b0.z; bt[3] = b0.w;
+    bt[4] = b1.x; bt[5] = b1.y; bt[6] = b1.z; bt[7] = b1.w;
+  }
+  // the affine form of the normalisation: a = x * sc + sh
+  float sc[8], sh[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    sc[e] = st.y * gm[e];
+    sh[e] = fmaf(-st.x, sc[e], bt[e]);
+  }
+  const int p0 = blockIdx.x * chunk_px;
+  const int p1 = min(HW, p0 + chunk_px);
+  const size_t base = static_cast<size_t>(n) * HW * VP + v;
+#pragma unroll 4
+  for (int p = p0 + r; p < p1; p += rows) {
+    const size_t i = base + static_cast<size_t>(p) * VP;
     float f[8];
     unpack8(__ldcs(x + i), f);
     uint32_t o[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      float a0 = fmaf((f[2 * e] - st.x) * st.y, gm[2 * e], bt[2 * e]);
-      float a1 = fmaf((f[2 * e + 1] - st.x) * st.y, gm[2 * e + 1], bt[2 * e + 1]);
+      float a0 = fmaf(f[2 * e], sc[2 * e], sh[2 * e]);
+      float a1 = fmaf(f[2 * e + 1], sc[2 * e + 1], sh[2 * e + 1]);
       a0 = __fdividef(a0, 1.f + __expf(-a0));
       a1 = __fdividef(a1, 1.f + __expf(-a1));
       o[e] = pack_bf16x2(a0, a1);
@@ -682,12 +702,15 @@ cudaError_t launch_group_norm_silu(const mf_bf16* x, const float* gamma, const f
   gn_finalize_kernel<<<N * G, kGnThreads, 0, st>>>(partial, G, chunks, eps, stats);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const long long total = static_cast<long long>(N) * HW * (C / 8);
-  long long blocks = (total + 255) / 256;
-  const long long cap = 8LL * sm_count();
-  if (blocks > cap) blocks = cap;
-  gn_silu_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-      reinterpret_cast<const uint4*>(x), gamma, beta, stats, total, HW, C, G,
+  // about eight 256-thread CTAs per SM over the whole tensor, each a run of pixels
+  const int rows = 256 / (C / 8);
+  long long nchunk = (8LL * sm_count() + N - 1) / N;
+  const long long max_chunk = (HW + rows - 1) / rows;
+  if (nchunk > max_chunk) nchunk = max_chunk;
+  if (nchunk < 1) nchunk = 1;
+  const int chunk_px2 = static_cast<int>((HW + nchunk - 1) / nchunk);
+  gn_silu_kernel<<<dim3(static_cast<unsigned>(nchunk), N), 256, 0, st>>>(
+      reinterpret_cast<const uint4*>(x), gamma, beta, stats, HW, C, G, chunk_px2,
       reinterpret_cast<uint4*>(y));
   return cudaGetLastError();
 }
