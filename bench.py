@@ -259,7 +259,7 @@ def run_reference(args, rank):
         "config": workload_config(w, args),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                          "sample": (f"each step: {w.name}, pack metadata, modulation vectors, "
-                                    f"then for every {stride}th token row adaLN and, "
+                                    f"then for one token row in {stride}, adaLN and, "
                                     f"for head 0 of {w.H}, RoPE + attention over the row's "
                                     f"sample + gated residual; fp64 NumPy ({api})")},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
