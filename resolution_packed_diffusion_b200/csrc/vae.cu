@@ -15,10 +15,11 @@
 // GroupNorm affine parameters and conv biases fp32.
 //
 // Kernels:
-//   gn_partial_kernel   per (pixel chunk, sample): each thread folds its
-//                       8-channel vectors into (count, mean, M2) (Chan's
-//                       pairwise update); the CTA merges them per group in a
-//                       fixed order and writes one partial per group.
+//   gn_partial_kernel   per (pixel chunk, sample): each thread sums its
+//                       8-channel vectors' values and squares about one of its
+//                       own values and turns them into (count, mean, M2); the
+//                       CTA merges those per group in a fixed order (Chan's
+//                       pairwise update) and writes one partial per group.
 //   gn_finalize_kernel  one CTA per (sample, group): merges the chunks'
 //                       partials in a fixed tree -> (mean, rstd). Deterministic.
 //   gn_silu_kernel      y = SiLU((x - mean) rstd gamma + beta), 16-byte vectors;
@@ -107,19 +108,28 @@ __global__ void __launch_bounds__(kGnThreads) gn_partial_kernel(
   const int n = blockIdx.y;
   const int p0 = blockIdx.x * chunk_px;
   const int p1 = min(HW, p0 + chunk_px);
-  Moments m = {0.f, 0.f, 0.f};
+  // this thread's pixels: sums of (value - K) and its square, K = its first
+  // value (a sample of the data keeps the shifted sums well conditioned), turned
+  // into (count, mean, M2) once at the end
   const uint4* xs = x + static_cast<size_t>(n) * HW * VP;
+  float K = 0.f, s1 = 0.f, s2 = 0.f, cnt = 0.f;
+  if (p0 + r < p1) K = __uint_as_float(__ldg(xs + static_cast<size_t>(p0 + r) * VP + v).x << 16);
+#pragma unroll 4
   for (int p = p0 + r; p < p1; p += rows) {
     float f[8];
     unpack8(__ldg(xs + static_cast<size_t>(p) * VP + v), f);
-    float s = 0.f;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) s += f[e];
-    const float bm = s * 0.125f;
-    float b2 = 0.f;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) b2 = fmaf(f[e] - bm, f[e] - bm, b2);
-    m = merge(m, Moments{8.f, bm, b2});
+    for (int e = 0; e < 8; ++e) {
+      const float d = f[e] - K;
+      s1 += d;
+      s2 = fmaf(d, d, s2);
+    }
+    cnt += 8.f;
+  }
+  Moments m = {0.f, 0.f, 0.f};
+  if (cnt > 0.f) {
+    const float dm = s1 / cnt;
+    m = Moments{cnt, K + dm, fmaxf(s2 - s1 * dm, 0.f)};
   }
   s_m[threadIdx.x] = m;
   __syncthreads();
