@@ -720,6 +720,29 @@ def check_gelu_bwd_vs_torch(gelu_tanh_bwd):
     assert np.allclose(gelu_tanh_bwd(z, dh), zt.grad.numpy(), rtol=0, atol=1e-12)
 
 
+def check_linear_bwd_vs_autograd(modality_linear_bwd):
+    """torch autograd (float64) through out[t] = x[t] @ W[m(t)]^T, the rows of
+    each modality routed by index (a library matmul per modality), gives the
+    same dx and dW; a modality without tokens gets dW[m] = 0."""
+    rng = np.random.default_rng(103)
+    T, K, N = 37, 24, 16
+    x = rng.standard_normal((T, K))
+    W = rng.standard_normal((2, N, K))
+    dout = rng.standard_normal((T, N))
+    for tok_mod in (rng.integers(0, 2, T).astype(np.uint8), np.zeros(T, dtype=np.uint8)):
+        xt = torch.tensor(x, requires_grad=True)
+        Wt = torch.tensor(W, requires_grad=True)
+        out = torch.zeros((T, N), dtype=torch.float64)
+        for m in (0, 1):
+            idx = torch.tensor(np.nonzero(tok_mod == m)[0])
+            out = out.index_add(0, idx, xt[idx] @ Wt[m].T)
+        out.backward(torch.tensor(dout))
+        dx, dW = modality_linear_bwd(x, W, tok_mod, dout)
+        assert np.allclose(dx, xt.grad.numpy(), rtol=0, atol=1e-12)
+        assert np.allclose(dW, Wt.grad.numpy(), rtol=0, atol=1e-12)
+    assert np.all(dW[1] == 0.0)  # the last case has no text token
+
+
 def check_mmdit_bwd_finite_diff(mmdit_block_bwd, mmdit_block_fwd):
     """Directional derivatives of L = <dy, y> of the unrounded whole block by
     central differences match <grad, direction> for x, all six weight tensors

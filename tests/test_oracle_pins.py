@@ -249,6 +249,10 @@ def test_gelu_bwd_vs_torch():
     pins.check_gelu_bwd_vs_torch(oracle.gelu_tanh_bwd)
 
 
+def test_linear_bwd_vs_autograd():
+    pins.check_linear_bwd_vs_autograd(oracle.modality_linear_bwd)
+
+
 def test_mmdit_bwd_finite_diff():
     pins.check_mmdit_bwd_finite_diff(oracle.mmdit_block_bwd, oracle.mmdit_block_fwd)
 
